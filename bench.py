@@ -1,0 +1,395 @@
+#!/usr/bin/env python
+"""Benchmark of the GPTQ layer solver on B200: Gparam/s and Hessian TFLOP/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload layer-1024x4096] [--no-cpu-baseline] [--no-e2e]
+
+One step = one pass of the whole path over one layer: H = 2.X.X^T from the
+calibration activations, preparation (damping, act-order, the Cholesky factor
+U) and quantization (sweep, lazy trailing updates, packing), inputs resident in
+HBM.  Each step is timed with CUDA events on the launching stream; L2 is
+flushed (a 256 MiB write) between steps, outside the timed events.
+
+With N > 1 (torchrun, one process per GPU) every rank quantizes its own,
+independently seeded layer: layers are independent problems, so there is no
+data-path collective and scaling is weak; the process group only carries the
+barrier and the max-over-ranks of the timings.
+
+`--impl reference` times the fp64 CPU oracle on rank 0 (the other ranks exit),
+each step on a bounded token sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic as S  # noqa: E402
+
+METRIC = "GPTQ layer quantize: weights/sec (Gparam/s) + Hessian TFLOP/s, % roofline, 1 B200"
+UNIT = "Gparam/s"
+DEFAULT_WORKLOAD = "layer-1024x4096"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------- #
+# helpers
+# --------------------------------------------------------------------------- #
+def env_rank():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["_source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["_source"] = "fallback"
+    return d
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.t is not None:
+            self.t.join(timeout=5)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None, "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------- #
+# CPU oracle leg (bounded sample)
+# --------------------------------------------------------------------------- #
+def oracle_sample(layer: S.Layer, st: S.QuantSettings, tokens: int):
+    """Run the oracle on the full layer with the first `tokens` calibration tokens.
+
+    Returns (seconds extrapolated to the full token count, sample description).
+    The Hessian's cost is linear in tokens; preparation and sweep do not depend on them.
+    """
+    from oracle import gptq_oracle as O  # the oracle is only ever run here, for the CPU baseline
+    W = S.make_w(layer.w)
+    x = S.make_x(layer.x, 0, tokens)
+    t0 = time.perf_counter()
+    H = O.hessian(x)
+    t1 = time.perf_counter()
+    prep = O.prepare(H, st.damp_percent, st.desc_act)
+    sw, codes = O.quantize_layer(W, prep, st.bits, st.group_size, st.sym, st.block)
+    O.pack(codes, st.bits)
+    O.g_idx(prep.perm, st.group_size)
+    t2 = time.perf_counter()
+    scale = layer.x.tokens / tokens
+    est = (t1 - t0) * scale + (t2 - t1)
+    desc = (f"full layer {layer.w.out}x{layer.w.n} (prepare, sweep, pack run in full); Hessian on the first "
+            f"{tokens} of {layer.x.tokens} tokens, its time scaled x{scale:g}; measured {t2 - t0:.1f} s")
+    return est, desc
+
+
+# --------------------------------------------------------------------------- #
+# reference arm: the oracle
+# --------------------------------------------------------------------------- #
+def run_reference(args):
+    rank, _, world = env_rank()
+    if rank != 0:
+        return 0
+    wl = S.workloads()[args.workload]
+    layer, st = wl.layers[0], wl.settings[0]
+    tokens = min(layer.x.tokens, args.ref_tokens)
+    times = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        est, desc = oracle_sample(layer, st, tokens)
+        if i >= args.warmup:
+            times.append(est)
+    t = statistics.mean(times)
+    value = layer.w.out * layer.w.n / t / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(args.workload, layer, st),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": host_cores(), "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(name, layer, st):
+    return {"workload": name, "out": layer.w.out, "in": layer.w.n, "tokens": layer.x.tokens,
+            "w_dtype": layer.w.dtype, "bits": st.bits, "group_size": st.group_size, "sym": st.sym,
+            "desc_act": st.desc_act, "damp_percent": st.damp_percent, "block": st.block,
+            "x": f"bf16 outlier/low-rank synthetic, rank {layer.x.rank}, {layer.x.outlier_frac:g} outliers "
+                 f"x{layer.x.outlier_mult:g}",
+            "l2": "flushed between steps (256 MiB write outside the per-step events)"}
+
+
+# --------------------------------------------------------------------------- #
+# our arm
+# --------------------------------------------------------------------------- #
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import post_weight_quantization_15_b200 as G
+
+    rank, local_rank, world = env_rank()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    wl = S.workloads()[args.workload]
+    layer0, st = wl.layers[0], wl.settings[0]
+    # independent problem per rank
+    import dataclasses
+    layer = dataclasses.replace(layer0, w=dataclasses.replace(layer0.w, seed=layer0.w.seed + rank),
+                                x=dataclasses.replace(layer0.x, seed=layer0.x.seed + rank))
+    out, n, N = layer.w.out, layer.w.n, layer.x.tokens
+
+    W_np = S.make_w(layer.w)
+    X_np = S.make_x(layer.x)
+    W_host = torch.from_numpy(W_np).pin_memory()
+    X_host = torch.from_numpy(X_np.view(np.int16)).pin_memory()
+    W = W_host.to(dev)
+    X = X_host.to(dev).view(torch.bfloat16)
+
+    stream = torch.cuda.current_stream()
+    status = G.new_status(dev)
+    H = torch.empty((n, n), dtype=torch.float32, device=dev)
+    hdiag = torch.empty(n, dtype=torch.float64, device=dev) if st.desc_act else None
+    prep_ws = G.workspace(G.lib().gptq_prepare_workspace_size(n), dev)
+    q_ws = G.workspace(G.quantize_workspace_size(out, n, st.block), dev)
+    prep = G.Prepared(U=torch.empty((n, n), dtype=torch.float32, device=dev),
+                      perm=torch.empty(n, dtype=torch.int32, device=dev),
+                      dead=torch.empty(n, dtype=torch.uint8, device=dev), status=status, desc_act=st.desc_act)
+    qout = G.alloc_quantized(out, n, st.bits, st.group_size, st.sym, dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+
+    def step(e=None):
+        G.status_reset(status)
+        H.zero_()
+        if hdiag is not None:
+            hdiag.zero_()
+        if e is not None:
+            e[0].record(stream)
+        G.hessian_accumulate(H, X, hdiag, status)
+        if e is not None:
+            e[1].record(stream)
+        G.prepare(H, st.damp_percent, st.desc_act, hdiag, status, ws=prep_ws, out=prep)
+        if e is not None:
+            e[2].record(stream)
+        G.quantize_layer(W, prep, st.bits, st.group_size, st.sym, st.block, ws=q_ws, out=qout)
+        if e is not None:
+            e[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+        flush.fill_(1.0)
+    torch.cuda.synchronize()
+    G.raise_on_status(status, "warm-up")
+
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    launches0 = G.kernel_launches()
+    t_wall0 = time.perf_counter()
+    for i in range(args.steps):
+        step(ev[i])
+        flush.fill_(1.0)
+    torch.cuda.synchronize()
+    t_wall1 = time.perf_counter()
+    launches = G.kernel_launches() - launches0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    G.raise_on_status(status, "timed steps")
+
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
+    hess_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    prep_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    quant_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    ms = statistics.mean(step_ms)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * out * n / (ms * 1e-3) / 1e9
+
+    # dominant kernel: the Hessian tile product (one launch per step)
+    peaks = load_peaks()
+    h_flops = float(n) * (n + 1) * N
+    h_s = statistics.mean(hess_ms) * 1e-3
+    achieved = h_flops / h_s / 1e12
+    peak = float(peaks["bf16_tflops"])
+    roofline = {"kernel": "hessian (K1)", "bound": "tensor", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                "peak_source": f"{peaks['_source']} bf16 burst",
+                "work": f"n(n+1)N = {h_flops:.4g} flop per launch (upper triangle incl. diagonal)"}
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(G, torch, W_host, X_host, st, n, out, dev, args.steps, flush)
+        if world > 1:
+            t = torch.tensor([e2e["ms_per_step"]], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e["ms_per_step"] = float(t.item())
+            e2e["value"] = world * out * n / (e2e["ms_per_step"] * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        est, desc = oracle_sample(layer, st, min(N, args.ref_tokens))
+        cpu = {"value": out * n / est / 1e9, "unit": UNIT, "cores": host_cores(), "kind": "oracle", "sample": desc}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16->f32 (Hessian), f32 (solver)", "data": "synthetic",
+        "config": config_dict(args.workload, layer0, st),
+        "hessian_tflops": achieved,
+        "stages_ms": {"hessian": statistics.mean(hess_ms), "prepare": statistics.mean(prep_ms),
+                      "quantize": statistics.mean(quant_ms)},
+        "wall_ms_per_step_incl_flush": (t_wall1 - t_wall0) * 1e3 / args.steps,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_e2e(G, torch, W_host, X_host, st, n, out, dev, steps, flush):
+    """Gparam/s through gptq_quantize with host inputs: H2D of W and X, D2H of the stored result."""
+    stream = torch.cuda.current_stream()
+    times = []
+    h2d = W_host.numel() * W_host.element_size() + X_host.numel() * X_host.element_size()
+    d2h = 0
+    res_host = None
+    for i in range(steps + 1):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        W = W_host.to(dev, non_blocking=True)
+        X = X_host.to(dev, non_blocking=True).view(torch.bfloat16)
+        q, prep, H = G.gptq_quantize(W, X, st.bits, st.group_size, st.sym, st.desc_act, st.damp_percent,
+                                     st.block, check=False)
+        if res_host is None:
+            res_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                        for t in (q.qweight, q.scales, q.zeros, q.g_idx)]
+            d2h = sum(t.numel() * t.element_size() for t in res_host)
+        for h, t in zip(res_host, (q.qweight, q.scales, q.zeros, q.g_idx)):
+            h.copy_(t, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        G.raise_on_status(prep.status, "e2e")
+        if i > 0:                       # the first pass also allocates the pinned result buffers
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.mean(times)
+    return {"value": out * n / (ms * 1e-3) / 1e9, "unit": UNIT, "ms_per_step": ms, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(S.workloads().keys()))
+    ap.add_argument("--ref-tokens", type=int, default=8192,
+                    help="token sample of the CPU oracle legs (its Hessian time is scaled to the full count)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

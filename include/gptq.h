@@ -1,0 +1,179 @@
+/*
+ * gptq.h - C ABI of the B200 GPTQ layer-solver library (libgptq.so).
+ *
+ * GPTQ quantizes one linear layer W [out, in] so that ||W.X - What.X||^2 is small
+ * ("polydesk.ai/glossaire/gptq", section "Comment fonctionne l'algorithme GPTQ"):
+ * columns are quantized one after another, and each column's rounding error is
+ * pushed onto the columns not yet quantized through the upper Cholesky factor of
+ * the damped inverse Hessian, in lazy batches of 128 columns (same page, "Etape 2"
+ * and "Etape 3").  The calls below are the steps of that path:
+ *
+ *   gptq_hessian_accumulate   H += 2 . X . X^T                    ("Etape 2")
+ *   gptq_prepare              dead inputs, act-order, damping, U  ("Etape 2"; desc_act)
+ *   gptq_quantize_layer       column sweep, lazy trailing update,
+ *                             packed qweight / fp16 scales, zeros / g_idx
+ *   gptq_pack                 the bit-packing step on its own
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensor pointers are DEVICE pointers to memory the caller owns.  The
+ *   library allocates nothing: calls that need scratch take a caller-provided
+ *   workspace whose size the matching *_workspace_size() call reports.
+ * - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *   Every call only enqueues work on that stream and returns; calls on one
+ *   stream run in order.  Calls on different streams that share buffers race.
+ * - Argument errors are returned synchronously (nothing is enqueued).
+ *   Errors found on the device (a non-positive Cholesky pivot, non-finite
+ *   values, a bounded wait that gave up) are recorded in a caller-provided
+ *   device status block `d_status` (int32[4]: code, info, stage, reserved):
+ *   the first error wins, and every later kernel that sees a non-zero code
+ *   skips its work.  Clear it with gptq_status_reset() before a layer and read
+ *   it with gptq_status_read(), which synchronizes the stream.
+ * - Matrices are row-major with the stated leading dimensions.
+ * - The library targets sm_100a (B200) only.
+ */
+#ifndef GPTQ_B200_H
+#define GPTQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GPTQ_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define GPTQ_API __attribute__((visibility("default")))
+#else
+#define GPTQ_API
+#endif
+
+typedef enum {
+  GPTQ_OK = 0,
+  GPTQ_ERR_INVALID_ARG = -1,  /* a pointer, size or stride is invalid               */
+  GPTQ_ERR_UNSUPPORTED = -2,  /* a valid combination this build does not implement */
+  GPTQ_ERR_NOT_SPD = -3,      /* damped Hessian not positive definite; info = pivot  */
+  GPTQ_ERR_NONFINITE = -4,    /* NaN/Inf in W or H; info = column or pivot           */
+  GPTQ_ERR_CUDA = -5,         /* a CUDA runtime call failed                          */
+  GPTQ_ERR_TIMEOUT = -6,      /* a bounded on-device wait gave up                    */
+  GPTQ_ERR_WORKSPACE = -7     /* workspace too small or misaligned                   */
+} gptq_status;
+
+typedef enum { GPTQ_F32 = 0, GPTQ_F16 = 1, GPTQ_BF16 = 2 } gptq_dtype;
+
+/* Library / ABI version (GPTQ_ABI_VERSION). */
+GPTQ_API int gptq_version(void);
+
+/* Number of kernels this library has enqueued since it was loaded (all
+ * devices, all streams; host-side counter, for accounting in benchmarks). */
+GPTQ_API uint64_t gptq_kernel_launches(void);
+
+/* Human-readable name of a gptq_status code (static string). */
+GPTQ_API const char* gptq_status_string(int status);
+
+/* Clears the device status block (int32[4]) on `stream`. */
+GPTQ_API int gptq_status_reset(int32_t* d_status, void* stream);
+
+/* Synchronizes `stream`, then returns the code stored in d_status[0]
+ * (GPTQ_OK if none) and, when `info` is not NULL, d_status[1] (the failing
+ * pivot or column).  Returns GPTQ_ERR_CUDA if the synchronization fails. */
+GPTQ_API int gptq_status_read(const int32_t* d_status, void* stream, int32_t* info);
+
+/*
+ * gptq_hessian_accumulate - H += 2 . X . X^T on the tensor cores.
+ *
+ * "polydesk.ai/glossaire/gptq", "Etape 2": the Hessian is approximated by
+ * H = 2.X.X^T from the calibration activations.  Calling this once per chunk
+ * of tokens accumulates the sum over all chunks.
+ *
+ *   H        fp32 [n, n], ld = n.  Only the upper triangle (j >= i) is updated
+ *            and later read; the lower triangle is left unspecified (diagonal
+ *            tiles may write it).  Zero it before the first chunk.
+ *   hdiag    optional fp64 [n] (NULL to skip): hdiag[i] += 2 . sum_t X[i,t]^2,
+ *            accumulated in fp64 from exact bf16 squares.  gptq_prepare uses it
+ *            as the act-order key, so that the order does not depend on the
+ *            fp32 summation order of H.
+ *   X        bf16 [n, tokens] (features x tokens, tokens contiguous), row
+ *            stride ld_x elements; ld_x % 8 == 0 and X 16-byte aligned.
+ *   tokens   may be 0 (no-op).  Any n >= 1 and tokens >= 0 are accepted.
+ *   d_status may be NULL; bounded waits that give up report GPTQ_ERR_TIMEOUT there.
+ */
+GPTQ_API int gptq_hessian_accumulate(float* H, double* hdiag, int n, const void* X, int64_t ld_x,
+                            int64_t tokens, int32_t* d_status, void* stream);
+
+/*
+ * gptq_prepare - dead inputs, act-order, damping and the Cholesky factor U.
+ *
+ * In this order (the readings are those of the library's oracle):
+ *  1. inputs with diag(H) == 0 are dead: H_ii := 1 and dead[i] = 1;
+ *  2. desc_act ("polydesk.ai/glossaire/gptq", desc_act: decreasing activation
+ *     magnitude): perm = stable descending order of the key (hdiag if given,
+ *     else diag(H); dead inputs have key 1); otherwise perm = identity;
+ *  3. damping ("skillmd.com/skills/artubss/gptq", damp_percent): the permuted H
+ *     gets lambda = damp_percent . mean(diag H) added to its diagonal;
+ *  4. U = the upper-triangular Cholesky factor of the damped, permuted H^-1
+ *     (H^-1 = U^T . U), computed in fp32 through a Cholesky factorization
+ *     ("polydesk.ai/glossaire/gptq", "Etape 2").
+ *
+ *   H        fp32 [n, n] (upper triangle read; not modified).
+ *   hdiag    optional fp64 [n] act-order key (see gptq_hessian_accumulate).
+ *   U        fp32 [n, n] output, row-major, strictly-lower part set to 0.
+ *   perm     int32 [n] output: processing position k holds input column perm[k].
+ *   dead     uint8 [n] output.
+ *   ws       workspace of at least gptq_prepare_workspace_size(n) bytes, 256-byte aligned.
+ *   d_status required: GPTQ_ERR_NOT_SPD (info = failing pivot, in processing
+ *            order) or GPTQ_ERR_NONFINITE.
+ */
+GPTQ_API size_t gptq_prepare_workspace_size(int n);
+GPTQ_API int gptq_prepare(const float* H, const double* hdiag, int n, float damp_percent, int desc_act,
+                 float* U, int32_t* perm, uint8_t* dead, void* ws, size_t ws_bytes,
+                 int32_t* d_status, void* stream);
+
+/*
+ * gptq_quantize_layer - the column sweep, the lazy trailing update and packing.
+ *
+ * For every column j in processing order ("polydesk.ai/glossaire/gptq",
+ * "Etape 2"): at a group start the group's per-row scale and zero point are
+ * computed from the current, already compensated weights; the column is
+ * quantized (round to nearest even, decided in fp32); e = (w - what) / U_jj;
+ * the remaining columns of the block absorb e . U[j, :]; after each block of
+ * `block` columns the later columns absorb Err . U[block, later] at once
+ * ("Etape 3").  Symmetric codes use the grid [-2^(b-1)+1, 2^(b-1)-1] offset by
+ * z = 2^(b-1) ("sym"); asymmetric codes use a zero point in [0, 2^b-1].
+ *
+ *   W          [out, n] row-major, dtype w_dtype (F32, F16 or BF16); not modified.
+ *   U, perm, dead   from gptq_prepare (perm and dead may be NULL: identity / none).
+ *   bits       2, 3, 4 or 8.     group_size 32, 64, 128, or -1 (one group per row).
+ *   block      128 (the pages' batch); block % group_size == 0 when group_size > 0.
+ *   n % 32 == 0, and n % group_size == 0 when group_size > 0.  out >= 1.
+ *   qweight    int32 [n*bits/32, out]: per output row, the codes of the input
+ *              columns in original order as a little-endian bit stream (column k
+ *              at stream bits k*bits ...), word-major.
+ *   scales, zeros   fp16 (as uint16) [G, out], G = n / group_size (1 if -1),
+ *              in group (processing) order; zeros hold integers.
+ *   g_idx      int32 [n]: group of each input column (original order).
+ *   codes      optional uint8 [out, n], original column order (NULL to skip).
+ *   err_sq     optional fp32 [out]: per row, sum_j e_j^2 (NULL to skip).
+ *   ws         >= gptq_quantize_workspace_size(out, n, block) bytes, 256-byte aligned.
+ */
+GPTQ_API size_t gptq_quantize_workspace_size(int out, int n, int block);
+GPTQ_API int gptq_quantize_layer(const void* W, int w_dtype, int out, int n, const float* U,
+                        const int32_t* perm, const uint8_t* dead, int bits, int group_size,
+                        int sym, int block, int32_t* qweight, uint16_t* scales, uint16_t* zeros,
+                        int32_t* g_idx, uint8_t* codes, float* err_sq, void* ws, size_t ws_bytes,
+                        int32_t* d_status, void* stream);
+
+/*
+ * gptq_pack - bit-packing on its own: codes uint8 [out, n] (original order)
+ * -> qweight int32 [n*bits/32, out], the layout gptq_quantize_layer writes.
+ * bits in {2, 3, 4, 8}; n*bits % 32 == 0; codes must be < 2^bits.
+ */
+GPTQ_API int gptq_pack(const uint8_t* codes, int out, int n, int bits, int32_t* qweight, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_B200_H */

@@ -30,7 +30,7 @@ functions below (each says "reading").  Floating point that decides an integer
 everything else is fp64.
 
 Library primitives used as steps: matrix products (numpy), the Cholesky
-factorization and triangular solves (numpy / scipy LAPACK).
+factorization and the triangular inverse (numpy / scipy LAPACK).
 """
 from __future__ import annotations
 
@@ -39,6 +39,7 @@ from typing import Optional, Tuple
 
 import numpy as np
 import scipy.linalg
+import scipy.linalg.lapack
 
 __all__ = [
     "bf16_bits_to_f64", "hessian", "act_order", "prepare", "Prepared",
@@ -126,7 +127,9 @@ def prepare(H: np.ndarray, damp_percent: float, desc_act: bool,
     lam = float(damp_percent) * float(np.mean(np.diag(Hp)))
     Hd = Hp + lam * np.eye(n)
     L = np.linalg.cholesky(Hd)                                            # H_d = L L^T
-    Linv = scipy.linalg.solve_triangular(L, np.eye(n), lower=True)       # L^-1
+    Linv, info = scipy.linalg.lapack.dtrtri(L, lower=1)                  # L^-1
+    if info != 0:
+        raise np.linalg.LinAlgError("triangular inverse failed")
     Hinv = Linv.T @ Linv                                                 # H_d^-1
     Hinv = 0.5 * (Hinv + Hinv.T)
     U = np.linalg.cholesky(Hinv).T                                       # H_d^-1 = U^T U

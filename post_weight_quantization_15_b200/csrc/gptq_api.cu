@@ -1,0 +1,117 @@
+// The C ABI (include/gptq.h): argument checks, workspace sizes, status block.
+// Every call only enqueues kernels on the caller's stream; nothing is allocated.
+#include <cuda_runtime.h>
+
+#include <atomic>
+
+#include "common.cuh"
+#include "internal.h"
+
+using namespace gptq;
+
+namespace gptq {
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace gptq
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+bool valid_bits(int bits) { return bits == 2 || bits == 3 || bits == 4 || bits == 8; }
+bool valid_gs(int gs) { return gs == -1 || gs == 32 || gs == 64 || gs == 128; }
+
+}  // namespace
+
+extern "C" {
+
+int gptq_version(void) { return GPTQ_ABI_VERSION; }
+
+uint64_t gptq_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* gptq_status_string(int status) {
+  switch (status) {
+    case GPTQ_OK: return "ok";
+    case GPTQ_ERR_INVALID_ARG: return "invalid argument";
+    case GPTQ_ERR_UNSUPPORTED: return "unsupported combination";
+    case GPTQ_ERR_NOT_SPD: return "damped Hessian is not positive definite";
+    case GPTQ_ERR_NONFINITE: return "non-finite value in W or H";
+    case GPTQ_ERR_CUDA: return "CUDA runtime error";
+    case GPTQ_ERR_TIMEOUT: return "bounded device wait gave up";
+    case GPTQ_ERR_WORKSPACE: return "workspace too small or misaligned";
+    default: return "unknown status";
+  }
+}
+
+int gptq_status_reset(int32_t* d_status, void* stream) {
+  if (d_status == nullptr) return GPTQ_ERR_INVALID_ARG;
+  GPTQ_CUDA_TRY(cudaMemsetAsync(d_status, 0, 4 * sizeof(int32_t), as_stream(stream)));
+  return GPTQ_OK;
+}
+
+int gptq_status_read(const int32_t* d_status, void* stream, int32_t* info) {
+  if (d_status == nullptr) return GPTQ_ERR_INVALID_ARG;
+  int32_t h[4] = {0, 0, 0, 0};
+  GPTQ_CUDA_TRY(cudaMemcpyAsync(h, d_status, sizeof(h), cudaMemcpyDeviceToHost, as_stream(stream)));
+  GPTQ_CUDA_TRY(cudaStreamSynchronize(as_stream(stream)));
+  if (info) *info = h[1];
+  return h[0];
+}
+
+int gptq_hessian_accumulate(float* H, double* hdiag, int n, const void* X, int64_t ld_x, int64_t tokens,
+                            int32_t* d_status, void* stream) {
+  if (H == nullptr || n <= 0 || tokens < 0) return GPTQ_ERR_INVALID_ARG;
+  if (tokens == 0) return GPTQ_OK;
+  if (X == nullptr || ld_x < tokens || ld_x % 8 != 0 || !aligned(X, 16)) return GPTQ_ERR_INVALID_ARG;
+  int rc = launch_hessian(H, n, X, ld_x, tokens, d_status, as_stream(stream));
+  if (rc != GPTQ_OK) return rc;
+  if (hdiag) rc = launch_hessian_diag64(hdiag, n, X, ld_x, tokens, d_status, as_stream(stream));
+  return rc;
+}
+
+size_t gptq_prepare_workspace_size(int n) { return n > 0 ? prepare_ws_bytes(n) : 0; }
+
+int gptq_prepare(const float* H, const double* hdiag, int n, float damp_percent, int desc_act, float* U,
+                 int32_t* perm, uint8_t* dead, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (H == nullptr || U == nullptr || perm == nullptr || dead == nullptr || d_status == nullptr || n <= 0)
+    return GPTQ_ERR_INVALID_ARG;
+  if (!(damp_percent >= 0.f) || !(damp_percent < 1e30f)) return GPTQ_ERR_INVALID_ARG;
+  if (ws == nullptr || ws_bytes < prepare_ws_bytes(n) || !aligned(ws, 256)) return GPTQ_ERR_WORKSPACE;
+  return launch_prepare(H, hdiag, n, damp_percent, desc_act ? 1 : 0, U, perm, dead, ws, d_status,
+                        as_stream(stream));
+}
+
+size_t gptq_quantize_workspace_size(int out, int n, int block) {
+  if (out <= 0 || n <= 0) return 0;
+  return quantize_ws_bytes(out, n, block);
+}
+
+int gptq_quantize_layer(const void* W, int w_dtype, int out, int n, const float* U, const int32_t* perm,
+                        const uint8_t* dead, int bits, int group_size, int sym, int block, int32_t* qweight,
+                        uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq,
+                        void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (W == nullptr || U == nullptr || qweight == nullptr || scales == nullptr || zeros == nullptr ||
+      g_idx == nullptr || d_status == nullptr)
+    return GPTQ_ERR_INVALID_ARG;
+  if (out <= 0 || n <= 0) return GPTQ_ERR_INVALID_ARG;
+  if (w_dtype != GPTQ_F32 && w_dtype != GPTQ_F16 && w_dtype != GPTQ_BF16) return GPTQ_ERR_INVALID_ARG;
+  if (!valid_bits(bits) || !valid_gs(group_size)) return GPTQ_ERR_UNSUPPORTED;
+  if (block != 128) return GPTQ_ERR_UNSUPPORTED;
+  if (n % 32 != 0) return GPTQ_ERR_UNSUPPORTED;
+  if (group_size > 0 && (n % group_size != 0 || block % group_size != 0)) return GPTQ_ERR_UNSUPPORTED;
+  if (ws == nullptr || ws_bytes < quantize_ws_bytes(out, n, block) || !aligned(ws, 256)) return GPTQ_ERR_WORKSPACE;
+  return launch_quantize(W, w_dtype, out, n, U, perm, dead, bits, group_size, sym ? 1 : 0, block, qweight, scales,
+                         zeros, g_idx, codes, err_sq, ws, d_status, as_stream(stream));
+}
+
+int gptq_pack(const uint8_t* codes, int out, int n, int bits, int32_t* qweight, void* stream) {
+  if (codes == nullptr || qweight == nullptr || out <= 0 || n <= 0) return GPTQ_ERR_INVALID_ARG;
+  if (!valid_bits(bits)) return GPTQ_ERR_UNSUPPORTED;
+  if (((int64_t)n * bits) % 32 != 0) return GPTQ_ERR_UNSUPPORTED;
+  return launch_pack(codes, nullptr, out, n, n, bits, qweight, nullptr, as_stream(stream));
+}
+
+}  // extern "C"

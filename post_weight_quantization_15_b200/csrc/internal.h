@@ -1,0 +1,29 @@
+// Host-side launchers of the individual stages (internal to libgptq.so).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gptq {
+
+// ---- K1: Hessian -----------------------------------------------------------
+int launch_hessian(float* H, int n, const void* X, int64_t ld_x, int64_t tokens, int32_t* st,
+                   cudaStream_t s);
+int launch_hessian_diag64(double* hdiag, int n, const void* X, int64_t ld_x, int64_t tokens,
+                          int32_t* st, cudaStream_t s);
+
+// ---- K2: prepare -------------------------------------------------------------
+size_t prepare_ws_bytes(int n);
+int launch_prepare(const float* H, const double* hdiag, int n, float damp, int desc_act, float* U,
+                   int32_t* perm, uint8_t* dead, void* ws, int32_t* st, cudaStream_t s);
+
+// ---- K0/K3/K4/K5: quantize ---------------------------------------------------
+size_t quantize_ws_bytes(int out, int n, int block);
+int launch_quantize(const void* W, int w_dtype, int out, int n, const float* U, const int32_t* perm,
+                    const uint8_t* dead, int bits, int gs, int sym, int block, int32_t* qweight,
+                    uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq,
+                    void* ws, int32_t* st, cudaStream_t s);
+int launch_pack(const uint8_t* codes, const int32_t* invperm, int out, int n, int ld_codes, int bits,
+                int32_t* qweight, const int32_t* st, cudaStream_t s);
+
+}  // namespace gptq

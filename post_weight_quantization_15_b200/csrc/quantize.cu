@@ -1,0 +1,426 @@
+// K0 ingest, K3 column sweep, K4 lazy trailing update, K5 packing.
+//
+// "polydesk.ai/glossaire/gptq":
+//   "Etape 2" - per column: quantize (rounding + scale), take the error, push it
+//               onto the remaining columns through the inverse Hessian's
+//               Cholesky factor;
+//   "Etape 3" - the updates are batched per block of 128 columns;
+//   "sym"     - symmetric grid [-2^(b-1)+1, 2^(b-1)-1] with an exact zero, or an
+//               asymmetric zero point;
+//   group_size - groups sharing one scale (-1: one per row).
+// "dev.ayinedjimi-consultants.fr ... ia-quantization-gptq-gguf-awq",
+// "Calibration et dataset": scale and zero point are stored in FP16.
+#include <math.h>
+
+#include <algorithm>
+#include <type_traits>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace gptq {
+
+namespace {
+
+constexpr int BLK = 128;           // columns per lazy batch
+
+struct QuantWs {
+  float* Wf;          // [out, n] working weights, processing order
+  float* Err;         // [out, BLK] scaled errors of the current block
+  uint8_t* codes_p;   // [out, n] codes, processing order
+  int32_t* invperm;   // [n] processing position of every input column
+  float* rows;        // [out] row-wide scale, [out] row-wide zero (group_size = -1)
+};
+
+QuantWs carve(void* ws, int out, int n) {
+  char* p = static_cast<char*>(ws);
+  QuantWs w;
+  w.Wf = reinterpret_cast<float*>(p);        p += align_up((size_t)out * n * 4, 256);
+  w.Err = reinterpret_cast<float*>(p);       p += align_up((size_t)out * BLK * 4, 256);
+  w.codes_p = reinterpret_cast<uint8_t*>(p); p += align_up((size_t)out * n, 256);
+  w.invperm = reinterpret_cast<int32_t*>(p); p += align_up((size_t)n * 4, 256);
+  w.rows = reinterpret_cast<float*>(p);
+  return w;
+}
+
+// ---------------------------------------------------------------------------
+// The quantizer.  Every operation is one IEEE fp32 operation (round to nearest
+// even), so identical inputs give identical decisions on any IEEE machine.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float to_f16_scale(float s) {
+  // Round to FP16 (the stored precision) before use; keep within fp16's positive range.
+  const float kMin = 5.9604644775390625e-08f;  // 2^-24, the smallest fp16 subnormal
+  s = fminf(fmaxf(s, kMin), 65504.f);
+  return fmaxf(__half2float(__float2half_rn(s)), kMin);
+}
+
+struct QParams { float s, z; };
+
+__device__ __forceinline__ QParams params_asym(float lo, float hi, float maxq) {
+  lo = fminf(lo, 0.f);
+  hi = fmaxf(hi, 0.f);
+  if (hi == lo) { lo = -1.f; hi = 1.f; }
+  QParams p;
+  p.s = to_f16_scale(__fdiv_rn(__fsub_rn(hi, lo), maxq));
+  p.z = fminf(fmaxf(rintf(__fdiv_rn(-lo, p.s)), 0.f), maxq);
+  return p;
+}
+
+__device__ __forceinline__ QParams params_sym(float amax, int bits) {
+  if (amax == 0.f) amax = 1.f;
+  QParams p;
+  p.s = to_f16_scale(__fdiv_rn(amax, (float)((1 << (bits - 1)) - 1)));
+  p.z = (float)(1 << (bits - 1));
+  return p;
+}
+
+__device__ __forceinline__ float quant_code(float w, QParams p, int bits, bool sym) {
+  const float q = rintf(__fdiv_rn(w, p.s));
+  if (sym) {
+    const float h = (float)((1 << (bits - 1)) - 1);
+    return fminf(fmaxf(q, -h), h) + p.z;
+  }
+  return fminf(fmaxf(q + p.z, 0.f), (float)((1 << bits) - 1));
+}
+
+// ---------------------------------------------------------------------------
+// K0: Wf[r][k] = W[r][perm[k]] (0 for dead inputs), invperm, g_idx.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void ingest_kernel(const T* W, int out, int n, const int32_t* perm, const uint8_t* dead, int gs,
+                              float* Wf, int32_t* invperm, int32_t* g_idx, int32_t* st) {
+  if (has_error(st)) return;
+  const int k = blockIdx.x * 32 + threadIdx.x;
+  const int r = blockIdx.y * 8 + threadIdx.y;
+  if (k >= n) return;
+  const int src = perm ? perm[k] : k;
+  if (r == 0) {
+    invperm[src] = k;
+    g_idx[src] = gs > 0 ? k / gs : 0;
+  }
+  if (r >= out) return;
+  float v = load_as_float<T>(W + (int64_t)r * n + src);
+  if (!isfinite(v)) set_error(st, GPTQ_ERR_NONFINITE, src, STAGE_INGEST);
+  if (dead && dead[src]) v = 0.f;
+  Wf[(int64_t)r * n + k] = v;
+}
+
+// group_size = -1: one scale / zero per row, from the whole (uncompensated) row.
+__global__ void __launch_bounds__(256) row_params_kernel(const float* Wf, int out, int n, int bits, int sym,
+                                                         float* rows, uint16_t* scales, uint16_t* zeros,
+                                                         const int32_t* st) {
+  if (has_error(st)) return;
+  const int r = blockIdx.x;
+  if (r >= out) return;
+  float lo = INFINITY, hi = -INFINITY, amax = 0.f;
+  for (int k = threadIdx.x; k < n; k += blockDim.x) {
+    const float v = Wf[(int64_t)r * n + k];
+    lo = fminf(lo, v); hi = fmaxf(hi, v); amax = fmaxf(amax, fabsf(v));
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  }
+  __shared__ float red[3][8];
+  if ((threadIdx.x & 31) == 0) { red[0][threadIdx.x >> 5] = lo; red[1][threadIdx.x >> 5] = hi; red[2][threadIdx.x >> 5] = amax; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < 8; ++w) { lo = fminf(lo, red[0][w]); hi = fmaxf(hi, red[1][w]); amax = fmaxf(amax, red[2][w]); }
+    lo = fminf(lo, red[0][0]); hi = fmaxf(hi, red[1][0]); amax = fmaxf(amax, red[2][0]);
+    const QParams p = sym ? params_sym(amax, bits) : params_asym(lo, hi, (float)((1 << bits) - 1));
+    rows[r] = p.s;
+    rows[out + r] = p.z;
+    scales[r] = __half_as_ushort(__float2half_rn(p.s));
+    zeros[r] = __half_as_ushort(__float2half_rn(p.z));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K3: the sweep of one block [b0, b0 + bw) of columns.
+//
+// TPR lanes of one warp own one row; lane `seg` of the row holds the block's
+// columns [seg.SEG, seg.SEG + SEG) in registers.  For column j the owning lane's
+// error e is broadcast with a shuffle and every lane applies e . U[j, :] to its own
+// columns.  The U block sits in shared memory with its strictly-lower part
+// zeroed, so the update needs no masking: columns before j see U = 0, and the
+// owner overwrites column j with e afterwards.  Rows are independent given U
+// ("polydesk.ai/glossaire/gptq", "Etape 1": the inverse-Hessian work is shared by
+// all rows), so rows never synchronize.
+// GS = group size (32/64/128), or 0 for row-wide parameters given in `rows`.
+// ---------------------------------------------------------------------------
+template <int TPR>
+struct SweepShape {
+  static constexpr int SEG = BLK / TPR;          // columns per lane
+  static constexpr int SEGP = SEG + 4;           // padded segment stride in shared memory
+  static constexpr int LDU = TPR * SEGP;         // padded U row stride
+  static constexpr int THREADS = 128;
+  static constexpr int ROWS = THREADS / TPR;     // rows per CTA
+  static constexpr size_t SMEM = (size_t)BLK * LDU * sizeof(float) + BLK * sizeof(float);
+};
+
+template <int GS, int TPR>
+__global__ void __launch_bounds__(128)
+sweep_kernel(float* Wf, int out, int n, int b0, int bw, const float* U, float* Err, uint8_t* codes_p,
+             uint16_t* scales, uint16_t* zeros, const float* rows, float* err_sq, int bits, int sym,
+             const int32_t* st) {
+  using SS = SweepShape<TPR>;
+  constexpr int SEG = SS::SEG;
+  if (has_error(st)) return;
+  extern __shared__ float smem[];
+  float* Us = smem;                       // [BLK][LDU]
+  float* dinv = smem + BLK * SS::LDU;     // [BLK] 1 / U_jj
+  for (int idx = threadIdx.x; idx < BLK * BLK; idx += blockDim.x) {
+    const int j = idx / BLK, c = idx % BLK;
+    const float v = (j < bw && c < bw && c >= j) ? U[(int64_t)(b0 + j) * n + b0 + c] : 0.f;
+    Us[j * SS::LDU + (c / SEG) * SS::SEGP + (c % SEG)] = v;
+    if (c == j) dinv[j] = (j < bw) ? 1.f / v : 0.f;
+  }
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31;
+  const int seg = lane % TPR;
+  const int r = blockIdx.x * SS::ROWS + threadIdx.x / TPR;
+  const bool live = r < out;
+  const int rr = live ? r : 0;
+  float w[SEG];
+  {
+    const float* src = Wf + (int64_t)rr * n + b0 + seg * SEG;
+    const bool inb = live && seg * SEG < bw;
+#pragma unroll
+    for (int k = 0; k < SEG; k += 4) {
+      float4 v = inb ? *reinterpret_cast<const float4*>(src + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+      w[k] = v.x; w[k + 1] = v.y; w[k + 2] = v.z; w[k + 3] = v.w;
+    }
+  }
+  const bool symq = sym != 0;
+  const float maxq = (float)((1 << bits) - 1);
+  QParams p;
+  if (GS == 0) { p.s = rows[rr]; p.z = rows[out + rr]; }
+  else { p.s = 1.f; p.z = 0.f; }
+  float esq = 0.f;
+  uint32_t cw[SEG / 4];
+#pragma unroll
+  for (int k = 0; k < SEG / 4; ++k) cw[k] = 0u;
+  const int group_lane0 = lane & ~(TPR - 1);
+
+  for (int jb = 0; jb < TPR; ++jb) {
+    if (jb * SEG >= bw) break;
+    const bool owner = seg == jb;
+#pragma unroll
+    for (int jj = 0; jj < SEG; ++jj) {
+      const int j = jb * SEG + jj;
+      if (GS > 0 && jj == 0 && ((b0 + j) % (GS > 0 ? GS : 1)) == 0) {
+        // group [j, j + GS): lanes whose segment lies inside it contribute
+        const int g_lo = j, g_hi = j + GS;
+        const bool in = seg * SEG >= g_lo && seg * SEG + SEG <= g_hi;
+        float lo = INFINITY, hi = -INFINITY, amax = 0.f;
+        if (in) {
+#pragma unroll
+          for (int k = 0; k < SEG; ++k) { lo = fminf(lo, w[k]); hi = fmaxf(hi, w[k]); amax = fmaxf(amax, fabsf(w[k])); }
+        }
+#pragma unroll
+        for (int o = 1; o < TPR; o <<= 1) {
+          lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+          hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        }
+        p = symq ? params_sym(amax, bits) : params_asym(lo, hi, maxq);
+        if (owner && live) {
+          const int g = (b0 + j) / (GS > 0 ? GS : 1);
+          scales[(int64_t)g * out + r] = __half_as_ushort(__float2half_rn(p.s));
+          zeros[(int64_t)g * out + r] = __half_as_ushort(__float2half_rn(p.z));
+        }
+      }
+      const float c = quant_code(w[jj], p, bits, symq);
+      const float e_own = (w[jj] - p.s * (c - p.z)) * dinv[j];
+      const float e = __shfl_sync(0xffffffffu, e_own, group_lane0 | jb);
+      const float* urow = Us + j * SS::LDU + seg * SS::SEGP;
+#pragma unroll
+      for (int k = 0; k < SEG; k += 4) {
+        const float4 u = *reinterpret_cast<const float4*>(urow + k);
+        w[k] = fmaf(-e, u.x, w[k]);
+        w[k + 1] = fmaf(-e, u.y, w[k + 1]);
+        w[k + 2] = fmaf(-e, u.z, w[k + 2]);
+        w[k + 3] = fmaf(-e, u.w, w[k + 3]);
+      }
+      if (owner) {
+        w[jj] = e;
+        esq = fmaf(e, e, esq);
+        cw[jj / 4] |= ((uint32_t)c) << (8 * (jj % 4));
+      }
+    }
+  }
+  if (!live || seg * SEG >= bw) {
+    // nothing to store for this lane
+  } else {
+    float* erow = Err + (int64_t)r * BLK + seg * SEG;
+#pragma unroll
+    for (int k = 0; k < SEG; k += 4) *reinterpret_cast<float4*>(erow + k) = make_float4(w[k], w[k + 1], w[k + 2], w[k + 3]);
+    uint8_t* crow = codes_p + (int64_t)r * n + b0 + seg * SEG;
+#pragma unroll
+    for (int k = 0; k < SEG; k += 16)
+      *reinterpret_cast<uint4*>(crow + k) = make_uint4(cw[k / 4], cw[k / 4 + 1], cw[k / 4 + 2], cw[k / 4 + 3]);
+  }
+#pragma unroll
+  for (int o = 1; o < TPR; o <<= 1) esq += __shfl_xor_sync(0xffffffffu, esq, o);
+  if (err_sq && live && seg == 0) err_sq[r] += esq;
+}
+
+// ---------------------------------------------------------------------------
+// K4: Wf[:, e:] -= Err . U[b0:b0+bw, e:]   (CUDA-core fp32 tiles)
+// ---------------------------------------------------------------------------
+constexpr int TT = 64;
+constexpr int TK = 16;
+
+__global__ void __launch_bounds__(256)
+trailing_kernel(float* Wf, int out, int n, int e, const float* Err, int bw, const float* Ub, const int32_t* st) {
+  if (has_error(st)) return;
+  __shared__ float As[TK][TT + 4];
+  __shared__ float Bs[TK][TT + 4];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int rbase = blockIdx.y * TT, cbase = e + blockIdx.x * TT;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < bw; k0 += TK) {
+    for (int idx = threadIdx.x; idx < TT * TK; idx += 256) {
+      {
+        const int r = idx / TK, k = idx % TK;
+        const int gr = rbase + r;
+        As[k][r] = (gr < out && k0 + k < bw) ? Err[(int64_t)gr * BLK + k0 + k] : 0.f;
+      }
+      {
+        const int k = idx / TT, c = idx % TT;
+        const int gc = cbase + c;
+        Bs[k][c] = (gc < n && k0 + k < bw) ? Ub[(int64_t)(k0 + k) * n + gc] : 0.f;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < TK; ++k) {
+      float a[4], b[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) { a[u] = As[k][ty * 4 + u]; b[u] = Bs[k][tx * 4 + u]; }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(a[u], b[v], acc[u][v]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int gr = rbase + ty * 4 + u;
+    if (gr >= out) continue;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int gc = cbase + tx * 4 + v;
+      if (gc < n) Wf[(int64_t)gr * n + gc] -= acc[u][v];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K5: qweight[w][o] = bits of the codes of input columns k with k.bits in
+// [32w, 32w + 32), original order; code of column k = codes[o][invperm[k]].
+// ---------------------------------------------------------------------------
+__global__ void pack_kernel(const uint8_t* codes, const int32_t* invperm, int out, int n, int ld_codes,
+                            int bits, int32_t* qweight, const int32_t* st) {
+  if (has_error(st)) return;
+  const int o = blockIdx.x * blockDim.x + threadIdx.x;
+  const int wi = blockIdx.y;
+  if (o >= out) return;
+  const int pos0 = wi * 32;
+  const int k_lo = pos0 / bits, k_hi = (pos0 + 31) / bits;
+  uint64_t acc = 0;
+  const uint8_t* crow = codes + (int64_t)o * ld_codes;
+  for (int k = k_lo; k <= k_hi && k < n; ++k) {
+    const int src = invperm ? invperm[k] : k;
+    const uint64_t c = crow[src] & ((1u << bits) - 1u);
+    const int sh = k * bits - pos0;  // may be negative for a code straddling in from the left
+    if (sh >= 0) acc |= c << sh; else acc |= c >> (-sh);
+  }
+  qweight[(int64_t)wi * out + o] = (int32_t)(uint32_t)(acc & 0xFFFFFFFFull);
+}
+
+// Optional output: codes in the original column order.
+__global__ void codes_out_kernel(const uint8_t* codes_p, const int32_t* invperm, int out, int n, uint8_t* codes,
+                                 const int32_t* st) {
+  if (has_error(st)) return;
+  const int k = blockIdx.x * 32 + threadIdx.x;
+  const int r = blockIdx.y * 8 + threadIdx.y;
+  if (k >= n || r >= out) return;
+  codes[(int64_t)r * n + k] = codes_p[(int64_t)r * n + invperm[k]];
+}
+
+}  // namespace
+
+size_t quantize_ws_bytes(int out, int n, int block) {
+  (void)block;
+  return align_up((size_t)out * n * 4, 256) + align_up((size_t)out * BLK * 4, 256) + align_up((size_t)out * n, 256) +
+         align_up((size_t)n * 4, 256) + align_up((size_t)out * 8, 256);
+}
+
+int launch_pack(const uint8_t* codes, const int32_t* invperm, int out, int n, int ld_codes, int bits,
+                int32_t* qweight, const int32_t* st, cudaStream_t s) {
+  const int words = n * bits / 32;
+  dim3 grd((unsigned)cdiv(out, 128), (unsigned)words);
+  pack_kernel<<<grd, 128, 0, s>>>(codes, invperm, out, n, ld_codes, bits, qweight, st);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
+int launch_quantize(const void* W, int w_dtype, int out, int n, const float* U, const int32_t* perm,
+                    const uint8_t* dead, int bits, int gs, int sym, int block, int32_t* qweight,
+                    uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq,
+                    void* ws, int32_t* st, cudaStream_t s) {
+  (void)block;
+  QuantWs w = carve(ws, out, n);
+  {
+    dim3 blk(32, 8), grd((unsigned)cdiv(n, 32), (unsigned)cdiv(std::max(out, 1), 8));
+    if (w_dtype == GPTQ_F32)
+      ingest_kernel<float><<<grd, blk, 0, s>>>(static_cast<const float*>(W), out, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
+    else if (w_dtype == GPTQ_F16)
+      ingest_kernel<__half><<<grd, blk, 0, s>>>(static_cast<const __half*>(W), out, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
+    else
+      ingest_kernel<__nv_bfloat16><<<grd, blk, 0, s>>>(static_cast<const __nv_bfloat16*>(W), out, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
+    GPTQ_LAUNCH_CHECK();
+  }
+  if (err_sq) GPTQ_CUDA_TRY(cudaMemsetAsync(err_sq, 0, (size_t)out * 4, s));
+  if (gs <= 0) {
+    row_params_kernel<<<out, 256, 0, s>>>(w.Wf, out, n, bits, sym, w.rows, scales, zeros, st);
+    GPTQ_LAUNCH_CHECK();
+  }
+  // Few rows: 8 lanes per row (more parallelism); many rows: 4 (less redundant work).
+  const bool wide = out < 4096;
+  auto pick = [&](auto tpr_tag) {
+    constexpr int T = decltype(tpr_tag)::value;
+    return gs == 32 ? sweep_kernel<32, T> : gs == 64 ? sweep_kernel<64, T> : gs == 128 ? sweep_kernel<128, T>
+                                                                                      : sweep_kernel<0, T>;
+  };
+  auto sweep = wide ? pick(std::integral_constant<int, 8>{}) : pick(std::integral_constant<int, 4>{});
+  const size_t smem = wide ? SweepShape<8>::SMEM : SweepShape<4>::SMEM;
+  const int rows_per_cta = wide ? SweepShape<8>::ROWS : SweepShape<4>::ROWS;
+  GPTQ_CUDA_TRY(cudaFuncSetAttribute(sweep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  for (int b0 = 0; b0 < n; b0 += BLK) {
+    const int bw = std::min(BLK, n - b0);
+    sweep<<<(unsigned)cdiv(out, rows_per_cta), 128, smem, s>>>(w.Wf, out, n, b0, bw, U, w.Err, w.codes_p, scales,
+                                                                zeros, w.rows, err_sq, bits, sym, st);
+    GPTQ_LAUNCH_CHECK();
+    const int e = b0 + bw;
+    if (e < n) {
+      dim3 grd((unsigned)cdiv(n - e, TT), (unsigned)cdiv(out, TT));
+      trailing_kernel<<<grd, 256, 0, s>>>(w.Wf, out, n, e, w.Err, bw, U + (int64_t)b0 * n, st);
+      GPTQ_LAUNCH_CHECK();
+    }
+  }
+  int rc = launch_pack(w.codes_p, w.invperm, out, n, n, bits, qweight, st, s);
+  if (rc != GPTQ_OK) return rc;
+  if (codes) {
+    dim3 blk(32, 8), grd((unsigned)cdiv(n, 32), (unsigned)cdiv(out, 8));
+    codes_out_kernel<<<grd, blk, 0, s>>>(w.codes_p, w.invperm, out, n, codes, st);
+    GPTQ_LAUNCH_CHECK();
+  }
+  return GPTQ_OK;
+}
+
+}  // namespace gptq

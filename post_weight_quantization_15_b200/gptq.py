@@ -1,0 +1,293 @@
+"""Python binding of libgptq.so (ctypes): argument marshalling only.
+
+Every step of the path runs in the library's CUDA kernels.  PyTorch is used for
+device memory (the output tensors and the workspaces handed to the library) and
+for the current stream.  There is no fallback: if the library or a CUDA device is
+missing, every call raises.
+
+The calls mirror include/gptq.h:
+
+    hessian_accumulate(H, X, hdiag=None)          H += 2 . X . X^T
+    prepare(H, damp_percent, desc_act, hdiag)     -> Prepared(U, perm, dead)
+    quantize_layer(W, prep, bits, group_size, sym, block=128)
+                                                  -> QuantizedLayer(qweight, scales, zeros, g_idx, ...)
+    pack(codes, bits)                             -> qweight
+    gptq_quantize(W, X, ...)                      the whole path for one layer
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptq.so")
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED = -2
+ERR_NOT_SPD = -3
+ERR_NONFINITE = -4
+ERR_CUDA = -5
+ERR_TIMEOUT = -6
+ERR_WORKSPACE = -7
+
+F32, F16, BF16 = 0, 1, 2
+_DTYPE_CODE = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
+
+_lib = None
+
+
+class GptqError(RuntimeError):
+    def __init__(self, code: int, where: str, info: Optional[int] = None):
+        self.code = code
+        self.info = info
+        msg = f"{where}: {status_string(code)} ({code})"
+        if info is not None:
+            msg += f", info={info}"
+        super().__init__(msg)
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgptq.so (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"libgptq.so is not built ({_LIB_PATH}); run "
+                           "`python -m post_weight_quantization_15_b200.build`")
+    L = ctypes.CDLL(_LIB_PATH)
+    P, I, I64, SZ, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+    L.gptq_version.restype = I
+    L.gptq_version.argtypes = []
+    L.gptq_kernel_launches.restype = ctypes.c_uint64
+    L.gptq_kernel_launches.argtypes = []
+    L.gptq_status_string.restype = ctypes.c_char_p
+    L.gptq_status_string.argtypes = [I]
+    L.gptq_status_reset.restype = I
+    L.gptq_status_reset.argtypes = [P, P]
+    L.gptq_status_read.restype = I
+    L.gptq_status_read.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
+    L.gptq_hessian_accumulate.restype = I
+    L.gptq_hessian_accumulate.argtypes = [P, P, I, P, I64, I64, P, P]
+    L.gptq_prepare_workspace_size.restype = SZ
+    L.gptq_prepare_workspace_size.argtypes = [I]
+    L.gptq_prepare.restype = I
+    L.gptq_prepare.argtypes = [P, P, I, F, I, P, P, P, P, SZ, P, P]
+    L.gptq_quantize_workspace_size.restype = SZ
+    L.gptq_quantize_workspace_size.argtypes = [I, I, I]
+    L.gptq_quantize_layer.restype = I
+    L.gptq_quantize_layer.argtypes = [P, I, I, I, P, P, P, I, I, I, I, P, P, P, P, P, P, P, SZ, P, P]
+    L.gptq_pack.restype = I
+    L.gptq_pack.argtypes = [P, I, I, I, P, P]
+    _lib = L
+    return L
+
+
+def kernel_launches() -> int:
+    """Kernels enqueued by the library since it was loaded (host-side counter)."""
+    return int(lib().gptq_kernel_launches())
+
+
+def status_string(code: int) -> str:
+    try:
+        return lib().gptq_status_string(int(code)).decode()
+    except RuntimeError:
+        return str(code)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != OK:
+        raise GptqError(rc, where)
+
+
+def _require_cuda(*ts: Optional[torch.Tensor]):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A 256-byte-aligned device buffer of at least nbytes (torch allocations are)."""
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+# --------------------------------------------------------------------------- #
+# status block
+# --------------------------------------------------------------------------- #
+def new_status(device) -> torch.Tensor:
+    return torch.zeros(4, dtype=torch.int32, device=device)
+
+
+def status_reset(st: torch.Tensor, stream=None):
+    _check(lib().gptq_status_reset(_ptr(st), _stream(stream)), "gptq_status_reset")
+
+
+def status_read(st: torch.Tensor, stream=None):
+    info = ctypes.c_int32(0)
+    rc = lib().gptq_status_read(_ptr(st), _stream(stream), ctypes.byref(info))
+    return rc, info.value
+
+
+def raise_on_status(st: torch.Tensor, where: str, stream=None):
+    rc, info = status_read(st, stream)
+    if rc != OK:
+        raise GptqError(rc, where, info)
+
+
+# --------------------------------------------------------------------------- #
+# K1
+# --------------------------------------------------------------------------- #
+def hessian_accumulate(H: torch.Tensor, X: torch.Tensor, hdiag: Optional[torch.Tensor] = None,
+                       status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """H += 2 . X . X^T.  H fp32 [n, n]; X bf16 [n, tokens] (row stride may exceed tokens)."""
+    _require_cuda(H, X, hdiag, status)
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.stride(1) != 1:
+        raise ValueError("X must be a bf16 [n, tokens] tensor with contiguous rows")
+    n = X.shape[0]
+    if H.dtype != torch.float32 or tuple(H.shape) != (n, n) or not H.is_contiguous():
+        raise ValueError("H must be a contiguous fp32 [n, n] tensor")
+    if hdiag is not None and (hdiag.dtype != torch.float64 or hdiag.numel() != n):
+        raise ValueError("hdiag must be fp64 [n]")
+    _check(lib().gptq_hessian_accumulate(_ptr(H), _ptr(hdiag), n, _ptr(X), X.stride(0), X.shape[1],
+                                         _ptr(status), _stream(stream)), "gptq_hessian_accumulate")
+    return H
+
+
+# --------------------------------------------------------------------------- #
+# K2
+# --------------------------------------------------------------------------- #
+@dataclasses.dataclass
+class Prepared:
+    U: torch.Tensor       # fp32 [n, n] upper
+    perm: torch.Tensor    # int32 [n]
+    dead: torch.Tensor    # uint8 [n]
+    status: torch.Tensor  # int32 [4]
+    desc_act: bool
+
+
+def prepare(H: torch.Tensor, damp_percent: float = 0.01, desc_act: bool = False,
+            hdiag: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+            ws: Optional[torch.Tensor] = None, out: Optional[Prepared] = None, stream=None) -> Prepared:
+    _require_cuda(H, hdiag, status, ws)
+    n = H.shape[0]
+    if H.dtype != torch.float32 or tuple(H.shape) != (n, n) or not H.is_contiguous():
+        raise ValueError("H must be a contiguous fp32 [n, n] tensor")
+    dev = H.device
+    if status is None:
+        status = new_status(dev)
+    need = lib().gptq_prepare_workspace_size(n)
+    if ws is None or ws.numel() < need:
+        ws = workspace(need, dev)
+    if out is None:
+        out = Prepared(U=torch.empty((n, n), dtype=torch.float32, device=dev),
+                       perm=torch.empty(n, dtype=torch.int32, device=dev),
+                       dead=torch.empty(n, dtype=torch.uint8, device=dev), status=status, desc_act=bool(desc_act))
+    out.status = status
+    _check(lib().gptq_prepare(_ptr(H), _ptr(hdiag), n, float(damp_percent), int(bool(desc_act)), _ptr(out.U),
+                              _ptr(out.perm), _ptr(out.dead), _ptr(ws), ws.numel(), _ptr(status), _stream(stream)),
+           "gptq_prepare")
+    return out
+
+
+# --------------------------------------------------------------------------- #
+# K0 / K3 / K4 / K5
+# --------------------------------------------------------------------------- #
+@dataclasses.dataclass
+class QuantizedLayer:
+    qweight: torch.Tensor          # int32 [n*bits/32, out]
+    scales: torch.Tensor           # fp16 [G, out]
+    zeros: torch.Tensor            # fp16 [G, out]
+    g_idx: torch.Tensor            # int32 [n]
+    codes: Optional[torch.Tensor]  # uint8 [out, n] (original order) if requested
+    err_sq: Optional[torch.Tensor]  # fp32 [out] if requested
+    bits: int
+    group_size: int
+    sym: bool
+
+
+def quantize_workspace_size(out: int, n: int, block: int = 128) -> int:
+    return int(lib().gptq_quantize_workspace_size(out, n, block))
+
+
+def alloc_quantized(out: int, n: int, bits: int, group_size: int, sym: bool, device, want_codes=False,
+                    want_err=False) -> QuantizedLayer:
+    G = 1 if group_size == -1 else n // group_size
+    return QuantizedLayer(
+        qweight=torch.empty((n * bits // 32, out), dtype=torch.int32, device=device),
+        scales=torch.empty((G, out), dtype=torch.float16, device=device),
+        zeros=torch.empty((G, out), dtype=torch.float16, device=device),
+        g_idx=torch.empty(n, dtype=torch.int32, device=device),
+        codes=torch.empty((out, n), dtype=torch.uint8, device=device) if want_codes else None,
+        err_sq=torch.empty(out, dtype=torch.float32, device=device) if want_err else None,
+        bits=bits, group_size=group_size, sym=bool(sym))
+
+
+def quantize_layer(W: torch.Tensor, prep: Prepared, bits: int = 4, group_size: int = 128, sym: bool = False,
+                   block: int = 128, want_codes: bool = False, want_err: bool = False,
+                   ws: Optional[torch.Tensor] = None, out: Optional[QuantizedLayer] = None,
+                   stream=None) -> QuantizedLayer:
+    _require_cuda(W, ws)
+    if W.dim() != 2 or not W.is_contiguous() or W.dtype not in _DTYPE_CODE:
+        raise ValueError("W must be a contiguous fp32/fp16/bf16 [out, n] tensor")
+    o, n = W.shape
+    if prep.U.shape[0] != n:
+        raise ValueError("W and U disagree on n")
+    dev = W.device
+    need = quantize_workspace_size(o, n, block)
+    if ws is None or ws.numel() < need:
+        ws = workspace(need, dev)
+    if out is None:
+        out = alloc_quantized(o, n, bits, group_size, sym, dev, want_codes, want_err)
+    _check(lib().gptq_quantize_layer(_ptr(W), _DTYPE_CODE[W.dtype], o, n, _ptr(prep.U), _ptr(prep.perm),
+                                     _ptr(prep.dead), int(bits), int(group_size), int(bool(sym)), int(block),
+                                     _ptr(out.qweight), _ptr(out.scales), _ptr(out.zeros), _ptr(out.g_idx),
+                                     _ptr(out.codes), _ptr(out.err_sq), _ptr(ws), ws.numel(), _ptr(prep.status),
+                                     _stream(stream)), "gptq_quantize_layer")
+    return out
+
+
+def pack(codes: torch.Tensor, bits: int, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    _require_cuda(codes, out)
+    if codes.dtype != torch.uint8 or codes.dim() != 2 or not codes.is_contiguous():
+        raise ValueError("codes must be a contiguous uint8 [out, n] tensor")
+    o, n = codes.shape
+    if out is None:
+        out = torch.empty((n * bits // 32, o), dtype=torch.int32, device=codes.device)
+    _check(lib().gptq_pack(_ptr(codes), o, n, int(bits), _ptr(out), _stream(stream)), "gptq_pack")
+    return out
+
+
+# --------------------------------------------------------------------------- #
+# The whole path for one layer
+# --------------------------------------------------------------------------- #
+def gptq_quantize(W: torch.Tensor, X: torch.Tensor, bits: int = 4, group_size: int = 128, sym: bool = False,
+                  desc_act: bool = False, damp_percent: float = 0.01, block: int = 128,
+                  want_codes: bool = False, want_err: bool = False, check: bool = True):
+    """H = 2.X.X^T, prepare, quantize.  Returns (QuantizedLayer, Prepared, H)."""
+    n = X.shape[0]
+    dev = X.device
+    st = new_status(dev)
+    H = torch.zeros((n, n), dtype=torch.float32, device=dev)
+    hdiag = torch.zeros(n, dtype=torch.float64, device=dev) if desc_act else None
+    hessian_accumulate(H, X, hdiag, st)
+    prep = prepare(H, damp_percent, desc_act, hdiag, st)
+    q = quantize_layer(W, prep, bits, group_size, sym, block, want_codes, want_err)
+    if check:
+        raise_on_status(st, "gptq_quantize")
+    return q, prep, H

@@ -59,13 +59,21 @@ def _rng(seed: int, *key: int) -> np.random.Generator:
 # --------------------------------------------------------------------------- #
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round fp32 values to bf16 (round to nearest, ties to even); return the bit patterns."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
-    lsb = (u >> np.uint32(16)) & np.uint32(1)
-    r = (u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)
-    nan = np.isnan(x)
+    u = np.array(x, dtype=np.float32, copy=True).view(np.uint32)
+    nan = np.isnan(u.view(np.float32))
+    _round_bf16_inplace(u)
     if nan.any():
-        r = np.where(nan, np.uint32(0x7FC0), r)
-    return r.astype(np.uint16)
+        u[nan] = 0x7FC0
+    return u.astype(np.uint16)
+
+
+def _round_bf16_inplace(u: np.ndarray) -> None:
+    """u: uint32 view of finite fp32 values; leaves the bf16 pattern in the low 16 bits."""
+    t = np.right_shift(u, 16)
+    np.bitwise_and(t, 1, out=t)
+    t += np.uint32(0x7FFF)
+    u += t
+    np.right_shift(u, 16, out=u)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
@@ -115,10 +123,14 @@ def make_x(spec: XSpec, t0: int = 0, t1: Optional[int] = None) -> np.ndarray:
         w = b - a
         zr = _rng(spec.seed, spec.stream, _TAG_ZR, c).standard_normal((G.shape[1], w), dtype=np.float32)
         zn = _rng(spec.seed, spec.stream, _TAG_ZN, c).standard_normal((spec.n, w), dtype=np.float32)
-        blk = (G32 @ zr) + zn
+        blk = G32 @ zr
+        blk += zn
+        del zn
         blk *= s32[:, None]
+        u = blk.view(np.uint32)
+        _round_bf16_inplace(u)
         lo, hi = max(a, t0), min(b, t1)
-        out[:, lo - t0:hi - t0] = f32_to_bf16_bits(blk[:, lo - a:hi - a])
+        out[:, lo - t0:hi - t0] = u[:, lo - a:hi - a]
 
     chunks = range(t0 // X_CHUNK, (t1 + X_CHUNK - 1) // X_CHUNK)
     workers = max(1, min(len(chunks), os.cpu_count() or 1, 16))

@@ -1,0 +1,68 @@
+"""Comparison helpers shared by the GPU parity tests and the smoke check.
+
+The tolerances are those of the method's statement: codes may differ from the
+oracle's for at most 0.5 % of the weights (floating-point ties flip and the
+flips cascade through the compensation), the layer error ||WX - What X||^2 /
+||WX||^2 must be within 2 % of the oracle's, and scales / zeros within 1e-3
+relative on groups whose codes all match.  Packing and g_idx are bit-exact.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+from oracle import gptq_oracle as O
+
+CODE_MISMATCH_MAX = 0.005
+REL_ERR_TOL = 0.02
+SCALE_TOL = 1e-3
+
+
+@dataclasses.dataclass
+class Comparison:
+    code_mismatch: float
+    rel_err_gpu: float
+    rel_err_oracle: float
+    rel_err_ratio: float
+    scale_max_rel: float
+    zero_max_rel: float
+    groups_compared: int
+    pack_exact: bool
+    gidx_exact: bool
+    perm_equal: bool
+
+    def ok(self) -> bool:
+        return (self.code_mismatch <= CODE_MISMATCH_MAX and abs(self.rel_err_ratio - 1.0) <= REL_ERR_TOL
+                and self.scale_max_rel <= SCALE_TOL and self.zero_max_rel <= SCALE_TOL and self.pack_exact
+                and self.gidx_exact and self.perm_equal)
+
+
+def compare_layer(W: np.ndarray, H64: np.ndarray, ora: "O.LayerResult", qweight: np.ndarray, scales16: np.ndarray,
+                  zeros16: np.ndarray, gidx: np.ndarray, codes: np.ndarray, perm: np.ndarray, bits: int,
+                  group_size: int) -> Comparison:
+    n = W.shape[1]
+    perm_equal = np.array_equal(perm.astype(np.int64), ora.perm)
+    mism = float(np.mean(codes != ora.codes))
+    What = O.dequantize(qweight, scales16, zeros16, gidx, bits, n)
+    rel_g = O.layer_error(W, What, H64)
+    ratio = rel_g / ora.rel_err if ora.rel_err > 0 else (1.0 if rel_g == 0 else np.inf)
+    pack_exact = np.array_equal(O.pack(codes, bits).view(np.uint32), qweight.view(np.uint32))
+    gidx_exact = np.array_equal(O.g_idx(perm.astype(np.int64), group_size), gidx)
+    # groups (processing order) whose codes all match
+    gs = n if group_size == -1 else group_size
+    cp_g = codes[:, ora.perm]
+    cp_o = ora.codes[:, ora.perm]
+    G = n // gs
+    same = (cp_g == cp_o).reshape(codes.shape[0], G, gs).all(axis=2).T       # [G, out]
+    sg = scales16.astype(np.float64)
+    so = ora.scales.astype(np.float64)
+    zg = zeros16.astype(np.float64)
+    zo = ora.zeros.astype(np.float64)
+    if same.any():
+        s_rel = float(np.max(np.abs(sg[same] - so[same]) / np.maximum(np.abs(so[same]), 1e-30)))
+        z_rel = float(np.max(np.abs(zg[same] - zo[same]) / np.maximum(np.abs(zo[same]), 1.0)))
+    else:
+        s_rel = z_rel = 0.0
+    return Comparison(mism, rel_g, ora.rel_err, ratio, s_rel, z_rel, int(same.sum()), pack_exact, gidx_exact,
+                      perm_equal)

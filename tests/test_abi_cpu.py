@@ -1,0 +1,68 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+symbol include/gptq.h declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "gptq.h")) as f:
+        src = f.read()
+    return sorted(set(re.findall(r"GPTQ_API\s+[\w\s\*]+?\b(gptq_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    import post_weight_quantization_15_b200 as G
+    return G.lib()
+
+
+def test_header_declares_the_path():
+    names = _declared()
+    for required in ("gptq_hessian_accumulate", "gptq_prepare", "gptq_quantize_layer", "gptq_pack",
+                     "gptq_prepare_workspace_size", "gptq_quantize_workspace_size", "gptq_status_read"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_version_and_status_strings(L):
+    import post_weight_quantization_15_b200 as G
+    assert L.gptq_version() == 1
+    assert G.status_string(0) == "ok"
+    assert "positive definite" in G.status_string(-3)
+
+
+def test_workspace_sizes(L):
+    import post_weight_quantization_15_b200 as G
+    n = 4096
+    assert L.gptq_prepare_workspace_size(n) >= 2 * n * n * 4
+    assert G.quantize_workspace_size(1024, n) >= 1024 * n * 5
+    assert L.gptq_prepare_workspace_size(0) == 0
+
+
+def test_bad_arguments_rejected_without_a_gpu(L):
+    P = ctypes.c_void_p
+    fake = P(256)   # never dereferenced: every call below fails its argument checks first
+    assert L.gptq_quantize_layer(None, 0, 8, 128, fake, None, None, 4, 128, 0, 128, fake, fake, fake, fake,
+                                 None, None, fake, 1 << 30, fake, None) == -1
+    assert L.gptq_quantize_layer(fake, 0, 8, 128, fake, None, None, 5, 128, 0, 128, fake, fake, fake, fake,
+                                 None, None, fake, 1 << 30, fake, None) == -2
+    assert L.gptq_quantize_layer(fake, 0, 8, 100, fake, None, None, 4, 32, 0, 128, fake, fake, fake, fake,
+                                 None, None, fake, 1 << 30, fake, None) == -2
+    assert L.gptq_quantize_layer(fake, 0, 8, 128, fake, None, None, 4, 128, 0, 64, fake, fake, fake, fake,
+                                 None, None, fake, 1 << 30, fake, None) == -2
+    assert L.gptq_quantize_layer(fake, 0, 8, 128, fake, None, None, 4, 128, 0, 128, fake, fake, fake, fake,
+                                 None, None, fake, 16, fake, None) == -7
+    assert L.gptq_prepare(fake, None, 0, ctypes.c_float(0.01), 0, fake, fake, fake, fake, 1 << 30, fake, None) == -1
+    assert L.gptq_prepare(fake, None, 64, ctypes.c_float(0.01), 0, fake, fake, fake, fake, 16, fake, None) == -7
+    assert L.gptq_hessian_accumulate(fake, None, 64, fake, 100, 100, None, None) == -1   # ld_x % 8 != 0
+    assert L.gptq_hessian_accumulate(fake, None, 64, fake, 96, 0, None, None) == 0        # empty chunk
+    assert L.gptq_pack(fake, 4, 33, 4, fake, None) == -2

@@ -1,0 +1,217 @@
+"""CUDA path against the fp64 oracle, element by element, through the C ABI.
+
+Every input comes from the seeded generator; every expected value from the oracle.
+"""
+import numpy as np
+import pytest
+
+import synthetic as S
+from oracle import gptq_oracle as O
+from tests.parity import CODE_MISMATCH_MAX, REL_ERR_TOL, compare_layer
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import post_weight_quantization_15_b200 as G
+
+
+def _dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")
+
+
+def _to_dev_x(x_bits, dev):
+    """X on the device as a [n, tokens] view of a buffer whose row stride is a multiple of 8."""
+    n, t = x_bits.shape
+    ld = (t + 7) // 8 * 8
+    buf = torch.zeros((n, ld), dtype=torch.int16, device=dev)
+    buf[:, :t] = torch.from_numpy(x_bits.view(np.int16)).to(dev)
+    return buf.view(torch.bfloat16)[:, :t]
+
+
+def _w_tensor(W, dev):
+    return torch.from_numpy(np.ascontiguousarray(W)).to(dev)
+
+
+def _run_gpu(W, x_bits, bits, gs, sym, act, damp=0.01):
+    dev = _dev()
+    q, prep, H = G.gptq_quantize(_w_tensor(W, dev), _to_dev_x(x_bits, dev), bits, gs, sym, act, damp,
+                                 want_codes=True, want_err=True)
+    torch.cuda.synchronize()
+    return q, prep, H
+
+
+def _compare(W, x_bits, bits, gs, sym, act, H64=None):
+    q, prep, Hg = _run_gpu(W, x_bits, bits, gs, sym, act)
+    if H64 is None:
+        H64 = O.hessian(x_bits)
+    ora = O.gptq_layer(W, None, bits, gs, sym, act, H=H64)
+    c = compare_layer(W, H64, ora, q.qweight.cpu().numpy(), q.scales.cpu().numpy(), q.zeros.cpu().numpy(),
+                      q.g_idx.cpu().numpy(), q.codes.cpu().numpy(), prep.perm.cpu().numpy(), bits, gs)
+    return c, q, prep, Hg, H64, ora
+
+
+# --------------------------------------------------------------------------- #
+# Whole path
+# --------------------------------------------------------------------------- #
+def test_small_workload_full_path():
+    wl = S.workloads()["layer-256x512"]
+    L, st = wl.layers[0], wl.settings[0]
+    W, x = S.make_w(L.w), S.make_x(L.x)
+    c, *_ = _compare(W, x, st.bits, st.group_size, st.sym, st.desc_act)
+    print(c)
+    assert c.ok(), c
+
+
+@pytest.mark.parametrize("out,n,tokens,bits,gs,sym,act", [
+    (200, 384, 1000, 4, 128, False, True),      # ragged rows, 3 blocks, ragged tokens, act-order
+    (77, 256, 700, 3, 64, True, False),
+    (130, 320, 900, 2, 32, False, True),        # n = 2.5 blocks (ragged last block)
+    (64, 512, 1500, 8, 128, True, True),
+    (96, 256, 1024, 4, -1, False, False),       # one group per row
+    (5000, 128, 600, 4, 128, True, True),       # many rows: 4 lanes per row
+])
+def test_ragged_shapes_and_settings(out, n, tokens, bits, gs, sym, act):
+    W, x = S.small_case(out, n, tokens, seed=out + n, rank=8, frac=0.02, mult=20.0)
+    c, q, prep, Hg, H64, ora = _compare(W, x, bits, gs, sym, act)
+    print(c)
+    assert c.ok(), c
+
+
+def test_hessian_and_diag_against_oracle():
+    dev = _dev()
+    W, x = S.small_case(8, 300, 2504, seed=3)          # n not a multiple of any tile, ragged tokens
+    X = _to_dev_x(x, dev)
+    H = torch.zeros((300, 300), dtype=torch.float32, device=dev)
+    hd = torch.zeros(300, dtype=torch.float64, device=dev)
+    G.hessian_accumulate(H, X[:, :1200], hd)              # two chunks
+    G.hessian_accumulate(H, X[:, 1200:].contiguous(), hd)
+    torch.cuda.synchronize()
+    H64 = O.hessian(x)
+    Hg = H.cpu().numpy().astype(np.float64)
+    iu = np.triu_indices(300)
+    rel = np.abs(Hg[iu] - H64[iu]) / np.sqrt(np.outer(np.diag(H64), np.diag(H64)))[iu]
+    assert rel.max() < 2e-6, rel.max()
+    assert np.allclose(hd.cpu().numpy(), np.diag(H64), rtol=1e-13, atol=0)
+
+
+def test_prepare_u_and_perm():
+    dev = _dev()
+    _, x = S.small_case(8, 384, 3000, seed=4)
+    H64 = O.hessian(x)
+    Ht = torch.from_numpy(H64.astype(np.float32)).to(dev)
+    hd = torch.from_numpy(np.diag(H64).copy()).to(dev)
+    p = G.prepare(Ht, 0.01, True, hd)
+    G.raise_on_status(p.status, "prepare")
+    ora = O.prepare(H64, 0.01, True)
+    assert np.array_equal(p.perm.cpu().numpy(), ora.perm)
+    U = p.U.cpu().numpy().astype(np.float64)
+    assert np.all(np.tril(U, -1) == 0) and np.all(np.diag(U) > 0)
+    R = U.T @ U @ ora.Hd
+    assert np.abs(R - np.eye(384)).max() < 1e-3
+    assert np.abs(U - ora.U).max() / np.abs(ora.U).max() < 1e-4
+
+
+def test_identity_hessian_is_bit_exact_round_to_nearest():
+    dev = _dev()
+    W = S.make_w(S.WSpec(300, 512, 0.02, "f16", 5, 100))
+    for bits, gs, sym in [(4, 128, False), (3, 64, True), (2, 32, False), (4, -1, True)]:
+        H = torch.eye(512, dtype=torch.float32, device=dev)
+        p = G.prepare(H, 0.01, False)
+        q = G.quantize_layer(_w_tensor(W, dev), p, bits, gs, sym, want_codes=True)
+        G.raise_on_status(p.status, "rtn")
+        rc, rs, rz = O.rtn(W, bits, gs, sym)
+        assert np.array_equal(q.codes.cpu().numpy(), rc)
+        assert np.array_equal(q.scales.cpu().numpy(), rs.astype(np.float16))
+        assert np.array_equal(q.zeros.cpu().numpy(), rz.astype(np.float16))
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_pack_bit_exact_on_oracle_codes(bits):
+    dev = _dev()
+    rng = np.random.default_rng(bits)
+    codes = rng.integers(0, 2 ** bits, (333, 256)).astype(np.uint8)
+    qg = G.pack(torch.from_numpy(codes).to(dev), bits).cpu().numpy()
+    assert np.array_equal(qg.view(np.uint32), O.pack(codes, bits).view(np.uint32))
+
+
+def test_err_sq_matches_loss_identity():
+    """sum_j e_j^2 = (w - what)^T H_d (w - what) per row, from the GPU's own outputs."""
+    W, x = S.small_case(64, 256, 1200, seed=6)
+    c, q, prep, Hg, H64, ora = _compare(W, x, 4, 64, True, True)
+    assert c.perm_equal
+    What = O.dequantize(q.qweight.cpu().numpy(), q.scales.cpu().numpy(), q.zeros.cpu().numpy(),
+                        q.g_idx.cpu().numpy(), 4, 256)[:, ora.perm]
+    d = W.astype(np.float64)[:, ora.perm] - What
+    rhs = np.einsum("ij,jk,ik->i", d, ora.prep.Hd, d)
+    lhs = q.err_sq.cpu().numpy().astype(np.float64)
+    assert np.allclose(lhs, rhs, rtol=2e-2)
+
+
+# --------------------------------------------------------------------------- #
+# Errors
+# --------------------------------------------------------------------------- #
+def test_not_spd_is_reported():
+    dev = _dev()
+    n = 256
+    H = torch.eye(n, dtype=torch.float32, device=dev)
+    H[10, 10] = -50.0
+    p = G.prepare(H, 0.01, False)
+    rc, info = G.status_read(p.status)
+    assert rc == G.gptq.ERR_NOT_SPD
+    assert 0 <= info < n
+
+
+def test_nonfinite_weight_is_reported():
+    dev = _dev()
+    W = S.make_w(S.WSpec(16, 128, 0.02, "f32", 1, 100))
+    W[3, 17] = np.nan
+    H = torch.eye(128, dtype=torch.float32, device=dev)
+    p = G.prepare(H, 0.01, False)
+    G.quantize_layer(_w_tensor(W, dev), p, 4, 128, False)
+    rc, info = G.status_read(p.status)
+    assert rc == G.gptq.ERR_NONFINITE and info == 17
+
+
+def test_invalid_arguments_are_synchronous():
+    dev = _dev()
+    W = torch.zeros((8, 100), dtype=torch.float32, device=dev)    # n % 32 != 0
+    H = torch.eye(100, dtype=torch.float32, device=dev)
+    p = G.prepare(H, 0.01, False)
+    with pytest.raises(G.GptqError) as e:
+        G.quantize_layer(W, p, 4, 32, False)
+    assert e.value.code == G.gptq.ERR_UNSUPPORTED
+    W2 = torch.zeros((8, 128), dtype=torch.float32, device=dev)
+    H2 = torch.eye(128, dtype=torch.float32, device=dev)
+    p2 = G.prepare(H2, 0.01, False)
+    with pytest.raises(G.GptqError) as e:
+        G.quantize_layer(W2, p2, 5, 32, False)
+    assert e.value.code == G.gptq.ERR_UNSUPPORTED
+    with pytest.raises(G.GptqError) as e:
+        G.quantize_layer(W2, p2, 4, 128, False, block=64)
+    assert e.value.code == G.gptq.ERR_UNSUPPORTED
+
+
+def test_empty_token_chunk_is_a_no_op():
+    dev = _dev()
+    H = torch.zeros((64, 64), dtype=torch.float32, device=dev)
+    X = torch.zeros((64, 0), dtype=torch.bfloat16, device=dev)
+    G.hessian_accumulate(H, X)
+    torch.cuda.synchronize()
+    assert float(H.abs().max()) == 0.0
+
+
+# --------------------------------------------------------------------------- #
+# The worked-example layer at full size: [1024, 4096], 65,536 tokens
+# --------------------------------------------------------------------------- #
+def test_worked_example_layer_full_size():
+    wl = S.workloads()["layer-1024x4096"]
+    L, st = wl.layers[0], wl.settings[0]
+    W, x = S.make_w(L.w), S.make_x(L.x)
+    c, q, prep, Hg, H64, ora = _compare(W, x, st.bits, st.group_size, st.sym, st.desc_act)
+    print(c)
+    assert q.scales.numel() == 32768
+    assert c.code_mismatch <= CODE_MISMATCH_MAX and abs(c.rel_err_ratio - 1) <= REL_ERR_TOL
+    assert c.ok(), c
