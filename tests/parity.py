@@ -4,7 +4,9 @@ The tolerances are those of the method's statement: codes may differ from the
 oracle's for at most 0.5 % of the weights (floating-point ties flip and the
 flips cascade through the compensation), the layer error ||WX - What X||^2 /
 ||WX||^2 must be within 2 % of the oracle's, and scales / zeros within 1e-3
-relative on groups whose codes all match.  Packing and g_idx are bit-exact.
+relative on groups whose codes match (read as: the group's codes and those of
+every earlier column of its row, since the group's parameters are computed from
+weights all those decisions compensated).  Packing and g_idx are bit-exact.
 """
 from __future__ import annotations
 
@@ -49,12 +51,16 @@ def compare_layer(W: np.ndarray, H64: np.ndarray, ora: "O.LayerResult", qweight:
     ratio = rel_g / ora.rel_err if ora.rel_err > 0 else (1.0 if rel_g == 0 else np.inf)
     pack_exact = np.array_equal(O.pack(codes, bits).view(np.uint32), qweight.view(np.uint32))
     gidx_exact = np.array_equal(O.g_idx(perm.astype(np.int64), group_size), gidx)
-    # groups (processing order) whose codes all match
+    # Groups (processing order) whose codes match, together with every earlier
+    # column of the same row: a group's scale and zero are computed from weights
+    # that every earlier decision of the row has compensated, so they are only
+    # determined up to rounding when all those decisions agree.
     gs = n if group_size == -1 else group_size
     cp_g = codes[:, ora.perm]
     cp_o = ora.codes[:, ora.perm]
     G = n // gs
-    same = (cp_g == cp_o).reshape(codes.shape[0], G, gs).all(axis=2).T       # [G, out]
+    gmatch = (cp_g == cp_o).reshape(codes.shape[0], G, gs).all(axis=2)      # [out, G]
+    same = np.logical_and.accumulate(gmatch, axis=1).T                     # [G, out]
     sg = scales16.astype(np.float64)
     so = ora.scales.astype(np.float64)
     zg = zeros16.astype(np.float64)
