@@ -172,6 +172,38 @@ GPTQ_API int gptq_quantize_layer(const void* W, int w_dtype, int out, int n, con
  */
 GPTQ_API int gptq_pack(const uint8_t* codes, int out, int n, int bits, int32_t* qweight, void* stream);
 
+/*
+ * gptq_quantize_layer_noalloc - gptq_quantize_layer without a caller workspace.
+ *
+ * The GPTQ pages have no counterpart to this call: it exists for callers that
+ * cannot allocate device memory where they quantize (a plugin whose host
+ * application owns all device allocations, code that may run while a stream is
+ * being captured, a service that must not grow its footprint after start-up).
+ * Arguments, layouts, results and errors are those of gptq_quantize_layer; the
+ * caller still provides every input and output.  The scratch comes from a
+ * static device array of GPTQ_NOALLOC_SCRATCH_BYTES inside the library instead
+ * of `ws`:
+ *
+ * - A layer whose gptq_quantize_workspace_size(out, n, block) exceeds
+ *   GPTQ_NOALLOC_SCRATCH_BYTES is rejected with GPTQ_ERR_WORKSPACE before
+ *   anything is enqueued.
+ * - Every GPU that loads the library holds one copy of the array until the
+ *   process exits.  The first call on a device looks up the array's device
+ *   address (cudaGetSymbolAddress, with that device current) and caches it;
+ *   make that first call before any stream capture.
+ * - All calls on a device share the array, which keeps the last call's
+ *   contents (every byte a call reads from it is written by the same call
+ *   first).  Calls whose work overlaps on the GPU - on different streams, or
+ *   from host threads that do not order them - race on it.
+ * - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define GPTQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+GPTQ_API int gptq_quantize_layer_noalloc(const void* W, int w_dtype, int out, int n, const float* U,
+                                         const int32_t* perm, const uint8_t* dead, int bits, int group_size,
+                                         int sym, int block, int32_t* qweight, uint16_t* scales,
+                                         uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq,
+                                         int32_t* d_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

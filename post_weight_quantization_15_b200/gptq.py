@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
     L.gptq_quantize_layer.argtypes = [P, I, I, I, P, P, P, I, I, I, I, P, P, P, P, P, P, P, SZ, P, P]
     L.gptq_pack.restype = I
     L.gptq_pack.argtypes = [P, I, I, I, P, P]
+    L.gptq_quantize_layer_noalloc.restype = I
+    L.gptq_quantize_layer_noalloc.argtypes = [P, I, I, I, P, P, P, I, I, I, I, P, P, P, P, P, P, P, P]
     _lib = L
     return L
 
@@ -291,3 +293,31 @@ def gptq_quantize(W: torch.Tensor, X: torch.Tensor, bits: int = 4, group_size: i
     if check:
         raise_on_status(st, "gptq_quantize")
     return q, prep, H
+
+
+# --------------------------------------------------------------------------- #
+# Static-scratch variant (no workspace)
+# --------------------------------------------------------------------------- #
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def quantize_layer_noalloc(W: torch.Tensor, prep: Prepared, out: QuantizedLayer, block: int = 128,
+                           stream=None) -> QuantizedLayer:
+    """quantize_layer for callers that cannot allocate device memory.
+
+    The library takes its scratch from a static 16 MiB device array instead of a
+    workspace, so this call allocates nothing; the caller passes preallocated
+    outputs (see alloc_quantized).  Layers whose workspace would exceed the array
+    raise GptqError(ERR_WORKSPACE).  Calls that overlap on the GPU race on the
+    shared array.
+    """
+    _require_cuda(W)
+    if W.dim() != 2 or not W.is_contiguous() or W.dtype not in _DTYPE_CODE:
+        raise ValueError("W must be a contiguous fp32/fp16/bf16 [out, n] tensor")
+    o, n = W.shape
+    _check(lib().gptq_quantize_layer_noalloc(_ptr(W), _DTYPE_CODE[W.dtype], o, n, _ptr(prep.U), _ptr(prep.perm),
+                                             _ptr(prep.dead), int(out.bits), int(out.group_size), int(out.sym),
+                                             int(block), _ptr(out.qweight), _ptr(out.scales), _ptr(out.zeros),
+                                             _ptr(out.g_idx), _ptr(out.codes), _ptr(out.err_sq), _ptr(prep.status),
+                                             _stream(stream)), "gptq_quantize_layer_noalloc")
+    return out
