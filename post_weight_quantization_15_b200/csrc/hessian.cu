@@ -1,9 +1,11 @@
-// K1: H += 2 . X . X^T  ("polydesk.ai/glossaire/gptq", "Etape 2": H = 2.X.X^T).
+// K1: H += 2 . X . X^T  ("polydesk.ai/glossaire/gptq", "Etape 2": H = 2.X.X^T),
+// a dense contraction over the calibration tokens on the tcgen05 tensor cores.
 //
 // hessian_diag64_kernel: the act-order key, 2 . sum_t x_it^2 in fp64 (every bf16
 // square is exact in fp64).
 #include "common.cuh"
 #include "internal.h"
+#include "tc_common.cuh"
 
 namespace gptq {
 
@@ -33,53 +35,214 @@ hessian_diag64_kernel(double* hdiag, int n, const __nv_bfloat16* X, int64_t ld_x
   }
 }
 
-// Plain CUDA-core version of the Hessian tile product: one 64x64 upper tile per
-// CTA, 4x4 outputs per thread, tokens staged through shared memory.
-constexpr int HT = 64;
-constexpr int HK = 32;
+// ---------------------------------------------------------------------------
+// Tensor-core tile product.  One CTA computes one 128 x 256 tile of 2.X.X^T
+// (rows [128 bi, +128), columns [256 bj, +256), for tiles that reach the upper
+// triangle) over all tokens:
+//   warp 0      TMA producer: 64 tokens of the 128 A rows and 256 B rows per
+//               stage (128-byte swizzled rows), 4-stage ring;
+//   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32 accumulators) and
+//               one thread issues tcgen05.mma (bf16 x bf16 -> fp32, M=128, N=256);
+//   warps 2..9  epilogue.
+// The tensor cores' fp32 accumulation is not rounded to nearest, and its error
+// grows with the number of accumulation steps.  So the MMA accumulates chunks of
+// CHUNK tokens from zero into the two TMEM accumulators alternately, and the
+// epilogue warps add each finished chunk into fp32 registers (round to nearest)
+// while the next chunk is computed.  At the end H += 2 . acc.
+// When the A rows lie inside the B rows (tiles on the diagonal) only the B tile
+// is loaded and A reads its half of it.
+// Every wait is bounded; a wait that gives up raises GPTQ_ERR_TIMEOUT, drains the
+// copies and MMAs in flight (again bounded) and frees TMEM.
+// ---------------------------------------------------------------------------
+constexpr int HBM_ = 128;                     // tile rows (A)
+constexpr int HBN = 256;                      // tile columns (B)
+constexpr int HKB = 64;                       // tokens per stage (128 bytes of bf16)
+constexpr int HSTAGES = 4;
+constexpr int CHUNK_KB = 4;                   // stages per accumulation chunk (256 tokens)
+constexpr int A_BYTES = HBM_ * HKB * 2;       // 16 KB
+constexpr int B_BYTES = HBN * HKB * 2;        // 32 KB
+constexpr uint32_t HESS_IDESC = tc::idesc_f32acc(1, 128, 256);
+constexpr int EPI_WARPS = 8;
+constexpr int HESS_THREADS = 64 + EPI_WARPS * 32;
 
-__global__ void __launch_bounds__(256)
-hessian_simple_kernel(float* H, int n, const __nv_bfloat16* X, int64_t ld_x, int64_t tokens,
-                      const int32_t* st) {
-  if (has_error(st)) return;
-  const int T = (int)cdiv(n, HT);
-  int t = blockIdx.x, bi = 0;
-  while (t >= T - bi) { t -= T - bi; ++bi; }
-  const int bj = bi + t;
-  __shared__ float As[HK][HT + 4];
-  __shared__ float Bs[HK][HT + 4];
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4] = {};
-  for (int64_t k0 = 0; k0 < tokens; k0 += HK) {
-    for (int idx = threadIdx.x; idx < HT * HK; idx += 256) {
-      const int r = idx / HK, k = idx % HK;
-      const int64_t gk = k0 + k;
-      const int gi = bi * HT + r, gj = bj * HT + r;
-      As[k][r] = (gi < n && gk < tokens) ? __bfloat162float(X[(int64_t)gi * ld_x + gk]) : 0.f;
-      Bs[k][r] = (gj < n && gk < tokens) ? __bfloat162float(X[(int64_t)gj * ld_x + gk]) : 0.f;
+struct HessSmem {
+  uint8_t b[HSTAGES][B_BYTES];
+  uint8_t a[HSTAGES][A_BYTES];
+  uint64_t full[HSTAGES];
+  uint64_t empty[HSTAGES];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int skip;
+};
+constexpr size_t HESS_SMEM = sizeof(HessSmem) + 1024;
+
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = tc::globaltimer();
+  while (!tc::mbar_try_wait(bar, parity)) {
+    if (tc::globaltimer() - t0 > 1000000000ull) return false;
+  }
+  return true;
+}
+
+// Tiles (bi, bj) with 256 bj + 255 >= 128 bi, i.e. bj >= bi / 2, row-major.
+__device__ __forceinline__ void hess_tile(int t, int TB, int& bi, int& bj) {
+  bi = 0;
+  for (;;) {
+    const int cnt = TB - bi / 2;
+    if (t < cnt) break;
+    t -= cnt;
+    ++bi;
+  }
+  bj = bi / 2 + t;
+}
+
+__global__ void __launch_bounds__(HESS_THREADS, 1)
+hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* H, int n, int kblocks, int32_t* st) {
+  extern __shared__ uint8_t smem_raw[];
+  HessSmem& S = *reinterpret_cast<HessSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int TB = (int)cdiv(n, HBN);
+  int bi, bj;
+  hess_tile(blockIdx.x, TB, bi, bj);
+  const bool inside = (bi / 2) == bj;          // A rows are half of the B rows
+  const int a_half = bi & 1;
+  const int nchunks = (int)cdiv(kblocks, CHUNK_KB);
+
+  if (threadIdx.x == 0) {
+    S.skip = has_error(st) ? 1 : 0;
+    S.abort = 0;
+    for (int s = 0; s < HSTAGES; ++s) { tc::mbar_init(&S.full[s], 1); tc::mbar_init(&S.empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { tc::mbar_init(&S.acc_full[b], 1); tc::mbar_init(&S.acc_empty[b], EPI_WARPS); }
+    tc::mbar_init(&S.drain, 1);
+    tc::fence_barrier_init();
+    tc::prefetch_tensormap(&tmap);
+  }
+  if (warp == 1) tc::tmem_alloc<512>(&S.tmem_base);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t taddr = S.tmem_base;
+  const bool skip = S.skip != 0;
+  volatile int* abort_flag = &S.abort;
+
+  int armed[HSTAGES] = {0, 0, 0, 0};
+  bool mma_committed = false;
+
+  if (!skip) {
+    if (warp == 0 && lane == 0) {
+      // ---------------- producer ----------------
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = kb % HSTAGES;
+        const uint32_t ph = (uint32_t)(kb / HSTAGES) & 1u;
+        if (!tc::mbar_wait(&S.empty[s], ph ^ 1u, abort_flag)) break;
+        tc::mbar_arrive_expect_tx(&S.full[s], inside ? B_BYTES : A_BYTES + B_BYTES);
+        tc::tma_load_2d(S.b[s], &tmap, &S.full[s], kb * HKB, bj * HBN);
+        tc::tma_load_2d(S.b[s] + A_BYTES, &tmap, &S.full[s], kb * HKB, bj * HBN + HBM_);
+        if (!inside) tc::tma_load_2d(S.a[s], &tmap, &S.full[s], kb * HKB, bi * HBM_);
+        ++armed[s];
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ---------------- MMA issuer ----------------
+      int kb = 0;
+      for (int c = 0; c < nchunks && !*abort_flag; ++c) {
+        const int buf = c & 1;
+        if (!tc::mbar_wait(&S.acc_empty[buf], ((uint32_t)(c >> 1) & 1u) ^ 1u, abort_flag)) break;
+        tc::tc_fence_after();
+        const int kb_end = min(kblocks, (c + 1) * CHUNK_KB);
+        bool first = true;
+        for (; kb < kb_end; ++kb) {
+          const int s = kb % HSTAGES;
+          const uint32_t ph = (uint32_t)(kb / HSTAGES) & 1u;
+          if (!tc::mbar_wait(&S.full[s], ph, abort_flag)) break;
+          tc::tc_fence_after();
+          const uint32_t b0 = tc::smem_u32(S.b[s]);
+          const uint32_t a0 = inside ? b0 + a_half * (HBM_ * 128) : tc::smem_u32(S.a[s]);
+#pragma unroll
+          for (int kk = 0; kk < HKB / 16; ++kk) {
+            tc::mma_f16(taddr + buf * HBN, tc::sdesc_k_sw128(a0 + kk * 32), tc::sdesc_k_sw128(b0 + kk * 32),
+                        HESS_IDESC, !first);
+            first = false;
+          }
+          tc::mma_commit(&S.empty[s]);
+        }
+        if (*abort_flag) break;
+        tc::mma_commit(&S.acc_full[buf]);
+      }
+      // Track every MMA this thread issued; wait for them before teardown so that
+      // no tcgen05 arrival can land after the CTA's shared memory is released.
+      tc::mma_commit(&S.drain);
+      mma_committed = true;
+      if (!*abort_flag) drain_wait(&S.drain, 0);
+    } else if (warp >= 2) {
+      // ---------------- epilogue ----------------
+      const int q = warp & 3;                  // TMEM lane quarter this warp may access
+      const int hc = (warp - 2) >> 2;          // which 128 of the 256 columns
+      const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+      float acc[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+      bool ok = true;
+      for (int c = 0; c < nchunks; ++c) {
+        const int buf = c & 1;
+        int ready = 0;
+        if (lane == 0) ready = tc::mbar_wait(&S.acc_full[buf], (uint32_t)(c >> 1) & 1u, abort_flag);
+        ready = __shfl_sync(0xffffffffu, ready, 0);
+        if (!ready) { ok = false; break; }
+        tc::tc_fence_after();
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float v[32];
+          tc::tmem_ld_32x32b_x32(taddr + lane_base + buf * HBN + hc * 128 + c4 * 32, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[c4 * 32 + i] += v[i];
+        }
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&S.acc_empty[buf]);
+      }
+      if (ok && !*abort_flag) {
+        const int row = bi * HBM_ + q * 32 + lane;
+        const int col0 = bj * HBN + hc * 128;
+        if (row < n && col0 < n) {
+          float* dst = H + (int64_t)row * n + col0;
+          if ((n & 3) == 0 && col0 + 128 <= n) {
+#pragma unroll
+            for (int i = 0; i < 128; i += 4) {
+              float4 o = *reinterpret_cast<float4*>(dst + i);
+              o.x = fmaf(2.f, acc[i], o.x); o.y = fmaf(2.f, acc[i + 1], o.y);
+              o.z = fmaf(2.f, acc[i + 2], o.z); o.w = fmaf(2.f, acc[i + 3], o.w);
+              *reinterpret_cast<float4*>(dst + i) = o;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+              if (col0 + i < n) dst[i] = fmaf(2.f, acc[i], dst[i]);
+          }
+        }
+      }
     }
-    __syncthreads();
-#pragma unroll 8
-    for (int k = 0; k < HK; ++k) {
-      float a[4], b[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) { a[u] = As[k][ty * 4 + u]; b[u] = Bs[k][tx * 4 + u]; }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(a[u], b[v], acc[u][v]);
+  }
+
+  // ---------------- teardown ----------------
+  tc::tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    // drain what this CTA still has in flight before its shared memory and TMEM go away
+    if (warp == 0 && lane == 0) {
+      for (int s = 0; s < HSTAGES; ++s)
+        if (armed[s] > 0) drain_wait(&S.full[s], (uint32_t)(armed[s] - 1) & 1u);
     }
+    if (warp == 1 && lane == 0 && mma_committed) drain_wait(&S.drain, 0);
+    if (threadIdx.x == 0) set_error(st, GPTQ_ERR_TIMEOUT, blockIdx.x, STAGE_HESSIAN);
     __syncthreads();
   }
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int gi = bi * HT + ty * 4 + u;
-    if (gi >= n) continue;
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int gj = bj * HT + tx * 4 + v;
-      if (gj < n) H[(int64_t)gi * n + gj] += 2.f * acc[u][v];
-    }
+  if (warp == 1) {
+    __syncwarp();
+    tc::tmem_dealloc<512>(taddr);
   }
 }
 
@@ -95,9 +258,18 @@ int launch_hessian_diag64(double* hdiag, int n, const void* X, int64_t ld_x, int
 
 int launch_hessian(float* H, int n, const void* X, int64_t ld_x, int64_t tokens, int32_t* st,
                    cudaStream_t s) {
-  const int T = (int)cdiv(n, HT);
-  const int tiles = T * (T + 1) / 2;
-  hessian_simple_kernel<<<tiles, 256, 0, s>>>(H, n, static_cast<const __nv_bfloat16*>(X), ld_x, tokens, st);
+  CUtensorMap map;
+  // One map serves both operands: its box is 64 tokens x 128 rows; the B tile is two boxes.
+  int rc = make_tmap_2d(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)tokens, (uint64_t)n,
+                        (uint64_t)ld_x * 2, HKB, HBM_, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != GPTQ_OK) return rc;
+  const int TB = (int)cdiv(n, HBN);
+  const int TA = (int)cdiv(n, HBM_);
+  int tiles = 0;
+  for (int bi = 0; bi < TA; ++bi) tiles += TB - bi / 2;
+  const int kblocks = (int)cdiv(tokens, HKB);
+  GPTQ_CUDA_TRY(cudaFuncSetAttribute(hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)HESS_SMEM));
+  hessian_tc_kernel<<<tiles, HESS_THREADS, HESS_SMEM, s>>>(map, H, n, kblocks, st);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }

@@ -92,10 +92,12 @@ def test_hessian_and_diag_against_oracle():
     H64 = O.hessian(x)
     Hg = H.cpu().numpy().astype(np.float64)
     iu = np.triu_indices(300)
-    # fp32 accumulation of N products: |error| <= N . 2^-24 . sum_t |x_it x_jt|
-    # <= N . 2^-24 . sqrt(H_ii H_jj) (Cauchy-Schwarz); the products are exact.
+    # fp32 accumulation of N exact products, each addition off by at most one ulp
+    # (the tensor cores need not round to nearest): |error| <= N . 2^-23 .
+    # sum_t |x_it x_jt| <= N . 2^-23 . sqrt(H_ii H_jj) (Cauchy-Schwarz).
     rel = np.abs(Hg[iu] - H64[iu]) / np.sqrt(np.outer(np.diag(H64), np.diag(H64)))[iu]
-    assert rel.max() <= 2504 * 2.0 ** -24, rel.max()
+    assert rel.max() <= 2504 * 2.0 ** -23, rel.max()
+    print("hessian max normalised error", rel.max())
     assert np.allclose(hd.cpu().numpy(), np.diag(H64), rtol=1e-13, atol=0)
 
 
