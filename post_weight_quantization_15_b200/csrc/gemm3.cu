@@ -1,0 +1,288 @@
+// C -= A . B^T in fp32-level precision on the tcgen05 tensor cores (3 x TF32).
+//
+// The lazy trailing update of the column sweep ("polydesk.ai/glossaire/gptq",
+// "Etape 3") and the trailing updates of the blocked Cholesky factorization and
+// triangular inverse are dense contractions whose results feed rounding
+// decisions; a single TF32 pass (10-bit mantissa) perturbs them too much.  Every
+// fp32 operand x is split once, outside this kernel, into hi = x with its low 13
+// mantissa bits cleared (exact in TF32) and lo = x - hi (exact in fp32), and
+//     A . B^T  ~  A_hi.B_hi^T + A_hi.B_lo^T + A_lo.B_hi^T
+// (the dropped A_lo.B_lo^T term is below 2^-20 of the product).
+//
+// One CTA computes one 128 x GN tile of C (GN = 256, or 128 for narrow C):
+//   warp 0      TMA producer: 32-wide K slices of A_hi, A_lo (128 rows) and
+//               B_hi, B_lo (GN rows), 128-byte swizzled, 2- or 3-stage ring;
+//   warp 1      allocates GN TMEM columns; one thread issues the tcgen05.mma
+//               kind::tf32 instructions (M = 128, N = GN, K = 8);
+//   warps 2..5  epilogue: TMEM -> registers -> C -= acc, or C = acc, and
+//               optionally the TF32 split of the result (Chi, Clo) for a later
+//               product.
+// All operands are row-major with K contiguous (K-major).  `lower` skips tiles
+// that lie entirely above the diagonal of a square C.
+// Every wait is bounded (GPTQ_ERR_TIMEOUT).
+#include "common.cuh"
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace gptq {
+
+namespace {
+
+constexpr int GM = 128;
+constexpr int GK = 32;                      // fp32 per 128-byte row
+constexpr int A_TILE = GM * GK * 4;         // 16 KB
+constexpr int G_THREADS = 192;
+
+template <int GN>
+struct GemmCfg {
+  static constexpr int STAGES = GN == 256 ? 2 : 3;
+  static constexpr int B_TILE = GN * GK * 4;
+  static constexpr uint32_t IDESC = tc::idesc_f32acc(2, GM, GN);
+};
+
+template <int GN>
+struct GemmSmem {
+  static constexpr int ST = GemmCfg<GN>::STAGES;
+  uint8_t bhi[ST][GemmCfg<GN>::B_TILE];
+  uint8_t blo[ST][GemmCfg<GN>::B_TILE];
+  uint8_t ahi[ST][A_TILE];
+  uint8_t alo[ST][A_TILE];
+  uint64_t full[ST];
+  uint64_t empty[ST];
+  uint64_t acc_full;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int skip;
+};
+
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = tc::globaltimer();
+  while (!tc::mbar_try_wait(bar, parity)) {
+    if (tc::globaltimer() - t0 > 1000000000ull) return false;
+  }
+  return true;
+}
+
+struct GemmMaps {
+  CUtensorMap ahi, alo, bhi, blo;
+};
+
+struct GemmOut {
+  float* C;
+  int ldc;
+  int store;        // 0: C -= acc, 1: C = acc
+  float* Chi;       // optional TF32 split of the result (same row/column origin as C)
+  float* Clo;
+  int ldh;
+};
+
+__device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
+
+template <int GN>
+__global__ void __launch_bounds__(G_THREADS, 1)
+gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, int K, int lower, int tiles_n,
+             int32_t* st) {
+  using Cfg = GemmCfg<GN>;
+  constexpr int ST = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  GemmSmem<GN>& S =
+      *reinterpret_cast<GemmSmem<GN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ti = blockIdx.x / tiles_n, tj = blockIdx.x % tiles_n;
+  const bool skip_tile = lower && (tj * GN > ti * GM + GM - 1);
+  if (skip_tile) return;                      // CTA-uniform, before any barrier or TMEM use
+  const int kblocks = (int)cdiv(K, GK);
+
+  if (threadIdx.x == 0) {
+    S.skip = has_error(st) ? 1 : 0;
+    S.abort = 0;
+    for (int s = 0; s < ST; ++s) { tc::mbar_init(&S.full[s], 1); tc::mbar_init(&S.empty[s], 1); }
+    tc::mbar_init(&S.acc_full, 1);
+    tc::mbar_init(&S.drain, 1);
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) tc::tmem_alloc<GN>(&S.tmem_base);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t taddr = S.tmem_base;
+  const bool skip = S.skip != 0;
+  volatile int* abort_flag = &S.abort;
+  int armed[ST] = {};
+  bool mma_committed = false;
+
+  if (!skip) {
+    if (warp == 0 && lane == 0) {
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = kb % ST;
+        const uint32_t ph = (uint32_t)(kb / ST) & 1u;
+        if (!tc::mbar_wait(&S.empty[s], ph ^ 1u, abort_flag)) break;
+        tc::mbar_arrive_expect_tx(&S.full[s], 2 * (A_TILE + Cfg::B_TILE));
+        tc::tma_load_2d(S.ahi[s], &maps.ahi, &S.full[s], kb * GK, ti * GM);
+        tc::tma_load_2d(S.alo[s], &maps.alo, &S.full[s], kb * GK, ti * GM);
+        tc::tma_load_2d(S.bhi[s], &maps.bhi, &S.full[s], kb * GK, tj * GN);
+        tc::tma_load_2d(S.blo[s], &maps.blo, &S.full[s], kb * GK, tj * GN);
+        ++armed[s];
+      }
+    } else if (warp == 1 && lane == 0) {
+      for (int kb = 0; kb < kblocks; ++kb) {
+        const int s = kb % ST;
+        const uint32_t ph = (uint32_t)(kb / ST) & 1u;
+        if (!tc::mbar_wait(&S.full[s], ph, abort_flag)) break;
+        tc::tc_fence_after();
+        const uint32_t ah = tc::smem_u32(S.ahi[s]), al = tc::smem_u32(S.alo[s]);
+        const uint32_t bh = tc::smem_u32(S.bhi[s]), bl = tc::smem_u32(S.blo[s]);
+#pragma unroll
+        for (int kk = 0; kk < GK / 8; ++kk) {
+          const uint32_t o = kk * 32;
+          tc::mma_tf32(taddr, tc::sdesc_k_sw128(al + o), tc::sdesc_k_sw128(bh + o), Cfg::IDESC, kb > 0 || kk > 0);
+          tc::mma_tf32(taddr, tc::sdesc_k_sw128(ah + o), tc::sdesc_k_sw128(bl + o), Cfg::IDESC, true);
+          tc::mma_tf32(taddr, tc::sdesc_k_sw128(ah + o), tc::sdesc_k_sw128(bh + o), Cfg::IDESC, true);
+        }
+        tc::mma_commit(&S.empty[s]);
+      }
+      if (!*abort_flag) tc::mma_commit(&S.acc_full);
+      tc::mma_commit(&S.drain);
+      mma_committed = true;
+      if (!*abort_flag) drain_wait(&S.drain, 0);
+    } else if (warp >= 2) {
+      int ready = 0;
+      if (lane == 0) ready = tc::mbar_wait(&S.acc_full, 0, abort_flag) && !*abort_flag;
+      ready = __shfl_sync(0xffffffffu, ready, 0);
+      if (ready) {
+        tc::tc_fence_after();
+        const int q = warp & 3;
+        const int row = ti * GM + q * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+#pragma unroll 1
+        for (int c = 0; c < GN / 32; ++c) {
+          float v[32];
+          tc::tmem_ld_32x32b_x32(taddr + lane_base + c * 32, v);
+          const int col0 = tj * GN + c * 32;
+          if (row < M && col0 < N) {
+            float* dst = out.C + (int64_t)row * out.ldc + col0;
+            const bool vec = ((out.ldc & 3) == 0) && col0 + 32 <= N;
+            if (!out.store) {
+              if (vec) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                  float4 o = *reinterpret_cast<float4*>(dst + i);
+                  o.x -= v[i]; o.y -= v[i + 1]; o.z -= v[i + 2]; o.w -= v[i + 3];
+                  *reinterpret_cast<float4*>(dst + i) = o;
+                  v[i] = o.x; v[i + 1] = o.y; v[i + 2] = o.z; v[i + 3] = o.w;
+                }
+              } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                  if (col0 + i < N) { dst[i] -= v[i]; v[i] = dst[i]; }
+              }
+            } else {
+              if (vec) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                  *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                  if (col0 + i < N) dst[i] = v[i];
+              }
+            }
+            if (out.Chi != nullptr) {
+              float* hi = out.Chi + (int64_t)row * out.ldh + col0;
+              float* lo = out.Clo + (int64_t)row * out.ldh + col0;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                if (col0 + i < N) {
+                  const float h = tf32_hi(v[i]);
+                  hi[i] = h;
+                  lo[i] = v[i] - h;
+                }
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    if (warp == 0 && lane == 0) {
+      for (int s = 0; s < ST; ++s)
+        if (armed[s] > 0) drain_wait(&S.full[s], (uint32_t)(armed[s] - 1) & 1u);
+    }
+    if (warp == 1 && lane == 0 && mma_committed) drain_wait(&S.drain, 0);
+    if (threadIdx.x == 0) set_error(st, GPTQ_ERR_TIMEOUT, blockIdx.x, STAGE_TRAILING);
+    __syncthreads();
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tc::tmem_dealloc<GN>(taddr);
+  }
+}
+
+// hi = x with the low 13 mantissa bits cleared, lo = x - hi.
+__global__ void split_tf32_kernel(const float* X, int rows, int cols, int ldx, float* hi, float* lo, int ldo,
+                                  const int32_t* st) {
+  if (has_error(st)) return;
+  const int c = blockIdx.x * 32 + threadIdx.x;
+  const int r = blockIdx.y * 8 + threadIdx.y;
+  if (r >= rows || c >= cols) return;
+  const float x = X[(int64_t)r * ldx + c];
+  const float h = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
+  hi[(int64_t)r * ldo + c] = h;
+  lo[(int64_t)r * ldo + c] = x - h;
+}
+
+int launch_split_tf32_impl(const float* X, int rows, int cols, int ldx, float* hi, float* lo, int ldo,
+                      const int32_t* st, cudaStream_t s) {
+  if (rows <= 0 || cols <= 0) return GPTQ_OK;
+  dim3 blk(32, 8), grd((unsigned)cdiv(cols, 32), (unsigned)cdiv(rows, 8));
+  split_tf32_kernel<<<grd, blk, 0, s>>>(X, rows, cols, ldx, hi, lo, ldo, st);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
+template <int GN>
+int launch_gemm3_t(const GemmOut& out, int M, int N, int K, const float* Ahi, const float* Alo, int lda,
+                   const float* Bhi, const float* Blo, int ldb, bool lower, int32_t* st, cudaStream_t s) {
+  GemmMaps maps;
+  int rc = make_tmap_2d(&maps.ahi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Ahi, (uint64_t)K, (uint64_t)M,
+                        (uint64_t)lda * 4, GK, GM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc == GPTQ_OK)
+    rc = make_tmap_2d(&maps.alo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Alo, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 4,
+                      GK, GM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc == GPTQ_OK)
+    rc = make_tmap_2d(&maps.bhi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Bhi, (uint64_t)K, (uint64_t)N, (uint64_t)ldb * 4,
+                      GK, GN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc == GPTQ_OK)
+    rc = make_tmap_2d(&maps.blo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Blo, (uint64_t)K, (uint64_t)N, (uint64_t)ldb * 4,
+                      GK, GN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != GPTQ_OK) return rc;
+  const int tm = (int)cdiv(M, GM), tn = (int)cdiv(N, GN);
+  const size_t smem = sizeof(GemmSmem<GN>) + 1024;
+  GPTQ_CUDA_TRY(cudaFuncSetAttribute(gemm3_kernel<GN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  gemm3_kernel<GN><<<tm * tn, G_THREADS, smem, s>>>(maps, out, M, N, K, lower ? 1 : 0, tn, st);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
+}  // namespace
+
+int launch_split_tf32(const float* X, int rows, int cols, int ldx, float* hi, float* lo, int ldo,
+                      const int32_t* st, cudaStream_t s) {
+  return launch_split_tf32_impl(X, rows, cols, ldx, hi, lo, ldo, st, s);
+}
+
+int launch_gemm3(float* C, int ldc, int M, int N, int K, const float* Ahi, const float* Alo, int lda,
+                 const float* Bhi, const float* Blo, int ldb, bool lower, int32_t* st, cudaStream_t s,
+                 bool store, float* Chi, float* Clo, int ldh) {
+  if (M <= 0 || N <= 0 || K <= 0) return GPTQ_OK;
+  GemmOut out{C, ldc, store ? 1 : 0, Chi, Clo, ldh};
+  if (N <= 128) return launch_gemm3_t<128>(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, st, s);
+  return launch_gemm3_t<256>(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, st, s);
+}
+
+}  // namespace gptq

@@ -26,7 +26,10 @@ constexpr int BLK = 128;           // columns per lazy batch
 
 struct QuantWs {
   float* Wf;          // [out, n] working weights, processing order
-  float* Err;         // [out, BLK] scaled errors of the current block
+  float* Ehi;         // [out, BLK] scaled errors of the current block, TF32-exact high part
+  float* Elo;         // [out, BLK] and the remainder
+  float* Bhi;         // [n, BLK] U[block rows, later columns]^T, high part (K-major operand)
+  float* Blo;         // [n, BLK] and the remainder
   uint8_t* codes_p;   // [out, n] codes, processing order
   int32_t* invperm;   // [n] processing position of every input column
   float* rows;        // [out] row-wide scale, [out] row-wide zero (group_size = -1)
@@ -36,12 +39,17 @@ QuantWs carve(void* ws, int out, int n) {
   char* p = static_cast<char*>(ws);
   QuantWs w;
   w.Wf = reinterpret_cast<float*>(p);        p += align_up((size_t)out * n * 4, 256);
-  w.Err = reinterpret_cast<float*>(p);       p += align_up((size_t)out * BLK * 4, 256);
+  w.Ehi = reinterpret_cast<float*>(p);       p += align_up((size_t)out * BLK * 4, 256);
+  w.Elo = reinterpret_cast<float*>(p);       p += align_up((size_t)out * BLK * 4, 256);
+  w.Bhi = reinterpret_cast<float*>(p);       p += align_up((size_t)n * BLK * 4, 256);
+  w.Blo = reinterpret_cast<float*>(p);       p += align_up((size_t)n * BLK * 4, 256);
   w.codes_p = reinterpret_cast<uint8_t*>(p); p += align_up((size_t)out * n, 256);
   w.invperm = reinterpret_cast<int32_t*>(p); p += align_up((size_t)n * 4, 256);
   w.rows = reinterpret_cast<float*>(p);
   return w;
 }
+
+__device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
 
 // ---------------------------------------------------------------------------
 // The quantizer.  Every operation is one IEEE fp32 operation (round to nearest
@@ -161,7 +169,7 @@ struct SweepShape {
 
 template <int GS, int TPR>
 __global__ void __launch_bounds__(128)
-sweep_kernel(float* Wf, int out, int n, int b0, int bw, const float* U, float* Err, uint8_t* codes_p,
+sweep_kernel(float* Wf, int out, int n, int b0, int bw, const float* U, float* Ehi, float* Elo, uint8_t* codes_p,
              uint16_t* scales, uint16_t* zeros, const float* rows, float* err_sq, int bits, int sym,
              const int32_t* st) {
   using SS = SweepShape<TPR>;
@@ -170,11 +178,25 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, const float* U, float* E
   extern __shared__ float smem[];
   float* Us = smem;                       // [BLK][LDU]
   float* dinv = smem + BLK * SS::LDU;     // [BLK] 1 / U_jj
-  for (int idx = threadIdx.x; idx < BLK * BLK; idx += blockDim.x) {
-    const int j = idx / BLK, c = idx % BLK;
-    const float v = (j < bw && c < bw && c >= j) ? U[(int64_t)(b0 + j) * n + b0 + c] : 0.f;
-    Us[j * SS::LDU + (c / SEG) * SS::SEGP + (c % SEG)] = v;
-    if (c == j) dinv[j] = (j < bw) ? 1.f / v : 0.f;
+  // Stage U[b0 + j][b0 + c] (j, c < bw) in 16-byte asynchronous copies, all in
+  // flight together; U is zero below its diagonal, so the lower part arrives zeroed.
+  for (int idx = threadIdx.x; idx < BLK * (BLK / 4); idx += blockDim.x) {
+    const int j = idx / (BLK / 4), c = (idx % (BLK / 4)) * 4;
+    float* dst = Us + j * SS::LDU + (c / SEG) * SS::SEGP + (c % SEG);
+    if (j < bw && c < bw) {
+      const float* src = U + (int64_t)(b0 + j) * n + b0 + c;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                   "l"(src)
+                   : "memory");
+    } else {
+      *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
+  for (int j = threadIdx.x; j < BLK; j += blockDim.x) {
+    const float d = Us[j * SS::LDU + (j / SEG) * SS::SEGP + (j % SEG)];
+    dinv[j] = (j < bw) ? 1.f / d : 0.f;
   }
   __syncthreads();
 
@@ -254,9 +276,14 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, const float* U, float* E
   if (!live || seg * SEG >= bw) {
     // nothing to store for this lane
   } else {
-    float* erow = Err + (int64_t)r * BLK + seg * SEG;
+    float* ehi = Ehi + (int64_t)r * BLK + seg * SEG;
+    float* elo = Elo + (int64_t)r * BLK + seg * SEG;
 #pragma unroll
-    for (int k = 0; k < SEG; k += 4) *reinterpret_cast<float4*>(erow + k) = make_float4(w[k], w[k + 1], w[k + 2], w[k + 3]);
+    for (int k = 0; k < SEG; k += 4) {
+      const float4 h = make_float4(tf32_hi(w[k]), tf32_hi(w[k + 1]), tf32_hi(w[k + 2]), tf32_hi(w[k + 3]));
+      *reinterpret_cast<float4*>(ehi + k) = h;
+      *reinterpret_cast<float4*>(elo + k) = make_float4(w[k] - h.x, w[k + 1] - h.y, w[k + 2] - h.z, w[k + 3] - h.w);
+    }
     uint8_t* crow = codes_p + (int64_t)r * n + b0 + seg * SEG;
 #pragma unroll
     for (int k = 0; k < SEG; k += 16)
@@ -268,53 +295,28 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, const float* U, float* E
 }
 
 // ---------------------------------------------------------------------------
-// K4: Wf[:, e:] -= Err . U[b0:b0+bw, e:]   (CUDA-core fp32 tiles)
+// K4 operand: B[c - e][k] = U[b0 + k][c] for c in [e, n), k < bw, split into its
+// TF32 high part and remainder (rows of 128, K-major for the tensor cores).
+// 32 x 32 tiles through shared memory keep both the read and the write coalesced.
 // ---------------------------------------------------------------------------
-constexpr int TT = 64;
-constexpr int TK = 16;
-
-__global__ void __launch_bounds__(256)
-trailing_kernel(float* Wf, int out, int n, int e, const float* Err, int bw, const float* Ub, const int32_t* st) {
+__global__ void u_block_transpose_split_kernel(const float* U, int n, int b0, int bw, int e, float* Bhi, float* Blo,
+                                               const int32_t* st) {
   if (has_error(st)) return;
-  __shared__ float As[TK][TT + 4];
-  __shared__ float Bs[TK][TT + 4];
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const int rbase = blockIdx.y * TT, cbase = e + blockIdx.x * TT;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < bw; k0 += TK) {
-    for (int idx = threadIdx.x; idx < TT * TK; idx += 256) {
-      {
-        const int r = idx / TK, k = idx % TK;
-        const int gr = rbase + r;
-        As[k][r] = (gr < out && k0 + k < bw) ? Err[(int64_t)gr * BLK + k0 + k] : 0.f;
-      }
-      {
-        const int k = idx / TT, c = idx % TT;
-        const int gc = cbase + c;
-        Bs[k][c] = (gc < n && k0 + k < bw) ? Ub[(int64_t)(k0 + k) * n + gc] : 0.f;
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < TK; ++k) {
-      float a[4], b[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) { a[u] = As[k][ty * 4 + u]; b[u] = Bs[k][tx * 4 + u]; }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(a[u], b[v], acc[u][v]);
-    }
-    __syncthreads();
+  __shared__ float t[32][33];
+  const int c0 = e + blockIdx.x * 32;      // U column tile
+  const int k0 = blockIdx.y * 32;          // U row tile within the block
+  for (int yy = threadIdx.y; yy < 32; yy += 8) {
+    const int k = k0 + yy, c = c0 + threadIdx.x;
+    t[yy][threadIdx.x] = (k < bw && c < n) ? U[(int64_t)(b0 + k) * n + c] : 0.f;
   }
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int gr = rbase + ty * 4 + u;
-    if (gr >= out) continue;
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int gc = cbase + tx * 4 + v;
-      if (gc < n) Wf[(int64_t)gr * n + gc] -= acc[u][v];
+  __syncthreads();
+  for (int yy = threadIdx.y; yy < 32; yy += 8) {
+    const int c = c0 + yy, k = k0 + threadIdx.x;
+    if (c < n && k < BLK) {
+      const float x = t[threadIdx.x][yy];
+      const float h = tf32_hi(x);
+      Bhi[(int64_t)(c - e) * BLK + k] = h;
+      Blo[(int64_t)(c - e) * BLK + k] = x - h;
     }
   }
 }
@@ -356,8 +358,9 @@ __global__ void codes_out_kernel(const uint8_t* codes_p, const int32_t* invperm,
 
 size_t quantize_ws_bytes(int out, int n, int block) {
   (void)block;
-  return align_up((size_t)out * n * 4, 256) + align_up((size_t)out * BLK * 4, 256) + align_up((size_t)out * n, 256) +
-         align_up((size_t)n * 4, 256) + align_up((size_t)out * 8, 256);
+  return align_up((size_t)out * n * 4, 256) + 2 * align_up((size_t)out * BLK * 4, 256) +
+         2 * align_up((size_t)n * BLK * 4, 256) + align_up((size_t)out * n, 256) + align_up((size_t)n * 4, 256) +
+         align_up((size_t)out * 8, 256);
 }
 
 int launch_pack(const uint8_t* codes, const int32_t* invperm, int out, int n, int ld_codes, int bits,
@@ -403,14 +406,17 @@ int launch_quantize(const void* W, int w_dtype, int out, int n, const float* U, 
   GPTQ_CUDA_TRY(cudaFuncSetAttribute(sweep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   for (int b0 = 0; b0 < n; b0 += BLK) {
     const int bw = std::min(BLK, n - b0);
-    sweep<<<(unsigned)cdiv(out, rows_per_cta), 128, smem, s>>>(w.Wf, out, n, b0, bw, U, w.Err, w.codes_p, scales,
-                                                                zeros, w.rows, err_sq, bits, sym, st);
+    sweep<<<(unsigned)cdiv(out, rows_per_cta), 128, smem, s>>>(w.Wf, out, n, b0, bw, U, w.Ehi, w.Elo, w.codes_p,
+                                                                scales, zeros, w.rows, err_sq, bits, sym, st);
     GPTQ_LAUNCH_CHECK();
     const int e = b0 + bw;
     if (e < n) {
-      dim3 grd((unsigned)cdiv(n - e, TT), (unsigned)cdiv(out, TT));
-      trailing_kernel<<<grd, 256, 0, s>>>(w.Wf, out, n, e, w.Err, bw, U + (int64_t)b0 * n, st);
+      dim3 blk(32, 8), grd((unsigned)cdiv(n - e, 32), (unsigned)(BLK / 32));
+      u_block_transpose_split_kernel<<<grd, blk, 0, s>>>(U, n, b0, bw, e, w.Bhi, w.Blo, st);
       GPTQ_LAUNCH_CHECK();
+      // Wf[:, e:] -= Err . U[b0:b0+bw, e:]
+      const int rc = launch_gemm3(w.Wf + e, n, out, n - e, BLK, w.Ehi, w.Elo, BLK, w.Bhi, w.Blo, BLK, false, st, s);
+      if (rc != GPTQ_OK) return rc;
     }
   }
   int rc = launch_pack(w.codes_p, w.invperm, out, n, n, bits, qweight, st, s);
