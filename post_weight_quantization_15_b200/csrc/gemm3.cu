@@ -24,6 +24,11 @@
 #include "internal.h"
 #include "tc_common.cuh"
 
+// Timeline marks for probes; empty in the library build.
+#ifndef GPTQ_GEMM_MARK
+#define GPTQ_GEMM_MARK(i)
+#endif
+
 namespace gptq {
 
 namespace {
@@ -93,6 +98,7 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
   const bool skip_tile = lower && (tj * GN > ti * GM + GM - 1);
   if (skip_tile) return;                      // CTA-uniform, before any barrier or TMEM use
   const int kblocks = (int)cdiv(K, GK);
+  GPTQ_GEMM_MARK(0);
 
   if (threadIdx.x == 0) {
     S.skip = has_error(st) ? 1 : 0;
@@ -106,6 +112,7 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
+  GPTQ_GEMM_MARK(1);
   const uint32_t taddr = S.tmem_base;
   const bool skip = S.skip != 0;
   volatile int* abort_flag = &S.abort;
@@ -131,6 +138,7 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
         const uint32_t ph = (uint32_t)(kb / ST) & 1u;
         if (!tc::mbar_wait(&S.full[s], ph, abort_flag)) break;
         tc::tc_fence_after();
+        if (kb == 0) GPTQ_GEMM_MARK(2);
         const uint32_t ah = tc::smem_u32(S.ahi[s]), al = tc::smem_u32(S.alo[s]);
         const uint32_t bh = tc::smem_u32(S.bhi[s]), bl = tc::smem_u32(S.blo[s]);
 #pragma unroll
@@ -142,6 +150,7 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
         }
         tc::mma_commit(&S.empty[s]);
       }
+      GPTQ_GEMM_MARK(3);
       if (!*abort_flag) tc::mma_commit(&S.acc_full);
       tc::mma_commit(&S.drain);
       mma_committed = true;
@@ -152,51 +161,80 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
       ready = __shfl_sync(0xffffffffu, ready, 0);
       if (ready) {
         tc::tc_fence_after();
+        if (warp == 2 && lane == 0) GPTQ_GEMM_MARK(4);
         const int q = warp & 3;
         const int row = ti * GM + q * 32 + lane;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        // Each warp owns TMEM lanes (rows) [32 q, 32 q + 32).  It stages its 32 x GN
+        // slice of C in shared memory (the stage buffers are free once the
+        // accumulator is complete): 16-byte pieces, piece p of row rr stored at
+        // slot p ^ (rr & 7), so that both the row-wise combine (lane = row) and the
+        // coalesced global accesses (lane = piece) stay within 4-way bank sharing.
+        constexpr int P = GN / 4;                                    // pieces per row
+        float* tile = reinterpret_cast<float*>(S.bhi[0]) + q * (32 * GN);
+        const int row0 = ti * GM + q * 32;
+        const bool vec = (out.ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(out.C) & 15) == 0;
+        auto slot = [](int rr, int p) { return rr * GN + ((p ^ (rr & 7)) << 2); };
+        if (!out.store) {
+          for (int g = lane; g < 32 * P; g += 32) {
+            const int rr = g / P, p = g % P;
+            const int r = row0 + rr, col = tj * GN + 4 * p;
+            float* dst = tile + slot(rr, p);
+            if (vec && r < M && col + 3 < N) {
+              asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)),
+                           "l"(out.C + (int64_t)r * out.ldc + col)
+                           : "memory");
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                dst[e] = (r < M && col + e < N) ? out.C[(int64_t)r * out.ldc + col + e] : 0.f;
+            }
+          }
+          asm volatile("cp.async.wait_all;" ::: "memory");
+          __syncwarp();
+        }
 #pragma unroll 1
         for (int c = 0; c < GN / 32; ++c) {
           float v[32];
           tc::tmem_ld_32x32b_x32(taddr + lane_base + c * 32, v);
-          const int col0 = tj * GN + c * 32;
-          if (row < M && col0 < N) {
-            float* dst = out.C + (int64_t)row * out.ldc + col0;
-            const bool vec = ((out.ldc & 3) == 0) && col0 + 32 <= N;
-            if (!out.store) {
-              if (vec) {
+          // lane = row: combine with C
 #pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                  float4 o = *reinterpret_cast<float4*>(dst + i);
-                  o.x -= v[i]; o.y -= v[i + 1]; o.z -= v[i + 2]; o.w -= v[i + 3];
-                  *reinterpret_cast<float4*>(dst + i) = o;
-                  v[i] = o.x; v[i + 1] = o.y; v[i + 2] = o.z; v[i + 3] = o.w;
-                }
-              } else {
+          for (int pp = 0; pp < 8; ++pp) {
+            float* e = tile + slot(lane, 8 * c + pp);
+            float4 x = *reinterpret_cast<float4*>(e);
+            if (out.store) x = make_float4(v[4 * pp], v[4 * pp + 1], v[4 * pp + 2], v[4 * pp + 3]);
+            else x = make_float4(x.x - v[4 * pp], x.y - v[4 * pp + 1], x.z - v[4 * pp + 2], x.w - v[4 * pp + 3]);
+            *reinterpret_cast<float4*>(e) = x;
+          }
+        }
+        __syncwarp();
+        // lane = piece: coalesced stores of C and of its split
+        for (int g = lane; g < 32 * P; g += 32) {
+          const int rr = g / P, p = g % P;
+          const int r = row0 + rr, col = tj * GN + 4 * p;
+          if (r >= M || col >= N) continue;
+          const float4 x = *reinterpret_cast<const float4*>(tile + slot(rr, p));
+          const float xs[4] = {x.x, x.y, x.z, x.w};
+          if (vec && col + 3 < N) {
+            *reinterpret_cast<float4*>(out.C + (int64_t)r * out.ldc + col) = x;
+          } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                  if (col0 + i < N) { dst[i] -= v[i]; v[i] = dst[i]; }
-              }
+            for (int e = 0; e < 4; ++e)
+              if (col + e < N) out.C[(int64_t)r * out.ldc + col + e] = xs[e];
+          }
+          if (out.Chi != nullptr) {
+            float hs[4], ls[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) { hs[e] = tf32_hi(xs[e]); ls[e] = xs[e] - hs[e]; }
+            if ((out.ldh & 3) == 0 && col + 3 < N) {
+              *reinterpret_cast<float4*>(out.Chi + (int64_t)r * out.ldh + col) = make_float4(hs[0], hs[1], hs[2], hs[3]);
+              *reinterpret_cast<float4*>(out.Clo + (int64_t)r * out.ldh + col) = make_float4(ls[0], ls[1], ls[2], ls[3]);
             } else {
-              if (vec) {
 #pragma unroll
-                for (int i = 0; i < 32; i += 4)
-                  *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-              } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                  if (col0 + i < N) dst[i] = v[i];
-              }
-            }
-            if (out.Chi != nullptr) {
-              float* hi = out.Chi + (int64_t)row * out.ldh + col0;
-              float* lo = out.Clo + (int64_t)row * out.ldh + col0;
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                if (col0 + i < N) {
-                  const float h = tf32_hi(v[i]);
-                  hi[i] = h;
-                  lo[i] = v[i] - h;
+              for (int e = 0; e < 4; ++e) {
+                if (col + e < N) {
+                  out.Chi[(int64_t)r * out.ldh + col + e] = hs[e];
+                  out.Clo[(int64_t)r * out.ldh + col + e] = ls[e];
                 }
               }
             }
@@ -208,6 +246,7 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
 
   tc::tc_fence_before();
   __syncthreads();
+  GPTQ_GEMM_MARK(5);
   if (*abort_flag) {
     if (warp == 0 && lane == 0) {
       for (int s = 0; s < ST; ++s)

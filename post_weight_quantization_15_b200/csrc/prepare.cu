@@ -42,10 +42,10 @@ struct PrepWs {
   float* A;        // [n, ldn] lower triangle: the reversed, permuted, damped H, then L
   float* Xt;       // [n, ldn] upper triangle: (L^-1)^T
   float* Phi; float* Plo;     // [n, PB] split of the panel A21 before the solve
-  float* Lhi; float* Llo;     // [n, PB] split of L21
+  float* Lhi[2]; float* Llo[2];   // [n, PB] split of L21 (two panels in flight)
   float* XPhi; float* XPlo;   // [n, PB] split of Xt[:k0, k] before the solve
   float* XQhi; float* XQlo;   // [n, PB] split of the finished Xt[:, k]
-  float* LIhi; float* LIlo;   // [PB, PB] split of L_kk^-1
+  float* LIhi[2]; float* LIlo[2]; // [PB, PB] split of L_kk^-1 (two panels in flight)
   double* key;     // [n] act-order key
   float* dfix;     // [n] diag(H) with dead inputs set to 1
   double* scal;    // [0] sum of dfix, [1] lambda
@@ -61,11 +61,16 @@ PrepWs carve(void* ws, int n) {
   w.A = reinterpret_cast<float*>(take(nn));
   w.Xt = reinterpret_cast<float*>(take(nn));
   w.Phi = reinterpret_cast<float*>(take(panel));  w.Plo = reinterpret_cast<float*>(take(panel));
-  w.Lhi = reinterpret_cast<float*>(take(panel));  w.Llo = reinterpret_cast<float*>(take(panel));
+  for (int b = 0; b < 2; ++b) {
+    w.Lhi[b] = reinterpret_cast<float*>(take(panel));
+    w.Llo[b] = reinterpret_cast<float*>(take(panel));
+  }
   w.XPhi = reinterpret_cast<float*>(take(panel)); w.XPlo = reinterpret_cast<float*>(take(panel));
   w.XQhi = reinterpret_cast<float*>(take(panel)); w.XQlo = reinterpret_cast<float*>(take(panel));
-  w.LIhi = reinterpret_cast<float*>(take((size_t)PB * PB * 4));
-  w.LIlo = reinterpret_cast<float*>(take((size_t)PB * PB * 4));
+  for (int b = 0; b < 2; ++b) {
+    w.LIhi[b] = reinterpret_cast<float*>(take((size_t)PB * PB * 4));
+    w.LIlo[b] = reinterpret_cast<float*>(take((size_t)PB * PB * 4));
+  }
   w.key = reinterpret_cast<double*>(take((size_t)n * 8));
   w.dfix = reinterpret_cast<float*>(take((size_t)n * 4));
   w.scal = reinterpret_cast<double*>(take(256));
@@ -159,137 +164,175 @@ __global__ void prep_gather_kernel(const float* H, const float* dfix, const int3
 // ---------------------------------------------------------------------------
 // (5) The diagonal block of panel k: Cholesky L_kk and its inverse T = L_kk^-1
 // (rows/columns past nb padded with the identity), in one pass over the 128
-// pivots.  256 threads form a 16 x 16 grid; thread (ty, tx) keeps the entries
-// (ty + 16a, tx + 16b), a, b < 8, of L and of T in registers.  Pivot j:
-//   1. the owners of column j scale it by 1 / L_jj (published to shared memory),
-//      and the owners of row j of T scale it by the same factor (row j of T is
-//      final: T = L^-1 is the forward elimination of the identity);
-//   2. every thread applies the rank-1 updates L[i][k] -= L_ij L_kj (j < k <= i)
-//      and T[i][c] -= L_ij T_jc (i > j, c <= j), and the owner of the next
-//      pivot computes its square root and reciprocal.
-// The pivot loop is unrolled over its eight 16-pivot slot blocks, so every
-// register index is a compile-time constant and finished slots are skipped at
-// compile time.
+// pivots with one CTA barrier per pivot.
+//   Layout: warp w owns the columns k = w + 8c (c < 16), lane l the rows
+//   i = l + 32r (r < 4); every thread keeps those 64 entries of L and of T in
+//   registers.
+//   Pivot s, phase A (the warp owning column s only): the pivot comes from the
+//   owning lane by a shuffle; the warp scales its column and publishes it
+//   (zero for rows <= s) together with 1 / L_ss.
+//   Barrier.
+//   Phase B (every warp): L[i][k] -= L_is L_ks; T absorbs the previous pivot,
+//   T[i][c] -= L_i,s-1 T_s-1,c; then the lanes holding row s of T scale it by
+//   1 / L_ss (row s is final: T = L^-1 is the forward elimination of the
+//   identity) and publish it for the next pivot.
+//   The published vectors rotate through three buffers, so no second barrier
+//   is needed.  The pivot loop is unrolled over its 16 column-slot blocks, so
+//   every register index is a compile-time constant.
 // ---------------------------------------------------------------------------
 constexpr int POTRF_THREADS = 256;
-constexpr size_t POTRF_SMEM = 0;
-
-__device__ __forceinline__ void pivot_publish(float d, int j, float* piv, int* bad, int k0, int n, int32_t* st) {
-  if (!(d > 0.f) || !isfinite(d)) {
-    if (!*bad) {
-      *bad = 1;
-      set_error(st, isfinite(d) ? GPTQ_ERR_NOT_SPD : GPTQ_ERR_NONFINITE, n - 1 - (k0 + j), STAGE_POTRF);
-    }
-    d = 1.f;   // keep the arithmetic finite; every later stage sees the error and skips
-  }
-  const float sq = sqrtf(d);
-  piv[0] = sq;
-  piv[1] = __frcp_rn(sq);
-}
+constexpr int SLD = PB + 1;
+constexpr size_t POTRF_SMEM = (size_t)PB * SLD * sizeof(float);
 
 __global__ void __launch_bounds__(POTRF_THREADS)
 potrf_inv_kernel(float* A, int lda, int k0, int nb, int n, float* LIhi, float* LIlo, float* Xt, int ldx,
                  float* XQhi, float* XQlo, int32_t* st) {
-  __shared__ float colL[PB];
-  __shared__ float rowT[PB];
-  __shared__ float piv[2];
+  extern __shared__ float stage[];          // [PB][SLD] input / output staging
+  __shared__ float colL[3][PB];
+  __shared__ float rowT[3][PB];
+  __shared__ float piv[3];
   __shared__ int bad;
   if (has_error(st)) return;
-  const int tid = threadIdx.x;
-  const int ty = tid >> 4, tx = tid & 15;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) bad = 0;
-  if (tid < PB) { colL[tid] = 0.f; rowT[tid] = 0.f; }
 
-  float l[8][8], t[8][8];
+  // coalesced load of the lower triangle (identity past nb)
+  for (int idx = tid; idx < PB * PB; idx += POTRF_THREADS * 8) {
+    float v[8];
 #pragma unroll
-  for (int a = 0; a < 8; ++a)
+    for (int u = 0; u < 8; ++u) {
+      const int e = idx + u * POTRF_THREADS;
+      const int r = e / PB, c = e % PB;
+      v[u] = (e < PB * PB && r < nb && c <= r) ? A[(int64_t)(k0 + r) * lda + k0 + c] : 0.f;
+    }
 #pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      const int i = ty + 16 * a, k = tx + 16 * b;
-      float v = 0.f;
-      if (b <= a) v = (i < nb && k <= i) ? A[(int64_t)(k0 + i) * lda + k0 + k] : (i == k ? 1.f : 0.f);
-      l[a][b] = v;
-      t[a][b] = (i == k) ? 1.f : 0.f;
+    for (int u = 0; u < 8; ++u) {
+      const int e = idx + u * POTRF_THREADS;
+      const int r = e / PB, c = e % PB;
+      if (e < PB * PB) stage[r * SLD + c] = (r >= nb && r == c) ? 1.f : v[u];
+    }
+  }
+  __syncthreads();
+  float l[4][16], t[4][16];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int i = lane + 32 * r, k = warp + 8 * c;
+      l[r][c] = k <= i ? stage[i * SLD + k] : 0.f;
+      t[r][c] = i == k ? 1.f : 0.f;
     }
   __syncthreads();
   GPTQ_PHASE_MARK(0);
-  if (tid == 0) pivot_publish(l[0][0], 0, piv, &bad, k0, n, st);   // thread (0, 0) owns (0, 0)
-  __syncthreads();
 
 #pragma unroll
-  for (int J = 0; J < 8; ++J) {
+  for (int C = 0; C < 16; ++C) {
+    const int R = C / 4;                       // row slot of the pivots of this block
 #pragma unroll 1
-    for (int jj = 0; jj < 16; ++jj) {
-      const int j = 16 * J + jj;
-      const float sq = piv[0], rinv = piv[1];
-      // 1. column j of L (owners: tx == jj, slot b = J) and row j of T (owners: ty == jj, slot a = J).
-      //    colL[i] is 0 for every row i <= j (a row's entry is zeroed when it is the
-      //    pivot and never rewritten), and rowT[c] is 0 for every c > j (never
-      //    written yet), so the updates below need no masks.
-      if (tx == jj) {
-#pragma unroll
-        for (int a = J; a < 8; ++a) {
-          const int i = ty + 16 * a;
-          if (i > j) { l[a][J] *= rinv; colL[i] = l[a][J]; }
-          else if (i == j) { l[a][J] = sq; colL[j] = 0.f; }
+    for (int ws = 0; ws < 8; ++ws) {
+      const int s = 8 * C + ws;
+      const int buf = s % 3, prev = (s + 2) % 3;
+      // ---- phase A: the warp owning column s ----
+      if (warp == ws) {
+        float d = __shfl_sync(0xffffffffu, l[R][C], 8 * (C % 4) + ws);
+        const bool badp = !(d > 0.f) || !isfinite(d);
+        if (badp) {
+          if (lane == 0 && !bad) {
+            bad = 1;
+            set_error(st, isfinite(d) ? GPTQ_ERR_NOT_SPD : GPTQ_ERR_NONFINITE, n - 1 - (k0 + s), STAGE_POTRF);
+          }
+          d = 1.f;   // keep the arithmetic finite; every later stage sees the error and skips
         }
-      }
-      if (ty == jj) {
+        const float sq = sqrtf(d);
+        const float rinv = __frcp_rn(sq);
 #pragma unroll
-        for (int b = 0; b <= J; ++b) {
-          const int c = tx + 16 * b;
-          if (c <= j) { t[J][b] *= rinv; rowT[c] = t[J][b]; }
+        for (int r = 0; r < 4; ++r) {
+          const int i = lane + 32 * r;
+          float v = l[r][C];
+          if (i > s) v *= rinv;
+          else if (i == s) v = sq;
+          if (i >= s) l[r][C] = v;
+          colL[buf][i] = i > s ? v : 0.f;
         }
+        if (lane == 0) piv[buf] = rinv;
       }
       __syncthreads();
-      // 2. rank-1 updates (branch-free): L[i][k] -= L_ij L_kj and T[i][c] -= L_ij T_jc.
-      //    Entries above the diagonal of the diagonal slots also change; they are
-      //    never read.
-      float lk[8];
+      // ---- phase B: every warp ----
+      {
+        float li[4];
 #pragma unroll
-      for (int b = J; b < 8; ++b) lk[b] = colL[tx + 16 * b];
-      float tr[8];
+        for (int r = R; r < 4; ++r) li[r] = colL[buf][lane + 32 * r];
 #pragma unroll
-      for (int b = 0; b <= J; ++b) tr[b] = rowT[tx + 16 * b];
+        for (int c = C; c < 16; ++c) {
+          const float lk = colL[buf][warp + 8 * c];
 #pragma unroll
-      for (int a = J; a < 8; ++a) {
-        const float li = colL[ty + 16 * a];
+          for (int r = R; r < 4; ++r) l[r][c] = fmaf(-li[r], lk, l[r][c]);
+        }
+        if (s > 0) {
+          // T absorbs pivot s - 1 (rows <= s - 1 have a zero multiplier, columns > s - 1 a zero row entry)
+          float lp[4];
 #pragma unroll
-        for (int b = J; b <= a; ++b) l[a][b] = fmaf(-li, lk[b], l[a][b]);
+          for (int r = R; r < 4; ++r) lp[r] = colL[prev][lane + 32 * r];
 #pragma unroll
-        for (int b = 0; b <= J; ++b) t[a][b] = fmaf(-li, tr[b], t[a][b]);
+          for (int c = 0; c <= C; ++c) {
+            const float tk = rowT[prev][warp + 8 * c];
+#pragma unroll
+            for (int r = R; r < 4; ++r) t[r][c] = fmaf(-lp[r], tk, t[r][c]);
+          }
+        }
+        if (lane == 8 * (C % 4) + ws) {
+          // row s of T is final after scaling
+          const float rinv = piv[buf];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            if (c <= C) t[R][c] *= rinv;
+            rowT[buf][warp + 8 * c] = t[R][c];
+          }
+        }
       }
-      // the owner of pivot j + 1 publishes it
-      if (jj < 15) {
-        if (ty == jj + 1 && tx == jj + 1) pivot_publish(l[J][J], j + 1, piv, &bad, k0, n, st);
-      } else if (J < 7) {
-        if (ty == 0 && tx == 0) pivot_publish(l[J + 1][J + 1], j + 1, piv, &bad, k0, n, st);
-      }
-      __syncthreads();
     }
   }
+  __syncthreads();
   GPTQ_PHASE_MARK(13);
   if (bad) return;
 
-  // outputs
+  // outputs, staged through shared memory for coalesced global access
 #pragma unroll
-  for (int a = 0; a < 8; ++a)
+  for (int r = 0; r < 4; ++r)
 #pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      const int i = ty + 16 * a, k = tx + 16 * b;
-      if (b <= a && i < nb && k <= i) A[(int64_t)(k0 + i) * lda + k0 + k] = l[a][b];
+    for (int c = 0; c < 16; ++c) stage[(lane + 32 * r) * SLD + warp + 8 * c] = l[r][c];
+  __syncthreads();
+  for (int idx = tid; idx < PB * PB; idx += POTRF_THREADS) {
+    const int i = idx / PB, k = idx % PB;
+    if (i < nb && k <= i) A[(int64_t)(k0 + i) * lda + k0 + k] = stage[i * SLD + k];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 16; ++c) stage[(lane + 32 * r) * SLD + warp + 8 * c] = t[r][c];
+  __syncthreads();
+  for (int idx = tid; idx < PB * PB; idx += POTRF_THREADS) {
+    {
       // split of L_kk^-1 (B operand rows i, K index k), zero outside nb
-      const float tv = (i < nb && k < nb) ? t[a][b] : 0.f;
+      const int i = idx / PB, k = idx % PB;
+      const float tv = (i < nb && k < nb) ? stage[i * SLD + k] : 0.f;
       const float th = tf32_hi(tv);
       LIhi[i * PB + k] = th;
       LIlo[i * PB + k] = tv - th;
+    }
+    {
       // transposed: Xt[k0 + k][k0 + i] = T[i][k] and its split XQ[k0 + k][i]
+      const int k = idx / PB, i = idx % PB;
       if (i < nb && k < nb) {
+        const float tv = stage[i * SLD + k];
+        const float th = tf32_hi(tv);
         Xt[(int64_t)(k0 + k) * ldx + k0 + i] = tv;
         XQhi[(int64_t)(k0 + k) * PB + i] = th;
         XQlo[(int64_t)(k0 + k) * PB + i] = tv - th;
       }
     }
+  }
 }
 
 // (6) U[i][j] = (L^-1)[n-1-i][n-1-j] = Xt[n-1-j][n-1-i] for j >= i, 0 below the diagonal.
@@ -308,13 +351,39 @@ __global__ void write_u_kernel(const float* Xt, int n, int ldx, float* U, const 
   }
 }
 
+// The blocked inverse's updates run on an auxiliary stream next to the
+// factorization: one non-blocking stream and a few events per host thread and
+// device, created on first use and kept for the life of the process.
+struct AuxStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, panel = nullptr, join = nullptr, done[2] = {nullptr, nullptr};
+};
+
+int aux_stream(AuxStream** out) {
+  // one set per host thread and device, so concurrent callers never share it
+  thread_local AuxStream per_dev[64];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GPTQ_ERR_CUDA;
+  AuxStream& a = per_dev[dev];
+  if (a.s == nullptr) {
+    if (cudaStreamCreateWithFlags(&a.s, cudaStreamNonBlocking) != cudaSuccess) return GPTQ_ERR_CUDA;
+    const unsigned f = cudaEventDisableTiming;
+    if (cudaEventCreateWithFlags(&a.fork, f) != cudaSuccess || cudaEventCreateWithFlags(&a.panel, f) != cudaSuccess ||
+        cudaEventCreateWithFlags(&a.join, f) != cudaSuccess || cudaEventCreateWithFlags(&a.done[0], f) != cudaSuccess ||
+        cudaEventCreateWithFlags(&a.done[1], f) != cudaSuccess)
+      return GPTQ_ERR_CUDA;
+  }
+  *out = &a;
+  return GPTQ_OK;
+}
+
 }  // namespace
 
 size_t prepare_ws_bytes(int n) {
   const int ldn = ld_of(n);
   const size_t nn = align_up((size_t)n * ldn * sizeof(float), 256);
   const size_t panel = align_up((size_t)n * PB * sizeof(float), 256);
-  return 2 * nn + 8 * panel + 2 * align_up((size_t)PB * PB * 4, 256) + align_up((size_t)n * 8, 256) +
+  return 2 * nn + 10 * panel + 4 * align_up((size_t)PB * PB * 4, 256) + align_up((size_t)n * 8, 256) +
          align_up((size_t)n * 4, 256) + 256;
 }
 
@@ -336,41 +405,61 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
   }
   GPTQ_CUDA_TRY(cudaMemsetAsync(w.Xt, 0, (size_t)n * ldn * sizeof(float), s));
 
-  for (int k0 = 0; k0 < n; k0 += PB) {
+  GPTQ_CUDA_TRY(cudaFuncSetAttribute(potrf_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)POTRF_SMEM));
+  AuxStream* aux = nullptr;
+  int rc = aux_stream(&aux);
+  if (rc != GPTQ_OK) return rc;
+  cudaStream_t s2 = aux->s;
+  GPTQ_CUDA_TRY(cudaEventRecord(aux->fork, s));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s2, aux->fork, 0));
+
+  int panel = 0;
+  for (int k0 = 0; k0 < n; k0 += PB, ++panel) {
     const int nb = std::min(PB, n - k0);
     const int rest = n - k0 - nb;
-    potrf_inv_kernel<<<1, POTRF_THREADS, 0, s>>>(w.A, ldn, k0, nb, n, w.LIhi, w.LIlo, w.Xt, ldn, w.XQhi,
-                                                          w.XQlo, st);
+    const int b = panel & 1;
+    // the inverse's chain must be done with this buffer's previous use (panel - 2)
+    if (panel >= 2) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->done[b], 0));
+    potrf_inv_kernel<<<1, POTRF_THREADS, POTRF_SMEM, s>>>(w.A, ldn, k0, nb, n, w.LIhi[b], w.LIlo[b], w.Xt, ldn,
+                                                           w.XQhi, w.XQlo, st);
     GPTQ_LAUNCH_CHECK();
-    int rc = GPTQ_OK;
     if (rest > 0) {
       float* A21 = w.A + (int64_t)(k0 + nb) * ldn + k0;
       // L21 = A21 . L_kk^-T (stored in place of A21), with its split
       rc = launch_split_tf32(A21, rest, nb, ldn, w.Phi, w.Plo, PB, st, s);
       if (rc == GPTQ_OK)
-        rc = launch_gemm3(A21, ldn, rest, nb, nb, w.Phi, w.Plo, PB, w.LIhi, w.LIlo, PB, false, st, s, true, w.Lhi,
-                          w.Llo, PB);
-      // A22 -= L21 . L21^T (lower tiles)
-      if (rc == GPTQ_OK)
-        rc = launch_gemm3(w.A + (int64_t)(k0 + nb) * ldn + (k0 + nb), ldn, rest, rest, nb, w.Lhi, w.Llo, PB, w.Lhi,
-                          w.Llo, PB, true, st, s);
+        rc = launch_gemm3(A21, ldn, rest, nb, nb, w.Phi, w.Plo, PB, w.LIhi[b], w.LIlo[b], PB, false, st, s, true,
+                          w.Lhi[b], w.Llo[b], PB);
+      if (rc != GPTQ_OK) return rc;
     }
-    if (rc != GPTQ_OK) return rc;
+    GPTQ_CUDA_TRY(cudaEventRecord(aux->panel, s));
+    if (rest > 0) {
+      // A22 -= L21 . L21^T (lower tiles)
+      rc = launch_gemm3(w.A + (int64_t)(k0 + nb) * ldn + (k0 + nb), ldn, rest, rest, nb, w.Lhi[b], w.Llo[b], PB,
+                        w.Lhi[b], w.Llo[b], PB, true, st, s);
+      if (rc != GPTQ_OK) return rc;
+    }
+    // ---- the inverse's block column k, on the auxiliary stream ----
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(s2, aux->panel, 0));
     if (k0 > 0) {
       // Xt[:k0, k] = Xt[:k0, k] . L_kk^-T, with its split (rows 0..k0 of XQ)
       float* Xk = w.Xt + k0;
-      rc = launch_split_tf32(Xk, k0, nb, ldn, w.XPhi, w.XPlo, PB, st, s);
+      rc = launch_split_tf32(Xk, k0, nb, ldn, w.XPhi, w.XPlo, PB, st, s2);
       if (rc == GPTQ_OK)
-        rc = launch_gemm3(Xk, ldn, k0, nb, nb, w.XPhi, w.XPlo, PB, w.LIhi, w.LIlo, PB, false, st, s, true, w.XQhi,
-                          w.XQlo, PB);
+        rc = launch_gemm3(Xk, ldn, k0, nb, nb, w.XPhi, w.XPlo, PB, w.LIhi[b], w.LIlo[b], PB, false, st, s2, true,
+                          w.XQhi, w.XQlo, PB);
       if (rc != GPTQ_OK) return rc;
     }
     if (rest > 0) {
       // Xt[:k0+nb, later] -= Xt[:k0+nb, k] . L21^T
-      rc = launch_gemm3(w.Xt + (k0 + nb), ldn, k0 + nb, rest, nb, w.XQhi, w.XQlo, PB, w.Lhi, w.Llo, PB, false, st, s);
+      rc = launch_gemm3(w.Xt + (k0 + nb), ldn, k0 + nb, rest, nb, w.XQhi, w.XQlo, PB, w.Lhi[b], w.Llo[b], PB, false,
+                        st, s2);
       if (rc != GPTQ_OK) return rc;
     }
+    GPTQ_CUDA_TRY(cudaEventRecord(aux->done[b], s2));
   }
+  GPTQ_CUDA_TRY(cudaEventRecord(aux->join, s2));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->join, 0));
   {
     dim3 blk(32, 8), grd((unsigned)cdiv(n, 32), (unsigned)cdiv(n, 32));
     write_u_kernel<<<grd, blk, 0, s>>>(w.Xt, n, ldn, U, st);
