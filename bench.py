@@ -50,6 +50,29 @@ def env_rank():
             int(os.environ.get("WORLD_SIZE", "1")))
 
 
+def rank_layer(layer: "S.Layer", rank: int) -> "S.Layer":
+    """Each rank quantizes its own, independently seeded layer of the same shape."""
+    import dataclasses
+    return dataclasses.replace(layer, w=dataclasses.replace(layer.w, seed=layer.w.seed + rank),
+                               x=dataclasses.replace(layer.x, seed=layer.x.seed + rank))
+
+
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """The slowest rank's time (all ranks take this collective in the same order)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gparams_per_s(world: int, out: int, n: int, ms: float) -> float:
+    """Whole-job throughput: every rank quantized one out x n layer in (at most) ms."""
+    return world * out * n / (ms * 1e-3) / 1e9
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -211,10 +234,7 @@ def run_ours(args):
 
     wl = S.workloads()[args.workload]
     layer0, st = wl.layers[0], wl.settings[0]
-    # independent problem per rank
-    import dataclasses
-    layer = dataclasses.replace(layer0, w=dataclasses.replace(layer0.w, seed=layer0.w.seed + rank),
-                                x=dataclasses.replace(layer0.x, seed=layer0.x.seed + rank))
+    layer = rank_layer(layer0, rank)      # independent problem per rank
     out, n, N = layer.w.out, layer.w.n, layer.x.tokens
 
     W_np = S.make_w(layer.w)
@@ -284,12 +304,8 @@ def run_ours(args):
     hess_ms = [e[0].elapsed_time(e[1]) for e in ev]
     prep_ms = [e[1].elapsed_time(e[2]) for e in ev]
     quant_ms = [e[2].elapsed_time(e[3]) for e in ev]
-    ms = statistics.mean(step_ms)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * out * n / (ms * 1e-3) / 1e9
+    ms = max_over_ranks(statistics.mean(step_ms), world, dev)
+    value = job_gparams_per_s(world, out, n, ms)
 
     # dominant kernel: the Hessian tile product (one launch per step)
     peaks = load_peaks()
@@ -306,11 +322,8 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(G, torch, W_host, X_host, st, n, out, dev, args.steps, flush)
-        if world > 1:
-            t = torch.tensor([e2e["ms_per_step"]], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e["ms_per_step"] = float(t.item())
-            e2e["value"] = world * out * n / (e2e["ms_per_step"] * 1e-3) / 1e9
+        e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], world, dev)
+        e2e["value"] = job_gparams_per_s(world, out, n, e2e["ms_per_step"])
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
