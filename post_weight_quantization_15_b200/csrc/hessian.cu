@@ -3,6 +3,9 @@
 //
 // hessian_diag64_kernel: the act-order key, 2 . sum_t x_it^2 in fp64 (every bf16
 // square is exact in fp64).
+#include <stdlib.h>
+#include <string.h>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
@@ -100,7 +103,8 @@ __device__ __forceinline__ void hess_tile(int t, int TB, int& bi, int& bj) {
 }
 
 __global__ void __launch_bounds__(HESS_THREADS, 1)
-hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* H, int n, int kblocks, int32_t* st) {
+hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* H, int n, int kblocks, int32_t* st, int stall,
+                  uint64_t wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   HessSmem& S = *reinterpret_cast<HessSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -135,10 +139,12 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* H, int n, int
   if (!skip) {
     if (warp == 0 && lane == 0) {
       // ---------------- producer ----------------
-      for (int kb = 0; kb < kblocks; ++kb) {
+      // (stall: the failure test withholds every load so that the MMA side's
+      // bounded wait runs out)
+      for (int kb = 0; kb < kblocks && !stall; ++kb) {
         const int s = kb % HSTAGES;
         const uint32_t ph = (uint32_t)(kb / HSTAGES) & 1u;
-        if (!tc::mbar_wait(&S.empty[s], ph ^ 1u, abort_flag)) break;
+        if (!tc::mbar_wait(&S.empty[s], ph ^ 1u, abort_flag, wait_ns)) break;
         tc::mbar_arrive_expect_tx(&S.full[s], inside ? B_BYTES : A_BYTES + B_BYTES);
         tc::tma_load_2d(S.b[s], &tmap, &S.full[s], kb * HKB, bj * HBN);
         tc::tma_load_2d(S.b[s] + A_BYTES, &tmap, &S.full[s], kb * HKB, bj * HBN + HBM_);
@@ -150,14 +156,14 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* H, int n, int
       int kb = 0;
       for (int c = 0; c < nchunks && !*abort_flag; ++c) {
         const int buf = c & 1;
-        if (!tc::mbar_wait(&S.acc_empty[buf], ((uint32_t)(c >> 1) & 1u) ^ 1u, abort_flag)) break;
+        if (!tc::mbar_wait(&S.acc_empty[buf], ((uint32_t)(c >> 1) & 1u) ^ 1u, abort_flag, wait_ns)) break;
         tc::tc_fence_after();
         const int kb_end = min(kblocks, (c + 1) * CHUNK_KB);
         bool first = true;
         for (; kb < kb_end; ++kb) {
           const int s = kb % HSTAGES;
           const uint32_t ph = (uint32_t)(kb / HSTAGES) & 1u;
-          if (!tc::mbar_wait(&S.full[s], ph, abort_flag)) break;
+          if (!tc::mbar_wait(&S.full[s], ph, abort_flag, wait_ns)) break;
           tc::tc_fence_after();
           const uint32_t b0 = tc::smem_u32(S.b[s]);
           const uint32_t a0 = inside ? b0 + a_half * (HBM_ * 128) : tc::smem_u32(S.a[s]);
@@ -189,7 +195,7 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* H, int n, int
       for (int c = 0; c < nchunks; ++c) {
         const int buf = c & 1;
         int ready = 0;
-        if (lane == 0) ready = tc::mbar_wait(&S.acc_full[buf], (uint32_t)(c >> 1) & 1u, abort_flag);
+        if (lane == 0) ready = tc::mbar_wait(&S.acc_full[buf], (uint32_t)(c >> 1) & 1u, abort_flag, wait_ns);
         ready = __shfl_sync(0xffffffffu, ready, 0);
         if (!ready) { ok = false; break; }
         tc::tc_fence_after();
@@ -268,8 +274,14 @@ int launch_hessian(float* H, int n, const void* X, int64_t ld_x, int64_t tokens,
   int tiles = 0;
   for (int bi = 0; bi < TA; ++bi) tiles += TB - bi / 2;
   const int kblocks = (int)cdiv(tokens, HKB);
+  // Failure test switch (host side, read per call): GPTQ_FAULT_INJECT=hessian_stall
+  // withholds the operand loads and shortens the wait limit to 200 ms, so the
+  // kernel's bounded waits run out and it reports GPTQ_ERR_TIMEOUT.
+  const char* fi = getenv("GPTQ_FAULT_INJECT");
+  const int stall = (fi != nullptr && strcmp(fi, "hessian_stall") == 0) ? 1 : 0;
+  const uint64_t wait_ns = stall ? 200000000ull : tc::kWaitLimitNs;
   GPTQ_CUDA_TRY(cudaFuncSetAttribute(hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)HESS_SMEM));
-  hessian_tc_kernel<<<tiles, HESS_THREADS, HESS_SMEM, s>>>(map, H, n, kblocks, st);
+  hessian_tc_kernel<<<tiles, HESS_THREADS, HESS_SMEM, s>>>(map, H, n, kblocks, st, stall, wait_ns);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }

@@ -58,7 +58,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Waits for the phase of `parity` to complete.  Returns false (and raises the
 // CTA's abort flag) if the wait exceeds kWaitLimitNs or another role aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -66,7 +67,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       if (*abort_flag) return false;
       const uint64_t now = globaltimer();
       if (t0 == 0) t0 = now;
-      else if (now - t0 > kWaitLimitNs) { *abort_flag = 1; return false; }
+      else if (now - t0 > limit_ns) { *abort_flag = 1; return false; }
     }
   }
 }
