@@ -23,13 +23,15 @@ namespace gptq {
 namespace {
 
 constexpr int BLK = 128;           // columns per lazy batch
+constexpr int SUPER = 4;           // lazy batches per super-block
+constexpr int SBK = SUPER * BLK;   // columns per super-block
 
 struct QuantWs {
   float* Wf;          // [out, n] working weights, processing order
-  float* Ehi;         // [out, BLK] scaled errors of the current block, TF32-exact high part
-  float* Elo;         // [out, BLK] and the remainder
-  float* Bhi;         // [n, BLK] U[block rows, later columns]^T, high part (K-major operand)
-  float* Blo;         // [n, BLK] and the remainder
+  float* Ehi;         // [out, SBK] scaled errors of the current super-block, TF32-exact high part
+  float* Elo;         // [out, SBK] and the remainder
+  float* Bhi;         // [n, SBK] U[super-block rows, later columns]^T, high part (K-major operand)
+  float* Blo;         // [n, SBK] and the remainder
   uint8_t* codes_p;   // [out, n] codes, processing order
   int32_t* invperm;   // [n] processing position of every input column
   float* rows;        // [out] row-wide scale, [out] row-wide zero (group_size = -1)
@@ -39,10 +41,10 @@ QuantWs carve(void* ws, int out, int n) {
   char* p = static_cast<char*>(ws);
   QuantWs w;
   w.Wf = reinterpret_cast<float*>(p);        p += align_up((size_t)out * n * 4, 256);
-  w.Ehi = reinterpret_cast<float*>(p);       p += align_up((size_t)out * BLK * 4, 256);
-  w.Elo = reinterpret_cast<float*>(p);       p += align_up((size_t)out * BLK * 4, 256);
-  w.Bhi = reinterpret_cast<float*>(p);       p += align_up((size_t)n * BLK * 4, 256);
-  w.Blo = reinterpret_cast<float*>(p);       p += align_up((size_t)n * BLK * 4, 256);
+  w.Ehi = reinterpret_cast<float*>(p);       p += align_up((size_t)out * SBK * 4, 256);
+  w.Elo = reinterpret_cast<float*>(p);       p += align_up((size_t)out * SBK * 4, 256);
+  w.Bhi = reinterpret_cast<float*>(p);       p += align_up((size_t)n * SBK * 4, 256);
+  w.Blo = reinterpret_cast<float*>(p);       p += align_up((size_t)n * SBK * 4, 256);
   w.codes_p = reinterpret_cast<uint8_t*>(p); p += align_up((size_t)out * n, 256);
   w.invperm = reinterpret_cast<int32_t*>(p); p += align_up((size_t)n * 4, 256);
   w.rows = reinterpret_cast<float*>(p);
@@ -62,7 +64,7 @@ __device__ __forceinline__ float to_f16_scale(float s) {
   return fmaxf(__half2float(__float2half_rn(s)), kMin);
 }
 
-struct QParams { float s, z; };
+struct QParams { float s, z, rs; };   // scale, zero point, fp32 reciprocal of the scale
 
 __device__ __forceinline__ QParams params_asym(float lo, float hi, float maxq) {
   lo = fminf(lo, 0.f);
@@ -71,6 +73,7 @@ __device__ __forceinline__ QParams params_asym(float lo, float hi, float maxq) {
   QParams p;
   p.s = to_f16_scale(__fdiv_rn(__fsub_rn(hi, lo), maxq));
   p.z = fminf(fmaxf(rintf(__fdiv_rn(-lo, p.s)), 0.f), maxq);
+  p.rs = __frcp_rn(p.s);
   return p;
 }
 
@@ -79,11 +82,23 @@ __device__ __forceinline__ QParams params_sym(float amax, int bits) {
   QParams p;
   p.s = to_f16_scale(__fdiv_rn(amax, (float)((1 << (bits - 1)) - 1)));
   p.z = (float)(1 << (bits - 1));
+  p.rs = __frcp_rn(p.s);
   return p;
 }
 
+// rint(w / s) with the quotient rounded as IEEE division rounds it.  t = w . fl(1/s)
+// is within |w/s| . 2^-23 of w/s, and fl(w/s) within |w/s| . 2^-24: for |t| <= 2^10
+// both lie within 2^-12 of each other, so rint(t) == rint(fl(w/s)) unless t is within
+// 2^-12 of a half-integer.  Those rare cases (and huge quotients) take the division.
+__device__ __forceinline__ float rint_div(float w, QParams p) {
+  const float t = w * p.rs;
+  const float f = t - floorf(t);
+  if (fabsf(t) < 1024.f && fabsf(f - 0.5f) > 2.44140625e-4f) return rintf(t);
+  return rintf(__fdiv_rn(w, p.s));
+}
+
 __device__ __forceinline__ float quant_code(float w, QParams p, int bits, bool sym) {
-  const float q = rintf(__fdiv_rn(w, p.s));
+  const float q = rint_div(w, p);
   if (sym) {
     const float h = (float)((1 << (bits - 1)) - 1);
     return fminf(fmaxf(q, -h), h) + p.z;
@@ -164,12 +179,14 @@ struct SweepShape {
   static constexpr int LDU = TPR * SEGP;         // padded U row stride
   static constexpr int THREADS = 128;
   static constexpr int ROWS = THREADS / TPR;     // rows per CTA
-  static constexpr size_t SMEM = (size_t)BLK * LDU * sizeof(float) + BLK * sizeof(float);
+  static constexpr size_t SMEM =
+      (size_t)BLK * LDU * sizeof(float) + BLK * sizeof(float) + (size_t)ROWS * (BLK + 1) * sizeof(float);
 };
 
 template <int GS, int TPR>
 __global__ void __launch_bounds__(128)
-sweep_kernel(float* Wf, int out, int n, int b0, int bw, const float* U, float* Ehi, float* Elo, uint8_t* codes_p,
+sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const float* U, float* Ehi, float* Elo,
+             uint8_t* codes_p,
              uint16_t* scales, uint16_t* zeros, const float* rows, float* err_sq, int bits, int sym,
              const int32_t* st) {
   using SS = SweepShape<TPR>;
@@ -218,8 +235,8 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, const float* U, float* E
   const bool symq = sym != 0;
   const float maxq = (float)((1 << bits) - 1);
   QParams p;
-  if (GS == 0) { p.s = rows[rr]; p.z = rows[out + rr]; }
-  else { p.s = 1.f; p.z = 0.f; }
+  if (GS == 0) { p.s = rows[rr]; p.z = rows[out + rr]; p.rs = __frcp_rn(p.s); }
+  else { p.s = 1.f; p.z = 0.f; p.rs = 1.f; }
   float esq = 0.f;
   uint32_t cw[SEG / 4];
 #pragma unroll
@@ -276,8 +293,8 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, const float* U, float* E
   if (!live || seg * SEG >= bw) {
     // nothing to store for this lane
   } else {
-    float* ehi = Ehi + (int64_t)r * BLK + seg * SEG;
-    float* elo = Elo + (int64_t)r * BLK + seg * SEG;
+    float* ehi = Ehi + (int64_t)r * SBK + eoff + seg * SEG;
+    float* elo = Elo + (int64_t)r * SBK + eoff + seg * SEG;
 #pragma unroll
     for (int k = 0; k < SEG; k += 4) {
       const float4 h = make_float4(tf32_hi(w[k]), tf32_hi(w[k + 1]), tf32_hi(w[k + 2]), tf32_hi(w[k + 3]));
@@ -292,31 +309,86 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, const float* U, float* E
 #pragma unroll
   for (int o = 1; o < TPR; o <<= 1) esq += __shfl_xor_sync(0xffffffffu, esq, o);
   if (err_sq && live && seg == 0) err_sq[r] += esq;
+
+  // Near update: the rest of this super-block, columns [b0 + bw, se), absorbs this
+  // block's errors, W[r][c] -= sum_j e_j U[b0 + j][c], in fp32 on the CUDA cores,
+  // 128 columns at a time with the U rows staged in shared memory.  The columns past
+  // the super-block are updated once per super-block by the tensor-core GEMM.
+  if (b0 + bw < se) {
+    float* Es = dinv + BLK;                        // [ROWS][BLK + 1] this block's errors per row
+    const int rloc = threadIdx.x / TPR;
+#pragma unroll
+    for (int k = 0; k < SEG; ++k) Es[rloc * (BLK + 1) + seg * SEG + k] = (seg * SEG < bw) ? w[k] : 0.f;
+    for (int c0n = b0 + bw; c0n < se; c0n += BLK) {
+      const int cwid = min(BLK, se - c0n);
+      __syncthreads();                             // Us is free; Es is complete
+      for (int idx = threadIdx.x; idx < BLK * (BLK / 4); idx += blockDim.x) {
+        const int j = idx / (BLK / 4), c = (idx % (BLK / 4)) * 4;
+        float* dst = Us + j * SS::LDU + (c / SEG) * SS::SEGP + (c % SEG);
+        if (j < bw && c < cwid) {
+          const float* src = U + (int64_t)(b0 + j) * n + c0n + c;
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                       "l"(src)
+                       : "memory");
+        } else {
+          *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      __syncthreads();
+      float acc[SEG];
+#pragma unroll
+      for (int k = 0; k < SEG; ++k) acc[k] = 0.f;
+      const float* erow = Es + rloc * (BLK + 1);
+#pragma unroll 4
+      for (int j = 0; j < bw; ++j) {
+        const float ej = erow[j];
+        const float* urow = Us + j * SS::LDU + seg * SS::SEGP;
+#pragma unroll
+        for (int k = 0; k < SEG; k += 4) {
+          const float4 u = *reinterpret_cast<const float4*>(urow + k);
+          acc[k] = fmaf(ej, u.x, acc[k]);
+          acc[k + 1] = fmaf(ej, u.y, acc[k + 1]);
+          acc[k + 2] = fmaf(ej, u.z, acc[k + 2]);
+          acc[k + 3] = fmaf(ej, u.w, acc[k + 3]);
+        }
+      }
+      if (live && seg * SEG < cwid) {
+        float* dst = Wf + (int64_t)r * n + c0n + seg * SEG;
+#pragma unroll
+        for (int k = 0; k < SEG; k += 4) {
+          float4 o = *reinterpret_cast<float4*>(dst + k);
+          o.x -= acc[k]; o.y -= acc[k + 1]; o.z -= acc[k + 2]; o.w -= acc[k + 3];
+          *reinterpret_cast<float4*>(dst + k) = o;
+        }
+      }
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
-// K4 operand: B[c - e][k] = U[b0 + k][c] for c in [e, n), k < bw, split into its
-// TF32 high part and remainder (rows of 128, K-major for the tensor cores).
+// K4 operand: B[c - e][k] = U[b0 + k][c] for c in [e, n), k < kw, split into its
+// TF32 high part and remainder (rows of ldk, K-major for the tensor cores).
 // 32 x 32 tiles through shared memory keep both the read and the write coalesced.
 // ---------------------------------------------------------------------------
-__global__ void u_block_transpose_split_kernel(const float* U, int n, int b0, int bw, int e, float* Bhi, float* Blo,
-                                               const int32_t* st) {
+__global__ void u_block_transpose_split_kernel(const float* U, int n, int b0, int kw, int e, float* Bhi, float* Blo,
+                                               int ldk, const int32_t* st) {
   if (has_error(st)) return;
   __shared__ float t[32][33];
   const int c0 = e + blockIdx.x * 32;      // U column tile
-  const int k0 = blockIdx.y * 32;          // U row tile within the block
+  const int k0 = blockIdx.y * 32;          // U row tile within the super-block
   for (int yy = threadIdx.y; yy < 32; yy += 8) {
     const int k = k0 + yy, c = c0 + threadIdx.x;
-    t[yy][threadIdx.x] = (k < bw && c < n) ? U[(int64_t)(b0 + k) * n + c] : 0.f;
+    t[yy][threadIdx.x] = (k < kw && c < n) ? U[(int64_t)(b0 + k) * n + c] : 0.f;
   }
   __syncthreads();
   for (int yy = threadIdx.y; yy < 32; yy += 8) {
     const int c = c0 + yy, k = k0 + threadIdx.x;
-    if (c < n && k < BLK) {
+    if (c < n && k < ldk) {
       const float x = t[threadIdx.x][yy];
       const float h = tf32_hi(x);
-      Bhi[(int64_t)(c - e) * BLK + k] = h;
-      Blo[(int64_t)(c - e) * BLK + k] = x - h;
+      Bhi[(int64_t)(c - e) * ldk + k] = h;
+      Blo[(int64_t)(c - e) * ldk + k] = x - h;
     }
   }
 }
@@ -358,8 +430,8 @@ __global__ void codes_out_kernel(const uint8_t* codes_p, const int32_t* invperm,
 
 size_t quantize_ws_bytes(int out, int n, int block) {
   (void)block;
-  return align_up((size_t)out * n * 4, 256) + 2 * align_up((size_t)out * BLK * 4, 256) +
-         2 * align_up((size_t)n * BLK * 4, 256) + align_up((size_t)out * n, 256) + align_up((size_t)n * 4, 256) +
+  return align_up((size_t)out * n * 4, 256) + 2 * align_up((size_t)out * SBK * 4, 256) +
+         2 * align_up((size_t)n * SBK * 4, 256) + align_up((size_t)out * n, 256) + align_up((size_t)n * 4, 256) +
          align_up((size_t)out * 8, 256);
 }
 
@@ -404,18 +476,25 @@ int launch_quantize(const void* W, int w_dtype, int out, int n, const float* U, 
   const size_t smem = wide ? SweepShape<8>::SMEM : SweepShape<4>::SMEM;
   const int rows_per_cta = wide ? SweepShape<8>::ROWS : SweepShape<4>::ROWS;
   GPTQ_CUDA_TRY(cudaFuncSetAttribute(sweep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  for (int b0 = 0; b0 < n; b0 += BLK) {
-    const int bw = std::min(BLK, n - b0);
-    sweep<<<(unsigned)cdiv(out, rows_per_cta), 128, smem, s>>>(w.Wf, out, n, b0, bw, U, w.Ehi, w.Elo, w.codes_p,
-                                                                scales, zeros, w.rows, err_sq, bits, sym, st);
-    GPTQ_LAUNCH_CHECK();
-    const int e = b0 + bw;
-    if (e < n) {
-      dim3 blk(32, 8), grd((unsigned)cdiv(n - e, 32), (unsigned)(BLK / 32));
-      u_block_transpose_split_kernel<<<grd, blk, 0, s>>>(U, n, b0, bw, e, w.Bhi, w.Blo, st);
+  // Two-level lazy batches: blocks of 128 columns inside super-blocks of 512.  A
+  // block's sweep also updates the rest of its super-block; the columns after a
+  // super-block absorb its 512 errors at once on the tensor cores.
+  for (int s0 = 0; s0 < n; s0 += SBK) {
+    const int se = std::min(n, s0 + SBK);
+    for (int b0 = s0; b0 < se; b0 += BLK) {
+      const int bw = std::min(BLK, n - b0);
+      sweep<<<(unsigned)cdiv(out, rows_per_cta), 128, smem, s>>>(w.Wf, out, n, b0, bw, b0 - s0, se, U, w.Ehi, w.Elo,
+                                                                  w.codes_p, scales, zeros, w.rows, err_sq, bits, sym,
+                                                                  st);
       GPTQ_LAUNCH_CHECK();
-      // Wf[:, e:] -= Err . U[b0:b0+bw, e:]
-      const int rc = launch_gemm3(w.Wf + e, n, out, n - e, BLK, w.Ehi, w.Elo, BLK, w.Bhi, w.Blo, BLK, false, st, s);
+    }
+    if (se < n) {
+      const int kw = se - s0;   // == SBK
+      dim3 blk(32, 8), grd((unsigned)cdiv(n - se, 32), (unsigned)(SBK / 32));
+      u_block_transpose_split_kernel<<<grd, blk, 0, s>>>(U, n, s0, kw, se, w.Bhi, w.Blo, SBK, st);
+      GPTQ_LAUNCH_CHECK();
+      // Wf[:, se:] -= Err[:, super-block] . U[super-block, se:]
+      const int rc = launch_gemm3(w.Wf + se, n, out, n - se, kw, w.Ehi, w.Elo, SBK, w.Bhi, w.Blo, SBK, false, st, s);
       if (rc != GPTQ_OK) return rc;
     }
   }
