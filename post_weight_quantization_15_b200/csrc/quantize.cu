@@ -18,6 +18,11 @@
 #include "common.cuh"
 #include "internal.h"
 
+// Timeline marks for probes; empty in the library build.
+#ifndef GPTQ_SWEEP_MARK
+#define GPTQ_SWEEP_MARK(i)
+#endif
+
 namespace gptq {
 
 namespace {
@@ -86,24 +91,39 @@ __device__ __forceinline__ QParams params_sym(float amax, int bits) {
   return p;
 }
 
-// rint(w / s) with the quotient rounded as IEEE division rounds it.  t = w . fl(1/s)
-// is within |w/s| . 2^-23 of w/s, and fl(w/s) within |w/s| . 2^-24: for |t| <= 2^10
-// both lie within 2^-12 of each other, so rint(t) == rint(fl(w/s)) unless t is within
-// 2^-12 of a half-integer.  Those rare cases (and huge quotients) take the division.
+// rint(fl(w / s)), fl = IEEE round-to-nearest division, without dividing and
+// without branches (the column loop stays one basic block).
+//   t = w . fl(1/s) is within |w/s| . 2^-22 of w/s, so for |t| < 1024 the decision
+//   is between k = floor(t) and k + 1, i.e. on which side of h = k + 1/2 the
+//   rounded quotient lies.  d = fma(-h, s, w) = RN(w - h.s): h.s is exact (h has
+//   at most 13 significant bits, s is an fp16 value), so the sign of d is the sign
+//   of w/s - h, and d itself is exact whenever w/s is within 1/4 of h (Sterbenz).
+//   The rounded quotient equals h exactly iff |w/s - h| <= ulp(h)/2, i.e.
+//   |d| <= s . ulp(h)/2 (h's last mantissa bit is 0 for |h| < 2^22, so a tie
+//   rounds to h); then rint picks the even one of k, k + 1.
+//   For |t| >= 1024 every code saturates, and rint(t) clamps to the same code.
 __device__ __forceinline__ float rint_div(float w, QParams p) {
   const float t = w * p.rs;
-  const float f = t - floorf(t);
-  if (fabsf(t) < 1024.f && fabsf(f - 0.5f) > 2.44140625e-4f) return rintf(t);
-  return rintf(__fdiv_rn(w, p.s));
+  const float k = floorf(t);
+  const float h = k + 0.5f;
+  const float d = fmaf(-h, p.s, w);
+  const float ulp_h = __uint_as_float((__float_as_uint(h) & 0x7F800000u) - (23u << 23));
+  const float thr = p.s * ulp_h * 0.5f;
+  const float k_even = (((int)k) & 1) ? k + 1.f : k;
+  const float r = fabsf(d) <= thr ? k_even : (d > 0.f ? k + 1.f : k);
+  return fabsf(t) < 1024.f ? r : rintf(t);
 }
 
-__device__ __forceinline__ float quant_code(float w, QParams p, int bits, bool sym) {
-  const float q = rint_div(w, p);
+__device__ __forceinline__ float code_from_q(float q, QParams p, int bits, bool sym) {
   if (sym) {
     const float h = (float)((1 << (bits - 1)) - 1);
     return fminf(fmaxf(q, -h), h) + p.z;
   }
   return fminf(fmaxf(q + p.z, 0.f), (float)((1 << bits) - 1));
+}
+
+__device__ __forceinline__ float quant_code(float w, QParams p, int bits, bool sym) {
+  return code_from_q(rint_div(w, p), p, bits, sym);
 }
 
 // ---------------------------------------------------------------------------
@@ -179,8 +199,9 @@ struct SweepShape {
   static constexpr int LDU = TPR * SEGP;         // padded U row stride
   static constexpr int THREADS = 128;
   static constexpr int ROWS = THREADS / TPR;     // rows per CTA
+  static constexpr int LDE = BLK + 4;            // error row stride (16-byte aligned rows)
   static constexpr size_t SMEM =
-      (size_t)BLK * LDU * sizeof(float) + BLK * sizeof(float) + (size_t)ROWS * (BLK + 1) * sizeof(float);
+      (size_t)BLK * LDU * sizeof(float) + BLK * sizeof(float) + (size_t)ROWS * LDE * sizeof(float);
 };
 
 template <int GS, int TPR>
@@ -192,6 +213,7 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
   using SS = SweepShape<TPR>;
   constexpr int SEG = SS::SEG;
   if (has_error(st)) return;
+  GPTQ_SWEEP_MARK(0);
   extern __shared__ float smem[];
   float* Us = smem;                       // [BLK][LDU]
   float* dinv = smem + BLK * SS::LDU;     // [BLK] 1 / U_jj
@@ -216,6 +238,7 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
     dinv[j] = (j < bw) ? 1.f / d : 0.f;
   }
   __syncthreads();
+  GPTQ_SWEEP_MARK(1);
 
   const int lane = threadIdx.x & 31;
   const int seg = lane % TPR;
@@ -243,6 +266,11 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
   for (int k = 0; k < SEG / 4; ++k) cw[k] = 0u;
   const int group_lane0 = lane & ~(TPR - 1);
 
+  // The owner of column j quantizes it from `wq`, a scalar that already holds every
+  // update up to column j - 1: the update by column j - 1 is applied to it with the
+  // owner's own error, so the broadcast of that error (needed by the other lanes)
+  // overlaps the next column's decision instead of preceding it.
+  float wq = 0.f;
   for (int jb = 0; jb < TPR; ++jb) {
     if (jb * SEG >= bw) break;
     const bool owner = seg == jb;
@@ -271,10 +299,12 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
           zeros[(int64_t)g * out + r] = __half_as_ushort(__float2half_rn(p.z));
         }
       }
-      const float c = quant_code(w[jj], p, bits, symq);
-      const float e_own = (w[jj] - p.s * (c - p.z)) * dinv[j];
-      const float e = __shfl_sync(0xffffffffu, e_own, group_lane0 | jb);
+      if (jj == 0) wq = w[0];           // a new segment (owner): the array holds every update
+      const float c = code_from_q(rint_div(wq, p), p, bits, symq);
+      const float e_own = (wq - p.s * (c - p.z)) * dinv[j];
       const float* urow = Us + j * SS::LDU + seg * SS::SEGP;
+      if (jj + 1 < SEG) wq = fmaf(-e_own, urow[jj + 1], w[jj + 1]);   // the owner's next column
+      const float e = __shfl_sync(0xffffffffu, e_own, group_lane0 | jb);
 #pragma unroll
       for (int k = 0; k < SEG; k += 4) {
         const float4 u = *reinterpret_cast<const float4*>(urow + k);
@@ -290,6 +320,7 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
       }
     }
   }
+  GPTQ_SWEEP_MARK(2);
   if (!live || seg * SEG >= bw) {
     // nothing to store for this lane
   } else {
@@ -309,16 +340,17 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
 #pragma unroll
   for (int o = 1; o < TPR; o <<= 1) esq += __shfl_xor_sync(0xffffffffu, esq, o);
   if (err_sq && live && seg == 0) err_sq[r] += esq;
+  GPTQ_SWEEP_MARK(3);
 
   // Near update: the rest of this super-block, columns [b0 + bw, se), absorbs this
   // block's errors, W[r][c] -= sum_j e_j U[b0 + j][c], in fp32 on the CUDA cores,
   // 128 columns at a time with the U rows staged in shared memory.  The columns past
   // the super-block are updated once per super-block by the tensor-core GEMM.
   if (b0 + bw < se) {
-    float* Es = dinv + BLK;                        // [ROWS][BLK + 1] this block's errors per row
+    float* Es = dinv + BLK;                        // [ROWS][LDE] this block's errors per row
     const int rloc = threadIdx.x / TPR;
 #pragma unroll
-    for (int k = 0; k < SEG; ++k) Es[rloc * (BLK + 1) + seg * SEG + k] = (seg * SEG < bw) ? w[k] : 0.f;
+    for (int k = 0; k < SEG; ++k) Es[rloc * SS::LDE + seg * SEG + k] = (seg * SEG < bw) ? w[k] : 0.f;
     for (int c0n = b0 + bw; c0n < se; c0n += BLK) {
       const int cwid = min(BLK, se - c0n);
       __syncthreads();                             // Us is free; Es is complete
@@ -336,21 +368,27 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
       }
       asm volatile("cp.async.wait_all;" ::: "memory");
       __syncthreads();
+      GPTQ_SWEEP_MARK(4);
       float acc[SEG];
 #pragma unroll
       for (int k = 0; k < SEG; ++k) acc[k] = 0.f;
-      const float* erow = Es + rloc * (BLK + 1);
-#pragma unroll 4
-      for (int j = 0; j < bw; ++j) {
-        const float ej = erow[j];
-        const float* urow = Us + j * SS::LDU + seg * SS::SEGP;
+      const float* erow = Es + rloc * SS::LDE;
+      // four errors and four U rows per step; the errors past bw are zero
+#pragma unroll 1
+      for (int j = 0; j < bw; j += 4) {
+        const float4 e4 = *reinterpret_cast<const float4*>(erow + j);
+        const float ev[4] = {e4.x, e4.y, e4.z, e4.w};
 #pragma unroll
-        for (int k = 0; k < SEG; k += 4) {
-          const float4 u = *reinterpret_cast<const float4*>(urow + k);
-          acc[k] = fmaf(ej, u.x, acc[k]);
-          acc[k + 1] = fmaf(ej, u.y, acc[k + 1]);
-          acc[k + 2] = fmaf(ej, u.z, acc[k + 2]);
-          acc[k + 3] = fmaf(ej, u.w, acc[k + 3]);
+        for (int q = 0; q < 4; ++q) {
+          const float* urow = Us + (j + q) * SS::LDU + seg * SS::SEGP;
+#pragma unroll
+          for (int k = 0; k < SEG; k += 4) {
+            const float4 u = *reinterpret_cast<const float4*>(urow + k);
+            acc[k] = fmaf(ev[q], u.x, acc[k]);
+            acc[k + 1] = fmaf(ev[q], u.y, acc[k + 1]);
+            acc[k + 2] = fmaf(ev[q], u.z, acc[k + 2]);
+            acc[k + 3] = fmaf(ev[q], u.w, acc[k + 3]);
+          }
         }
       }
       if (live && seg * SEG < cwid) {
@@ -362,6 +400,7 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
           *reinterpret_cast<float4*>(dst + k) = o;
         }
       }
+      GPTQ_SWEEP_MARK(5);
     }
   }
 }
@@ -465,16 +504,17 @@ int launch_quantize(const void* W, int w_dtype, int out, int n, const float* U, 
     row_params_kernel<<<out, 256, 0, s>>>(w.Wf, out, n, bits, sym, w.rows, scales, zeros, st);
     GPTQ_LAUNCH_CHECK();
   }
-  // Few rows: 8 lanes per row (more parallelism); many rows: 4 (less redundant work).
+  // Few rows: 16 lanes per row (more parallelism, less work per lane); many rows: 4
+  // (less redundant work).
   const bool wide = out < 4096;
   auto pick = [&](auto tpr_tag) {
     constexpr int T = decltype(tpr_tag)::value;
     return gs == 32 ? sweep_kernel<32, T> : gs == 64 ? sweep_kernel<64, T> : gs == 128 ? sweep_kernel<128, T>
                                                                                       : sweep_kernel<0, T>;
   };
-  auto sweep = wide ? pick(std::integral_constant<int, 8>{}) : pick(std::integral_constant<int, 4>{});
-  const size_t smem = wide ? SweepShape<8>::SMEM : SweepShape<4>::SMEM;
-  const int rows_per_cta = wide ? SweepShape<8>::ROWS : SweepShape<4>::ROWS;
+  auto sweep = wide ? pick(std::integral_constant<int, 16>{}) : pick(std::integral_constant<int, 4>{});
+  const size_t smem = wide ? SweepShape<16>::SMEM : SweepShape<4>::SMEM;
+  const int rows_per_cta = wide ? SweepShape<16>::ROWS : SweepShape<4>::ROWS;
   GPTQ_CUDA_TRY(cudaFuncSetAttribute(sweep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   // Two-level lazy batches: blocks of 128 columns inside super-blocks of 512.  A
   // block's sweep also updates the rest of its super-block; the columns after a

@@ -315,3 +315,38 @@ def test_bounded_wait_reports_timeout_and_the_context_survives(monkeypatch):
     H64 = O.hessian(x)
     iu = np.triu_indices(256)
     assert np.allclose(H.cpu().numpy().astype(np.float64)[iu], H64[iu], rtol=1e-4, atol=1e-3)
+
+
+@pytest.mark.parametrize("sym", [True, False])
+def test_rounding_boundaries_are_bit_exact(sym):
+    """Weights placed on and within a few ulps of (k + 1/2).s, where the fp32 quotient
+    decides the code by its last bit; with H = I there is no compensation, so the
+    codes must equal round-to-nearest of the IEEE quotient exactly."""
+    dev = _dev()
+    rng = np.random.default_rng(7 + sym)
+    out, n, gs = 512, 512, 128
+    s0 = np.float16(np.exp(rng.uniform(-9, -3, (out, n // gs)))).astype(np.float32)   # fp16 scales
+    W = np.zeros((out, n), np.float32)
+    for g in range(n // gs):
+        s = s0[:, g:g + 1]
+        k = rng.integers(-7, 7, (out, gs)).astype(np.float32)
+        base = ((k + np.float32(0.5)) * s).astype(np.float32)
+        steps = rng.integers(-3, 4, (out, gs))
+        w = base.copy()
+        for _ in range(3):
+            move = np.abs(steps) > _
+            w = np.where(move, np.nextafter(w, np.where(steps > 0, np.inf, -np.inf).astype(np.float32)), w)
+        if sym:
+            w[:, 0] = 7 * s[:, 0]          # amax = 7 s  ->  scale = fp16(7 s / 7) = s
+            w[:, 1] = -7 * s[:, 0]
+        else:
+            w[:, 0] = -7 * s[:, 0]         # lo = -7 s, hi = 8 s  ->  scale = fp16(15 s / 15) = s, zero = 7
+            w[:, 1] = 8 * s[:, 0]
+        W[:, g * gs:(g + 1) * gs] = np.clip(w, -7 * s, (7 if sym else 8) * s)
+    H = torch.eye(n, dtype=torch.float32, device=dev)
+    p = G.prepare(H, 0.01, False)
+    q = G.quantize_layer(_w_tensor(W, dev), p, 4, gs, sym, want_codes=True)
+    G.raise_on_status(p.status, "boundaries")
+    rc, rs, rz = O.rtn(W, 4, gs, sym)
+    assert np.array_equal(rs, s0.T)
+    assert np.array_equal(q.codes.cpu().numpy(), rc)
