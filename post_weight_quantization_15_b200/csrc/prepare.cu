@@ -351,12 +351,15 @@ __global__ void write_u_kernel(const float* Xt, int n, int ldx, float* U, const 
   }
 }
 
-// The blocked inverse's updates run on an auxiliary stream next to the
-// factorization: one non-blocking stream and a few events per host thread and
-// device, created on first use and kept for the life of the process.
+// The blocked inverse's updates and the trailing updates beyond the next panel run
+// on two auxiliary streams next to the factorization: two non-blocking streams and
+// a few events per host thread and device, created on first use and kept for the
+// life of the process.
 struct AuxStream {
-  cudaStream_t s = nullptr;
+  cudaStream_t s = nullptr;    // the inverse's chain
+  cudaStream_t t = nullptr;    // the trailing updates beyond the next panel
   cudaEvent_t fork = nullptr, panel = nullptr, join = nullptr, done[2] = {nullptr, nullptr};
+  cudaEvent_t rest = nullptr, tjoin = nullptr;
 };
 
 int aux_stream(AuxStream** out) {
@@ -367,10 +370,12 @@ int aux_stream(AuxStream** out) {
   AuxStream& a = per_dev[dev];
   if (a.s == nullptr) {
     if (cudaStreamCreateWithFlags(&a.s, cudaStreamNonBlocking) != cudaSuccess) return GPTQ_ERR_CUDA;
+    if (cudaStreamCreateWithFlags(&a.t, cudaStreamNonBlocking) != cudaSuccess) return GPTQ_ERR_CUDA;
     const unsigned f = cudaEventDisableTiming;
     if (cudaEventCreateWithFlags(&a.fork, f) != cudaSuccess || cudaEventCreateWithFlags(&a.panel, f) != cudaSuccess ||
         cudaEventCreateWithFlags(&a.join, f) != cudaSuccess || cudaEventCreateWithFlags(&a.done[0], f) != cudaSuccess ||
-        cudaEventCreateWithFlags(&a.done[1], f) != cudaSuccess)
+        cudaEventCreateWithFlags(&a.done[1], f) != cudaSuccess || cudaEventCreateWithFlags(&a.rest, f) != cudaSuccess ||
+        cudaEventCreateWithFlags(&a.tjoin, f) != cudaSuccess)
       return GPTQ_ERR_CUDA;
   }
   *out = &a;
@@ -410,8 +415,11 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
   int rc = aux_stream(&aux);
   if (rc != GPTQ_OK) return rc;
   cudaStream_t s2 = aux->s;
+  cudaStream_t s3 = aux->t;
   GPTQ_CUDA_TRY(cudaEventRecord(aux->fork, s));
   GPTQ_CUDA_TRY(cudaStreamWaitEvent(s2, aux->fork, 0));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s3, aux->fork, 0));
+  bool rest_pending = false;
 
   int panel = 0;
   for (int k0 = 0; k0 < n; k0 += PB, ++panel) {
@@ -434,10 +442,26 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
     }
     GPTQ_CUDA_TRY(cudaEventRecord(aux->panel, s));
     if (rest > 0) {
-      // A22 -= L21 . L21^T (lower tiles)
-      rc = launch_gemm3(w.A + (int64_t)(k0 + nb) * ldn + (k0 + nb), ldn, rest, rest, nb, w.Lhi[b], w.Llo[b], PB,
-                        w.Lhi[b], w.Llo[b], PB, true, st, s);
+      // A22 -= L21 . L21^T.  Look-ahead: the next panel's column block on this
+      // stream (the next diagonal factorization needs only it); the lower tiles
+      // beyond it on the trailing stream, overlapping the next panel's work.
+      const int nb2 = std::min(PB, rest);
+      float* A22 = w.A + (int64_t)(k0 + nb) * ldn + (k0 + nb);
+      // the trailing stream's previous update overlaps this column block
+      if (rest_pending) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->rest, 0));
+      rc = launch_gemm3(A22, ldn, rest, nb2, nb, w.Lhi[b], w.Llo[b], PB, w.Lhi[b], w.Llo[b], PB, false, st, s);
       if (rc != GPTQ_OK) return rc;
+      if (rest > nb2) {
+        GPTQ_CUDA_TRY(cudaStreamWaitEvent(s3, aux->panel, 0));
+        rc = launch_gemm3(A22 + (int64_t)nb2 * ldn + nb2, ldn, rest - nb2, rest - nb2, nb, w.Lhi[b] + (int64_t)nb2 * PB,
+                          w.Llo[b] + (int64_t)nb2 * PB, PB, w.Lhi[b] + (int64_t)nb2 * PB, w.Llo[b] + (int64_t)nb2 * PB,
+                          PB, true, st, s3);
+        if (rc != GPTQ_OK) return rc;
+        GPTQ_CUDA_TRY(cudaEventRecord(aux->rest, s3));
+        rest_pending = true;
+      } else {
+        rest_pending = false;
+      }
     }
     // ---- the inverse's block column k, on the auxiliary stream ----
     GPTQ_CUDA_TRY(cudaStreamWaitEvent(s2, aux->panel, 0));
@@ -460,6 +484,8 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
   }
   GPTQ_CUDA_TRY(cudaEventRecord(aux->join, s2));
   GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->join, 0));
+  GPTQ_CUDA_TRY(cudaEventRecord(aux->tjoin, s3));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->tjoin, 0));
   {
     dim3 blk(32, 8), grd((unsigned)cdiv(n, 32), (unsigned)cdiv(n, 32));
     write_u_kernel<<<grd, blk, 0, s>>>(w.Xt, n, ldn, U, st);
