@@ -9,7 +9,8 @@
 //     A . B^T  ~  A_hi.B_hi^T + A_hi.B_lo^T + A_lo.B_hi^T
 // (the dropped A_lo.B_lo^T term is below 2^-20 of the product).
 //
-// One CTA computes one 128 x GN tile of C (GN = 256, or 128 for narrow C):
+// One CTA computes one 128 x GN tile of C (GN = 256; 128, 64 or 32 for narrow C,
+// so that a skinny product still spreads over most of the SMs):
 //   warp 0      TMA producer: 32-wide K slices of A_hi, A_lo (128 rows) and
 //               B_hi, B_lo (GN rows), 128-byte swizzled, 2- or 3-stage ring;
 //   warp 1      allocates GN TMEM columns; one thread issues the tcgen05.mma
@@ -40,7 +41,7 @@ constexpr int G_THREADS = 192;
 
 template <int GN>
 struct GemmCfg {
-  static constexpr int STAGES = GN == 256 ? 2 : 3;
+  static constexpr int STAGES = GN == 256 ? 2 : (GN == 128 ? 3 : 4);
   static constexpr int B_TILE = GN * GK * 4;
   static constexpr uint32_t IDESC = tc::idesc_f32acc(2, GM, GN);
 };
@@ -320,6 +321,12 @@ int launch_gemm3(float* C, int ldc, int M, int N, int K, const float* Ahi, const
                  bool store, float* Chi, float* Clo, int ldh) {
   if (M <= 0 || N <= 0 || K <= 0) return GPTQ_OK;
   GemmOut out{C, ldc, store ? 1 : 0, Chi, Clo, ldh};
+  // the widest tile that still gives about one CTA per SM
+  const int64_t tm = (int64_t)cdiv(M, GM);
+  if (N <= 128 && tm * (int64_t)cdiv(N, 64) < 148)
+    return launch_gemm3_t<32>(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, st, s);
+  if (N <= 128 && tm * (int64_t)cdiv(N, 128) < 148)
+    return launch_gemm3_t<64>(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, st, s);
   if (N <= 128) return launch_gemm3_t<128>(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, st, s);
   return launch_gemm3_t<256>(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, st, s);
 }

@@ -163,176 +163,340 @@ __global__ void prep_gather_kernel(const float* H, const float* dfix, const int3
 
 // ---------------------------------------------------------------------------
 // (5) The diagonal block of panel k: Cholesky L_kk and its inverse T = L_kk^-1
-// (rows/columns past nb padded with the identity), in one pass over the 128
-// pivots with one CTA barrier per pivot.
-//   Layout: warp w owns the columns k = w + 8c (c < 16), lane l the rows
-//   i = l + 32r (r < 4); every thread keeps those 64 entries of L and of T in
-//   registers.
-//   Pivot s, phase A (the warp owning column s only): the pivot comes from the
-//   owning lane by a shuffle; the warp scales its column and publishes it
-//   (zero for rows <= s) together with 1 / L_ss.
-//   Barrier.
-//   Phase B (every warp): L[i][k] -= L_is L_ks; T absorbs the previous pivot,
-//   T[i][c] -= L_i,s-1 T_s-1,c; then the lanes holding row s of T scale it by
-//   1 / L_ss (row s is final: T = L^-1 is the forward elimination of the
-//   identity) and publish it for the next pivot.
-//   The published vectors rotate through three buffers, so no second barrier
-//   is needed.  The pivot loop is unrolled over its 16 column-slot blocks, so
-//   every register index is a compile-time constant.
+// (rows/columns past nb padded with the identity), blocked by 32-wide
+// sub-blocks q = 32p, p = 0..3, with the block and its inverse in shared memory:
+//   A  one warp factors the 32 x 32 diagonal sub-block (lane i keeps row i).  At
+//      pivot j the column j of L goes through a shared buffer (kept: it is also
+//      the operand of the triangular solves) and updates the later columns; the
+//      next pivot is derived by its own lane and broadcast before that update, so
+//      its reciprocal square root overlaps it.
+//   B  forward substitution with L_pp, one right-hand side per lane: the rows of
+//      L21 = A21 . L_pp^-T (in place, and into a scratch panel) and the columns
+//      of T_pp = L_pp^-1; next to it Y = L[p, 0:q] . T[0:q, 0:q].
+//   C  A22 -= L21 . L21^T (lower block triangle) and T[p, 0:q] = -T_pp . Y
+//      (L T = I gives L_pp T_pr = -sum_{r<=m<p} L_pm T_mr).
+// The products of B and C run on mma.sync (m16n8k8, TF32) with every operand
+// split into hi + lo and three products (hi.hi + hi.lo + lo.hi), fp32-level
+// accuracy; one warp computes one 16 x 32 tile.
 // ---------------------------------------------------------------------------
-constexpr int POTRF_THREADS = 256;
-constexpr int SLD = PB + 1;
-constexpr size_t POTRF_SMEM = (size_t)PB * SLD * sizeof(float);
+constexpr int DT = 384;            // threads (12 warps)
+constexpr int NWARP = DT / 32;
+constexpr int LDL = 132;           // row stride (floats) of the L and T stages
+constexpr int LDY = 104;           // row stride of Y
+constexpr int LDP = 36;            // row stride of the scratch panel
+constexpr int OFF_T = PB * LDL;
+constexpr int OFF_Y = 2 * PB * LDL;
+constexpr int OFF_P = OFF_Y + 32 * LDY;
+constexpr int OFF_C = OFF_P + (PB - 32) * LDP;
+constexpr int OFF_R = OFF_C + 32 * 32;
+constexpr size_t POTRF_SMEM = (size_t)(OFF_R + PB) * sizeof(float);
 
-__global__ void __launch_bounds__(POTRF_THREADS)
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = __float_as_uint(x) & 0xFFFFE000u;
+  lo = __float_as_uint(x - __uint_as_float(hi));
+}
+
+__device__ __forceinline__ void mma_m16n8k8_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// acc (16 x 32, fragment layout) += A (16 x K) . B (K x 32):
+//   A(r, k) = A[r * lda + k];  B(k, n) = B[k * ldb + n] (NN) or B[n * ldb + k] (NT).
+// acc[s][e] holds the element (g + 8 (e >> 1), 8 s + 2 t + (e & 1)), g = lane / 4, t = lane % 4.
+template <bool NN>
+__device__ __forceinline__ void mma_tile_16x32(const float* A, int lda, const float* B, int ldb, int K, int lane,
+                                               float (&acc)[4][4]) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll 1
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    uint32_t ah[4], al[4];
+    split_tf32(A[g * lda + k0 + t], ah[0], al[0]);
+    split_tf32(A[(g + 8) * lda + k0 + t], ah[1], al[1]);
+    split_tf32(A[g * lda + k0 + t + 4], ah[2], al[2]);
+    split_tf32(A[(g + 8) * lda + k0 + t + 4], ah[3], al[3]);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const float x0 = NN ? B[(k0 + t) * ldb + 8 * s + g] : B[(8 * s + g) * ldb + k0 + t];
+      const float x1 = NN ? B[(k0 + t + 4) * ldb + 8 * s + g] : B[(8 * s + g) * ldb + k0 + t + 4];
+      uint32_t bh0, bl0, bh1, bl1;
+      split_tf32(x0, bh0, bl0);
+      split_tf32(x1, bh1, bl1);
+      mma_m16n8k8_tf32(acc[s], al, bh0, bh1);
+      mma_m16n8k8_tf32(acc[s], ah, bl0, bl1);
+      mma_m16n8k8_tf32(acc[s], ah, bh0, bh1);
+    }
+  }
+}
+
+// 1 / sqrt(d): the hardware estimate refined by one Newton step, y += y (1 - d y^2) / 2.
+__device__ __forceinline__ float rsqrt_refined(float d) {
+  float y = rsqrtf(d);
+  const float e = fmaf(-d * y, y, 1.f);
+  return fmaf(0.5f * y, e, y);
+}
+
+// Phase A: Cholesky of the 32 x 32 sub-block at (q, q) in place.  One warp.
+// Cs[j][k] = L_kj (k > j, else 0) and Rv[j] = 1 / L_jj are kept for phase B.
+// *bad receives the first failing pivot (or -1), *bad_nan its kind.
+__device__ __forceinline__ void chol32(float* Ls, float* Cs, float* Rv, int q, int lane, int* bad, int* bad_nan) {
+  float a[32];
+  float* row = Ls + (q + lane) * LDL + q;
+#pragma unroll
+  for (int k = 0; k < 32; k += 4) {
+    const float4 v = *reinterpret_cast<const float4*>(row + k);
+    a[k] = k <= lane ? v.x : 0.f;
+    a[k + 1] = k + 1 <= lane ? v.y : 0.f;
+    a[k + 2] = k + 2 <= lane ? v.z : 0.f;
+    a[k + 3] = k + 3 <= lane ? v.w : 0.f;
+  }
+  // A failing pivot is replaced by 1, which keeps the arithmetic finite (every
+  // later stage sees the error and skips); lane j keeps pivot j as it came.
+  float mine = 1.f;
+  auto fix = [&](float& d, int j) {
+    if (lane == j) mine = d;
+    d = (d > 0.f && isfinite(d)) ? d : 1.f;
+  };
+  float d = __shfl_sync(0xffffffffu, a[0], 0);
+  fix(d, 0);
+  float y = rsqrt_refined(d);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float lij = lane > j ? a[j] * y : (lane == j ? d * y : 0.f);
+    a[j] = lij;
+    Cs[j * 32 + lane] = lane > j ? lij : 0.f;
+    if (lane == j) Rv[j] = y;
+    // lane j + 1 holds the next pivot once this column's term is removed
+    float dn = j + 1 < 32 ? __shfl_sync(0xffffffffu, fmaf(-lij, lij, a[(j + 1) & 31]), (j + 1) & 31) : 1.f;
+    __syncwarp();
+    float4 c4[8];
+#pragma unroll
+    for (int k4 = (j + 1) & ~3; k4 < 32; k4 += 4) c4[k4 / 4] = *reinterpret_cast<const float4*>(Cs + j * 32 + k4);
+    float yn = 1.f;
+    if (j + 1 < 32) {
+      fix(dn, j + 1);
+      yn = rsqrt_refined(dn);
+    }
+#pragma unroll
+    for (int k4 = (j + 1) & ~3; k4 < 32; k4 += 4) {
+      const float cc[4] = {c4[k4 / 4].x, c4[k4 / 4].y, c4[k4 / 4].z, c4[k4 / 4].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (k4 + u > j) a[k4 + u] = fmaf(-lij, cc[u], a[k4 + u]);
+    }
+    d = dn;
+    y = yn;
+  }
+#pragma unroll
+  for (int k = 0; k < 32; k += 4)
+    *reinterpret_cast<float4*>(row + k) = make_float4(a[k], a[k + 1], a[k + 2], a[k + 3]);
+  const uint32_t badm = __ballot_sync(0xffffffffu, !(mine > 0.f && isfinite(mine)));
+  const uint32_t nanm = __ballot_sync(0xffffffffu, !isfinite(mine));
+  *bad = badm ? __ffs(badm) - 1 : -1;
+  *bad_nan = badm ? (int)((nanm >> (__ffs(badm) - 1)) & 1u) : 0;
+}
+
+// x = L_pp^-1 b for one right-hand side per lane: x_j = b_j / L_jj, then
+// b_k -= L_kj x_j for k > j (column j of L_pp from Cs).  b is overwritten by x.
+__device__ __forceinline__ void fwd_subst32(const float* Cs, const float* Rv, float (&b)[32]) {
+  float4 cur[8], nxt[8];
+  float rcur = Rv[0], rnxt = 1.f;
+#pragma unroll
+  for (int k4 = 0; k4 < 32; k4 += 4) cur[k4 / 4] = *reinterpret_cast<const float4*>(Cs + k4);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    if (j + 1 < 32) {   // the next column, one step ahead
+      rnxt = Rv[(j + 1) & 31];
+#pragma unroll
+      for (int k4 = (j + 2) & ~3; k4 < 32; k4 += 4)
+        nxt[k4 / 4] = *reinterpret_cast<const float4*>(Cs + ((j + 1) & 31) * 32 + k4);
+    }
+    b[j] *= rcur;
+#pragma unroll
+    for (int k4 = (j + 1) & ~3; k4 < 32; k4 += 4) {
+      const float cc[4] = {cur[k4 / 4].x, cur[k4 / 4].y, cur[k4 / 4].z, cur[k4 / 4].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (k4 + u > j) b[k4 + u] = fmaf(-cc[u], b[j], b[k4 + u]);
+    }
+#pragma unroll
+    for (int k4 = 0; k4 < 32; k4 += 4) cur[k4 / 4] = nxt[k4 / 4];
+    rcur = rnxt;
+  }
+}
+
+__global__ void __launch_bounds__(DT, 1)
 potrf_inv_kernel(float* A, int lda, int k0, int nb, int n, float* LIhi, float* LIlo, float* Xt, int ldx,
                  float* XQhi, float* XQlo, int32_t* st) {
-  extern __shared__ float stage[];          // [PB][SLD] input / output staging
-  __shared__ float colL[3][PB];
-  __shared__ float rowT[3][PB];
-  __shared__ float piv[3];
+  extern __shared__ __align__(16) float sm[];
+  float* Ls = sm;
+  float* Ts = sm + OFF_T;
+  float* Ys = sm + OFF_Y;
+  float* Ps = sm + OFF_P;
+  float* Cs = sm + OFF_C;
+  float* Rv = sm + OFF_R;
   __shared__ int bad;
   if (has_error(st)) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t4 = lane & 3;
   if (tid == 0) bad = 0;
 
-  // coalesced load of the lower triangle (identity past nb)
-  for (int idx = tid; idx < PB * PB; idx += POTRF_THREADS * 8) {
-    float v[8];
+  // the lower triangle (identity past nb), 16-byte pieces; T starts at zero
+  for (int idx = tid; idx < PB * PB / 4; idx += DT) {
+    const int r = idx / (PB / 4), c = 4 * (idx % (PB / 4));
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < nb && c <= r) v = *reinterpret_cast<const float4*>(A + (int64_t)(k0 + r) * lda + k0 + c);
+    float e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int e = idx + u * POTRF_THREADS;
-      const int r = e / PB, c = e % PB;
-      v[u] = (e < PB * PB && r < nb && c <= r) ? A[(int64_t)(k0 + r) * lda + k0 + c] : 0.f;
+    for (int u = 0; u < 4; ++u) {
+      if (c + u > r) e[u] = 0.f;
+      if (r >= nb && r == c + u) e[u] = 1.f;
     }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int e = idx + u * POTRF_THREADS;
-      const int r = e / PB, c = e % PB;
-      if (e < PB * PB) stage[r * SLD + c] = (r >= nb && r == c) ? 1.f : v[u];
-    }
+    *reinterpret_cast<float4*>(Ls + r * LDL + c) = make_float4(e[0], e[1], e[2], e[3]);
+    *reinterpret_cast<float4*>(Ts + r * LDL + c) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  __syncthreads();
-  float l[4][16], t[4][16];
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const int i = lane + 32 * r, k = warp + 8 * c;
-      l[r][c] = k <= i ? stage[i * SLD + k] : 0.f;
-      t[r][c] = i == k ? 1.f : 0.f;
-    }
   __syncthreads();
   GPTQ_PHASE_MARK(0);
 
-#pragma unroll
-  for (int C = 0; C < 16; ++C) {
-    const int R = C / 4;                       // row slot of the pivots of this block
 #pragma unroll 1
-    for (int ws = 0; ws < 8; ++ws) {
-      const int s = 8 * C + ws;
-      const int buf = s % 3, prev = (s + 2) % 3;
-      // ---- phase A: the warp owning column s ----
-      if (warp == ws) {
-        float d = __shfl_sync(0xffffffffu, l[R][C], 8 * (C % 4) + ws);
-        const bool badp = !(d > 0.f) || !isfinite(d);
-        if (badp) {
-          if (lane == 0 && !bad) {
-            bad = 1;
-            set_error(st, isfinite(d) ? GPTQ_ERR_NOT_SPD : GPTQ_ERR_NONFINITE, n - 1 - (k0 + s), STAGE_POTRF);
-          }
-          d = 1.f;   // keep the arithmetic finite; every later stage sees the error and skips
-        }
-        const float sq = sqrtf(d);
-        const float rinv = __frcp_rn(sq);
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int i = lane + 32 * r;
-          float v = l[r][C];
-          if (i > s) v *= rinv;
-          else if (i == s) v = sq;
-          if (i >= s) l[r][C] = v;
-          colL[buf][i] = i > s ? v : 0.f;
-        }
-        if (lane == 0) piv[buf] = rinv;
+  for (int p = 0; p < 4; ++p) {
+    const int q = 32 * p;
+    const int R = PB - q - 32;          // rows below the sub-block
+    // ---- A ----
+    if (warp == 0) {
+      int bj, bn;
+      chol32(Ls, Cs, Rv + q, q, lane, &bj, &bn);
+      if (bj >= 0 && lane == 0 && !bad) {
+        bad = 1;
+        set_error(st, bn ? GPTQ_ERR_NONFINITE : GPTQ_ERR_NOT_SPD, n - 1 - (k0 + q + bj), STAGE_POTRF);
       }
-      __syncthreads();
-      // ---- phase B: every warp ----
-      {
-        float li[4];
+    }
+    __syncthreads();
+    GPTQ_PHASE_MARK(1 + 3 * p);
+    // ---- B ----
+    const int wl = R / 32;              // warps on the rows of L21
+    if (warp < wl) {
+      const int i = q + 32 + 32 * warp + lane;
+      float* row = Ls + i * LDL + q;
+      float b[32];
 #pragma unroll
-        for (int r = R; r < 4; ++r) li[r] = colL[buf][lane + 32 * r];
+      for (int k = 0; k < 32; k += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(row + k);
+        b[k] = v.x; b[k + 1] = v.y; b[k + 2] = v.z; b[k + 3] = v.w;
+      }
+      fwd_subst32(Cs, Rv + q, b);
+      float* prow = Ps + (i - q - 32) * LDP;
 #pragma unroll
-        for (int c = C; c < 16; ++c) {
-          const float lk = colL[buf][warp + 8 * c];
+      for (int k = 0; k < 32; k += 4) {
+        const float4 v = make_float4(b[k], b[k + 1], b[k + 2], b[k + 3]);
+        *reinterpret_cast<float4*>(row + k) = v;
+        *reinterpret_cast<float4*>(prow + k) = v;
+      }
+    } else if (warp == wl) {
+      float b[32];
 #pragma unroll
-          for (int r = R; r < 4; ++r) l[r][c] = fmaf(-li[r], lk, l[r][c]);
+      for (int k = 0; k < 32; ++k) b[k] = k == lane ? 1.f : 0.f;
+      fwd_subst32(Cs, Rv + q, b);
+#pragma unroll
+      for (int k = 0; k < 32; ++k) Ts[(q + k) * LDL + q + lane] = b[k];
+    } else if (warp - wl - 1 < 2 * p) {
+      // Y rows a0..a0+15, columns 32 ch..: T[m][c] = 0 for m < 32 ch
+      const int u = warp - wl - 1;
+      const int a0 = 16 * (u & 1), ch = u >> 1;
+      float acc[4][4] = {};
+      mma_tile_16x32<true>(Ls + (q + a0) * LDL + 32 * ch, LDL, Ts + 32 * ch * LDL + 32 * ch, LDL, q - 32 * ch, lane,
+                           acc);
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        float* y0 = Ys + (a0 + g) * LDY + 32 * ch + 8 * s + 2 * t4;
+        *reinterpret_cast<float2*>(y0) = make_float2(acc[s][0], acc[s][1]);
+        *reinterpret_cast<float2*>(y0 + 8 * LDY) = make_float2(acc[s][2], acc[s][3]);
+      }
+    }
+    __syncthreads();
+    GPTQ_PHASE_MARK(2 + 3 * p);
+    // ---- C ----
+    const int rt_n = R / 16;            // trailing row tiles (16 rows), column chunks <= rt / 2
+    int ntc = 0;
+    for (int rt = 0; rt < rt_n; ++rt) ntc += rt / 2 + 1;
+    const int ntasks = ntc + 2 * p;
+#pragma unroll 1
+    for (int task = warp; task < ntasks; task += NWARP) {
+      float acc[4][4] = {};
+      if (task < ntc) {
+        int rt = 0, rem = task;
+        while (rem >= rt / 2 + 1) { rem -= rt / 2 + 1; ++rt; }
+        const int ch = rem;
+        mma_tile_16x32<false>(Ps + 16 * rt * LDP, LDP, Ps + 32 * ch * LDP, LDP, 32, lane, acc);
+        const int i0 = q + 32 + 16 * rt, c0 = q + 32 + 32 * ch;
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          float2* e0 = reinterpret_cast<float2*>(Ls + (i0 + g) * LDL + c0 + 8 * s + 2 * t4);
+          float2* e1 = reinterpret_cast<float2*>(Ls + (i0 + g + 8) * LDL + c0 + 8 * s + 2 * t4);
+          float2 v0 = *e0, v1 = *e1;
+          v0.x -= acc[s][0]; v0.y -= acc[s][1]; v1.x -= acc[s][2]; v1.y -= acc[s][3];
+          *e0 = v0; *e1 = v1;
         }
-        if (s > 0) {
-          // T absorbs pivot s - 1 (rows <= s - 1 have a zero multiplier, columns > s - 1 a zero row entry)
-          float lp[4];
+      } else {
+        // T[q + a][c] = -sum_b T_pp[a][b] Y[b][c]; T_pp[a][b] = 0 for b > a
+        const int u = task - ntc;
+        const int a0 = 16 * (u & 1), ch = u >> 1;
+        mma_tile_16x32<true>(Ts + (q + a0) * LDL + q, LDL, Ys + 32 * ch, LDY, a0 + 16, lane, acc);
 #pragma unroll
-          for (int r = R; r < 4; ++r) lp[r] = colL[prev][lane + 32 * r];
-#pragma unroll
-          for (int c = 0; c <= C; ++c) {
-            const float tk = rowT[prev][warp + 8 * c];
-#pragma unroll
-            for (int r = R; r < 4; ++r) t[r][c] = fmaf(-lp[r], tk, t[r][c]);
-          }
-        }
-        if (lane == 8 * (C % 4) + ws) {
-          // row s of T is final after scaling
-          const float rinv = piv[buf];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            if (c <= C) t[R][c] *= rinv;
-            rowT[buf][warp + 8 * c] = t[R][c];
-          }
+        for (int s = 0; s < 4; ++s) {
+          float* t0 = Ts + (q + a0 + g) * LDL + 32 * ch + 8 * s + 2 * t4;
+          *reinterpret_cast<float2*>(t0) = make_float2(-acc[s][0], -acc[s][1]);
+          *reinterpret_cast<float2*>(t0 + 8 * LDL) = make_float2(-acc[s][2], -acc[s][3]);
         }
       }
     }
+    __syncthreads();
+    GPTQ_PHASE_MARK(3 + 3 * p);
   }
-  __syncthreads();
-  GPTQ_PHASE_MARK(13);
   if (bad) return;
 
-  // outputs, staged through shared memory for coalesced global access
+  // outputs (L_kk itself is not needed later: the trailing steps use L21 and T):
+  // the TF32 split of T, and T transposed into Xt with its split XQ
+  for (int idx = tid; idx < PB * PB / 4; idx += DT) {
+    const int i = idx / (PB / 4), k = 4 * (idx % (PB / 4));
+    const float4 v = *reinterpret_cast<const float4*>(Ts + i * LDL + k);
+    float e[4] = {v.x, v.y, v.z, v.w}, h[4], l[4];
 #pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int c = 0; c < 16; ++c) stage[(lane + 32 * r) * SLD + warp + 8 * c] = l[r][c];
-  __syncthreads();
-  for (int idx = tid; idx < PB * PB; idx += POTRF_THREADS) {
-    const int i = idx / PB, k = idx % PB;
-    if (i < nb && k <= i) A[(int64_t)(k0 + i) * lda + k0 + k] = stage[i * SLD + k];
-  }
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int c = 0; c < 16; ++c) stage[(lane + 32 * r) * SLD + warp + 8 * c] = t[r][c];
-  __syncthreads();
-  for (int idx = tid; idx < PB * PB; idx += POTRF_THREADS) {
-    {
-      // split of L_kk^-1 (B operand rows i, K index k), zero outside nb
-      const int i = idx / PB, k = idx % PB;
-      const float tv = (i < nb && k < nb) ? stage[i * SLD + k] : 0.f;
-      const float th = tf32_hi(tv);
-      LIhi[i * PB + k] = th;
-      LIlo[i * PB + k] = tv - th;
+    for (int u = 0; u < 4; ++u) {
+      if (i >= nb || k + u >= nb) e[u] = 0.f;
+      h[u] = tf32_hi(e[u]);
+      l[u] = e[u] - h[u];
     }
-    {
-      // transposed: Xt[k0 + k][k0 + i] = T[i][k] and its split XQ[k0 + k][i]
-      const int k = idx / PB, i = idx % PB;
-      if (i < nb && k < nb) {
-        const float tv = stage[i * SLD + k];
-        const float th = tf32_hi(tv);
-        Xt[(int64_t)(k0 + k) * ldx + k0 + i] = tv;
-        XQhi[(int64_t)(k0 + k) * PB + i] = th;
-        XQlo[(int64_t)(k0 + k) * PB + i] = tv - th;
-      }
-    }
+    *reinterpret_cast<float4*>(LIhi + i * PB + k) = make_float4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<float4*>(LIlo + i * PB + k) = make_float4(l[0], l[1], l[2], l[3]);
   }
+  for (int idx = tid; idx < PB * PB / 4; idx += DT) {
+    // Xt[k0 + k][k0 + i] = T[i][k] and XQ[k0 + k][i], four consecutive i
+    const int k = idx / (PB / 4), i = 4 * (idx % (PB / 4));
+    if (k >= nb || i >= nb) continue;
+    float e[4], h[4], l[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      e[u] = Ts[(i + u) * LDL + k];
+      h[u] = tf32_hi(e[u]);
+      l[u] = e[u] - h[u];
+    }
+    float* xrow = Xt + (int64_t)(k0 + k) * ldx + k0 + i;
+    if (i + 4 <= nb) {
+      *reinterpret_cast<float4*>(xrow) = make_float4(e[0], e[1], e[2], e[3]);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) if (i + u < nb) xrow[u] = e[u];
+    }
+    // XQ rows are PB wide: the entries past nb are zero (T is the identity there, masked)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) if (i + u >= nb) { h[u] = 0.f; l[u] = 0.f; }
+    *reinterpret_cast<float4*>(XQhi + (int64_t)(k0 + k) * PB + i) = make_float4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<float4*>(XQlo + (int64_t)(k0 + k) * PB + i) = make_float4(l[0], l[1], l[2], l[3]);
+  }
+  GPTQ_PHASE_MARK(13);
 }
 
 // (6) U[i][j] = (L^-1)[n-1-i][n-1-j] = Xt[n-1-j][n-1-i] for j >= i, 0 below the diagonal.
@@ -420,6 +584,7 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
   GPTQ_CUDA_TRY(cudaStreamWaitEvent(s2, aux->fork, 0));
   GPTQ_CUDA_TRY(cudaStreamWaitEvent(s3, aux->fork, 0));
   bool rest_pending = false;
+  int phi_row = 0;   // the row of Phi/Plo that holds the split of this panel's first A21 row
 
   int panel = 0;
   for (int k0 = 0; k0 < n; k0 += PB, ++panel) {
@@ -428,15 +593,19 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
     const int b = panel & 1;
     // the inverse's chain must be done with this buffer's previous use (panel - 2)
     if (panel >= 2) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->done[b], 0));
-    potrf_inv_kernel<<<1, POTRF_THREADS, POTRF_SMEM, s>>>(w.A, ldn, k0, nb, n, w.LIhi[b], w.LIlo[b], w.Xt, ldn,
+    potrf_inv_kernel<<<1, DT, POTRF_SMEM, s>>>(w.A, ldn, k0, nb, n, w.LIhi[b], w.LIlo[b], w.Xt, ldn,
                                                            w.XQhi, w.XQlo, st);
     GPTQ_LAUNCH_CHECK();
     if (rest > 0) {
       float* A21 = w.A + (int64_t)(k0 + nb) * ldn + k0;
-      // L21 = A21 . L_kk^-T (stored in place of A21), with its split
-      rc = launch_split_tf32(A21, rest, nb, ldn, w.Phi, w.Plo, PB, st, s);
+      // L21 = A21 . L_kk^-T (stored in place of A21), with its split.  The split of
+      // A21 comes from the previous panel's update of this block column; the first
+      // panel has none.
+      if (panel == 0) rc = launch_split_tf32(A21, rest, nb, ldn, w.Phi, w.Plo, PB, st, s);
+      const float* Ph = w.Phi + (int64_t)phi_row * PB;
+      const float* Pl = w.Plo + (int64_t)phi_row * PB;
       if (rc == GPTQ_OK)
-        rc = launch_gemm3(A21, ldn, rest, nb, nb, w.Phi, w.Plo, PB, w.LIhi[b], w.LIlo[b], PB, false, st, s, true,
+        rc = launch_gemm3(A21, ldn, rest, nb, nb, Ph, Pl, PB, w.LIhi[b], w.LIlo[b], PB, false, st, s, true,
                           w.Lhi[b], w.Llo[b], PB);
       if (rc != GPTQ_OK) return rc;
     }
@@ -449,8 +618,12 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
       float* A22 = w.A + (int64_t)(k0 + nb) * ldn + (k0 + nb);
       // the trailing stream's previous update overlaps this column block
       if (rest_pending) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->rest, 0));
-      rc = launch_gemm3(A22, ldn, rest, nb2, nb, w.Lhi[b], w.Llo[b], PB, w.Lhi[b], w.Llo[b], PB, false, st, s);
+      // (its result is final: the split goes to Phi/Plo for the next panel, whose
+      // A21 starts nb2 rows down)
+      rc = launch_gemm3(A22, ldn, rest, nb2, nb, w.Lhi[b], w.Llo[b], PB, w.Lhi[b], w.Llo[b], PB, false, st, s, false,
+                        w.Phi, w.Plo, PB);
       if (rc != GPTQ_OK) return rc;
+      phi_row = nb2;
       if (rest > nb2) {
         GPTQ_CUDA_TRY(cudaStreamWaitEvent(s3, aux->panel, 0));
         rc = launch_gemm3(A22 + (int64_t)nb2 * ldn + nb2, ldn, rest - nb2, rest - nb2, nb, w.Lhi[b] + (int64_t)nb2 * PB,
