@@ -164,7 +164,6 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
         tc::tc_fence_after();
         if (warp == 2 && lane == 0) GPTQ_GEMM_MARK(4);
         const int q = warp & 3;
-        const int row = ti * GM + q * 32 + lane;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         // Each warp owns TMEM lanes (rows) [32 q, 32 q + 32).  It stages its 32 x GN
         // slice of C in shared memory (the stage buffers are free once the

@@ -231,19 +231,16 @@ __device__ __forceinline__ void mma_tile_16x32(const float* A, int lda, const fl
   }
 }
 
-// 1 / sqrt(d): the hardware estimate refined by one Newton step, y += y (1 - d y^2) / 2.
-__device__ __forceinline__ float rsqrt_refined(float d) {
-  float y = rsqrtf(d);
-  const float e = fmaf(-d * y, y, 1.f);
-  return fmaf(0.5f * y, e, y);
-}
-
-// Phase A: Cholesky of the 32 x 32 sub-block at (q, q) in place.  One warp.
-// Cs[j][k] = L_kj (k > j, else 0) and Rv[j] = 1 / L_jj are kept for phase B.
+// Phase A: Cholesky of the 32 x 32 sub-block at (q, q).  One warp.  The factor
+// is kept as Cs[j][k] = L_kj (k > j, else 0) and Rv[j] = 1 / L_jj, the operands
+// of phase B; L_jj itself is never needed.  1 / L_jj is the hardware reciprocal
+// square root of the pivot (a few ulp); every later use takes that same value,
+// so the factor stays consistent and the backward error stays at the fp32
+// rounding level.
 // *bad receives the first failing pivot (or -1), *bad_nan its kind.
-__device__ __forceinline__ void chol32(float* Ls, float* Cs, float* Rv, int q, int lane, int* bad, int* bad_nan) {
+__device__ __forceinline__ void chol32(const float* Ls, float* Cs, float* Rv, int q, int lane, int* bad, int* bad_nan) {
   float a[32];
-  float* row = Ls + (q + lane) * LDL + q;
+  const float* row = Ls + (q + lane) * LDL + q;
 #pragma unroll
   for (int k = 0; k < 32; k += 4) {
     const float4 v = *reinterpret_cast<const float4*>(row + k);
@@ -252,19 +249,18 @@ __device__ __forceinline__ void chol32(float* Ls, float* Cs, float* Rv, int q, i
     a[k + 2] = k + 2 <= lane ? v.z : 0.f;
     a[k + 3] = k + 3 <= lane ? v.w : 0.f;
   }
-  // A failing pivot is replaced by 1, which keeps the arithmetic finite (every
+  // A failing pivot gets 1 / L_jj = 1, which keeps the arithmetic finite (every
   // later stage sees the error and skips); lane j keeps pivot j as it came.
   float mine = 1.f;
-  auto fix = [&](float& d, int j) {
+  auto inv_root = [&](float d, int j) {
     if (lane == j) mine = d;
-    d = (d > 0.f && isfinite(d)) ? d : 1.f;
+    const float y = rsqrtf(d);
+    return (d > 0.f && isfinite(d)) ? y : 1.f;
   };
-  float d = __shfl_sync(0xffffffffu, a[0], 0);
-  fix(d, 0);
-  float y = rsqrt_refined(d);
+  float y = inv_root(__shfl_sync(0xffffffffu, a[0], 0), 0);
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
-    const float lij = lane > j ? a[j] * y : (lane == j ? d * y : 0.f);
+    const float lij = lane > j ? a[j] * y : 0.f;
     a[j] = lij;
     Cs[j * 32 + lane] = lane > j ? lij : 0.f;
     if (lane == j) Rv[j] = y;
@@ -274,11 +270,7 @@ __device__ __forceinline__ void chol32(float* Ls, float* Cs, float* Rv, int q, i
     float4 c4[8];
 #pragma unroll
     for (int k4 = (j + 1) & ~3; k4 < 32; k4 += 4) c4[k4 / 4] = *reinterpret_cast<const float4*>(Cs + j * 32 + k4);
-    float yn = 1.f;
-    if (j + 1 < 32) {
-      fix(dn, j + 1);
-      yn = rsqrt_refined(dn);
-    }
+    const float yn = j + 1 < 32 ? inv_root(dn, j + 1) : 1.f;
 #pragma unroll
     for (int k4 = (j + 1) & ~3; k4 < 32; k4 += 4) {
       const float cc[4] = {c4[k4 / 4].x, c4[k4 / 4].y, c4[k4 / 4].z, c4[k4 / 4].w};
@@ -286,12 +278,8 @@ __device__ __forceinline__ void chol32(float* Ls, float* Cs, float* Rv, int q, i
       for (int u = 0; u < 4; ++u)
         if (k4 + u > j) a[k4 + u] = fmaf(-lij, cc[u], a[k4 + u]);
     }
-    d = dn;
     y = yn;
   }
-#pragma unroll
-  for (int k = 0; k < 32; k += 4)
-    *reinterpret_cast<float4*>(row + k) = make_float4(a[k], a[k + 1], a[k + 2], a[k + 3]);
   const uint32_t badm = __ballot_sync(0xffffffffu, !(mine > 0.f && isfinite(mine)));
   const uint32_t nanm = __ballot_sync(0xffffffffu, !isfinite(mine));
   *bad = badm ? __ffs(badm) - 1 : -1;
@@ -328,8 +316,7 @@ __device__ __forceinline__ void fwd_subst32(const float* Cs, const float* Rv, fl
 }
 
 __global__ void __launch_bounds__(DT, 1)
-potrf_inv_kernel(float* A, int lda, int k0, int nb, int n, float* LIhi, float* LIlo, float* Xt, int ldx,
-                 float* XQhi, float* XQlo, int32_t* st) {
+potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, float* LIhi, float* LIlo, int32_t* st) {
   extern __shared__ __align__(16) float sm[];
   float* Ls = sm;
   float* Ts = sm + OFF_T;
@@ -457,8 +444,8 @@ potrf_inv_kernel(float* A, int lda, int k0, int nb, int n, float* LIhi, float* L
   }
   if (bad) return;
 
-  // outputs (L_kk itself is not needed later: the trailing steps use L21 and T):
-  // the TF32 split of T, and T transposed into Xt with its split XQ
+  // output: the TF32 split of T (L_kk itself is not needed later: the trailing
+  // steps use L21 and T; the block of Xt comes from this split, off this chain)
   for (int idx = tid; idx < PB * PB / 4; idx += DT) {
     const int i = idx / (PB / 4), k = 4 * (idx % (PB / 4));
     const float4 v = *reinterpret_cast<const float4*>(Ts + i * LDL + k);
@@ -472,31 +459,30 @@ potrf_inv_kernel(float* A, int lda, int k0, int nb, int n, float* LIhi, float* L
     *reinterpret_cast<float4*>(LIhi + i * PB + k) = make_float4(h[0], h[1], h[2], h[3]);
     *reinterpret_cast<float4*>(LIlo + i * PB + k) = make_float4(l[0], l[1], l[2], l[3]);
   }
-  for (int idx = tid; idx < PB * PB / 4; idx += DT) {
-    // Xt[k0 + k][k0 + i] = T[i][k] and XQ[k0 + k][i], four consecutive i
-    const int k = idx / (PB / 4), i = 4 * (idx % (PB / 4));
-    if (k >= nb || i >= nb) continue;
-    float e[4], h[4], l[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      e[u] = Ts[(i + u) * LDL + k];
-      h[u] = tf32_hi(e[u]);
-      l[u] = e[u] - h[u];
-    }
-    float* xrow = Xt + (int64_t)(k0 + k) * ldx + k0 + i;
-    if (i + 4 <= nb) {
-      *reinterpret_cast<float4*>(xrow) = make_float4(e[0], e[1], e[2], e[3]);
-    } else {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) if (i + u < nb) xrow[u] = e[u];
-    }
-    // XQ rows are PB wide: the entries past nb are zero (T is the identity there, masked)
-#pragma unroll
-    for (int u = 0; u < 4; ++u) if (i + u >= nb) { h[u] = 0.f; l[u] = 0.f; }
-    *reinterpret_cast<float4*>(XQhi + (int64_t)(k0 + k) * PB + i) = make_float4(h[0], h[1], h[2], h[3]);
-    *reinterpret_cast<float4*>(XQlo + (int64_t)(k0 + k) * PB + i) = make_float4(l[0], l[1], l[2], l[3]);
-  }
   GPTQ_PHASE_MARK(13);
+}
+
+// (5b) The diagonal block of Xt = (L^-1)^T and the last nb rows of its split XQ,
+// from the split of T = L_kk^-1: Xt[k0 + k][k0 + i] = T[i][k] (hi + lo is exact),
+// XQ[k0 + k][i] = (hi, lo)(T[i][k]).  32 x 32 tiles through shared memory.
+__global__ void xt_diag_kernel(const float* LIhi, const float* LIlo, int k0, int nb, float* Xt, int ldx, float* XQhi,
+                               float* XQlo, const int32_t* st) {
+  if (has_error(st)) return;
+  __shared__ float th[32][33], tl[32][33];
+  const int i0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  for (int yy = threadIdx.y; yy < 32; yy += 8) {
+    th[yy][threadIdx.x] = LIhi[(i0 + yy) * PB + c0 + threadIdx.x];
+    tl[yy][threadIdx.x] = LIlo[(i0 + yy) * PB + c0 + threadIdx.x];
+  }
+  __syncthreads();
+  for (int yy = threadIdx.y; yy < 32; yy += 8) {
+    const int k = c0 + yy, i = i0 + threadIdx.x;
+    if (k >= nb) continue;
+    const float h = th[threadIdx.x][yy], l = tl[threadIdx.x][yy];
+    if (i < nb) Xt[(int64_t)(k0 + k) * ldx + k0 + i] = h + l;
+    XQhi[(int64_t)(k0 + k) * PB + i] = h;
+    XQlo[(int64_t)(k0 + k) * PB + i] = l;
+  }
 }
 
 // (6) U[i][j] = (L^-1)[n-1-i][n-1-j] = Xt[n-1-j][n-1-i] for j >= i, 0 below the diagonal.
@@ -515,13 +501,17 @@ __global__ void write_u_kernel(const float* Xt, int n, int ldx, float* U, const 
   }
 }
 
-// The blocked inverse's updates and the trailing updates beyond the next panel run
-// on two auxiliary streams next to the factorization: two non-blocking streams and
-// a few events per host thread and device, created on first use and kept for the
-// life of the process.
+// The panel loop runs on three streams: the factorization's critical chain (the
+// diagonal blocks, L21 and the next block column) on a high-priority stream, so
+// that its small launches get SMs ahead of the bulk work; the blocked inverse's
+// updates and the trailing updates beyond the next block column on two
+// low-priority streams.  Streams and events exist once per host thread and
+// device, created on first use and kept for the life of the process.
 struct AuxStream {
+  cudaStream_t c = nullptr;    // the critical chain
   cudaStream_t s = nullptr;    // the inverse's chain
   cudaStream_t t = nullptr;    // the trailing updates beyond the next panel
+  cudaEvent_t cjoin = nullptr;
   cudaEvent_t fork = nullptr, panel = nullptr, join = nullptr, done[2] = {nullptr, nullptr};
   cudaEvent_t rest = nullptr, tjoin = nullptr;
 };
@@ -533,9 +523,13 @@ int aux_stream(AuxStream** out) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GPTQ_ERR_CUDA;
   AuxStream& a = per_dev[dev];
   if (a.s == nullptr) {
-    if (cudaStreamCreateWithFlags(&a.s, cudaStreamNonBlocking) != cudaSuccess) return GPTQ_ERR_CUDA;
-    if (cudaStreamCreateWithFlags(&a.t, cudaStreamNonBlocking) != cudaSuccess) return GPTQ_ERR_CUDA;
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return GPTQ_ERR_CUDA;
+    if (cudaStreamCreateWithPriority(&a.c, cudaStreamNonBlocking, greatest) != cudaSuccess) return GPTQ_ERR_CUDA;
+    if (cudaStreamCreateWithPriority(&a.s, cudaStreamNonBlocking, least) != cudaSuccess) return GPTQ_ERR_CUDA;
+    if (cudaStreamCreateWithPriority(&a.t, cudaStreamNonBlocking, least) != cudaSuccess) return GPTQ_ERR_CUDA;
     const unsigned f = cudaEventDisableTiming;
+    if (cudaEventCreateWithFlags(&a.cjoin, f) != cudaSuccess) return GPTQ_ERR_CUDA;
     if (cudaEventCreateWithFlags(&a.fork, f) != cudaSuccess || cudaEventCreateWithFlags(&a.panel, f) != cudaSuccess ||
         cudaEventCreateWithFlags(&a.join, f) != cudaSuccess || cudaEventCreateWithFlags(&a.done[0], f) != cudaSuccess ||
         cudaEventCreateWithFlags(&a.done[1], f) != cudaSuccess || cudaEventCreateWithFlags(&a.rest, f) != cudaSuccess ||
@@ -546,43 +540,10 @@ int aux_stream(AuxStream** out) {
   return GPTQ_OK;
 }
 
-}  // namespace
-
-size_t prepare_ws_bytes(int n) {
-  const int ldn = ld_of(n);
-  const size_t nn = align_up((size_t)n * ldn * sizeof(float), 256);
-  const size_t panel = align_up((size_t)n * PB * sizeof(float), 256);
-  return 2 * nn + 10 * panel + 4 * align_up((size_t)PB * PB * 4, 256) + align_up((size_t)n * 8, 256) +
-         align_up((size_t)n * 4, 256) + 256;
-}
-
-int launch_prepare(const float* H, const double* hdiag, int n, float damp, int desc_act, float* U,
-                   int32_t* perm, uint8_t* dead, void* ws, int32_t* st, cudaStream_t s) {
-  PrepWs w = carve(ws, n);
-  const int ldn = ld_of(n);
-  prep_diag_kernel<<<(int)cdiv(n, 256), 256, 0, s>>>(H, hdiag, n, desc_act, dead, w.key, w.dfix, st);
-  GPTQ_LAUNCH_CHECK();
-  prep_lambda_kernel<<<1, 1024, 0, s>>>(w.dfix, n, damp, w.scal, st);
-  GPTQ_LAUNCH_CHECK();
-  if (desc_act) prep_rank_kernel<<<(int)cdiv(n, 256), 256, 0, s>>>(w.key, n, perm, st);
-  else prep_identity_kernel<<<(int)cdiv(n, 256), 256, 0, s>>>(perm, n);
-  GPTQ_LAUNCH_CHECK();
-  {
-    dim3 blk(32, 8), grd((unsigned)cdiv(n, 32), (unsigned)cdiv(n, 8));
-    prep_gather_kernel<<<grd, blk, 0, s>>>(H, w.dfix, perm, n, ldn, w.scal, w.A, st);
-    GPTQ_LAUNCH_CHECK();
-  }
-  GPTQ_CUDA_TRY(cudaMemsetAsync(w.Xt, 0, (size_t)n * ldn * sizeof(float), s));
-
-  GPTQ_CUDA_TRY(cudaFuncSetAttribute(potrf_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)POTRF_SMEM));
-  AuxStream* aux = nullptr;
-  int rc = aux_stream(&aux);
-  if (rc != GPTQ_OK) return rc;
-  cudaStream_t s2 = aux->s;
-  cudaStream_t s3 = aux->t;
-  GPTQ_CUDA_TRY(cudaEventRecord(aux->fork, s));
-  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s2, aux->fork, 0));
-  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s3, aux->fork, 0));
+// The blocked factorization and inverse, panel by panel, on the three streams.
+int panel_loop(const PrepWs& w, int n, int ldn, AuxStream* aux, int32_t* st) {
+  cudaStream_t s = aux->c, s2 = aux->s, s3 = aux->t;
+  int rc = GPTQ_OK;
   bool rest_pending = false;
   int phi_row = 0;   // the row of Phi/Plo that holds the split of this panel's first A21 row
 
@@ -593,8 +554,7 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
     const int b = panel & 1;
     // the inverse's chain must be done with this buffer's previous use (panel - 2)
     if (panel >= 2) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->done[b], 0));
-    potrf_inv_kernel<<<1, DT, POTRF_SMEM, s>>>(w.A, ldn, k0, nb, n, w.LIhi[b], w.LIlo[b], w.Xt, ldn,
-                                                           w.XQhi, w.XQlo, st);
+    potrf_inv_kernel<<<1, DT, POTRF_SMEM, s>>>(w.A, ldn, k0, nb, n, w.LIhi[b], w.LIlo[b], st);
     GPTQ_LAUNCH_CHECK();
     if (rest > 0) {
       float* A21 = w.A + (int64_t)(k0 + nb) * ldn + k0;
@@ -638,6 +598,11 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
     }
     // ---- the inverse's block column k, on the auxiliary stream ----
     GPTQ_CUDA_TRY(cudaStreamWaitEvent(s2, aux->panel, 0));
+    {
+      dim3 blk(32, 8), grd(PB / 32, PB / 32);
+      xt_diag_kernel<<<grd, blk, 0, s2>>>(w.LIhi[b], w.LIlo[b], k0, nb, w.Xt, ldn, w.XQhi, w.XQlo, st);
+      GPTQ_LAUNCH_CHECK();
+    }
     if (k0 > 0) {
       // Xt[:k0, k] = Xt[:k0, k] . L_kk^-T, with its split (rows 0..k0 of XQ)
       float* Xk = w.Xt + k0;
@@ -655,10 +620,54 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
     }
     GPTQ_CUDA_TRY(cudaEventRecord(aux->done[b], s2));
   }
-  GPTQ_CUDA_TRY(cudaEventRecord(aux->join, s2));
+  return GPTQ_OK;
+}
+
+}  // namespace
+
+size_t prepare_ws_bytes(int n) {
+  const int ldn = ld_of(n);
+  const size_t nn = align_up((size_t)n * ldn * sizeof(float), 256);
+  const size_t panel = align_up((size_t)n * PB * sizeof(float), 256);
+  return 2 * nn + 10 * panel + 4 * align_up((size_t)PB * PB * 4, 256) + align_up((size_t)n * 8, 256) +
+         align_up((size_t)n * 4, 256) + 256;
+}
+
+int launch_prepare(const float* H, const double* hdiag, int n, float damp, int desc_act, float* U,
+                   int32_t* perm, uint8_t* dead, void* ws, int32_t* st, cudaStream_t s) {
+  PrepWs w = carve(ws, n);
+  const int ldn = ld_of(n);
+  prep_diag_kernel<<<(int)cdiv(n, 256), 256, 0, s>>>(H, hdiag, n, desc_act, dead, w.key, w.dfix, st);
+  GPTQ_LAUNCH_CHECK();
+  prep_lambda_kernel<<<1, 1024, 0, s>>>(w.dfix, n, damp, w.scal, st);
+  GPTQ_LAUNCH_CHECK();
+  if (desc_act) prep_rank_kernel<<<(int)cdiv(n, 256), 256, 0, s>>>(w.key, n, perm, st);
+  else prep_identity_kernel<<<(int)cdiv(n, 256), 256, 0, s>>>(perm, n);
+  GPTQ_LAUNCH_CHECK();
+  {
+    dim3 blk(32, 8), grd((unsigned)cdiv(n, 32), (unsigned)cdiv(n, 8));
+    prep_gather_kernel<<<grd, blk, 0, s>>>(H, w.dfix, perm, n, ldn, w.scal, w.A, st);
+    GPTQ_LAUNCH_CHECK();
+  }
+  GPTQ_CUDA_TRY(cudaMemsetAsync(w.Xt, 0, (size_t)n * ldn * sizeof(float), s));
+
+  GPTQ_CUDA_TRY(cudaFuncSetAttribute(potrf_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)POTRF_SMEM));
+  AuxStream* aux = nullptr;
+  int rc = aux_stream(&aux);
+  if (rc != GPTQ_OK) return rc;
+  GPTQ_CUDA_TRY(cudaEventRecord(aux->fork, s));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(aux->c, aux->fork, 0));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(aux->s, aux->fork, 0));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(aux->t, aux->fork, 0));
+  rc = panel_loop(w, n, ldn, aux, st);
+  // the three streams join the caller's stream, after an error too
+  GPTQ_CUDA_TRY(cudaEventRecord(aux->join, aux->s));
   GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->join, 0));
-  GPTQ_CUDA_TRY(cudaEventRecord(aux->tjoin, s3));
+  GPTQ_CUDA_TRY(cudaEventRecord(aux->tjoin, aux->t));
   GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->tjoin, 0));
+  GPTQ_CUDA_TRY(cudaEventRecord(aux->cjoin, aux->c));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->cjoin, 0));
+  if (rc != GPTQ_OK) return rc;
   {
     dim3 blk(32, 8), grd((unsigned)cdiv(n, 32), (unsigned)cdiv(n, 32));
     write_u_kernel<<<grd, blk, 0, s>>>(w.Xt, n, ldn, U, st);

@@ -122,10 +122,6 @@ __device__ __forceinline__ float code_from_q(float q, QParams p, int bits, bool 
   return fminf(fmaxf(q + p.z, 0.f), (float)((1 << bits) - 1));
 }
 
-__device__ __forceinline__ float quant_code(float w, QParams p, int bits, bool sym) {
-  return code_from_q(rint_div(w, p), p, bits, sym);
-}
-
 // ---------------------------------------------------------------------------
 // K0: Wf[r][k] = W[r][perm[k]] (0 for dead inputs), invperm, g_idx.
 // ---------------------------------------------------------------------------
