@@ -75,7 +75,7 @@ struct GemmMaps {
 };
 
 struct GemmOut {
-  float* C;
+  float* C;         // may be null with store = 1 and a split: only the split is written
   int ldc;
   int store;        // 0: C -= acc, 1: C = acc
   float* Chi;       // optional TF32 split of the result (same row/column origin as C)
@@ -91,9 +91,9 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
              int32_t* st) {
   using Cfg = GemmCfg<GN>;
   constexpr int ST = Cfg::STAGES;
-  extern __shared__ uint8_t smem_raw[];
-  GemmSmem<GN>& S =
-      *reinterpret_cast<GemmSmem<GN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // offset arithmetic on the shared array keeps every access a shared-memory one
+  GemmSmem<GN>& S = *reinterpret_cast<GemmSmem<GN>*>(smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ti = blockIdx.x / tiles_n, tj = blockIdx.x % tiles_n;
   const bool skip_tile = lower && (tj * GN > ti * GM + GM - 1);
@@ -173,7 +173,7 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
         constexpr int P = GN / 4;                                    // pieces per row
         float* tile = reinterpret_cast<float*>(S.bhi[0]) + q * (32 * GN);
         const int row0 = ti * GM + q * 32;
-        const bool vec = (out.ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(out.C) & 15) == 0;
+        const bool vec = out.C != nullptr && (out.ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(out.C) & 15) == 0;
         auto slot = [](int rr, int p) { return rr * GN + ((p ^ (rr & 7)) << 2); };
         if (!out.store) {
           for (int g = lane; g < 32 * P; g += 32) {
@@ -215,7 +215,9 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
           if (r >= M || col >= N) continue;
           const float4 x = *reinterpret_cast<const float4*>(tile + slot(rr, p));
           const float xs[4] = {x.x, x.y, x.z, x.w};
-          if (vec && col + 3 < N) {
+          if (out.C == nullptr) {
+            // split only
+          } else if (vec && col + 3 < N) {
             *reinterpret_cast<float4*>(out.C + (int64_t)r * out.ldc + col) = x;
           } else {
 #pragma unroll

@@ -105,8 +105,9 @@ __device__ __forceinline__ void hess_tile(int t, int TB, int& bi, int& bj) {
 __global__ void __launch_bounds__(HESS_THREADS, 1)
 hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* H, int n, int kblocks, int32_t* st, int stall,
                   uint64_t wait_ns) {
-  extern __shared__ uint8_t smem_raw[];
-  HessSmem& S = *reinterpret_cast<HessSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // offset arithmetic on the shared array keeps every access a shared-memory one
+  HessSmem& S = *reinterpret_cast<HessSmem*>(smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const int TB = (int)cdiv(n, HBN);

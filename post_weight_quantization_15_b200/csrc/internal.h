@@ -27,8 +27,9 @@ int launch_pack(const uint8_t* codes, const int32_t* invperm, int out, int n, in
                 int32_t* qweight, const int32_t* st, cudaStream_t s);
 
 // ---- tensor-core GEMM: C -= A . B^T in 3 x TF32 (operands pre-split) ---------
-// store = false: C -= A.B^T; store = true: C = A.B^T.  Chi/Clo (optional, leading dimension ldh)
-// receive the TF32 split of the result.  lower: only tiles reaching the lower triangle of square C.
+// store = false: C -= A.B^T; store = true: C = A.B^T (C may be null then, if Chi/Clo are given).
+// Chi/Clo (optional, leading dimension ldh) receive the TF32 split of the result.
+// lower: only tiles reaching the lower triangle of square C.
 int launch_gemm3(float* C, int ldc, int M, int N, int K, const float* Ahi, const float* Alo, int lda,
                  const float* Bhi, const float* Blo, int ldb, bool lower, int32_t* st, cudaStream_t s,
                  bool store = false, float* Chi = nullptr, float* Clo = nullptr, int ldh = 0);

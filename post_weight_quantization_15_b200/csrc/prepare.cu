@@ -24,6 +24,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc_common.cuh"
 
 // Phase marks of the diagonal-block kernel; empty in the library build.
 #ifndef GPTQ_PHASE_MARK
@@ -184,12 +185,16 @@ constexpr int NWARP = DT / 32;
 constexpr int LDL = 132;           // row stride (floats) of the L and T stages
 constexpr int LDY = 104;           // row stride of Y
 constexpr int LDP = 36;            // row stride of the scratch panel
-constexpr int OFF_T = PB * LDL;
-constexpr int OFF_Y = 2 * PB * LDL;
+constexpr int OPND_BYTES = 131072;  // the prologue's tensor-core operand tiles (then the T stage)
+constexpr int OFF_T = 0;
+constexpr int OFF_L = OPND_BYTES / 4;
+constexpr int OFF_Y = OFF_L + PB * LDL;
 constexpr int OFF_P = OFF_Y + 32 * LDY;
 constexpr int OFF_C = OFF_P + (PB - 32) * LDP;
 constexpr int OFF_R = OFF_C + 32 * 32;
-constexpr size_t POTRF_SMEM = (size_t)(OFF_R + PB) * sizeof(float);
+static_assert(PB * LDL <= OFF_L, "the T stage fits in the operand area");
+// + 1024: the base is rounded up to the 1024-byte alignment of the swizzled tiles
+constexpr size_t POTRF_SMEM = (size_t)(OFF_R + PB) * sizeof(float) + 1024;
 
 __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
   hi = __float_as_uint(x) & 0xFFFFE000u;
@@ -315,22 +320,44 @@ __device__ __forceinline__ void fwd_subst32(const float* Cs, const float* Rv, fl
   }
 }
 
-__global__ void __launch_bounds__(DT, 1)
-potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, float* LIhi, float* LIlo, int32_t* st) {
-  extern __shared__ __align__(16) float sm[];
-  float* Ls = sm;
-  float* Ts = sm + OFF_T;
-  float* Ys = sm + OFF_Y;
-  float* Ps = sm + OFF_P;
-  float* Cs = sm + OFF_C;
-  float* Rv = sm + OFF_R;
-  __shared__ int bad;
-  if (has_error(st)) return;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t4 = lane & 3;
-  if (tid == 0) bad = 0;
+// Tensor-core operand tiles: 128 rows x 32 fp32 (128-byte rows) in the
+// 128-byte-swizzled K-major layout, 16-byte piece j of row r at r * 128 + ((j ^ (r & 7)) << 4).
+__device__ __forceinline__ void sw_store4(uint8_t* tile, int r, int j, float4 v) {
+  *reinterpret_cast<float4*>(tile + r * 128 + ((j ^ (r & 7)) << 4)) = v;
+}
 
-  // the lower triangle (identity past nb), 16-byte pieces; T starts at zero
+__device__ __forceinline__ void split4(float4 x, float4& h, float4& l) {
+  h = make_float4(tf32_hi(x.x), tf32_hi(x.y), tf32_hi(x.z), tf32_hi(x.w));
+  l = make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w);
+}
+
+// D[tmem] (+)= A . B^T over one 32-wide K chunk in 3 x TF32 (128 x 128, K = 8 steps).
+__device__ __forceinline__ void mma_chunk_3x(uint32_t d, uint32_t ah, uint32_t al, uint32_t bh, uint32_t bl,
+                                             bool accumulate) {
+  constexpr uint32_t IDESC = tc::idesc_f32acc(2, 128, 128);
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    const uint32_t o = kk * 32;
+    tc::mma_tf32(d, tc::sdesc_k_sw128(al + o), tc::sdesc_k_sw128(bh + o), IDESC, accumulate || kk > 0);
+    tc::mma_tf32(d, tc::sdesc_k_sw128(ah + o), tc::sdesc_k_sw128(bl + o), IDESC, true);
+    tc::mma_tf32(d, tc::sdesc_k_sw128(ah + o), tc::sdesc_k_sw128(bh + o), IDESC, true);
+  }
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Lower-triangular 16 x 32 tiles of a 128 x 128 result: row tile rt (16 rows),
+// column chunk ch <= rt / 2 (32 columns); 20 tiles in all.
+__device__ __forceinline__ void lower_tile(int task, int& rt, int& ch) {
+  rt = 0;
+  while (task >= rt / 2 + 1) { task -= rt / 2 + 1; ++rt; }
+  ch = task;
+}
+
+// D (lower triangle of block (k, k), identity past nb) into a stage.
+__device__ __forceinline__ void load_diag_block(const float* A, int lda, int k0, int nb, float* D, int tid) {
   for (int idx = tid; idx < PB * PB / 4; idx += DT) {
     const int r = idx / (PB / 4), c = 4 * (idx % (PB / 4));
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -341,7 +368,164 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, float* LIhi, fl
       if (c + u > r) e[u] = 0.f;
       if (r >= nb && r == c + u) e[u] = 1.f;
     }
-    *reinterpret_cast<float4*>(Ls + r * LDL + c) = make_float4(e[0], e[1], e[2], e[3]);
+    *reinterpret_cast<float4*>(D + r * LDL + c) = make_float4(e[0], e[1], e[2], e[3]);
+  }
+}
+
+// kp < 0: the first panel; D = A[k0.., k0..] is final.
+// kp >= 0: the previous panel (columns kp .. kp + PB) has its inverse T' = Tphi + Tplo,
+// and A[k0.., k0..] lacks only that panel's term.  The kernel first forms
+// L(k, k-1) = A(k, k-1) . T'^T and D -= L(k, k-1) . L(k, k-1)^T itself, on the
+// tensor cores (tcgen05, 3 x TF32, accumulators in TMEM), so that the chain of
+// diagonal blocks is one launch per panel; the other rows of L21 and their
+// updates run off this chain.
+__global__ void __launch_bounds__(DT, 1)
+potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tphi, const float* Tplo, int kp,
+                 float* LIhi, float* LIlo, int32_t* st) {
+  extern __shared__ __align__(1024) uint8_t sm_raw[];
+  // offset arithmetic on the shared array keeps every access a shared-memory one
+  uint8_t* base = sm_raw + ((1024u - (tc::smem_u32(sm_raw) & 1023u)) & 1023u);
+  float* sm = reinterpret_cast<float*>(base);
+  float* Ls = sm + OFF_L;
+  float* Ts = sm + OFF_T;
+  float* Ys = sm + OFF_Y;
+  float* Ps = sm + OFF_P;
+  float* Cs = sm + OFF_C;
+  float* Rv = sm + OFF_R;
+  __shared__ int bad;
+  __shared__ uint64_t pbar[6];   // operand buffers of the two products (2 + 2), accumulator complete, drain
+  __shared__ uint32_t tmem_base;
+  __shared__ int pfail;
+  if (has_error(st)) return;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t4 = lane & 3;
+  if (tid == 0) bad = 0;
+
+  load_diag_block(A, lda, k0, nb, Ls, tid);
+  if (kp >= 0) {
+    if (tid == 0) {
+      for (int i = 0; i < 6; ++i) tc::mbar_init(&pbar[i], 1);
+      tc::fence_barrier_init();
+      pfail = 0;
+    }
+    if (warp == 0) tc::tmem_alloc<256>(&tmem_base);
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tm = tmem_base;
+    volatile int* fail = &pfail;
+    uint32_t done_parity = 0;
+    auto wait_bar = [&](uint64_t* bar, uint32_t parity) {   // thread 0 only
+      if (!*fail && !tc::mbar_wait(bar, parity, fail)) *fail = 1;
+    };
+    // ---- L(k, k-1) = A(k, k-1) . T'^T into TMEM columns [0, 128), by 32-wide K chunks
+    // through two 64 KB operand buffers (A hi, A lo, T' hi, T' lo) ----
+    for (int kc = 0; kc < 4; ++kc) {
+      const int bf = kc & 1;
+      uint8_t* ob = base + bf * 65536;
+      if (kc >= 2) {                         // chunk kc - 2's products read this buffer
+        if (tid == 0) wait_bar(&pbar[bf], 0);
+        __syncthreads();
+      }
+      for (int idx = tid; idx < PB * 8; idx += DT) {
+        const int r = idx >> 3, j = idx & 7, c = kc * 32 + 4 * j;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < nb) a = *reinterpret_cast<const float4*>(A + (int64_t)(k0 + r) * lda + kp + c);
+        float4 ah, al;
+        split4(a, ah, al);
+        sw_store4(ob, r, j, ah);
+        sw_store4(ob + 16384, r, j, al);
+        sw_store4(ob + 32768, r, j, *reinterpret_cast<const float4*>(Tphi + r * PB + c));
+        sw_store4(ob + 49152, r, j, *reinterpret_cast<const float4*>(Tplo + r * PB + c));
+      }
+      fence_proxy_async();
+      __syncthreads();
+      if (tid == 0 && !*fail) {
+        tc::tc_fence_after();
+        const uint32_t o = tc::smem_u32(ob);
+        mma_chunk_3x(tm, o, o + 16384, o + 32768, o + 49152, kc > 0);
+        tc::mma_commit(&pbar[bf]);
+      }
+    }
+    if (tid == 0) {
+      if (!*fail) tc::mma_commit(&pbar[4]);
+      wait_bar(&pbar[4], done_parity);
+      done_parity ^= 1;
+    }
+    __syncthreads();
+    tc::tc_fence_after();
+    // ---- D -= L . L^T into TMEM columns [128, 256): L leaves TMEM by 32-column chunks,
+    // split into one tile pair (hi, lo) that is both operands ----
+    for (int kc = 0; kc < 4; ++kc) {
+      const int bf = kc & 1;
+      uint8_t* lb = base + bf * 32768;
+      if (kc >= 2) {
+        if (tid == 0) wait_bar(&pbar[2 + bf], 0);
+        __syncthreads();
+      }
+      if (warp < 4 && !*fail) {
+        float v[32];
+        tc::tmem_ld_32x32b_x32(tm + ((uint32_t)(warp * 32) << 16) + kc * 32, v);
+        const int r = warp * 32 + lane;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float4 h, l;
+          split4(make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]), h, l);
+          sw_store4(lb, r, j, h);
+          sw_store4(lb + 16384, r, j, l);
+        }
+      }
+      fence_proxy_async();
+      tc::tc_fence_before();
+      __syncthreads();
+      if (tid == 0 && !*fail) {
+        tc::tc_fence_after();
+        const uint32_t o = tc::smem_u32(lb);
+        mma_chunk_3x(tm + 128, o, o + 16384, o, o + 16384, kc > 0);
+        tc::mma_commit(&pbar[2 + bf]);
+      }
+    }
+    if (tid == 0) {
+      if (!*fail) tc::mma_commit(&pbar[4]);
+      wait_bar(&pbar[4], done_parity);
+    }
+    __syncthreads();
+    tc::tc_fence_after();
+    if (warp < 4 && !*fail) {
+      const int r = warp * 32 + lane;
+#pragma unroll 1
+      for (int c0 = 0; c0 < PB; c0 += 32) {
+        float v[32];
+        tc::tmem_ld_32x32b_x32(tm + ((uint32_t)(warp * 32) << 16) + 128 + c0, v);
+        float* d = Ls + r * LDL + c0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float4 x = *reinterpret_cast<float4*>(d + 4 * j);
+          x.x -= v[4 * j]; x.y -= v[4 * j + 1]; x.z -= v[4 * j + 2]; x.w -= v[4 * j + 3];
+          *reinterpret_cast<float4*>(d + 4 * j) = x;
+        }
+      }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (*fail && tid == 0) {
+      // a wait gave up: let whatever was issued finish (bounded) before TMEM goes back
+      tc::mma_commit(&pbar[5]);
+      const uint64_t t0 = tc::globaltimer();
+      while (!tc::mbar_try_wait(&pbar[5], 0) && tc::globaltimer() - t0 < 1000000000ull) {
+      }
+      set_error(st, GPTQ_ERR_TIMEOUT, n - 1 - k0, STAGE_POTRF);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      __syncwarp();
+      tc::tmem_dealloc<256>(tm);
+    }
+    if (*fail) return;
+  }
+  // T starts at zero
+  for (int idx = tid; idx < PB * PB / 4; idx += DT) {
+    const int r = idx / (PB / 4), c = 4 * (idx % (PB / 4));
     *reinterpret_cast<float4*>(Ts + r * LDL + c) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   __syncthreads();
@@ -501,19 +685,22 @@ __global__ void write_u_kernel(const float* Xt, int n, int ldx, float* U, const 
   }
 }
 
-// The panel loop runs on three streams: the factorization's critical chain (the
-// diagonal blocks, L21 and the next block column) on a high-priority stream, so
-// that its small launches get SMs ahead of the bulk work; the blocked inverse's
-// updates and the trailing updates beyond the next block column on two
-// low-priority streams.  Streams and events exist once per host thread and
-// device, created on first use and kept for the life of the process.
+// The panel loop runs on four streams.  High priority, so that their small
+// launches get SMs ahead of the bulk work: the chain of diagonal blocks (one
+// launch per panel), and the rest of each panel's factorization (all rows of
+// L21, and the update of the next block column below its diagonal block).  Low
+// priority: the trailing updates beyond the next block column, and the blocked
+// inverse.  Streams and events exist once per host thread and device, created
+// on first use and kept for the life of the process.
 struct AuxStream {
-  cudaStream_t c = nullptr;    // the critical chain
-  cudaStream_t s = nullptr;    // the inverse's chain
-  cudaStream_t t = nullptr;    // the trailing updates beyond the next panel
-  cudaEvent_t cjoin = nullptr;
-  cudaEvent_t fork = nullptr, panel = nullptr, join = nullptr, done[2] = {nullptr, nullptr};
-  cudaEvent_t rest = nullptr, tjoin = nullptr;
+  cudaStream_t c = nullptr;    // diagonal blocks
+  cudaStream_t o = nullptr;    // L21 and the next block column
+  cudaStream_t t = nullptr;    // trailing updates
+  cudaStream_t s = nullptr;    // the inverse
+  cudaEvent_t fork = nullptr, join[4] = {};
+  // per panel parity: diagonal block done, L21 split ready, next block column
+  // updated, trailing update done, inverse done with the panel's buffers
+  cudaEvent_t diag[2] = {}, l21[2] = {}, next[2] = {}, trail[2] = {}, done[2] = {};
 };
 
 int aux_stream(AuxStream** out) {
@@ -525,86 +712,95 @@ int aux_stream(AuxStream** out) {
   if (a.s == nullptr) {
     int least = 0, greatest = 0;
     if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return GPTQ_ERR_CUDA;
-    if (cudaStreamCreateWithPriority(&a.c, cudaStreamNonBlocking, greatest) != cudaSuccess) return GPTQ_ERR_CUDA;
-    if (cudaStreamCreateWithPriority(&a.s, cudaStreamNonBlocking, least) != cudaSuccess) return GPTQ_ERR_CUDA;
-    if (cudaStreamCreateWithPriority(&a.t, cudaStreamNonBlocking, least) != cudaSuccess) return GPTQ_ERR_CUDA;
-    const unsigned f = cudaEventDisableTiming;
-    if (cudaEventCreateWithFlags(&a.cjoin, f) != cudaSuccess) return GPTQ_ERR_CUDA;
-    if (cudaEventCreateWithFlags(&a.fork, f) != cudaSuccess || cudaEventCreateWithFlags(&a.panel, f) != cudaSuccess ||
-        cudaEventCreateWithFlags(&a.join, f) != cudaSuccess || cudaEventCreateWithFlags(&a.done[0], f) != cudaSuccess ||
-        cudaEventCreateWithFlags(&a.done[1], f) != cudaSuccess || cudaEventCreateWithFlags(&a.rest, f) != cudaSuccess ||
-        cudaEventCreateWithFlags(&a.tjoin, f) != cudaSuccess)
+    if (cudaStreamCreateWithPriority(&a.c, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&a.o, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&a.t, cudaStreamNonBlocking, least) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&a.s, cudaStreamNonBlocking, least) != cudaSuccess)
       return GPTQ_ERR_CUDA;
+    const unsigned f = cudaEventDisableTiming;
+    cudaEvent_t* evs[] = {&a.fork, &a.join[0], &a.join[1], &a.join[2], &a.join[3], &a.diag[0], &a.diag[1],
+                          &a.l21[0], &a.l21[1], &a.next[0], &a.next[1], &a.trail[0], &a.trail[1], &a.done[0],
+                          &a.done[1]};
+    for (cudaEvent_t* e : evs)
+      if (cudaEventCreateWithFlags(e, f) != cudaSuccess) return GPTQ_ERR_CUDA;
   }
   *out = &a;
   return GPTQ_OK;
 }
 
-// The blocked factorization and inverse, panel by panel, on the three streams.
+// The blocked factorization and inverse, panel by panel.  Panel k (columns k0 ..
+// k0 + nb, buffers of parity b = k & 1):
+//   c  the diagonal block: its last update (the previous panel's term, formed in
+//      the kernel) and its factorization and inverse T_k -> LI[b].
+//      Waits for panel k - 2's next-block-column update and trailing update
+//      (the inputs of block k) and for the inverse's use of LI[b].
+//   o  L21 = A21 . T_k^T for all rows below (split only: Lhi/Llo[b]); then the
+//      next block column below its diagonal block, A(i, k+1) -= L(i, k) L(k+1, k)^T
+//      for i >= k + 2, whose split is the next panel's A21 (Phi/Plo).
+//   t  the trailing update of blocks >= k + 2 (lower triangle).
+//   s  the inverse's block column k (Xt = (L^-1)^T): its diagonal block from T_k,
+//      Xt[:k0, k] = Xt[:k0, k] . T_k^T, then Xt[:k0+nb, later] -= Xt[:, k] . L21^T.
+// Block (k+1, k+1) gets panel k's term in the next diagonal launch, not on o.
 int panel_loop(const PrepWs& w, int n, int ldn, AuxStream* aux, int32_t* st) {
-  cudaStream_t s = aux->c, s2 = aux->s, s3 = aux->t;
+  cudaStream_t c = aux->c, o = aux->o, t = aux->t, s2 = aux->s;
   int rc = GPTQ_OK;
-  bool rest_pending = false;
-  int phi_row = 0;   // the row of Phi/Plo that holds the split of this panel's first A21 row
-
   int panel = 0;
   for (int k0 = 0; k0 < n; k0 += PB, ++panel) {
     const int nb = std::min(PB, n - k0);
     const int rest = n - k0 - nb;
     const int b = panel & 1;
-    // the inverse's chain must be done with this buffer's previous use (panel - 2)
-    if (panel >= 2) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->done[b], 0));
-    potrf_inv_kernel<<<1, DT, POTRF_SMEM, s>>>(w.A, ldn, k0, nb, n, w.LIhi[b], w.LIlo[b], st);
+    // ---- the diagonal block ----
+    if (panel >= 2) {
+      GPTQ_CUDA_TRY(cudaStreamWaitEvent(c, aux->next[b], 0));
+      GPTQ_CUDA_TRY(cudaStreamWaitEvent(c, aux->trail[b], 0));
+      GPTQ_CUDA_TRY(cudaStreamWaitEvent(c, aux->done[b], 0));
+    }
+    potrf_inv_kernel<<<1, DT, POTRF_SMEM, c>>>(w.A, ldn, k0, nb, n, w.LIhi[b ^ 1], w.LIlo[b ^ 1],
+                                               panel > 0 ? k0 - PB : -1, w.LIhi[b], w.LIlo[b], st);
     GPTQ_LAUNCH_CHECK();
+    GPTQ_CUDA_TRY(cudaEventRecord(aux->diag[b], c));
     if (rest > 0) {
-      float* A21 = w.A + (int64_t)(k0 + nb) * ldn + k0;
-      // L21 = A21 . L_kk^-T (stored in place of A21), with its split.  The split of
-      // A21 comes from the previous panel's update of this block column; the first
-      // panel has none.
-      if (panel == 0) rc = launch_split_tf32(A21, rest, nb, ldn, w.Phi, w.Plo, PB, st, s);
-      const float* Ph = w.Phi + (int64_t)phi_row * PB;
-      const float* Pl = w.Plo + (int64_t)phi_row * PB;
+      // ---- L21 and the next block column ----
+      GPTQ_CUDA_TRY(cudaStreamWaitEvent(o, aux->diag[b], 0));
+      if (panel >= 2) {   // Lhi/Llo[b]: panel k - 2's trailing update and inverse are done with them
+        GPTQ_CUDA_TRY(cudaStreamWaitEvent(o, aux->trail[b], 0));
+        GPTQ_CUDA_TRY(cudaStreamWaitEvent(o, aux->done[b], 0));
+      }
+      // the split of A21 comes from the previous panel's update of this block column;
+      // the first panel has none
+      if (panel == 0) rc = launch_split_tf32(w.A + (int64_t)nb * ldn, rest, nb, ldn, w.Phi, w.Plo, PB, st, o);
       if (rc == GPTQ_OK)
-        rc = launch_gemm3(A21, ldn, rest, nb, nb, Ph, Pl, PB, w.LIhi[b], w.LIlo[b], PB, false, st, s, true,
+        rc = launch_gemm3(nullptr, 0, rest, nb, nb, w.Phi, w.Plo, PB, w.LIhi[b], w.LIlo[b], PB, false, st, o, true,
                           w.Lhi[b], w.Llo[b], PB);
       if (rc != GPTQ_OK) return rc;
-    }
-    GPTQ_CUDA_TRY(cudaEventRecord(aux->panel, s));
-    if (rest > 0) {
-      // A22 -= L21 . L21^T.  Look-ahead: the next panel's column block on this
-      // stream (the next diagonal factorization needs only it); the lower tiles
-      // beyond it on the trailing stream, overlapping the next panel's work.
+      GPTQ_CUDA_TRY(cudaEventRecord(aux->l21[b], o));
       const int nb2 = std::min(PB, rest);
-      float* A22 = w.A + (int64_t)(k0 + nb) * ldn + (k0 + nb);
-      // the trailing stream's previous update overlaps this column block
-      if (rest_pending) GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->rest, 0));
-      // (its result is final: the split goes to Phi/Plo for the next panel, whose
-      // A21 starts nb2 rows down)
-      rc = launch_gemm3(A22, ldn, rest, nb2, nb, w.Lhi[b], w.Llo[b], PB, w.Lhi[b], w.Llo[b], PB, false, st, s, false,
-                        w.Phi, w.Plo, PB);
-      if (rc != GPTQ_OK) return rc;
-      phi_row = nb2;
       if (rest > nb2) {
-        GPTQ_CUDA_TRY(cudaStreamWaitEvent(s3, aux->panel, 0));
-        rc = launch_gemm3(A22 + (int64_t)nb2 * ldn + nb2, ldn, rest - nb2, rest - nb2, nb, w.Lhi[b] + (int64_t)nb2 * PB,
-                          w.Llo[b] + (int64_t)nb2 * PB, PB, w.Lhi[b] + (int64_t)nb2 * PB, w.Llo[b] + (int64_t)nb2 * PB,
-                          PB, true, st, s3);
+        // A(i, k+1) for i >= k + 2; panel k - 1's trailing update reached it first
+        if (panel >= 1) GPTQ_CUDA_TRY(cudaStreamWaitEvent(o, aux->trail[b ^ 1], 0));
+        float* Anext = w.A + (int64_t)(k0 + nb + nb2) * ldn + (k0 + nb);
+        rc = launch_gemm3(Anext, ldn, rest - nb2, nb2, nb, w.Lhi[b] + (int64_t)nb2 * PB, w.Llo[b] + (int64_t)nb2 * PB,
+                          PB, w.Lhi[b], w.Llo[b], PB, false, st, o, false, w.Phi, w.Plo, PB);
         if (rc != GPTQ_OK) return rc;
-        GPTQ_CUDA_TRY(cudaEventRecord(aux->rest, s3));
-        rest_pending = true;
-      } else {
-        rest_pending = false;
+        GPTQ_CUDA_TRY(cudaEventRecord(aux->next[b], o));
+        // ---- the trailing update of blocks >= k + 2 ----
+        GPTQ_CUDA_TRY(cudaStreamWaitEvent(t, aux->l21[b], 0));
+        const float* Lh2 = w.Lhi[b] + (int64_t)nb2 * PB;
+        const float* Ll2 = w.Llo[b] + (int64_t)nb2 * PB;
+        rc = launch_gemm3(Anext + nb2, ldn, rest - nb2, rest - nb2, nb, Lh2, Ll2, PB, Lh2, Ll2, PB, true, st, t);
+        if (rc != GPTQ_OK) return rc;
+        GPTQ_CUDA_TRY(cudaEventRecord(aux->trail[b], t));
       }
     }
-    // ---- the inverse's block column k, on the auxiliary stream ----
-    GPTQ_CUDA_TRY(cudaStreamWaitEvent(s2, aux->panel, 0));
+    // ---- the inverse's block column k ----
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(s2, aux->diag[b], 0));
     {
       dim3 blk(32, 8), grd(PB / 32, PB / 32);
       xt_diag_kernel<<<grd, blk, 0, s2>>>(w.LIhi[b], w.LIlo[b], k0, nb, w.Xt, ldn, w.XQhi, w.XQlo, st);
       GPTQ_LAUNCH_CHECK();
     }
     if (k0 > 0) {
-      // Xt[:k0, k] = Xt[:k0, k] . L_kk^-T, with its split (rows 0..k0 of XQ)
+      // Xt[:k0, k] = Xt[:k0, k] . T_k^T, with its split (rows 0..k0 of XQ)
       float* Xk = w.Xt + k0;
       rc = launch_split_tf32(Xk, k0, nb, ldn, w.XPhi, w.XPlo, PB, st, s2);
       if (rc == GPTQ_OK)
@@ -614,6 +810,7 @@ int panel_loop(const PrepWs& w, int n, int ldn, AuxStream* aux, int32_t* st) {
     }
     if (rest > 0) {
       // Xt[:k0+nb, later] -= Xt[:k0+nb, k] . L21^T
+      GPTQ_CUDA_TRY(cudaStreamWaitEvent(s2, aux->l21[b], 0));
       rc = launch_gemm3(w.Xt + (k0 + nb), ldn, k0 + nb, rest, nb, w.XQhi, w.XQlo, PB, w.Lhi[b], w.Llo[b], PB, false,
                         st, s2);
       if (rc != GPTQ_OK) return rc;
@@ -655,18 +852,15 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
   AuxStream* aux = nullptr;
   int rc = aux_stream(&aux);
   if (rc != GPTQ_OK) return rc;
+  cudaStream_t loop_streams[4] = {aux->c, aux->o, aux->t, aux->s};
   GPTQ_CUDA_TRY(cudaEventRecord(aux->fork, s));
-  GPTQ_CUDA_TRY(cudaStreamWaitEvent(aux->c, aux->fork, 0));
-  GPTQ_CUDA_TRY(cudaStreamWaitEvent(aux->s, aux->fork, 0));
-  GPTQ_CUDA_TRY(cudaStreamWaitEvent(aux->t, aux->fork, 0));
+  for (cudaStream_t ls : loop_streams) GPTQ_CUDA_TRY(cudaStreamWaitEvent(ls, aux->fork, 0));
   rc = panel_loop(w, n, ldn, aux, st);
-  // the three streams join the caller's stream, after an error too
-  GPTQ_CUDA_TRY(cudaEventRecord(aux->join, aux->s));
-  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->join, 0));
-  GPTQ_CUDA_TRY(cudaEventRecord(aux->tjoin, aux->t));
-  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->tjoin, 0));
-  GPTQ_CUDA_TRY(cudaEventRecord(aux->cjoin, aux->c));
-  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->cjoin, 0));
+  // the loop's streams join the caller's stream, after an error too
+  for (int i = 0; i < 4; ++i) {
+    GPTQ_CUDA_TRY(cudaEventRecord(aux->join[i], loop_streams[i]));
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, aux->join[i], 0));
+  }
   if (rc != GPTQ_OK) return rc;
   {
     dim3 blk(32, 8), grd((unsigned)cdiv(n, 32), (unsigned)cdiv(n, 32));
