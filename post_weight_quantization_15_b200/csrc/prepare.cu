@@ -162,6 +162,40 @@ __global__ void prep_gather_kernel(const float* H, const float* dfix, const int3
   A[(int64_t)i * ldn + j] = v;
 }
 
+// (4') The same with the identity order, q(i) = n-1-i: row i of A is row n-1-i of
+// H read backwards, so reads and writes are both contiguous.  One block per row.
+__global__ void __launch_bounds__(256) prep_reverse_kernel(const float* H, const float* dfix, int n, int ldn,
+                                                           const double* scal, float* A, int32_t* st) {
+  if (has_error(st)) return;
+  const int i = blockIdx.x;
+  const float* h = H + (int64_t)(n - 1 - i) * n + (n - 1);   // h[-j] = H[n-1-i][n-1-j]
+  float* a = A + (int64_t)i * ldn;
+  const float diag = (float)((double)dfix[n - 1 - i] + scal[1]);
+  bool bad = false;
+  for (int j = 4 * threadIdx.x; j <= i; j += 4 * 256) {
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int jj = j + u;
+      v[u] = jj < i ? h[-jj] : (jj == i ? diag : 0.f);
+      bad = bad || (jj < i && !isfinite(v[u]));
+    }
+    *reinterpret_cast<float4*>(a + j) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+  if (bad) set_error(st, GPTQ_ERR_NONFINITE, n - 1 - i, STAGE_PREP_DIAG);
+}
+
+// (4'') Xt starts at zero right of its 128-wide block diagonal, where the blocked
+// inverse accumulates; its diagonal blocks are written whole and nothing reads
+// below them.
+__global__ void zero_upper_blocks_kernel(float* Xt, int n, int ldn) {
+  const int r = blockIdx.y;
+  const int c0 = (r / PB + 1) * PB;
+  float* row = Xt + (int64_t)r * ldn;
+  for (int c = c0 + 4 * (int)threadIdx.x; c < n; c += 4 * (int)blockDim.x)
+    *reinterpret_cast<float4*>(row + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
 // ---------------------------------------------------------------------------
 // (5) The diagonal block of panel k: Cholesky L_kk and its inverse T = L_kk^-1
 // (rows/columns past nb padded with the identity), blocked by 32-wide
@@ -420,6 +454,24 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tp
     };
     // ---- L(k, k-1) = A(k, k-1) . T'^T into TMEM columns [0, 128), by 32-wide K chunks
     // through two 64 KB operand buffers (A hi, A lo, T' hi, T' lo) ----
+    // each thread moves (up to) PF pieces of each operand per chunk; the next
+    // chunk's loads are in flight while this chunk is stored and multiplied
+    constexpr int PF = (PB * 8 + DT - 1) / DT;
+    float4 pa[PF], ph[PF], pl[PF];
+    auto fetch = [&](int kc) {
+#pragma unroll
+      for (int u = 0; u < PF; ++u) {
+        const int idx = tid + u * DT;
+        const int r = idx >> 3, c = kc * 32 + 4 * (idx & 7);
+        pa[u] = ph[u] = pl[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (idx < PB * 8) {
+          if (r < nb) pa[u] = *reinterpret_cast<const float4*>(A + (int64_t)(k0 + r) * lda + kp + c);
+          ph[u] = *reinterpret_cast<const float4*>(Tphi + r * PB + c);
+          pl[u] = *reinterpret_cast<const float4*>(Tplo + r * PB + c);
+        }
+      }
+    };
+    fetch(0);
     for (int kc = 0; kc < 4; ++kc) {
       const int bf = kc & 1;
       uint8_t* ob = base + bf * 65536;
@@ -427,17 +479,20 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tp
         if (tid == 0) wait_bar(&pbar[bf], 0);
         __syncthreads();
       }
-      for (int idx = tid; idx < PB * 8; idx += DT) {
-        const int r = idx >> 3, j = idx & 7, c = kc * 32 + 4 * j;
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r < nb) a = *reinterpret_cast<const float4*>(A + (int64_t)(k0 + r) * lda + kp + c);
-        float4 ah, al;
-        split4(a, ah, al);
-        sw_store4(ob, r, j, ah);
-        sw_store4(ob + 16384, r, j, al);
-        sw_store4(ob + 32768, r, j, *reinterpret_cast<const float4*>(Tphi + r * PB + c));
-        sw_store4(ob + 49152, r, j, *reinterpret_cast<const float4*>(Tplo + r * PB + c));
+#pragma unroll
+      for (int u = 0; u < PF; ++u) {
+        const int idx = tid + u * DT;
+        if (idx < PB * 8) {
+          const int r = idx >> 3, j = idx & 7;
+          float4 ah, al;
+          split4(pa[u], ah, al);
+          sw_store4(ob, r, j, ah);
+          sw_store4(ob + 16384, r, j, al);
+          sw_store4(ob + 32768, r, j, ph[u]);
+          sw_store4(ob + 49152, r, j, pl[u]);
+        }
       }
+      if (kc + 1 < 4) fetch(kc + 1);
       fence_proxy_async();
       __syncthreads();
       if (tid == 0 && !*fail) {
@@ -670,18 +725,32 @@ __global__ void xt_diag_kernel(const float* LIhi, const float* LIlo, int k0, int
 }
 
 // (6) U[i][j] = (L^-1)[n-1-i][n-1-j] = Xt[n-1-j][n-1-i] for j >= i, 0 below the diagonal.
-__global__ void write_u_kernel(const float* Xt, int n, int ldx, float* U, const int32_t* st) {
+// 64 x 64 tiles through shared memory (64 x 4 threads, 16 entries each); tiles
+// wholly below the diagonal only write zeros.
+__global__ void __launch_bounds__(256) write_u_kernel(const float* Xt, int n, int ldx, float* U,
+                                                      const int32_t* st) {
   if (has_error(st)) return;
-  __shared__ float t[32][33];
-  const int i0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
-  for (int yy = threadIdx.y; yy < 32; yy += 8) {
-    const int j = j0 + yy, i = i0 + threadIdx.x;
-    t[yy][threadIdx.x] = (i < n && j < n && j >= i) ? Xt[(int64_t)(n - 1 - j) * ldx + (n - 1 - i)] : 0.f;
+  __shared__ float t[64][65];
+  const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  if (j0 + 63 < i0) {
+#pragma unroll 4
+    for (int yy = ty; yy < 64; yy += 4) {
+      const int i = i0 + yy, j = j0 + tx;
+      if (i < n && j < n) U[(int64_t)i * n + j] = 0.f;
+    }
+    return;
+  }
+#pragma unroll 4
+  for (int yy = ty; yy < 64; yy += 4) {
+    const int j = j0 + yy, i = i0 + tx;
+    t[yy][tx] = (i < n && j < n && j >= i) ? Xt[(int64_t)(n - 1 - j) * ldx + (n - 1 - i)] : 0.f;
   }
   __syncthreads();
-  for (int yy = threadIdx.y; yy < 32; yy += 8) {
-    const int i = i0 + yy, j = j0 + threadIdx.x;
-    if (i < n && j < n) U[(int64_t)i * n + j] = t[threadIdx.x][yy];
+#pragma unroll 4
+  for (int yy = ty; yy < 64; yy += 4) {
+    const int i = i0 + yy, j = j0 + tx;
+    if (i < n && j < n) U[(int64_t)i * n + j] = t[tx][yy];
   }
 }
 
@@ -841,12 +910,18 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
   if (desc_act) prep_rank_kernel<<<(int)cdiv(n, 256), 256, 0, s>>>(w.key, n, perm, st);
   else prep_identity_kernel<<<(int)cdiv(n, 256), 256, 0, s>>>(perm, n);
   GPTQ_LAUNCH_CHECK();
-  {
+  if (desc_act) {
     dim3 blk(32, 8), grd((unsigned)cdiv(n, 32), (unsigned)cdiv(n, 8));
     prep_gather_kernel<<<grd, blk, 0, s>>>(H, w.dfix, perm, n, ldn, w.scal, w.A, st);
+  } else {
+    prep_reverse_kernel<<<n, 256, 0, s>>>(H, w.dfix, n, ldn, w.scal, w.A, st);
+  }
+  GPTQ_LAUNCH_CHECK();
+  if (n > PB) {
+    // rows above the last block row (which starts at the last multiple of PB below n)
+    zero_upper_blocks_kernel<<<dim3(1, (unsigned)((n - 1) / PB * PB)), 256, 0, s>>>(w.Xt, n, ldn);
     GPTQ_LAUNCH_CHECK();
   }
-  GPTQ_CUDA_TRY(cudaMemsetAsync(w.Xt, 0, (size_t)n * ldn * sizeof(float), s));
 
   GPTQ_CUDA_TRY(cudaFuncSetAttribute(potrf_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)POTRF_SMEM));
   AuxStream* aux = nullptr;
@@ -863,7 +938,7 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
   }
   if (rc != GPTQ_OK) return rc;
   {
-    dim3 blk(32, 8), grd((unsigned)cdiv(n, 32), (unsigned)cdiv(n, 32));
+    dim3 blk(64, 4), grd((unsigned)cdiv(n, 64), (unsigned)cdiv(n, 64));
     write_u_kernel<<<grd, blk, 0, s>>>(w.Xt, n, ldn, U, st);
     GPTQ_LAUNCH_CHECK();
   }
