@@ -69,7 +69,7 @@ __device__ __forceinline__ float to_f16_scale(float s) {
   return fmaxf(__half2float(__float2half_rn(s)), kMin);
 }
 
-struct QParams { float s, z, rs; };   // scale, zero point, fp32 reciprocal of the scale
+struct QParams { float s, z, rs, s24; };   // scale, zero point, fp32 reciprocal of the scale, s . 2^-24
 
 __device__ __forceinline__ QParams params_asym(float lo, float hi, float maxq) {
   lo = fminf(lo, 0.f);
@@ -79,6 +79,7 @@ __device__ __forceinline__ QParams params_asym(float lo, float hi, float maxq) {
   p.s = to_f16_scale(__fdiv_rn(__fsub_rn(hi, lo), maxq));
   p.z = fminf(fmaxf(rintf(__fdiv_rn(-lo, p.s)), 0.f), maxq);
   p.rs = __frcp_rn(p.s);
+  p.s24 = p.s * 5.9604644775390625e-08f;
   return p;
 }
 
@@ -88,30 +89,40 @@ __device__ __forceinline__ QParams params_sym(float amax, int bits) {
   p.s = to_f16_scale(__fdiv_rn(amax, (float)((1 << (bits - 1)) - 1)));
   p.z = (float)(1 << (bits - 1));
   p.rs = __frcp_rn(p.s);
+  p.s24 = p.s * 5.9604644775390625e-08f;
   return p;
 }
 
 // rint(fl(w / s)), fl = IEEE round-to-nearest division, without dividing and
-// without branches (the column loop stays one basic block).
-//   t = w . fl(1/s) is within |w/s| . 2^-22 of w/s, so for |t| < 1024 the decision
-//   is between k = floor(t) and k + 1, i.e. on which side of h = k + 1/2 the
-//   rounded quotient lies.  d = fma(-h, s, w) = RN(w - h.s): h.s is exact (h has
-//   at most 13 significant bits, s is an fp16 value), so the sign of d is the sign
-//   of w/s - h, and d itself is exact whenever w/s is within 1/4 of h (Sterbenz).
-//   The rounded quotient equals h exactly iff |w/s - h| <= ulp(h)/2, i.e.
-//   |d| <= s . ulp(h)/2 (h's last mantissa bit is 0 for |h| < 2^22, so a tie
-//   rounds to h); then rint picks the even one of k, k + 1.
-//   For |t| >= 1024 every code saturates, and rint(t) clamps to the same code.
-__device__ __forceinline__ float rint_div(float w, QParams p) {
-  const float t = w * p.rs;
-  const float k = floorf(t);
-  const float h = k + 0.5f;
+// without branches (the column loop stays one basic block).  With t = w . fl(1/s)
+// and a lower candidate k, the answer is k or k + 1; round_up tells which.
+//   t is within |w/s| . 2^-22 of w/s, so for |t| < 1024 the answer is floor(t) or
+//   floor(t) + 1, i.e. it is decided by the side of h = floor(t) + 1/2 on which the
+//   rounded quotient lies.  d = fma(-h, s, w) = RN(w - h.s): h.s is exact (h has at
+//   most 13 significant bits, s is an fp16 value), so the sign of d is the sign of
+//   w/s - h, and d itself is exact whenever w/s is within 1/4 of h (Sterbenz).  The
+//   rounded quotient equals h exactly iff |w/s - h| <= ulp(h)/2, i.e.
+//   |d| <= s . ulp(h)/2 (h's last mantissa bit is 0 for |h| < 2^22, so a tie rounds
+//   to h); then rint picks the even one of k, k + 1.
+//   The candidate is k = rint(t - 1/2), formed by adding and subtracting 1.5 . 2^23
+//   (no conversion instruction): it is floor(t), except that for an integer t it may
+//   be t - 1; then w/s lies half a unit above h = t - 1/2 and d > 0 picks k + 1 = t,
+//   the right answer again.  The sum's last mantissa bit is the parity of k.
+//   s . ulp(h)/2 = (s . 2^-24) . 2^e(h), 2^e(h) being the exponent bits of h alone.
+//   For |t| >= 1024 both candidates saturate to the same code (codes have at most 8
+//   bits), so the answer does not matter there.
+struct Cand { float k; bool odd; };
+
+__device__ __forceinline__ Cand lower_candidate(float t) {
+  const float y = (t - 0.5f) + 12582912.f;   // rint(t - 1/2) + 1.5 . 2^23
+  return {y - 12582912.f, (__float_as_uint(y) & 1u) != 0u};
+}
+
+__device__ __forceinline__ bool round_up(float w, Cand c, QParams p) {
+  const float h = c.k + 0.5f;
   const float d = fmaf(-h, p.s, w);
-  const float ulp_h = __uint_as_float((__float_as_uint(h) & 0x7F800000u) - (23u << 23));
-  const float thr = p.s * ulp_h * 0.5f;
-  const float k_even = (((int)k) & 1) ? k + 1.f : k;
-  const float r = fabsf(d) <= thr ? k_even : (d > 0.f ? k + 1.f : k);
-  return fabsf(t) < 1024.f ? r : rintf(t);
+  const float thr = p.s24 * __uint_as_float(__float_as_uint(h) & 0x7F800000u);
+  return fabsf(d) <= thr ? c.odd : d > 0.f;
 }
 
 __device__ __forceinline__ float code_from_q(float q, QParams p, int bits, bool sym) {
@@ -191,17 +202,18 @@ __global__ void __launch_bounds__(256) row_params_kernel(const float* Wf, int ou
 template <int TPR>
 struct SweepShape {
   static constexpr int SEG = BLK / TPR;          // columns per lane
-  static constexpr int SEGP = SEG + 4;           // padded segment stride in shared memory
+  // padded segment stride in shared memory (4-column segments are conflict-free as they are)
+  static constexpr int SEGP = SEG >= 8 ? SEG + 4 : SEG;
   static constexpr int LDU = TPR * SEGP;         // padded U row stride
-  static constexpr int THREADS = 128;
+  static constexpr int THREADS = TPR == 32 ? 256 : 128;
   static constexpr int ROWS = THREADS / TPR;     // rows per CTA
   static constexpr int LDE = BLK + 4;            // error row stride (16-byte aligned rows)
   static constexpr size_t SMEM =
       (size_t)BLK * LDU * sizeof(float) + BLK * sizeof(float) + (size_t)ROWS * LDE * sizeof(float);
 };
 
-template <int GS, int TPR>
-__global__ void __launch_bounds__(128)
+template <int GS, int TPR, bool SYM>
+__global__ void __launch_bounds__(SweepShape<TPR>::THREADS)
 sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const float* U, float* Ehi, float* Elo,
              uint8_t* codes_p,
              uint16_t* scales, uint16_t* zeros, const float* rows, float* err_sq, int bits, int sym,
@@ -230,8 +242,9 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
   for (int j = threadIdx.x; j < BLK; j += blockDim.x) {
-    const float d = Us[j * SS::LDU + (j / SEG) * SS::SEGP + (j % SEG)];
-    dinv[j] = (j < bw) ? 1.f / d : 0.f;
+    float* dj = Us + j * SS::LDU + (j / SEG) * SS::SEGP + (j % SEG);
+    dinv[j] = (j < bw) ? 1.f / *dj : 0.f;
+    *dj = 0.f;   // the update by column j then leaves columns <= j alone
   }
   __syncthreads();
   GPTQ_SWEEP_MARK(1);
@@ -251,29 +264,47 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
       w[k] = v.x; w[k + 1] = v.y; w[k + 2] = v.z; w[k + 3] = v.w;
     }
   }
-  const bool symq = sym != 0;
+  constexpr bool symq = SYM;   // a compile-time choice: the column loop has no branch on it
+  GPTQ_SWEEP_MARK(6);
   const float maxq = (float)((1 << bits) - 1);
   QParams p;
-  if (GS == 0) { p.s = rows[rr]; p.z = rows[out + rr]; p.rs = __frcp_rn(p.s); }
-  else { p.s = 1.f; p.z = 0.f; p.rs = 1.f; }
+  if (GS == 0) { p.s = rows[rr]; p.z = rows[out + rr]; p.rs = __frcp_rn(p.s); p.s24 = p.s * 5.9604644775390625e-08f; }
+  else { p.s = 1.f; p.z = 0.f; p.rs = 1.f; p.s24 = 5.9604644775390625e-08f; }
   float esq = 0.f;
   uint32_t cw[SEG / 4];
 #pragma unroll
   for (int k = 0; k < SEG / 4; ++k) cw[k] = 0u;
   const int group_lane0 = lane & ~(TPR - 1);
 
-  // The owner of column j quantizes it from `wq`, a scalar that already holds every
-  // update up to column j - 1: the update by column j - 1 is applied to it with the
-  // owner's own error, so the broadcast of that error (needed by the other lanes)
-  // overlaps the next column's decision instead of preceding it.
-  float wq = 0.f;
+  // Column j's error reaches the lanes' registers one column late: the update by
+  // column j - 1 is applied in step j, after column j's decision, so the broadcast of
+  // that error overlaps the decision instead of preceding it.  The owner of column j
+  // folds the pending term into its value itself (wq), from its own previous error
+  // inside its segment and from the broadcast one at a segment's first column.
+  // Group parameters read every lane's columns, so a group start applies the
+  // pending update first.
+  auto apply = [&](float e, const float* urow) {
+#pragma unroll
+    for (int k = 0; k < SEG; k += 4) {
+      const float4 u = *reinterpret_cast<const float4*>(urow + k);
+      w[k] = fmaf(-e, u.x, w[k]);
+      w[k + 1] = fmaf(-e, u.y, w[k + 1]);
+      w[k + 2] = fmaf(-e, u.z, w[k + 2]);
+      w[k + 3] = fmaf(-e, u.w, w[k + 3]);
+    }
+  };
+  float e_prev = 0.f;   // the pending (broadcast) error of column j - 1
+  float e_mine = 0.f;   // this lane's error of column j - 1 when it owned it
   for (int jb = 0; jb < TPR; ++jb) {
     if (jb * SEG >= bw) break;
     const bool owner = seg == jb;
 #pragma unroll
     for (int jj = 0; jj < SEG; ++jj) {
       const int j = jb * SEG + jj;
+      const float* urow_p = Us + (j > 0 ? j - 1 : 0) * SS::LDU + seg * SS::SEGP;   // U row j - 1
       if (GS > 0 && jj == 0 && ((b0 + j) % (GS > 0 ? GS : 1)) == 0) {
+        apply(e_prev, urow_p);
+        e_prev = 0.f;
         // group [j, j + GS): lanes whose segment lies inside it contribute
         const int g_lo = j, g_hi = j + GS;
         const bool in = seg * SEG >= g_lo && seg * SEG + SEG <= g_hi;
@@ -295,27 +326,35 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
           zeros[(int64_t)g * out + r] = __half_as_ushort(__float2half_rn(p.z));
         }
       }
-      if (jj == 0) wq = w[0];           // a new segment (owner): the array holds every update
-      const float c = code_from_q(rint_div(wq, p), p, bits, symq);
-      const float e_own = (wq - p.s * (c - p.z)) * dinv[j];
-      const float* urow = Us + j * SS::LDU + seg * SS::SEGP;
-      if (jj + 1 < SEG) wq = fmaf(-e_own, urow[jj + 1], w[jj + 1]);   // the owner's next column
-      const float e = __shfl_sync(0xffffffffu, e_own, group_lane0 | jb);
-#pragma unroll
-      for (int k = 0; k < SEG; k += 4) {
-        const float4 u = *reinterpret_cast<const float4*>(urow + k);
-        w[k] = fmaf(-e, u.x, w[k]);
-        w[k + 1] = fmaf(-e, u.y, w[k + 1]);
-        w[k + 2] = fmaf(-e, u.z, w[k + 2]);
-        w[k + 3] = fmaf(-e, u.w, w[k + 3]);
-      }
+      // the owner's column j with every update up to column j - 1 (U[j-1][j] is read by
+      // every lane at the owner's address: one broadcast)
+      const float ep = jj == 0 ? e_prev : e_mine;
+      const float u_pj = Us[(j > 0 ? j - 1 : 0) * SS::LDU + jb * SS::SEGP + jj];
+      const float wq = fmaf(-ep, u_pj, w[jj]);
+      // rint(fl(wq / s)) is k or k + 1 (round_up); both candidates' codes and errors
+      // are formed beside the decision, which then only selects
+      const float t = wq * p.rs;
+      const Cand kc = lower_candidate(t);
+      const float k = kc.k;
+      const float c_lo = code_from_q(k, p, bits, symq), c_hi = code_from_q(k + 1.f, p, bits, symq);
+      const float dj = dinv[j];
+      const float e_lo = (wq - p.s * (c_lo - p.z)) * dj;
+      const float e_hi = (wq - p.s * (c_hi - p.z)) * dj;
+      const bool up = round_up(wq, kc, p);
+      const float c = up ? c_hi : c_lo;
+      const float e_own = up ? e_hi : e_lo;
+      const float e_cur = __shfl_sync(0xffffffffu, e_own, group_lane0 | jb);
+      apply(e_prev, urow_p);            // the lagged update by column j - 1
       if (owner) {
-        w[jj] = e;
-        esq = fmaf(e, e, esq);
+        w[jj] = e_own;
+        esq = fmaf(e_own, e_own, esq);
         cw[jj / 4] |= ((uint32_t)c) << (8 * (jj % 4));
       }
+      e_mine = e_own;
+      e_prev = e_cur;
     }
   }
+  // (the update by the block's last column reaches no column of the block)
   GPTQ_SWEEP_MARK(2);
   if (!live || seg * SEG >= bw) {
     // nothing to store for this lane
@@ -328,10 +367,17 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
       *reinterpret_cast<float4*>(ehi + k) = h;
       *reinterpret_cast<float4*>(elo + k) = make_float4(w[k] - h.x, w[k + 1] - h.y, w[k + 2] - h.z, w[k + 3] - h.w);
     }
+    // this lane's SEG codes (n % 32 == 0 keeps every width aligned)
     uint8_t* crow = codes_p + (int64_t)r * n + b0 + seg * SEG;
+    if constexpr (SEG % 16 == 0) {
 #pragma unroll
-    for (int k = 0; k < SEG; k += 16)
-      *reinterpret_cast<uint4*>(crow + k) = make_uint4(cw[k / 4], cw[k / 4 + 1], cw[k / 4 + 2], cw[k / 4 + 3]);
+      for (int k = 0; k < SEG; k += 16)
+        *reinterpret_cast<uint4*>(crow + k) = make_uint4(cw[k / 4], cw[k / 4 + 1], cw[k / 4 + 2], cw[k / 4 + 3]);
+    } else if constexpr (SEG == 8) {
+      *reinterpret_cast<uint2*>(crow) = make_uint2(cw[0], cw[1]);
+    } else {
+      *reinterpret_cast<uint32_t*>(crow) = cw[0];
+    }
   }
 #pragma unroll
   for (int o = 1; o < TPR; o <<= 1) esq += __shfl_xor_sync(0xffffffffu, esq, o);
@@ -500,17 +546,25 @@ int launch_quantize(const void* W, int w_dtype, int out, int n, const float* U, 
     row_params_kernel<<<out, 256, 0, s>>>(w.Wf, out, n, bits, sym, w.rows, scales, zeros, st);
     GPTQ_LAUNCH_CHECK();
   }
-  // Few rows: 16 lanes per row (more parallelism, less work per lane); many rows: 4
-  // (less redundant work).
-  const bool wide = out < 4096;
-  auto pick = [&](auto tpr_tag) {
+  // Lanes per row: the sweep is a chain of dependent column steps per row, so with few
+  // rows a whole warp per row (more warps per SM to hide the chain's latency), with
+  // many rows 4 (less redundant work per row).
+  const int tpr = out <= 2048 ? 32 : (out < 4096 ? 16 : 4);
+  auto pick_gs = [&](auto tpr_tag, auto sym_tag) {
     constexpr int T = decltype(tpr_tag)::value;
-    return gs == 32 ? sweep_kernel<32, T> : gs == 64 ? sweep_kernel<64, T> : gs == 128 ? sweep_kernel<128, T>
-                                                                                      : sweep_kernel<0, T>;
+    constexpr bool Y = decltype(sym_tag)::value;
+    return gs == 32 ? sweep_kernel<32, T, Y> : gs == 64 ? sweep_kernel<64, T, Y>
+                                             : gs == 128 ? sweep_kernel<128, T, Y> : sweep_kernel<0, T, Y>;
   };
-  auto sweep = wide ? pick(std::integral_constant<int, 16>{}) : pick(std::integral_constant<int, 4>{});
-  const size_t smem = wide ? SweepShape<16>::SMEM : SweepShape<4>::SMEM;
-  const int rows_per_cta = wide ? SweepShape<16>::ROWS : SweepShape<4>::ROWS;
+  auto pick = [&](auto tpr_tag) {
+    return sym ? pick_gs(tpr_tag, std::true_type{}) : pick_gs(tpr_tag, std::false_type{});
+  };
+  auto sweep = tpr == 32 ? pick(std::integral_constant<int, 32>{})
+                         : tpr == 16 ? pick(std::integral_constant<int, 16>{}) : pick(std::integral_constant<int, 4>{});
+  const size_t smem = tpr == 32 ? SweepShape<32>::SMEM : tpr == 16 ? SweepShape<16>::SMEM : SweepShape<4>::SMEM;
+  const int rows_per_cta = tpr == 32 ? SweepShape<32>::ROWS : tpr == 16 ? SweepShape<16>::ROWS : SweepShape<4>::ROWS;
+  const int threads = tpr == 32 ? SweepShape<32>::THREADS : tpr == 16 ? SweepShape<16>::THREADS
+                                                                      : SweepShape<4>::THREADS;
   GPTQ_CUDA_TRY(cudaFuncSetAttribute(sweep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   // Two-level lazy batches: blocks of 128 columns inside super-blocks of 512.  A
   // block's sweep also updates the rest of its super-block; the columns after a
@@ -519,7 +573,7 @@ int launch_quantize(const void* W, int w_dtype, int out, int n, const float* U, 
     const int se = std::min(n, s0 + SBK);
     for (int b0 = s0; b0 < se; b0 += BLK) {
       const int bw = std::min(BLK, n - b0);
-      sweep<<<(unsigned)cdiv(out, rows_per_cta), 128, smem, s>>>(w.Wf, out, n, b0, bw, b0 - s0, se, U, w.Ehi, w.Elo,
+      sweep<<<(unsigned)cdiv(out, rows_per_cta), threads, smem, s>>>(w.Wf, out, n, b0, bw, b0 - s0, se, U, w.Ehi, w.Elo,
                                                                   w.codes_p, scales, zeros, w.rows, err_sq, bits, sym,
                                                                   st);
       GPTQ_LAUNCH_CHECK();
