@@ -36,6 +36,7 @@ namespace gptq {
 namespace {
 
 constexpr int PB = 128;          // panel width
+constexpr int NBUF = 3;          // panels in flight: per-panel buffers and events form a ring
 
 int ld_of(int n) { return (int)align_up((size_t)n, 32); }
 
@@ -43,10 +44,10 @@ struct PrepWs {
   float* A;        // [n, ldn] lower triangle: the reversed, permuted, damped H, then L
   float* Xt;       // [n, ldn] upper triangle: (L^-1)^T
   float* Phi; float* Plo;     // [n, PB] split of the panel A21 before the solve
-  float* Lhi[2]; float* Llo[2];   // [n, PB] split of L21 (two panels in flight)
+  float* Lhi[NBUF]; float* Llo[NBUF];     // [n, PB] split of L21 (a ring of panels in flight)
   float* XPhi; float* XPlo;   // [n, PB] split of Xt[:k0, k] before the solve
   float* XQhi; float* XQlo;   // [n, PB] split of the finished Xt[:, k]
-  float* LIhi[2]; float* LIlo[2]; // [PB, PB] split of L_kk^-1 (two panels in flight)
+  float* LIhi[NBUF]; float* LIlo[NBUF];   // [PB, PB] split of L_kk^-1 (the same ring)
   double* key;     // [n] act-order key
   float* dfix;     // [n] diag(H) with dead inputs set to 1
   double* scal;    // [0] sum of dfix, [1] lambda
@@ -62,13 +63,13 @@ PrepWs carve(void* ws, int n) {
   w.A = reinterpret_cast<float*>(take(nn));
   w.Xt = reinterpret_cast<float*>(take(nn));
   w.Phi = reinterpret_cast<float*>(take(panel));  w.Plo = reinterpret_cast<float*>(take(panel));
-  for (int b = 0; b < 2; ++b) {
+  for (int b = 0; b < NBUF; ++b) {
     w.Lhi[b] = reinterpret_cast<float*>(take(panel));
     w.Llo[b] = reinterpret_cast<float*>(take(panel));
   }
   w.XPhi = reinterpret_cast<float*>(take(panel)); w.XPlo = reinterpret_cast<float*>(take(panel));
   w.XQhi = reinterpret_cast<float*>(take(panel)); w.XQlo = reinterpret_cast<float*>(take(panel));
-  for (int b = 0; b < 2; ++b) {
+  for (int b = 0; b < NBUF; ++b) {
     w.LIhi[b] = reinterpret_cast<float*>(take((size_t)PB * PB * 4));
     w.LIlo[b] = reinterpret_cast<float*>(take((size_t)PB * PB * 4));
   }
@@ -767,9 +768,9 @@ struct AuxStream {
   cudaStream_t t = nullptr;    // trailing updates
   cudaStream_t s = nullptr;    // the inverse
   cudaEvent_t fork = nullptr, join[4] = {};
-  // per panel parity: diagonal block done, L21 split ready, next block column
+  // per panel (ring slot): diagonal block done, L21 split ready, next block column
   // updated, trailing update done, inverse done with the panel's buffers
-  cudaEvent_t diag[2] = {}, l21[2] = {}, next[2] = {}, trail[2] = {}, done[2] = {};
+  cudaEvent_t diag[NBUF] = {}, l21[NBUF] = {}, next[NBUF] = {}, trail[NBUF] = {}, done[NBUF] = {};
 };
 
 int aux_stream(AuxStream** out) {
@@ -787,11 +788,14 @@ int aux_stream(AuxStream** out) {
         cudaStreamCreateWithPriority(&a.s, cudaStreamNonBlocking, least) != cudaSuccess)
       return GPTQ_ERR_CUDA;
     const unsigned f = cudaEventDisableTiming;
-    cudaEvent_t* evs[] = {&a.fork, &a.join[0], &a.join[1], &a.join[2], &a.join[3], &a.diag[0], &a.diag[1],
-                          &a.l21[0], &a.l21[1], &a.next[0], &a.next[1], &a.trail[0], &a.trail[1], &a.done[0],
-                          &a.done[1]};
-    for (cudaEvent_t* e : evs)
-      if (cudaEventCreateWithFlags(e, f) != cudaSuccess) return GPTQ_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&a.fork, f) != cudaSuccess) return GPTQ_ERR_CUDA;
+    for (cudaEvent_t& e : a.join)
+      if (cudaEventCreateWithFlags(&e, f) != cudaSuccess) return GPTQ_ERR_CUDA;
+    for (int b = 0; b < NBUF; ++b) {
+      cudaEvent_t* evs[] = {&a.diag[b], &a.l21[b], &a.next[b], &a.trail[b], &a.done[b]};
+      for (cudaEvent_t* e : evs)
+        if (cudaEventCreateWithFlags(e, f) != cudaSuccess) return GPTQ_ERR_CUDA;
+    }
   }
   *out = &a;
   return GPTQ_OK;
@@ -817,21 +821,23 @@ int panel_loop(const PrepWs& w, int n, int ldn, AuxStream* aux, int32_t* st) {
   for (int k0 = 0; k0 < n; k0 += PB, ++panel) {
     const int nb = std::min(PB, n - k0);
     const int rest = n - k0 - nb;
-    const int b = panel & 1;
+    const int b = panel % NBUF;                       // this panel's ring slot
+    const int b1 = (panel + NBUF - 1) % NBUF;         // panel k - 1's
+    const int b2 = (panel + NBUF - 2) % NBUF;         // panel k - 2's
     // ---- the diagonal block ----
-    if (panel >= 2) {
-      GPTQ_CUDA_TRY(cudaStreamWaitEvent(c, aux->next[b], 0));
-      GPTQ_CUDA_TRY(cudaStreamWaitEvent(c, aux->trail[b], 0));
-      GPTQ_CUDA_TRY(cudaStreamWaitEvent(c, aux->done[b], 0));
+    if (panel >= 2) {   // its inputs: panel k - 2's next-column and trailing updates
+      GPTQ_CUDA_TRY(cudaStreamWaitEvent(c, aux->next[b2], 0));
+      GPTQ_CUDA_TRY(cudaStreamWaitEvent(c, aux->trail[b2], 0));
     }
-    potrf_inv_kernel<<<1, DT, POTRF_SMEM, c>>>(w.A, ldn, k0, nb, n, w.LIhi[b ^ 1], w.LIlo[b ^ 1],
+    if (panel >= NBUF) GPTQ_CUDA_TRY(cudaStreamWaitEvent(c, aux->done[b], 0));   // LI[b] is free again
+    potrf_inv_kernel<<<1, DT, POTRF_SMEM, c>>>(w.A, ldn, k0, nb, n, w.LIhi[b1], w.LIlo[b1],
                                                panel > 0 ? k0 - PB : -1, w.LIhi[b], w.LIlo[b], st);
     GPTQ_LAUNCH_CHECK();
     GPTQ_CUDA_TRY(cudaEventRecord(aux->diag[b], c));
     if (rest > 0) {
       // ---- L21 and the next block column ----
       GPTQ_CUDA_TRY(cudaStreamWaitEvent(o, aux->diag[b], 0));
-      if (panel >= 2) {   // Lhi/Llo[b]: panel k - 2's trailing update and inverse are done with them
+      if (panel >= NBUF) {   // Lhi/Llo[b]: the slot's previous trailing update and inverse are done
         GPTQ_CUDA_TRY(cudaStreamWaitEvent(o, aux->trail[b], 0));
         GPTQ_CUDA_TRY(cudaStreamWaitEvent(o, aux->done[b], 0));
       }
@@ -846,7 +852,7 @@ int panel_loop(const PrepWs& w, int n, int ldn, AuxStream* aux, int32_t* st) {
       const int nb2 = std::min(PB, rest);
       if (rest > nb2) {
         // A(i, k+1) for i >= k + 2; panel k - 1's trailing update reached it first
-        if (panel >= 1) GPTQ_CUDA_TRY(cudaStreamWaitEvent(o, aux->trail[b ^ 1], 0));
+        if (panel >= 1) GPTQ_CUDA_TRY(cudaStreamWaitEvent(o, aux->trail[b1], 0));
         float* Anext = w.A + (int64_t)(k0 + nb + nb2) * ldn + (k0 + nb);
         rc = launch_gemm3(Anext, ldn, rest - nb2, nb2, nb, w.Lhi[b] + (int64_t)nb2 * PB, w.Llo[b] + (int64_t)nb2 * PB,
                           PB, w.Lhi[b], w.Llo[b], PB, false, st, o, false, w.Phi, w.Plo, PB);
@@ -895,8 +901,8 @@ size_t prepare_ws_bytes(int n) {
   const int ldn = ld_of(n);
   const size_t nn = align_up((size_t)n * ldn * sizeof(float), 256);
   const size_t panel = align_up((size_t)n * PB * sizeof(float), 256);
-  return 2 * nn + 10 * panel + 4 * align_up((size_t)PB * PB * 4, 256) + align_up((size_t)n * 8, 256) +
-         align_up((size_t)n * 4, 256) + 256;
+  return 2 * nn + (6 + 2 * NBUF) * panel + 2 * NBUF * align_up((size_t)PB * PB * 4, 256) +
+         align_up((size_t)n * 8, 256) + align_up((size_t)n * 4, 256) + 256;
 }
 
 int launch_prepare(const float* H, const double* hdiag, int n, float damp, int desc_act, float* U,
