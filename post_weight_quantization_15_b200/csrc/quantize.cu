@@ -208,8 +208,9 @@ struct SweepShape {
   static constexpr int THREADS = TPR == 32 ? 256 : 128;
   static constexpr int ROWS = THREADS / TPR;     // rows per CTA
   static constexpr int LDE = BLK + 4;            // error row stride (16-byte aligned rows)
+  // two U stages (the block's U, then the near passes alternating), 1/U_jj, errors
   static constexpr size_t SMEM =
-      (size_t)BLK * LDU * sizeof(float) + BLK * sizeof(float) + (size_t)ROWS * LDE * sizeof(float);
+      2 * (size_t)BLK * LDU * sizeof(float) + BLK * sizeof(float) + (size_t)ROWS * LDE * sizeof(float);
 };
 
 template <int GS, int TPR, bool SYM>
@@ -223,23 +224,33 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
   if (has_error(st)) return;
   GPTQ_SWEEP_MARK(0);
   extern __shared__ float smem[];
-  float* Us = smem;                       // [BLK][LDU]
-  float* dinv = smem + BLK * SS::LDU;     // [BLK] 1 / U_jj
-  // Stage U[b0 + j][b0 + c] (j, c < bw) in 16-byte asynchronous copies, all in
-  // flight together; U is zero below its diagonal, so the lower part arrives zeroed.
-  for (int idx = threadIdx.x; idx < BLK * (BLK / 4); idx += blockDim.x) {
-    const int j = idx / (BLK / 4), c = (idx % (BLK / 4)) * 4;
-    float* dst = Us + j * SS::LDU + (c / SEG) * SS::SEGP + (c % SEG);
-    if (j < bw && c < bw) {
-      const float* src = U + (int64_t)(b0 + j) * n + b0 + c;
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
-                   "l"(src)
-                   : "memory");
-    } else {
-      *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+  float* Us = smem;                       // [BLK][LDU] the block's U; then near passes 1, 3
+  float* Us2 = smem + BLK * SS::LDU;      // [BLK][LDU] near passes 0, 2
+  float* dinv = smem + 2 * BLK * SS::LDU; // [BLK] 1 / U_jj
+  // U[r0 + j][c0 + c] (j < rows_n, c < cols_n, zero elsewhere) into a stage, in
+  // 16-byte asynchronous copies, all in flight together.
+  auto stage = [&](float* buf, int r0, int c0, int rows_n, int cols_n) {
+    for (int idx = threadIdx.x; idx < BLK * (BLK / 4); idx += blockDim.x) {
+      const int j = idx / (BLK / 4), c = (idx % (BLK / 4)) * 4;
+      float* dst = buf + j * SS::LDU + (c / SEG) * SS::SEGP + (c % SEG);
+      if (j < rows_n && c < cols_n) {
+        const float* src = U + (int64_t)(r0 + j) * n + c0 + c;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                     "l"(src)
+                     : "memory");
+      } else {
+        *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
-  }
-  asm volatile("cp.async.wait_all;" ::: "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  // The block's U (zero below its diagonal, so the lower part arrives zeroed); the
+  // first near pass's U rows are fetched behind it and land during the sweep.
+  stage(Us, b0, b0, bw, bw);
+  const bool has_near = b0 + bw < se;
+  if (has_near) stage(Us2, b0, b0 + bw, bw, min(BLK, se - b0 - bw));
+  if (has_near) asm volatile("cp.async.wait_group 1;" ::: "memory");
+  else asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
   for (int j = threadIdx.x; j < BLK; j += blockDim.x) {
     float* dj = Us + j * SS::LDU + (j / SEG) * SS::SEGP + (j % SEG);
@@ -388,51 +399,53 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
   // block's errors, W[r][c] -= sum_j e_j U[b0 + j][c], in fp32 on the CUDA cores,
   // 128 columns at a time with the U rows staged in shared memory.  The columns past
   // the super-block are updated once per super-block by the tensor-core GEMM.
-  if (b0 + bw < se) {
+  if (has_near) {
     float* Es = dinv + BLK;                        // [ROWS][LDE] this block's errors per row
     const int rloc = threadIdx.x / TPR;
 #pragma unroll
     for (int k = 0; k < SEG; ++k) Es[rloc * SS::LDE + seg * SEG + k] = (seg * SEG < bw) ? w[k] : 0.f;
-    for (int c0n = b0 + bw; c0n < se; c0n += BLK) {
+    int pass = 0;
+    for (int c0n = b0 + bw; c0n < se; c0n += BLK, ++pass) {
       const int cwid = min(BLK, se - c0n);
-      __syncthreads();                             // Us is free; Es is complete
-      for (int idx = threadIdx.x; idx < BLK * (BLK / 4); idx += blockDim.x) {
-        const int j = idx / (BLK / 4), c = (idx % (BLK / 4)) * 4;
-        float* dst = Us + j * SS::LDU + (c / SEG) * SS::SEGP + (c % SEG);
-        if (j < bw && c < cwid) {
-          const float* src = U + (int64_t)(b0 + j) * n + c0n + c;
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
-                       "l"(src)
-                       : "memory");
-        } else {
-          *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      }
-      asm volatile("cp.async.wait_all;" ::: "memory");
-      __syncthreads();
+      float* cur = (pass & 1) ? Us : Us2;
+      float* nxt = (pass & 1) ? Us2 : Us;
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      __syncthreads();                             // cur has landed; Es is complete; nxt is free
+      if (c0n + BLK < se) stage(nxt, b0, c0n + BLK, bw, min(BLK, se - c0n - BLK));   // the next pass's rows
       GPTQ_SWEEP_MARK(4);
-      float acc[SEG];
+      // two accumulators (even and odd groups of four rows) halve the dependent
+      // chains; the errors past bw are zero
+      float acc[SEG], acc2[SEG];
 #pragma unroll
-      for (int k = 0; k < SEG; ++k) acc[k] = 0.f;
+      for (int k = 0; k < SEG; ++k) { acc[k] = 0.f; acc2[k] = 0.f; }
       const float* erow = Es + rloc * SS::LDE;
-      // four errors and four U rows per step; the errors past bw are zero
-#pragma unroll 1
-      for (int j = 0; j < bw; j += 4) {
-        const float4 e4 = *reinterpret_cast<const float4*>(erow + j);
-        const float ev[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll 2
+      for (int j = 0; j < bw; j += 8) {
+        const float4 e4a = *reinterpret_cast<const float4*>(erow + j);
+        const float4 e4b = *reinterpret_cast<const float4*>(erow + j + 4);
+        const float ea[4] = {e4a.x, e4a.y, e4a.z, e4a.w};
+        const float eb[4] = {e4b.x, e4b.y, e4b.z, e4b.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const float* urow = Us + (j + q) * SS::LDU + seg * SS::SEGP;
+          const float* ua = cur + (j + q) * SS::LDU + seg * SS::SEGP;
+          const float* ub = cur + (j + 4 + q) * SS::LDU + seg * SS::SEGP;
 #pragma unroll
           for (int k = 0; k < SEG; k += 4) {
-            const float4 u = *reinterpret_cast<const float4*>(urow + k);
-            acc[k] = fmaf(ev[q], u.x, acc[k]);
-            acc[k + 1] = fmaf(ev[q], u.y, acc[k + 1]);
-            acc[k + 2] = fmaf(ev[q], u.z, acc[k + 2]);
-            acc[k + 3] = fmaf(ev[q], u.w, acc[k + 3]);
+            const float4 u = *reinterpret_cast<const float4*>(ua + k);
+            const float4 v = *reinterpret_cast<const float4*>(ub + k);
+            acc[k] = fmaf(ea[q], u.x, acc[k]);
+            acc[k + 1] = fmaf(ea[q], u.y, acc[k + 1]);
+            acc[k + 2] = fmaf(ea[q], u.z, acc[k + 2]);
+            acc[k + 3] = fmaf(ea[q], u.w, acc[k + 3]);
+            acc2[k] = fmaf(eb[q], v.x, acc2[k]);
+            acc2[k + 1] = fmaf(eb[q], v.y, acc2[k + 1]);
+            acc2[k + 2] = fmaf(eb[q], v.z, acc2[k + 2]);
+            acc2[k + 3] = fmaf(eb[q], v.w, acc2[k + 3]);
           }
         }
       }
+#pragma unroll
+      for (int k = 0; k < SEG; ++k) acc[k] += acc2[k];
       if (live && seg * SEG < cwid) {
         float* dst = Wf + (int64_t)r * n + c0n + seg * SEG;
 #pragma unroll
