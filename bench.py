@@ -251,6 +251,29 @@ def run_reference(args):
     return 0
 
 
+# DRAM bytes (read + write) of one hessian_tc_kernel launch on layer-1024x4096, from one ncu
+# capture (profiles/hessian_tc_layer-1024x4096.md), valid while the kernel's sources are the
+# ones that were captured (their SHA-256 below); otherwise the traffic is reported as null.
+HESSIAN_TRAFFIC = {"n": 4096, "tokens": 65536, "bytes": 941680128 + 24512000,
+                   "sha256": {"post_weight_quantization_15_b200/csrc/hessian.cu": "79a19330e3dc3175",
+                              "post_weight_quantization_15_b200/csrc/tc_common.cuh": "7955f242938f18ca"}}
+
+
+def hessian_traffic(n: int, tokens: int):
+    import hashlib
+    if n != HESSIAN_TRAFFIC["n"] or tokens != HESSIAN_TRAFFIC["tokens"]:
+        return None
+    root = os.path.dirname(os.path.abspath(__file__))
+    for rel, digest in HESSIAN_TRAFFIC["sha256"].items():
+        try:
+            with open(os.path.join(root, rel), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest()[:16] != digest:
+                    return None
+        except OSError:
+            return None
+    return HESSIAN_TRAFFIC["bytes"]
+
+
 def config_dict(name, layer, st):
     return {"workload": name, "out": layer.w.out, "in": layer.w.n, "tokens": layer.x.tokens,
             "w_dtype": layer.w.dtype, "bits": st.bits, "group_size": st.group_size, "sym": st.sym,
@@ -364,7 +387,8 @@ def run_ours(args):
     achieved = h_flops / h_s / 1e12
     peak = float(peaks["bf16_tflops"])
     roofline = {"kernel": "hessian (K1)", "bound": "tensor", "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": hessian_traffic(n, N),
+                "traffic_unit": "DRAM bytes read + written per launch (ncu)",
                 "peak_source": f"{peaks['_source']} bf16 burst",
                 "work": f"n(n+1)N = {h_flops:.4g} flop per launch (upper triangle incl. diagonal)"}
 
