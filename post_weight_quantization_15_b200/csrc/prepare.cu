@@ -436,6 +436,26 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tp
   const int g = lane >> 2, t4 = lane & 3;
   if (tid == 0) bad = 0;
 
+  // The prologue's operands move in chunks of 32 columns; each thread moves (up to)
+  // PF pieces of each operand per chunk, and the next chunk's loads are in flight
+  // while a chunk is stored and multiplied.  The first chunk's loads go out before
+  // the diagonal block's, so that the two latencies overlap.
+  constexpr int PF = (PB * 8 + DT - 1) / DT;
+  float4 pa[PF], ph[PF], pl[PF];
+  auto fetch = [&](int kc) {
+#pragma unroll
+    for (int u = 0; u < PF; ++u) {
+      const int idx = tid + u * DT;
+      const int r = idx >> 3, c = kc * 32 + 4 * (idx & 7);
+      pa[u] = ph[u] = pl[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (idx < PB * 8) {
+        if (r < nb) pa[u] = *reinterpret_cast<const float4*>(A + (int64_t)(k0 + r) * lda + kp + c);
+        ph[u] = *reinterpret_cast<const float4*>(Tphi + r * PB + c);
+        pl[u] = *reinterpret_cast<const float4*>(Tplo + r * PB + c);
+      }
+    }
+  };
+  if (kp >= 0) fetch(0);
   load_diag_block(A, lda, k0, nb, Ls, tid);
   if (kp >= 0) {
     if (tid == 0) {
@@ -455,24 +475,6 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tp
     };
     // ---- L(k, k-1) = A(k, k-1) . T'^T into TMEM columns [0, 128), by 32-wide K chunks
     // through two 64 KB operand buffers (A hi, A lo, T' hi, T' lo) ----
-    // each thread moves (up to) PF pieces of each operand per chunk; the next
-    // chunk's loads are in flight while this chunk is stored and multiplied
-    constexpr int PF = (PB * 8 + DT - 1) / DT;
-    float4 pa[PF], ph[PF], pl[PF];
-    auto fetch = [&](int kc) {
-#pragma unroll
-      for (int u = 0; u < PF; ++u) {
-        const int idx = tid + u * DT;
-        const int r = idx >> 3, c = kc * 32 + 4 * (idx & 7);
-        pa[u] = ph[u] = pl[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (idx < PB * 8) {
-          if (r < nb) pa[u] = *reinterpret_cast<const float4*>(A + (int64_t)(k0 + r) * lda + kp + c);
-          ph[u] = *reinterpret_cast<const float4*>(Tphi + r * PB + c);
-          pl[u] = *reinterpret_cast<const float4*>(Tplo + r * PB + c);
-        }
-      }
-    };
-    fetch(0);
     for (int kc = 0; kc < 4; ++kc) {
       const int bf = kc & 1;
       uint8_t* ob = base + bf * 65536;

@@ -215,7 +215,7 @@ struct SweepShape {
 
 template <int GS, int TPR, bool SYM>
 __global__ void __launch_bounds__(SweepShape<TPR>::THREADS)
-sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const float* U, float* Ehi, float* Elo,
+sweep_kernel(float* Wf, int out, int n, int s0, int se, const float* U, float* Ehi, float* Elo,
              uint8_t* codes_p,
              uint16_t* scales, uint16_t* zeros, const float* rows, float* err_sq, int bits, int sym,
              const int32_t* st) {
@@ -224,8 +224,7 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
   if (has_error(st)) return;
   GPTQ_SWEEP_MARK(0);
   extern __shared__ float smem[];
-  float* Us = smem;                       // [BLK][LDU] the block's U; then near passes 1, 3
-  float* Us2 = smem + BLK * SS::LDU;      // [BLK][LDU] near passes 0, 2
+  // two U stages of [BLK][LDU], at smem and smem + BLK * LDU
   float* dinv = smem + 2 * BLK * SS::LDU; // [BLK] 1 / U_jj
   // U[r0 + j][c0 + c] (j < rows_n, c < cols_n, zero elsewhere) into a stage, in
   // 16-byte asynchronous copies, all in flight together.
@@ -244,11 +243,33 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
-  // The block's U (zero below its diagonal, so the lower part arrives zeroed); the
-  // first near pass's U rows are fetched behind it and land during the sweep.
-  stage(Us, b0, b0, bw, bw);
+  const int lane = threadIdx.x & 31;
+  const int seg = lane % TPR;
+  const int r = blockIdx.x * SS::ROWS + threadIdx.x / TPR;
+  const bool live = r < out;
+  const int rr = live ? r : 0;
+  constexpr bool symq = SYM;   // a compile-time choice: the column loop has no branch on it
+  const float maxq = (float)((1 << bits) - 1);
+  QParams p;
+  if (GS == 0) { p.s = rows[rr]; p.z = rows[out + rr]; p.rs = __frcp_rn(p.s); p.s24 = p.s * 5.9604644775390625e-08f; }
+  else { p.s = 1.f; p.z = 0.f; p.rs = 1.f; p.s24 = 5.9604644775390625e-08f; }
+  float esq = 0.f;
+  const int group_lane0 = lane & ~(TPR - 1);
+
+  // The blocks of the super-block [s0, se) one after the other.  A block's U is
+  // staged during the previous block's last near pass (the first block's here); the
+  // block's first near pass is fetched behind it and lands during the sweep.
+  int d = 0;                                        // the stage holding this block's U
+  stage(smem, s0, s0, min(BLK, se - s0), min(BLK, se - s0));
+#pragma unroll 1
+  for (int b0 = s0; b0 < se; b0 += BLK) {
+  const int bw = min(BLK, se - b0);
+  const int eoff = b0 - s0;
   const bool has_near = b0 + bw < se;
-  if (has_near) stage(Us2, b0, b0 + bw, bw, min(BLK, se - b0 - bw));
+  float* Us = smem + d * (BLK * SS::LDU);           // the block's U; then near passes 1, 3
+  float* Uo = smem + (d ^ 1) * (BLK * SS::LDU);     // near passes 0, 2
+  __syncthreads();                                  // the previous block is done with Uo
+  if (has_near) stage(Uo, b0, b0 + bw, bw, min(BLK, se - b0 - bw));
   if (has_near) asm volatile("cp.async.wait_group 1;" ::: "memory");
   else asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
@@ -260,11 +281,6 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
   __syncthreads();
   GPTQ_SWEEP_MARK(1);
 
-  const int lane = threadIdx.x & 31;
-  const int seg = lane % TPR;
-  const int r = blockIdx.x * SS::ROWS + threadIdx.x / TPR;
-  const bool live = r < out;
-  const int rr = live ? r : 0;
   float w[SEG];
   {
     const float* src = Wf + (int64_t)rr * n + b0 + seg * SEG;
@@ -275,17 +291,10 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
       w[k] = v.x; w[k + 1] = v.y; w[k + 2] = v.z; w[k + 3] = v.w;
     }
   }
-  constexpr bool symq = SYM;   // a compile-time choice: the column loop has no branch on it
   GPTQ_SWEEP_MARK(6);
-  const float maxq = (float)((1 << bits) - 1);
-  QParams p;
-  if (GS == 0) { p.s = rows[rr]; p.z = rows[out + rr]; p.rs = __frcp_rn(p.s); p.s24 = p.s * 5.9604644775390625e-08f; }
-  else { p.s = 1.f; p.z = 0.f; p.rs = 1.f; p.s24 = 5.9604644775390625e-08f; }
-  float esq = 0.f;
   uint32_t cw[SEG / 4];
 #pragma unroll
   for (int k = 0; k < SEG / 4; ++k) cw[k] = 0u;
-  const int group_lane0 = lane & ~(TPR - 1);
 
   // Column j's error reaches the lanes' registers one column late: the update by
   // column j - 1 is applied in step j, after column j's decision, so the broadcast of
@@ -390,9 +399,6 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
       *reinterpret_cast<uint32_t*>(crow) = cw[0];
     }
   }
-#pragma unroll
-  for (int o = 1; o < TPR; o <<= 1) esq += __shfl_xor_sync(0xffffffffu, esq, o);
-  if (err_sq && live && seg == 0) err_sq[r] += esq;
   GPTQ_SWEEP_MARK(3);
 
   // Near update: the rest of this super-block, columns [b0 + bw, se), absorbs this
@@ -407,11 +413,18 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
     int pass = 0;
     for (int c0n = b0 + bw; c0n < se; c0n += BLK, ++pass) {
       const int cwid = min(BLK, se - c0n);
-      float* cur = (pass & 1) ? Us : Us2;
-      float* nxt = (pass & 1) ? Us2 : Us;
+      float* cur = (pass & 1) ? Us : Uo;
+      float* nxt = (pass & 1) ? Uo : Us;
       asm volatile("cp.async.wait_group 0;" ::: "memory");
       __syncthreads();                             // cur has landed; Es is complete; nxt is free
-      if (c0n + BLK < se) stage(nxt, b0, c0n + BLK, bw, min(BLK, se - c0n - BLK));   // the next pass's rows
+      if (c0n + BLK < se) {
+        stage(nxt, b0, c0n + BLK, bw, min(BLK, se - c0n - BLK));   // the next pass's rows
+      } else {
+        // the last pass: the next block's own U goes to the other stage
+        const int bn = b0 + BLK, bwn = min(BLK, se - bn);
+        stage(nxt, bn, bn, bwn, bwn);
+        d = (pass & 1) ? d ^ 1 : d;
+      }
       GPTQ_SWEEP_MARK(4);
       // two accumulators (even and odd groups of four rows) halve the dependent
       // chains; the errors past bw are zero
@@ -458,6 +471,10 @@ sweep_kernel(float* Wf, int out, int n, int b0, int bw, int eoff, int se, const 
       GPTQ_SWEEP_MARK(5);
     }
   }
+  }   // the blocks of the super-block
+#pragma unroll
+  for (int o = 1; o < TPR; o <<= 1) esq += __shfl_xor_sync(0xffffffffu, esq, o);
+  if (err_sq && live && seg == 0) err_sq[r] += esq;
 }
 
 // ---------------------------------------------------------------------------
@@ -584,13 +601,9 @@ int launch_quantize(const void* W, int w_dtype, int out, int n, const float* U, 
   // super-block absorb its 512 errors at once on the tensor cores.
   for (int s0 = 0; s0 < n; s0 += SBK) {
     const int se = std::min(n, s0 + SBK);
-    for (int b0 = s0; b0 < se; b0 += BLK) {
-      const int bw = std::min(BLK, n - b0);
-      sweep<<<(unsigned)cdiv(out, rows_per_cta), threads, smem, s>>>(w.Wf, out, n, b0, bw, b0 - s0, se, U, w.Ehi, w.Elo,
-                                                                  w.codes_p, scales, zeros, w.rows, err_sq, bits, sym,
-                                                                  st);
-      GPTQ_LAUNCH_CHECK();
-    }
+    sweep<<<(unsigned)cdiv(out, rows_per_cta), threads, smem, s>>>(w.Wf, out, n, s0, se, U, w.Ehi, w.Elo, w.codes_p,
+                                                                scales, zeros, w.rows, err_sq, bits, sym, st);
+    GPTQ_LAUNCH_CHECK();
     if (se < n) {
       const int kw = se - s0;   // == SBK
       dim3 blk(32, 8), grd((unsigned)cdiv(n - se, 32), (unsigned)(SBK / 32));
