@@ -42,7 +42,7 @@ import scipy.linalg
 import scipy.linalg.lapack
 
 __all__ = [
-    "bf16_bits_to_f64", "hessian", "act_order", "prepare", "Prepared",
+    "bf16_bits_to_f64", "hessian", "act_order", "prepare", "prepare_trailing", "Prepared",
     "group_params", "quantize_codes", "dequant_value", "sweep", "SweepResult",
     "g_idx", "unpermute_codes", "pack", "unpack", "dequantize", "layer_error",
     "rtn", "quantize_layer", "LayerResult", "gptq_layer",
@@ -134,6 +134,42 @@ def prepare(H: np.ndarray, damp_percent: float, desc_act: bool,
     Hinv = 0.5 * (Hinv + Hinv.T)
     U = np.linalg.cholesky(Hinv).T                                       # H_d^-1 = U^T U
     return Prepared(U=U, perm=perm, dead=dead, lam=lam, Hd=Hd)
+
+
+def prepare_trailing(H: np.ndarray, damp_percent: float, desc_act: bool, m: int,
+                     order_key: Optional[np.ndarray] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """The last m rows and columns of U (processing order) and the order, for large n.
+
+    Same steps as ``prepare``; steps 1-3 need only the diagonal of H, and step 4 is
+    taken on the trailing m x m block of the permuted, damped H alone.  Why that
+    block suffices: H_d^-1 = U^T U gives H_d = V V^T with V = U^-1 upper triangular,
+    and for an upper triangular V the trailing block of V V^T is V_22 V_22^T; so
+    V_22 is the same factor of H_d's trailing block, and U_22 = V_22^-1 is the upper
+    factor of that block's inverse, the last m rows and columns of U.
+    """
+    H = np.asarray(H)
+    n = H.shape[0]
+    d = np.diag(H).astype(np.float64).copy()
+    dead = d == 0.0
+    d[dead] = 1.0
+    if desc_act:
+        key = d.copy() if order_key is None else np.asarray(order_key, np.float64).copy()
+        if order_key is not None:
+            key[dead] = 1.0
+        perm = act_order(key)
+    else:
+        perm = np.arange(n, dtype=np.int64)
+    lam = float(damp_percent) * float(np.mean(d))
+    tail = perm[n - m:]
+    Hs = np.array(H[np.ix_(tail, tail)], dtype=np.float64)
+    Hs[np.arange(m), np.arange(m)] = d[tail] + lam
+    L = np.linalg.cholesky(Hs)
+    Linv, info = scipy.linalg.lapack.dtrtri(L, lower=1)
+    if info != 0:
+        raise np.linalg.LinAlgError("triangular inverse failed")
+    Hinv = Linv.T @ Linv
+    Hinv = 0.5 * (Hinv + Hinv.T)
+    return np.linalg.cholesky(Hinv).T, perm
 
 
 # --------------------------------------------------------------------------- #

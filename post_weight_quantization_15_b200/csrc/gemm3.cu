@@ -39,11 +39,21 @@ constexpr int GK = 32;                      // fp32 per 128-byte row
 constexpr int A_TILE = GM * GK * 4;         // 16 KB
 constexpr int G_THREADS = 192;
 
+// K is accumulated in chunks of CHUNK_KB k-blocks (128) for tiles up to 128 wide:
+// the tensor cores' fp32 accumulation is not rounded to nearest and its error grows
+// with the accumulation length, so each chunk starts from zero in one of two TMEM
+// accumulators and the epilogue warps add the finished chunks in fp32 registers
+// (round to nearest) while the next chunk is computed.  256-wide tiles serve
+// K <= 128 only (one chunk).
+constexpr int CHUNK_KB = 4;
+
 template <int GN>
 struct GemmCfg {
   static constexpr int STAGES = GN == 256 ? 2 : (GN == 128 ? 3 : 4);
   static constexpr int B_TILE = GN * GK * 4;
   static constexpr uint32_t IDESC = tc::idesc_f32acc(2, GM, GN);
+  static constexpr bool CHUNKED = GN <= 128;
+  static constexpr uint32_t TMEM_COLS = CHUNKED ? 2 * GN : GN;
 };
 
 template <int GN>
@@ -55,7 +65,8 @@ struct GemmSmem {
   uint8_t alo[ST][A_TILE];
   uint64_t full[ST];
   uint64_t empty[ST];
-  uint64_t acc_full;
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -105,11 +116,11 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
     S.skip = has_error(st) ? 1 : 0;
     S.abort = 0;
     for (int s = 0; s < ST; ++s) { tc::mbar_init(&S.full[s], 1); tc::mbar_init(&S.empty[s], 1); }
-    tc::mbar_init(&S.acc_full, 1);
+    for (int b = 0; b < 2; ++b) { tc::mbar_init(&S.acc_full[b], 1); tc::mbar_init(&S.acc_empty[b], 4); }
     tc::mbar_init(&S.drain, 1);
     tc::fence_barrier_init();
   }
-  if (warp == 1) tc::tmem_alloc<GN>(&S.tmem_base);
+  if (warp == 1) tc::tmem_alloc<Cfg::TMEM_COLS>(&S.tmem_base);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -134,37 +145,70 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
         ++armed[s];
       }
     } else if (warp == 1 && lane == 0) {
-      for (int kb = 0; kb < kblocks; ++kb) {
-        const int s = kb % ST;
-        const uint32_t ph = (uint32_t)(kb / ST) & 1u;
-        if (!tc::mbar_wait(&S.full[s], ph, abort_flag)) break;
+      const int chunk_kb = Cfg::CHUNKED ? CHUNK_KB : kblocks;
+      const int nchunks = (int)cdiv(kblocks, chunk_kb);
+      int kb = 0;
+      for (int c = 0; c < nchunks && !*abort_flag; ++c) {
+        const int buf = Cfg::CHUNKED ? (c & 1) : 0;
+        if (Cfg::CHUNKED && !tc::mbar_wait(&S.acc_empty[buf], ((uint32_t)(c >> 1) & 1u) ^ 1u, abort_flag)) break;
         tc::tc_fence_after();
-        if (kb == 0) GPTQ_GEMM_MARK(2);
-        const uint32_t ah = tc::smem_u32(S.ahi[s]), al = tc::smem_u32(S.alo[s]);
-        const uint32_t bh = tc::smem_u32(S.bhi[s]), bl = tc::smem_u32(S.blo[s]);
+        const uint32_t dacc = taddr + buf * GN;
+        const int kb_end = min(kblocks, (c + 1) * chunk_kb);
+        bool first = true;
+        for (; kb < kb_end; ++kb) {
+          const int s = kb % ST;
+          const uint32_t ph = (uint32_t)(kb / ST) & 1u;
+          if (!tc::mbar_wait(&S.full[s], ph, abort_flag)) break;
+          tc::tc_fence_after();
+          if (kb == 0) GPTQ_GEMM_MARK(2);
+          const uint32_t ah = tc::smem_u32(S.ahi[s]), al = tc::smem_u32(S.alo[s]);
+          const uint32_t bh = tc::smem_u32(S.bhi[s]), bl = tc::smem_u32(S.blo[s]);
 #pragma unroll
-        for (int kk = 0; kk < GK / 8; ++kk) {
-          const uint32_t o = kk * 32;
-          tc::mma_tf32(taddr, tc::sdesc_k_sw128(al + o), tc::sdesc_k_sw128(bh + o), Cfg::IDESC, kb > 0 || kk > 0);
-          tc::mma_tf32(taddr, tc::sdesc_k_sw128(ah + o), tc::sdesc_k_sw128(bl + o), Cfg::IDESC, true);
-          tc::mma_tf32(taddr, tc::sdesc_k_sw128(ah + o), tc::sdesc_k_sw128(bh + o), Cfg::IDESC, true);
+          for (int kk = 0; kk < GK / 8; ++kk) {
+            const uint32_t o = kk * 32;
+            tc::mma_tf32(dacc, tc::sdesc_k_sw128(al + o), tc::sdesc_k_sw128(bh + o), Cfg::IDESC, !first);
+            tc::mma_tf32(dacc, tc::sdesc_k_sw128(ah + o), tc::sdesc_k_sw128(bl + o), Cfg::IDESC, true);
+            tc::mma_tf32(dacc, tc::sdesc_k_sw128(ah + o), tc::sdesc_k_sw128(bh + o), Cfg::IDESC, true);
+            first = false;
+          }
+          tc::mma_commit(&S.empty[s]);
         }
-        tc::mma_commit(&S.empty[s]);
+        if (*abort_flag) break;
+        tc::mma_commit(&S.acc_full[buf]);
       }
       GPTQ_GEMM_MARK(3);
-      if (!*abort_flag) tc::mma_commit(&S.acc_full);
       tc::mma_commit(&S.drain);
       mma_committed = true;
       if (!*abort_flag) drain_wait(&S.drain, 0);
     } else if (warp >= 2) {
-      int ready = 0;
-      if (lane == 0) ready = tc::mbar_wait(&S.acc_full, 0, abort_flag) && !*abort_flag;
-      ready = __shfl_sync(0xffffffffu, ready, 0);
-      if (ready) {
+      const int q = warp & 3;
+      const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+      // chunked: this thread's row of the tile (TMEM lane) in registers
+      float acc[Cfg::CHUNKED ? GN : 1];
+      int ready = 1;
+      const int nchunks = Cfg::CHUNKED ? (int)cdiv(kblocks, CHUNK_KB) : 1;
+      for (int c = 0; c < nchunks && ready; ++c) {
+        const int buf = Cfg::CHUNKED ? (c & 1) : 0;
+        int ok = 0;
+        if (lane == 0) ok = tc::mbar_wait(&S.acc_full[buf], (uint32_t)(c >> 1) & 1u, abort_flag) && !*abort_flag;
+        ready = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ready) break;
         tc::tc_fence_after();
+        if constexpr (Cfg::CHUNKED) {
+#pragma unroll
+          for (int cc = 0; cc < GN / 32; ++cc) {
+            float v[32];
+            tc::tmem_ld_32x32b_x32(taddr + lane_base + buf * GN + cc * 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[cc * 32 + i] = c == 0 ? v[i] : acc[cc * 32 + i] + v[i];
+          }
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&S.acc_empty[buf]);
+        }
+      }
+      if (ready) {
         if (warp == 2 && lane == 0) GPTQ_GEMM_MARK(4);
-        const int q = warp & 3;
-        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         // Each warp owns TMEM lanes (rows) [32 q, 32 q + 32).  It stages its 32 x GN
         // slice of C in shared memory (the stage buffers are free once the
         // accumulator is complete): 16-byte pieces, piece p of row rr stored at
@@ -193,10 +237,15 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
           asm volatile("cp.async.wait_all;" ::: "memory");
           __syncwarp();
         }
-#pragma unroll 1
+#pragma unroll
         for (int c = 0; c < GN / 32; ++c) {
           float v[32];
-          tc::tmem_ld_32x32b_x32(taddr + lane_base + c * 32, v);
+          if constexpr (Cfg::CHUNKED) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = acc[c * 32 + i];
+          } else {
+            tc::tmem_ld_32x32b_x32(taddr + lane_base + c * 32, v);
+          }
           // lane = row: combine with C
 #pragma unroll
           for (int pp = 0; pp < 8; ++pp) {
@@ -260,7 +309,7 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
   }
   if (warp == 1) {
     __syncwarp();
-    tc::tmem_dealloc<GN>(taddr);
+    tc::tmem_dealloc<Cfg::TMEM_COLS>(taddr);
   }
 }
 
@@ -322,8 +371,10 @@ int launch_gemm3(float* C, int ldc, int M, int N, int K, const float* Ahi, const
                  bool store, float* Chi, float* Clo, int ldh) {
   if (M <= 0 || N <= 0 || K <= 0) return GPTQ_OK;
   GemmOut out{C, ldc, store ? 1 : 0, Chi, Clo, ldh};
-  // the widest tile that still gives about one CTA per SM
+  // the widest tile that still gives about one CTA per SM; K beyond one chunk takes
+  // the chunked (<= 128-wide) tiles
   const int64_t tm = (int64_t)cdiv(M, GM);
+  if (K > CHUNK_KB * GK) return launch_gemm3_t<128>(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, st, s);
   if (N <= 128 && tm * (int64_t)cdiv(N, 64) < 148)
     return launch_gemm3_t<32>(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, st, s);
   if (N <= 128 && tm * (int64_t)cdiv(N, 128) < 148)

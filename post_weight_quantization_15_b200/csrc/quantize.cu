@@ -609,7 +609,9 @@ int launch_quantize(const void* W, int w_dtype, int out, int n, const float* U, 
       dim3 blk(32, 8), grd((unsigned)cdiv(n - se, 32), (unsigned)(SBK / 32));
       u_block_transpose_split_kernel<<<grd, blk, 0, s>>>(U, n, s0, kw, se, w.Bhi, w.Blo, SBK, st);
       GPTQ_LAUNCH_CHECK();
-      // Wf[:, se:] -= Err[:, super-block] . U[super-block, se:]
+      // Wf[:, se:] -= Err[:, super-block] . U[super-block, se:] (K = 512, accumulated by
+      // the GEMM in 128-deep chunks summed in fp32 registers: one long tensor-core
+      // accumulation let the codes of a 28,672-column layer drift past 0.5 %)
       const int rc = launch_gemm3(w.Wf + se, n, out, n - se, kw, w.Ehi, w.Elo, SBK, w.Bhi, w.Blo, SBK, false, st, s);
       if (rc != GPTQ_OK) return rc;
     }

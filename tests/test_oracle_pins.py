@@ -164,6 +164,28 @@ def test_u_is_upper_cholesky_of_damped_inverse():
     assert np.allclose(p.Hd - Hp, p.lam * np.eye(48), atol=1e-12 * np.abs(H).max())
 
 
+@pytest.mark.parametrize("act,with_dead", [(False, False), (True, False), (True, True)])
+def test_trailing_block_of_u_comes_from_the_trailing_block_of_h(act, with_dead):
+    # U's last m rows and columns depend only on the trailing principal block of H_d
+    # (H_d = V V^T with V = U^-1 upper triangular): the block computed from it alone
+    # must equal the full factor's block.
+    H, _ = _spd_from_x(40, 300, 6)
+    if with_dead:
+        H[5, :] = 0.0
+        H[:, 5] = 0.0
+        H[22, :] = 0.0
+        H[:, 22] = 0.0
+    key = np.diag(H) * (1.0 + 1e-9 * np.arange(40))
+    full = O.prepare(H, 0.01, act, order_key=key)
+    for m in (1, 7, 16, 40):
+        Ut, perm = O.prepare_trailing(H, 0.01, act, m, order_key=key)
+        assert np.array_equal(perm, full.perm)
+        assert np.allclose(Ut, full.U[40 - m:, 40 - m:], rtol=1e-10, atol=1e-12 * np.abs(full.U).max())
+    # a planted mistake (the leading block instead of the trailing one) fails
+    Ul, _ = O.prepare_trailing(H[::-1, ::-1].copy(), 0.01, False, 16)
+    assert not np.allclose(Ul, O.prepare(H, 0.01, False).U[24:, 24:], rtol=1e-6)
+
+
 def test_act_order_descending_and_stable():
     d = np.array([3.0, 5.0, 3.0, 1.0, 5.0, 0.5])
     assert O.act_order(d).tolist() == [1, 4, 0, 2, 3, 5]
