@@ -104,6 +104,36 @@ GPTQ_API int gptq_hessian_accumulate(float* H, double* hdiag, int n, const void*
                             int64_t tokens, int32_t* d_status, void* stream);
 
 /*
+ * gptq_hessian_accumulate_host - the same accumulation with X in HOST memory.
+ *
+ * Same computation and arguments as gptq_hessian_accumulate ("polydesk.ai/glossaire/
+ * gptq", "Etape 2"), except that X stays on the host: it is copied to the device in
+ * chunks of tokens, one strided copy per chunk, into a caller-provided device staging
+ * area, and the tile product of each chunk runs while the next one is copied, so
+ * that the transfer of the activations hides the contraction.  This is the one call
+ * whose X pointer is a host pointer; everything else is as above.
+ *
+ *   X_host         bf16 [n, tokens] in host memory, row stride ld_x elements
+ *                  (ld_x >= tokens).  Page-locked (pinned) memory lets the copies run
+ *                  asynchronously; pageable memory still gives the right result but the
+ *                  copies then do not overlap the work.  The caller keeps X_host alive
+ *                  and unchanged until the stream has passed this call.
+ *   staging        device buffer of staging_bytes, 256-byte aligned, owned by the
+ *                  caller; it is split in two halves of n x C bf16, C the largest
+ *                  multiple of 64 tokens that fits (at least 64, else
+ *                  GPTQ_ERR_WORKSPACE).  Larger areas mean fewer, longer chunks.
+ *   stream         the tile products run on it; the copies run on a stream of the
+ *                  library's own (one per host thread and device, created on first use)
+ *                  that is ordered after the work already queued on `stream`, and every
+ *                  kernel waits for its chunk's copy, so `stream` is ordered after all of
+ *                  this call's copies and kernels.
+ * Errors: as gptq_hessian_accumulate; a failed copy returns GPTQ_ERR_CUDA.
+ */
+GPTQ_API int gptq_hessian_accumulate_host(float* H, double* hdiag, int n, const void* X_host, int64_t ld_x,
+                                          int64_t tokens, void* staging, size_t staging_bytes,
+                                          int32_t* d_status, void* stream);
+
+/*
  * gptq_prepare - dead inputs, act-order, damping and the Cholesky factor U.
  *
  * In this order (the readings are those of the library's oracle):

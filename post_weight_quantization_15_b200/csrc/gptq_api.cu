@@ -72,6 +72,16 @@ int gptq_hessian_accumulate(float* H, double* hdiag, int n, const void* X, int64
   return rc;
 }
 
+int gptq_hessian_accumulate_host(float* H, double* hdiag, int n, const void* X_host, int64_t ld_x, int64_t tokens,
+                                 void* staging, size_t staging_bytes, int32_t* d_status, void* stream) {
+  if (H == nullptr || n <= 0 || tokens < 0) return GPTQ_ERR_INVALID_ARG;
+  if (tokens == 0) return GPTQ_OK;
+  if (X_host == nullptr || ld_x < tokens) return GPTQ_ERR_INVALID_ARG;
+  if (staging == nullptr || !aligned(staging, 256) || hessian_host_chunk(n, staging_bytes) < 64)
+    return GPTQ_ERR_WORKSPACE;
+  return launch_hessian_host(H, hdiag, n, X_host, ld_x, tokens, staging, staging_bytes, d_status, as_stream(stream));
+}
+
 size_t gptq_prepare_workspace_size(int n) { return n > 0 ? prepare_ws_bytes(n) : 0; }
 
 int gptq_prepare(const float* H, const double* hdiag, int n, float damp_percent, int desc_act, float* U,

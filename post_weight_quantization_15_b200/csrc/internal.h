@@ -11,6 +11,9 @@ int launch_hessian(float* H, int n, const void* X, int64_t ld_x, int64_t tokens,
                    cudaStream_t s);
 int launch_hessian_diag64(double* hdiag, int n, const void* X, int64_t ld_x, int64_t tokens,
                           int32_t* st, cudaStream_t s);
+int64_t hessian_host_chunk(int n, size_t staging_bytes);
+int launch_hessian_host(float* H, double* hdiag, int n, const void* X_host, int64_t ld_x_host, int64_t tokens,
+                        void* staging, size_t staging_bytes, int32_t* st, cudaStream_t s);
 
 // ---- K2: prepare -------------------------------------------------------------
 size_t prepare_ws_bytes(int n);

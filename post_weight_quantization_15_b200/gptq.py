@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
     L.gptq_status_read.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
     L.gptq_hessian_accumulate.restype = I
     L.gptq_hessian_accumulate.argtypes = [P, P, I, P, I64, I64, P, P]
+    L.gptq_hessian_accumulate_host.restype = I
+    L.gptq_hessian_accumulate_host.argtypes = [P, P, I, P, I64, I64, P, SZ, P, P]
     L.gptq_prepare_workspace_size.restype = SZ
     L.gptq_prepare_workspace_size.argtypes = [I]
     L.gptq_prepare.restype = I
@@ -168,6 +170,32 @@ def hessian_accumulate(H: torch.Tensor, X: torch.Tensor, hdiag: Optional[torch.T
         raise ValueError("hdiag must be fp64 [n]")
     _check(lib().gptq_hessian_accumulate(_ptr(H), _ptr(hdiag), n, _ptr(X), X.stride(0), X.shape[1],
                                          _ptr(status), _stream(stream)), "gptq_hessian_accumulate")
+    return H
+
+
+def hessian_accumulate_host(H: torch.Tensor, X_host: torch.Tensor, hdiag: Optional[torch.Tensor] = None,
+                            status: Optional[torch.Tensor] = None, staging: Optional[torch.Tensor] = None,
+                            chunk_tokens: int = 8192, stream=None) -> torch.Tensor:
+    """H += 2 . X . X^T with X in host memory (pinned for overlap), copied in token chunks.
+
+    ``staging`` is a device byte buffer (allocated here if None: two halves of
+    n x chunk_tokens bf16); the copies of chunk i + 1 overlap the product of chunk i.
+    """
+    _require_cuda(H, hdiag, status, staging)
+    if X_host.device.type != "cpu" or X_host.dtype not in (torch.bfloat16, torch.int16, torch.uint16) \
+            or X_host.dim() != 2 or X_host.stride(1) != 1:
+        raise ValueError("X_host must be a host [n, tokens] bf16 tensor with contiguous rows")
+    n = X_host.shape[0]
+    if H.dtype != torch.float32 or tuple(H.shape) != (n, n) or not H.is_contiguous():
+        raise ValueError("H must be a contiguous fp32 [n, n] tensor")
+    if hdiag is not None and (hdiag.dtype != torch.float64 or hdiag.numel() != n):
+        raise ValueError("hdiag must be fp64 [n]")
+    if staging is None:
+        chunk = max(64, min(int(chunk_tokens), (X_host.shape[1] + 63) // 64 * 64)) // 64 * 64
+        staging = workspace(2 * n * chunk * 2, H.device)
+    _check(lib().gptq_hessian_accumulate_host(_ptr(H), _ptr(hdiag), n, ctypes.c_void_p(X_host.data_ptr()),
+                                              X_host.stride(0), X_host.shape[1], _ptr(staging), staging.numel(),
+                                              _ptr(status), _stream(stream)), "gptq_hessian_accumulate_host")
     return H
 
 
@@ -281,13 +309,22 @@ def pack(codes: torch.Tensor, bits: int, out: Optional[torch.Tensor] = None, str
 def gptq_quantize(W: torch.Tensor, X: torch.Tensor, bits: int = 4, group_size: int = 128, sym: bool = False,
                   desc_act: bool = False, damp_percent: float = 0.01, block: int = 128,
                   want_codes: bool = False, want_err: bool = False, check: bool = True):
-    """H = 2.X.X^T, prepare, quantize.  Returns (QuantizedLayer, Prepared, H)."""
+    """H = 2.X.X^T, prepare, quantize.  Returns (QuantizedLayer, Prepared, H).
+
+    W and X on the device, or both in host memory (pinned for overlap): then X crosses
+    to the device in token chunks while the Hessian of the previous chunk is formed.
+    """
     n = X.shape[0]
-    dev = X.device
+    host = X.device.type == "cpu"
+    dev = torch.device("cuda", torch.cuda.current_device()) if host else X.device
     st = new_status(dev)
     H = torch.zeros((n, n), dtype=torch.float32, device=dev)
     hdiag = torch.zeros(n, dtype=torch.float64, device=dev) if desc_act else None
-    hessian_accumulate(H, X, hdiag, st)
+    if host:
+        W = W.to(dev, non_blocking=True)
+        hessian_accumulate_host(H, X, hdiag, st)
+    else:
+        hessian_accumulate(H, X, hdiag, st)
     prep = prepare(H, damp_percent, desc_act, hdiag, st)
     q = quantize_layer(W, prep, bits, group_size, sym, block, want_codes, want_err)
     if check:

@@ -101,6 +101,33 @@ def test_hessian_and_diag_against_oracle():
     assert np.allclose(hd.cpu().numpy(), np.diag(H64), rtol=1e-13, atol=0)
 
 
+def test_hessian_from_host_memory_in_chunks():
+    # X stays in pinned host memory; a small staging area forces five chunks, the last ragged
+    dev = _dev()
+    W, x = S.small_case(8, 300, 2504, seed=3)
+    X_host = torch.from_numpy(x.view(np.int16)).pin_memory()
+    H = torch.zeros((300, 300), dtype=torch.float32, device=dev)
+    hd = torch.zeros(300, dtype=torch.float64, device=dev)
+    staging = G.workspace(2 * 300 * 512 * 2, dev)
+    st = G.new_status(dev)
+    G.hessian_accumulate_host(H, X_host, hd, st, staging=staging)
+    G.raise_on_status(st, "host Hessian")
+    H64 = O.hessian(x)
+    Hg = H.cpu().numpy().astype(np.float64)
+    iu = np.triu_indices(300)
+    rel = np.abs(Hg[iu] - H64[iu]) / np.sqrt(np.outer(np.diag(H64), np.diag(H64)))[iu]
+    assert rel.max() <= 2504 * 2.0 ** -23, rel.max()
+    assert np.allclose(hd.cpu().numpy(), np.diag(H64), rtol=1e-13, atol=0)
+    # the whole path from host tensors gives the device path's result
+    W, x = S.small_case(48, 320, 2504, seed=4)
+    Wt = torch.from_numpy(np.ascontiguousarray(W))
+    X_host = torch.from_numpy(x.view(np.int16)).pin_memory()
+    q_h, p_h, _ = G.gptq_quantize(Wt.pin_memory(), X_host, 4, 32, False, True, want_codes=True)
+    q_d, p_d, _ = G.gptq_quantize(Wt.to(dev), _to_dev_x(x, dev), 4, 32, False, True, want_codes=True)
+    assert np.array_equal(p_h.perm.cpu().numpy(), p_d.perm.cpu().numpy())
+    assert float(np.mean(q_h.codes.cpu().numpy() != q_d.codes.cpu().numpy())) <= CODE_MISMATCH_MAX
+
+
 def test_prepare_u_and_perm():
     dev = _dev()
     _, x = S.small_case(8, 384, 3000, seed=4)
