@@ -136,23 +136,35 @@ __device__ __forceinline__ float code_from_q(float q, QParams p, int bits, bool 
 // ---------------------------------------------------------------------------
 // K0: Wf[r][k] = W[r][perm[k]] (0 for dead inputs), invperm, g_idx.
 // ---------------------------------------------------------------------------
+// Four consecutive columns per thread (n % 4 == 0): 16-byte stores, and the loads of a
+// warp cover 128 consecutive columns of a row for the identity order.
 template <typename T>
 __global__ void ingest_kernel(const T* W, int out, int n, const int32_t* perm, const uint8_t* dead, int gs,
                               float* Wf, int32_t* invperm, int32_t* g_idx, int32_t* st) {
   if (has_error(st)) return;
-  const int k = blockIdx.x * 32 + threadIdx.x;
+  const int k0 = 4 * (blockIdx.x * 32 + threadIdx.x);
   const int r = blockIdx.y * 8 + threadIdx.y;
-  if (k >= n) return;
-  const int src = perm ? perm[k] : k;
+  if (k0 >= n) return;
+  int src[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) src[u] = perm ? perm[k0 + u] : k0 + u;
   if (r == 0) {
-    invperm[src] = k;
-    g_idx[src] = gs > 0 ? k / gs : 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      invperm[src[u]] = k0 + u;
+      g_idx[src[u]] = gs > 0 ? (k0 + u) / gs : 0;
+    }
   }
   if (r >= out) return;
-  float v = load_as_float<T>(W + (int64_t)r * n + src);
-  if (!isfinite(v)) set_error(st, GPTQ_ERR_NONFINITE, src, STAGE_INGEST);
-  if (dead && dead[src]) v = 0.f;
-  Wf[(int64_t)r * n + k] = v;
+  const T* row = W + (int64_t)r * n;
+  float v[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    v[u] = load_as_float<T>(row + src[u]);
+    if (!isfinite(v[u])) set_error(st, GPTQ_ERR_NONFINITE, src[u], STAGE_INGEST);
+    if (dead && dead[src[u]]) v[u] = 0.f;
+  }
+  *reinterpret_cast<float4*>(Wf + (int64_t)r * n + k0) = make_float4(v[0], v[1], v[2], v[3]);
 }
 
 // group_size = -1: one scale / zero per row, from the whole (uncompensated) row.
@@ -507,24 +519,40 @@ __global__ void u_block_transpose_split_kernel(const float* U, int n, int b0, in
 // ---------------------------------------------------------------------------
 // K5: qweight[w][o] = bits of the codes of input columns k with k.bits in
 // [32w, 32w + 32), original order; code of column k = codes[o][invperm[k]].
+// A 32 x 32 tile of (rows o, words w) per block: a warp packs consecutive words of one
+// row (reading the row's codes in order), the tile turns through shared memory, and
+// a warp writes 32 consecutive o of one word.
 // ---------------------------------------------------------------------------
 __global__ void pack_kernel(const uint8_t* codes, const int32_t* invperm, int out, int n, int ld_codes,
                             int bits, int32_t* qweight, const int32_t* st) {
   if (has_error(st)) return;
-  const int o = blockIdx.x * blockDim.x + threadIdx.x;
-  const int wi = blockIdx.y;
-  if (o >= out) return;
-  const int pos0 = wi * 32;
-  const int k_lo = pos0 / bits, k_hi = (pos0 + 31) / bits;
-  uint64_t acc = 0;
-  const uint8_t* crow = codes + (int64_t)o * ld_codes;
-  for (int k = k_lo; k <= k_hi && k < n; ++k) {
-    const int src = invperm ? invperm[k] : k;
-    const uint64_t c = crow[src] & ((1u << bits) - 1u);
-    const int sh = k * bits - pos0;  // may be negative for a code straddling in from the left
-    if (sh >= 0) acc |= c << sh; else acc |= c >> (-sh);
+  __shared__ uint32_t tile[32][33];
+  const int words = n * bits / 32;
+  const int o0 = blockIdx.x * 32, w0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int o = o0 + ty + 8 * r, wi = w0 + tx;
+    uint64_t acc = 0;
+    if (o < out && wi < words) {
+      const int pos0 = wi * 32;
+      const int k_lo = pos0 / bits, k_hi = (pos0 + 31) / bits;
+      const uint8_t* crow = codes + (int64_t)o * ld_codes;
+      for (int k = k_lo; k <= k_hi && k < n; ++k) {
+        const int src = invperm ? invperm[k] : k;
+        const uint64_t c = crow[src] & ((1u << bits) - 1u);
+        const int sh = k * bits - pos0;  // may be negative for a code straddling in from the left
+        if (sh >= 0) acc |= c << sh; else acc |= c >> (-sh);
+      }
+    }
+    tile[ty + 8 * r][tx] = (uint32_t)(acc & 0xFFFFFFFFull);
   }
-  qweight[(int64_t)wi * out + o] = (int32_t)(uint32_t)(acc & 0xFFFFFFFFull);
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int wi = w0 + ty + 8 * r, o = o0 + tx;
+    if (wi < words && o < out) qweight[(int64_t)wi * out + o] = (int32_t)tile[tx][ty + 8 * r];
+  }
 }
 
 // Optional output: codes in the original column order.
@@ -549,8 +577,8 @@ size_t quantize_ws_bytes(int out, int n, int block) {
 int launch_pack(const uint8_t* codes, const int32_t* invperm, int out, int n, int ld_codes, int bits,
                 int32_t* qweight, const int32_t* st, cudaStream_t s) {
   const int words = n * bits / 32;
-  dim3 grd((unsigned)cdiv(out, 128), (unsigned)words);
-  pack_kernel<<<grd, 128, 0, s>>>(codes, invperm, out, n, ld_codes, bits, qweight, st);
+  dim3 blk(32, 8), grd((unsigned)cdiv(out, 32), (unsigned)cdiv(words, 32));
+  pack_kernel<<<grd, blk, 0, s>>>(codes, invperm, out, n, ld_codes, bits, qweight, st);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }
@@ -562,7 +590,7 @@ int launch_quantize(const void* W, int w_dtype, int out, int n, const float* U, 
   (void)block;
   QuantWs w = carve(ws, out, n);
   {
-    dim3 blk(32, 8), grd((unsigned)cdiv(n, 32), (unsigned)cdiv(std::max(out, 1), 8));
+    dim3 blk(32, 8), grd((unsigned)cdiv(n, 128), (unsigned)cdiv(std::max(out, 1), 8));
     if (w_dtype == GPTQ_F32)
       ingest_kernel<float><<<grd, blk, 0, s>>>(static_cast<const float*>(W), out, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
     else if (w_dtype == GPTQ_F16)
