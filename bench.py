@@ -251,9 +251,9 @@ def run_reference(args):
     return 0
 
 
-# DRAM bytes (read + write) of one hessian_tc_kernel launch on layer-1024x4096, from one ncu
-# capture (profiles/hessian_tc_layer-1024x4096.md), valid while the kernel's sources are the
-# ones that were captured (their SHA-256 below); otherwise the traffic is reported as null.
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one hessian_tc_kernel launch on
+# layer-1024x4096, from one ncu capture of this bench command, valid while the kernel's sources
+# are the ones that were captured (their SHA-256 below); otherwise the traffic is null.
 HESSIAN_TRAFFIC = {"n": 4096, "tokens": 65536, "bytes": 941680128 + 24512000,
                    "sha256": {"post_weight_quantization_15_b200/csrc/hessian.cu": "79a19330e3dc3175",
                               "post_weight_quantization_15_b200/csrc/tc_common.cuh": "7955f242938f18ca"}}
