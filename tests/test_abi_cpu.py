@@ -66,3 +66,9 @@ def test_bad_arguments_rejected_without_a_gpu(L):
     assert L.gptq_hessian_accumulate(fake, None, 64, fake, 100, 100, None, None) == -1   # ld_x % 8 != 0
     assert L.gptq_hessian_accumulate(fake, None, 64, fake, 96, 0, None, None) == 0        # empty chunk
     assert L.gptq_pack(fake, 4, 33, 4, fake, None) == -2
+    # the host-memory Hessian: ld_x < tokens, a staging area that holds less than two
+    # 64-token chunks, an unaligned staging area, and the empty chunk
+    assert L.gptq_hessian_accumulate_host(fake, None, 64, fake, 50, 100, fake, 1 << 20, None, None) == -1
+    assert L.gptq_hessian_accumulate_host(fake, None, 64, fake, 100, 100, fake, 2 * 64 * 63 * 2, None, None) == -7
+    assert L.gptq_hessian_accumulate_host(fake, None, 64, fake, 100, 100, P(258), 1 << 20, None, None) == -7
+    assert L.gptq_hessian_accumulate_host(fake, None, 64, fake, 100, 0, fake, 0, None, None) == 0
