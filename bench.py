@@ -458,6 +458,119 @@ def run_e2e(G, torch, W_host, X_host, st, n, out, dev, steps, flush):
             "d2h_bytes_per_step": d2h}
 
 
+# --------------------------------------------------------------------------- #
+# one whole decoder block
+# --------------------------------------------------------------------------- #
+# The inputs of a decoder block's linear layers: q, k and v read the same activations,
+# o reads the attention output, gate and up the same MLP input, down the MLP's inner
+# activations; H and U are formed once per input.
+BLOCK_INPUTS = (("q", "k", "v"), ("o",), ("gate", "up"), ("down",))
+
+
+def run_block(args):
+    """Time every layer of a decoder block on one GPU (Hessian and preparation once per
+    input, quantization once per layer); prints its own JSON line."""
+    import torch
+
+    import post_weight_quantization_15_b200 as G
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --block needs a CUDA device")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = S.workloads()[args.block]
+    st = wl.settings[0]
+    by = {l.name: l for l in wl.layers}
+    groups = [[by[nm] for nm in g if nm in by] for g in BLOCK_INPUTS]
+    groups = [g for g in groups if g]
+    xs = {}
+    work = []     # (n, X, [W...], tokens) per input
+    for g in groups:
+        xspec = g[0].x
+        key = (xspec.n, xspec.tokens)
+        if key not in xs:   # the synthetic activations of equal shape are the same array
+            xs[key] = torch.from_numpy(S.make_x(xspec).view(np.int16)).to(dev).view(torch.bfloat16)
+        Ws = [torch.from_numpy(S.make_w(l.w)).to(dev) for l in g]
+        work.append((xspec.n, xs[key], Ws, xspec.tokens, [l.name for l in g]))
+    status = G.new_status(dev)
+    stream = torch.cuda.current_stream()
+    bufs = []
+    for n, X, Ws, N, names in work:
+        H = torch.empty((n, n), dtype=torch.float32, device=dev)
+        hd = torch.empty(n, dtype=torch.float64, device=dev) if st.desc_act else None
+        ws = G.workspace(G.lib().gptq_prepare_workspace_size(n), dev)
+        prep = G.Prepared(U=torch.empty((n, n), dtype=torch.float32, device=dev),
+                          perm=torch.empty(n, dtype=torch.int32, device=dev),
+                          dead=torch.empty(n, dtype=torch.uint8, device=dev), status=status, desc_act=st.desc_act)
+        qws = G.workspace(max(G.quantize_workspace_size(W.shape[0], n, st.block) for W in Ws), dev)
+        outs = [G.alloc_quantized(W.shape[0], n, st.bits, st.group_size, st.sym, dev) for W in Ws]
+        bufs.append((H, hd, ws, prep, qws, outs))
+
+    def once(ev=None):
+        G.status_reset(status)
+        for gi, ((n, X, Ws, N, names), (H, hd, ws, prep, qws, outs)) in enumerate(zip(work, bufs)):
+            if ev is not None:
+                ev[gi][4].record(stream)
+            H.zero_()
+            if hd is not None:
+                hd.zero_()
+            if ev is not None:
+                ev[gi][0].record(stream)
+            G.hessian_accumulate(H, X, hd, status)
+            if ev is not None:
+                ev[gi][1].record(stream)
+            G.prepare(H, st.damp_percent, st.desc_act, hd, status, ws=ws, out=prep)
+            if ev is not None:
+                ev[gi][2].record(stream)
+            for W, q in zip(Ws, outs):
+                G.quantize_layer(W, prep, st.bits, st.group_size, st.sym, st.block, ws=qws, out=q)
+            if ev is not None:
+                ev[gi][3].record(stream)
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        once()
+    torch.cuda.synchronize()
+    G.raise_on_status(status, "block warm-up")
+    steps = max(1, min(args.steps, 3))
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in work] for _ in range(steps)]
+    clocks = ClockSampler(0)
+    clocks.start()
+    for i in range(steps):
+        once(evs[i])
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    G.raise_on_status(status, "block")
+    per_input = []
+    hess_flop, hess_s, total = 0.0, 0.0, 0.0
+    for gi, (n, X, Ws, N, names) in enumerate(work):
+        h = statistics.mean(evs[i][gi][0].elapsed_time(evs[i][gi][1]) for i in range(steps))
+        pr = statistics.mean(evs[i][gi][1].elapsed_time(evs[i][gi][2]) for i in range(steps))
+        qu = statistics.mean(evs[i][gi][2].elapsed_time(evs[i][gi][3]) for i in range(steps))
+        per_input.append({"layers": names, "in": n, "out": [int(W.shape[0]) for W in Ws], "hessian_ms": h,
+                          "prepare_ms": pr, "quantize_ms": qu})
+        hess_flop += float(n) * (n + 1) * N
+        hess_s += h * 1e-3
+        total += h + pr + qu
+    block_ms = statistics.mean(evs[i][0][4].elapsed_time(evs[i][-1][3]) for i in range(steps))   # clears included
+    weights = sum(int(W.numel()) for _, _, Ws, _, _ in work for W in Ws)
+    peaks = load_peaks()
+    achieved = hess_flop / hess_s / 1e12
+    line = {
+        "metric": f"GPTQ decoder block ({args.block}): seconds per block, 1 B200", "value": block_ms * 1e-3,
+        "unit": "s", "higher_is_better": False, "steps": steps, "n_gpus": 1, "data": "synthetic",
+        "config": {"workload": args.block, "bits": st.bits, "group_size": st.group_size, "sym": st.sym,
+                   "desc_act": st.desc_act, "inputs": "H and U once per input: q/k/v, o, gate/up, down"},
+        "gparam_per_s": weights / (block_ms * 1e-3) / 1e9,
+        "per_input": per_input,
+        "roofline": {"kernel": "hessian (K1), all inputs", "bound": "tensor", "achieved": achieved,
+                     "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
+                     "frac": achieved / float(peaks["bf16_tflops"]), "peak_source": f"{peaks['_source']} bf16 burst"},
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -469,11 +582,15 @@ def main():
                     help="token sample of the CPU oracle legs (its Hessian time is scaled to the full count)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--block", default=None, choices=["llama2-7b-block", "llama2-70b-block"],
+                    help="time every layer of a decoder block instead (its own JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.block:
+        return run_block(args)
     return run_ours(args)
 
 
