@@ -145,6 +145,20 @@ def test_prepare_u_and_perm():
     assert np.abs(U - ora.U).max() / np.abs(ora.U).max() < 1e-4
 
 
+@pytest.mark.parametrize("act", [False, True])
+def test_dead_inputs(act):
+    # features whose activations are all zero: H_ii = 0, so the column is dead (unit
+    # diagonal in the damped H, weights zeroed); act-order puts them by their unit key
+    W, x = S.small_case(64, 256, 1024, seed=9)
+    x = x.copy()
+    x[[3, 77, 200], :] = 0
+    c, q, prep, Hg, H64, ora = _compare(W, x, 4, 32, False, act)
+    print(c)
+    dead = prep.dead.cpu().numpy().astype(bool)
+    assert np.array_equal(np.flatnonzero(dead), [3, 77, 200])
+    assert c.ok(), c
+
+
 def test_identity_hessian_is_bit_exact_round_to_nearest():
     dev = _dev()
     W = S.make_w(S.WSpec(300, 512, 0.02, "f16", 5, 100))
