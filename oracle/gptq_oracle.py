@@ -45,7 +45,7 @@ __all__ = [
     "bf16_bits_to_f64", "hessian", "act_order", "prepare", "prepare_trailing", "Prepared",
     "group_params", "quantize_codes", "dequant_value", "sweep", "SweepResult",
     "g_idx", "unpermute_codes", "pack", "unpack", "dequantize", "layer_error",
-    "rtn", "quantize_layer", "LayerResult", "gptq_layer",
+    "rtn", "quantize_layer", "LayerResult", "gptq_layer", "pad_layer", "pack_zeros", "unpack_zeros",
 ]
 
 F16_MIN_SUBNORMAL = np.float32(2.0 ** -24)
@@ -473,3 +473,78 @@ def gptq_layer(W: np.ndarray, x_bits: Optional[np.ndarray], bits: int, group_siz
         rel_rtn = layer_error(W, dequantize(qr, rs.astype(np.float16), rz.astype(np.float16), gi, bits, n), H)
     return LayerResult(qweight=qw, scales=scales16, zeros=zeros16, g_idx=gi, codes=codes,
                        perm=prep.perm, prep=prep, sw=sw, rel_err=rel, rel_err_rtn=rel_rtn)
+
+
+# --------------------------------------------------------------------------- #
+# 7. Checkpoint variants: zero padding, packed zero points
+# --------------------------------------------------------------------------- #
+def pad_layer(W: np.ndarray, x_bits: Optional[np.ndarray], n: int) -> Tuple[np.ndarray, Optional[np.ndarray]]:
+    """The layer zero-padded to n inputs.
+
+    polydesk, "Limites de GPTQ" (divisibility): a width that the group size does
+    not divide is handled by padding the weights with zeros.  Reading: W gets
+    n - in zero columns and X (bf16 bit patterns) n - in zero rows, i.e. the padded
+    inputs carry no activation; the padded layer then goes through the ordinary
+    path, where those inputs are dead (zero diagonal) and count in the damping's
+    mean diagonal like any other input.
+    """
+    W = np.asarray(W)
+    out, k = W.shape
+    if n < k:
+        raise ValueError("padded width smaller than the layer")
+    Wp = np.zeros((out, n), dtype=W.dtype)
+    Wp[:, :k] = W
+    xp = None
+    if x_bits is not None:
+        x_bits = np.asarray(x_bits)
+        xp = np.zeros((n, x_bits.shape[1]), dtype=x_bits.dtype)     # bit pattern 0 is +0.0
+        xp[:k] = x_bits
+    return Wp, xp
+
+
+def pack_zeros(zeros: np.ndarray, bits: int, zero_offset: int = 0) -> np.ndarray:
+    """Zero points [G, out] -> int32 [G, out.bits/32], packed along the output dimension.
+
+    The pages store zero points in FP16 (ayinedjimi-consultants, "Calibration et
+    dataset") and warn that checkpoints of different tool versions differ
+    (polydesk, "Limites de GPTQ").  Reading for the packed integer form: per group,
+    the values (zero - zero_offset) mod 2^bits form a little-endian bit stream
+    along the outputs, output o at stream bits o.bits ... (the stream of ``pack``,
+    taken along the other dimension); zero_offset 1 is the older convention of
+    storing zero - 1.
+    """
+    z = np.asarray(zeros, dtype=np.float64)
+    if z.ndim != 2:
+        raise ValueError("zeros must be [G, out]")
+    if np.any(z != np.rint(z)) or np.any(z < 0) or np.any(z > 2 ** bits - 1):
+        raise ValueError("zero points must be integers in [0, 2^bits - 1]")
+    if zero_offset not in (0, 1):
+        raise ValueError("zero_offset must be 0 or 1")
+    G, out = z.shape
+    if (out * bits) % 32 != 0:
+        raise ValueError("out.bits must be a multiple of 32")
+    v = ((z.astype(np.int64) - zero_offset) % (2 ** bits)).astype(np.uint64)
+    words = np.zeros((G, out * bits // 32), dtype=np.uint64)
+    for o in range(out):
+        pos = o * bits
+        wi, off = pos // 32, pos % 32
+        words[:, wi] |= (v[:, o] << np.uint64(off)) & np.uint64(0xFFFFFFFF)
+        if off + bits > 32:
+            words[:, wi + 1] |= v[:, o] >> np.uint64(32 - off)
+    return words.astype(np.uint32).view(np.int32)
+
+
+def unpack_zeros(qzeros: np.ndarray, bits: int, out: int, zero_offset: int = 0) -> np.ndarray:
+    """Inverse of ``pack_zeros``: int32 [G, out.bits/32] -> zero points [G, out] (float64)."""
+    q = np.asarray(qzeros).view(np.uint32).astype(np.uint64)
+    G = q.shape[0]
+    z = np.zeros((G, out), dtype=np.float64)
+    mask = np.uint64(2 ** bits - 1)
+    for o in range(out):
+        pos = o * bits
+        wi, off = pos // 32, pos % 32
+        v = q[:, wi] >> np.uint64(off)
+        if off + bits > 32:
+            v |= q[:, wi + 1] << np.uint64(32 - off)
+        z[:, o] = ((v & mask).astype(np.int64) + zero_offset) % (2 ** bits)
+    return z

@@ -388,3 +388,98 @@ def test_planted_zero_offset_mistake_fails_range_pin(golden_dir, monkeypatch):
     g = _load(golden_dir, "quantizer_hand.json")["sym"]
     s, z = O.group_params(np.array([g["w"]], np.float32), 4, True)
     assert float(z[0]) != g["zero"]
+
+
+# --------------------------------------------------------------------------- #
+# Checkpoint variants: packed zero points, zero padding
+# --------------------------------------------------------------------------- #
+def test_pack_zeros_hand_examples(golden_dir):
+    for case in _load(golden_dir, "pack_zeros_hand.json")["cases"]:
+        z = np.array(case["zeros"], dtype=np.float64)
+        bits, off = case["bits"], case["zero_offset"]
+        qz = O.pack_zeros(z, bits, off).view(np.uint32).astype(np.int64)
+        assert [[int(h, 16) for h in row] for row in case["words_hex"]] == qz.tolist()
+        assert np.array_equal(O.unpack_zeros(O.pack_zeros(z, bits, off), bits, z.shape[1], off), z)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_pack_zeros_is_the_code_stream_along_the_outputs(bits):
+    # without the offset, group g's words are the stream the code packing forms for a
+    # row of codes, here taken along the outputs: pack of the [G, out] matrix, transposed
+    rng = np.random.default_rng(40 + bits)
+    z = rng.integers(0, 2 ** bits, (5, 96))
+    assert np.array_equal(O.pack_zeros(z, bits).view(np.uint32), O.pack(z.astype(np.uint8), bits).view(np.uint32).T)
+    # with it, every value moves down by one modulo 2^bits
+    assert np.array_equal(O.pack_zeros(z, bits, 1).view(np.uint32),
+                          O.pack(((z - 1) % 2 ** bits).astype(np.uint8), bits).view(np.uint32).T)
+    with pytest.raises(ValueError):
+        O.pack_zeros(z + 0.5, bits)
+    with pytest.raises(ValueError):
+        O.pack_zeros(z + 2 ** bits, bits)
+
+
+def _padded_case(n, n_pad, out=24, tokens=600, seed=31):
+    W, x = S.small_case(out, n, tokens, seed=seed, rank=6, frac=0.03, mult=15.0)
+    Wp, xp = O.pad_layer(W, x, n_pad)
+    return W, x, Wp, xp
+
+
+def test_padding_makes_dead_inputs_damped_by_the_padded_mean():
+    n, n_pad, damp = 300, 384, 0.01
+    W, x, Wp, xp = _padded_case(n, n_pad)
+    assert np.array_equal(Wp[:, :n], W) and not Wp[:, n:].any()
+    H, Hp = O.hessian(x), O.hessian(xp)
+    assert np.array_equal(Hp[:n, :n], H) and not Hp[n:].any() and not Hp[:, n:].any()
+    prep = O.prepare(Hp, damp, False)
+    assert np.array_equal(np.flatnonzero(prep.dead), np.arange(n, n_pad))
+    # the padded inputs' unit diagonal counts in the mean like any other input's
+    lam = damp * (np.trace(H) + (n_pad - n)) / n_pad
+    assert prep.lam == pytest.approx(lam, rel=1e-13)
+    # U is block diagonal: the real block is the upper factor of (H + lam I)^-1
+    # (numpy's inverse and Cholesky: the definition), the padded block (1 + lam)^-1/2 I
+    U_ref = np.linalg.cholesky(np.linalg.inv(H + lam * np.eye(n))).T
+    scale = np.abs(U_ref).max()
+    assert np.abs(prep.U[:n, :n] - U_ref).max() <= 1e-10 * scale
+    assert not prep.U[:n, n:].any() and not prep.U[n:, :n].any()
+    assert np.allclose(prep.U[n:, n:], np.eye(n_pad - n) / np.sqrt(1.0 + lam), rtol=1e-14, atol=0)
+    # planted mistake: damping by the mean over the real inputs alone misses the pin
+    lam_bad = damp * np.trace(H) / n
+    U_bad = np.linalg.cholesky(np.linalg.inv(H + lam_bad * np.eye(n))).T
+    assert np.abs(prep.U[:n, :n] - U_bad).max() > 1e-6 * scale
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_padded_layer_with_one_group_per_row_is_the_unpadded_layer(sym):
+    # one group per row: its parameters come from the whole initial row, and zero
+    # columns change neither its extremes (the range always holds 0) nor its largest
+    # magnitude, so the padded layer's real columns are the unpadded layer quantized
+    # with the padded damping
+    n, n_pad, damp = 300, 320, 0.01
+    W, x, Wp, xp = _padded_case(n, n_pad, seed=33)
+    res = O.gptq_layer(Wp, xp, 4, -1, sym, False, damp, with_rtn=False)
+    H = O.hessian(x)
+    lam = damp * (np.trace(H) + (n_pad - n)) / n_pad
+    prep_u = O.prepare(H, lam / np.mean(np.diag(H)), False)
+    sw = O.sweep(np.asarray(W, np.float64), prep_u.U, 4, -1, sym, 128)
+    assert np.array_equal(res.sw.scales, sw.scales) and np.array_equal(res.sw.zeros, sw.zeros)
+    assert np.mean(res.codes[:, :n] != sw.codes) <= 1e-3
+    # the padded columns take the zero point's code, which dequantizes to 0
+    assert np.array_equal(res.codes[:, n:], np.repeat(res.sw.zeros[0].astype(np.uint8)[:, None], n_pad - n, 1))
+    What = O.dequantize(res.qweight, res.scales, res.zeros, res.g_idx, 4, n_pad)
+    assert not What[:, n:].any()
+
+
+@pytest.mark.parametrize("bits,gs,sym,act", [(4, 128, False, False), (3, 64, True, True), (2, 32, False, True)])
+def test_padded_columns_quantize_to_zero_and_carry_no_error(bits, gs, sym, act):
+    n = 300
+    n_pad = -(-n // max(32, gs)) * max(32, gs)
+    W, x, Wp, xp = _padded_case(n, n_pad, seed=35 + bits)
+    res = O.gptq_layer(Wp, xp, bits, gs, sym, act, with_rtn=False)
+    pad = np.arange(n, n_pad)
+    What = O.dequantize(res.qweight, res.scales, res.zeros, res.g_idx, bits, n_pad)
+    assert not What[:, pad].any()
+    # processing positions of the padded columns: no error leaves them
+    pos = np.argsort(res.perm)[pad]
+    assert not res.sw.err[:, pos].any()
+    # their groups continue the processing order's numbering
+    assert np.array_equal(res.g_idx[pad], (pos // gs).astype(np.int32))
