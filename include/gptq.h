@@ -13,6 +13,8 @@
  *   gptq_quantize_layer       column sweep, lazy trailing update,
  *                             packed qweight / fp16 scales, zeros / g_idx
  *   gptq_pack                 the bit-packing step on its own
+ *   gptq_pack_zeros           zero points packed into int32 words
+ *   *_padded                  the same for a zero-padded layer ("Limites de GPTQ")
  *
  * Conventions shared by every call
  * --------------------------------
@@ -201,6 +203,68 @@ GPTQ_API int gptq_quantize_layer(const void* W, int w_dtype, int out, int n, con
  * bits in {2, 3, 4, 8}; n*bits % 32 == 0; codes must be < 2^bits.
  */
 GPTQ_API int gptq_pack(const uint8_t* codes, int out, int n, int bits, int32_t* qweight, void* stream);
+
+/*
+ * Zero padding of a layer whose width the group size or the packing does not
+ * divide.  "polydesk.ai/glossaire/gptq", section "Limites de GPTQ" (problems of
+ * divisibility): when a width is not a multiple of the group size, the weights
+ * are padded with zeros.  The padded layer has n >= w_cols input columns: W's
+ * columns w_cols .. n-1 and X's rows x_rows .. n-1 are zero.  The calls below
+ * compute exactly what the unpadded calls compute on those zero-padded arrays,
+ * without the arrays being formed:
+ *
+ * - gptq_hessian_accumulate_padded: H [n, n] from X's x_rows rows
+ *   (1 <= x_rows <= n).  Rows and columns x_rows .. n-1 of H receive nothing
+ *   (the caller zeroed H, so they stay 0); hdiag entries x_rows .. n-1 are not
+ *   touched.  Everything else as gptq_hessian_accumulate (X is [x_rows, ld_x]).
+ * - gptq_hessian_accumulate_host_padded: the same with X in host memory; only
+ *   x_rows rows cross, and the staging halves hold x_rows x C bf16.
+ * - gptq_prepare on that H (n) is the ordinary call: the padded inputs have a
+ *   zero diagonal, so step 1 makes them dead inputs, counted in the mean of the
+ *   damping like every other input.
+ * - gptq_quantize_layer_padded: W is [out, w_cols] (row stride w_cols,
+ *   1 <= w_cols <= n); columns w_cols .. n-1 are read as zeros.  Outputs are
+ *   those of the padded layer: qweight [n*bits/32, out], scales / zeros [G, out]
+ *   with G = n / group_size, g_idx [n], codes [out, n].  A padded column gets the
+ *   zero point's code, which dequantizes to 0.
+ * Pick n = the next multiple of max(32, group_size) (32 for group_size -1).
+ */
+GPTQ_API int gptq_hessian_accumulate_padded(float* H, double* hdiag, int n, const void* X, int x_rows,
+                                            int64_t ld_x, int64_t tokens, int32_t* d_status, void* stream);
+GPTQ_API int gptq_hessian_accumulate_host_padded(float* H, double* hdiag, int n, const void* X_host, int x_rows,
+                                                 int64_t ld_x, int64_t tokens, void* staging, size_t staging_bytes,
+                                                 int32_t* d_status, void* stream);
+GPTQ_API int gptq_quantize_layer_padded(const void* W, int w_dtype, int out, int w_cols, int n, const float* U,
+                                        const int32_t* perm, const uint8_t* dead, int bits, int group_size,
+                                        int sym, int block, int32_t* qweight, uint16_t* scales, uint16_t* zeros,
+                                        int32_t* g_idx, uint8_t* codes, float* err_sq, void* ws, size_t ws_bytes,
+                                        int32_t* d_status, void* stream);
+
+/*
+ * gptq_pack_zeros - the zero points packed into int32 words along the output
+ * dimension, for checkpoint layouts that store them that way.  The pages store
+ * scale and zero point in FP16 ("dev.ayinedjimi-consultants.fr ...
+ * ia-quantization-gptq-gguf-awq", "Calibration et dataset"), which is what
+ * gptq_quantize_layer writes, and warn that checkpoints of different tool
+ * versions are not all compatible ("polydesk.ai/glossaire/gptq", "Limites de
+ * GPTQ"); this call converts the fp16 zeros to the packed integer form.
+ *
+ *   zeros        fp16 (as uint16) [groups, out], integers in [0, 2^bits - 1]
+ *                (as gptq_quantize_layer writes them).
+ *   qzeros       int32 [groups, out*bits/32] output: row g is the little-endian
+ *                bit stream of (zeros[g][o] - zero_offset) mod 2^bits, column o
+ *                at stream bits o*bits ... (bit (o*bits) mod 32 of word
+ *                floor(o*bits/32)); a 3-bit value may continue into the next word.
+ *   zero_offset  0: the zero points as they are; 1: zero point - 1, the
+ *                convention of older checkpoints (a zero point of 0 wraps to
+ *                2^bits - 1).
+ *   bits in {2, 3, 4, 8}; out*bits % 32 == 0.
+ *   d_status     may be NULL; a zero that is not an integer in [0, 2^bits - 1]
+ *                records GPTQ_ERR_INVALID_ARG (info = g*out + o) and is packed
+ *                masked to bits.
+ */
+GPTQ_API int gptq_pack_zeros(const uint16_t* zeros, int groups, int out, int bits, int zero_offset,
+                             int32_t* qzeros, int32_t* d_status, void* stream);
 
 /*
  * gptq_quantize_layer_noalloc - gptq_quantize_layer without a caller workspace.

@@ -61,25 +61,38 @@ int gptq_status_read(const int32_t* d_status, void* stream, int32_t* info) {
   return h[0];
 }
 
-int gptq_hessian_accumulate(float* H, double* hdiag, int n, const void* X, int64_t ld_x, int64_t tokens,
-                            int32_t* d_status, void* stream) {
-  if (H == nullptr || n <= 0 || tokens < 0) return GPTQ_ERR_INVALID_ARG;
+int gptq_hessian_accumulate_padded(float* H, double* hdiag, int n, const void* X, int x_rows, int64_t ld_x,
+                                   int64_t tokens, int32_t* d_status, void* stream) {
+  if (H == nullptr || n <= 0 || x_rows <= 0 || x_rows > n || tokens < 0) return GPTQ_ERR_INVALID_ARG;
   if (tokens == 0) return GPTQ_OK;
   if (X == nullptr || ld_x < tokens || ld_x % 8 != 0 || !aligned(X, 16)) return GPTQ_ERR_INVALID_ARG;
-  int rc = launch_hessian(H, n, X, ld_x, tokens, d_status, as_stream(stream));
+  int rc = launch_hessian(H, n, X, x_rows, ld_x, tokens, d_status, as_stream(stream));
   if (rc != GPTQ_OK) return rc;
-  if (hdiag) rc = launch_hessian_diag64(hdiag, n, X, ld_x, tokens, d_status, as_stream(stream));
+  if (hdiag) rc = launch_hessian_diag64(hdiag, x_rows, X, ld_x, tokens, d_status, as_stream(stream));
   return rc;
+}
+
+int gptq_hessian_accumulate(float* H, double* hdiag, int n, const void* X, int64_t ld_x, int64_t tokens,
+                            int32_t* d_status, void* stream) {
+  return gptq_hessian_accumulate_padded(H, hdiag, n, X, n, ld_x, tokens, d_status, stream);
+}
+
+int gptq_hessian_accumulate_host_padded(float* H, double* hdiag, int n, const void* X_host, int x_rows,
+                                        int64_t ld_x, int64_t tokens, void* staging, size_t staging_bytes,
+                                        int32_t* d_status, void* stream) {
+  if (H == nullptr || n <= 0 || x_rows <= 0 || x_rows > n || tokens < 0) return GPTQ_ERR_INVALID_ARG;
+  if (tokens == 0) return GPTQ_OK;
+  if (X_host == nullptr || ld_x < tokens) return GPTQ_ERR_INVALID_ARG;
+  if (staging == nullptr || !aligned(staging, 256) || hessian_host_chunk(x_rows, staging_bytes) < 64)
+    return GPTQ_ERR_WORKSPACE;
+  return launch_hessian_host(H, hdiag, n, X_host, x_rows, ld_x, tokens, staging, staging_bytes, d_status,
+                             as_stream(stream));
 }
 
 int gptq_hessian_accumulate_host(float* H, double* hdiag, int n, const void* X_host, int64_t ld_x, int64_t tokens,
                                  void* staging, size_t staging_bytes, int32_t* d_status, void* stream) {
-  if (H == nullptr || n <= 0 || tokens < 0) return GPTQ_ERR_INVALID_ARG;
-  if (tokens == 0) return GPTQ_OK;
-  if (X_host == nullptr || ld_x < tokens) return GPTQ_ERR_INVALID_ARG;
-  if (staging == nullptr || !aligned(staging, 256) || hessian_host_chunk(n, staging_bytes) < 64)
-    return GPTQ_ERR_WORKSPACE;
-  return launch_hessian_host(H, hdiag, n, X_host, ld_x, tokens, staging, staging_bytes, d_status, as_stream(stream));
+  return gptq_hessian_accumulate_host_padded(H, hdiag, n, X_host, n, ld_x, tokens, staging, staging_bytes, d_status,
+                                             stream);
 }
 
 size_t gptq_prepare_workspace_size(int n) { return n > 0 ? prepare_ws_bytes(n) : 0; }
@@ -99,22 +112,30 @@ size_t gptq_quantize_workspace_size(int out, int n, int block) {
   return quantize_ws_bytes(out, n, block);
 }
 
-int gptq_quantize_layer(const void* W, int w_dtype, int out, int n, const float* U, const int32_t* perm,
-                        const uint8_t* dead, int bits, int group_size, int sym, int block, int32_t* qweight,
-                        uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq,
-                        void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+int gptq_quantize_layer_padded(const void* W, int w_dtype, int out, int w_cols, int n, const float* U,
+                               const int32_t* perm, const uint8_t* dead, int bits, int group_size, int sym, int block,
+                               int32_t* qweight, uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes,
+                               float* err_sq, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
   if (W == nullptr || U == nullptr || qweight == nullptr || scales == nullptr || zeros == nullptr ||
       g_idx == nullptr || d_status == nullptr)
     return GPTQ_ERR_INVALID_ARG;
-  if (out <= 0 || n <= 0) return GPTQ_ERR_INVALID_ARG;
+  if (out <= 0 || n <= 0 || w_cols <= 0 || w_cols > n) return GPTQ_ERR_INVALID_ARG;
   if (w_dtype != GPTQ_F32 && w_dtype != GPTQ_F16 && w_dtype != GPTQ_BF16) return GPTQ_ERR_INVALID_ARG;
   if (!valid_bits(bits) || !valid_gs(group_size)) return GPTQ_ERR_UNSUPPORTED;
   if (block != 128) return GPTQ_ERR_UNSUPPORTED;
   if (n % 32 != 0) return GPTQ_ERR_UNSUPPORTED;
   if (group_size > 0 && (n % group_size != 0 || block % group_size != 0)) return GPTQ_ERR_UNSUPPORTED;
   if (ws == nullptr || ws_bytes < quantize_ws_bytes(out, n, block) || !aligned(ws, 256)) return GPTQ_ERR_WORKSPACE;
-  return launch_quantize(W, w_dtype, out, n, U, perm, dead, bits, group_size, sym ? 1 : 0, block, qweight, scales,
-                         zeros, g_idx, codes, err_sq, ws, d_status, as_stream(stream));
+  return launch_quantize(W, w_dtype, out, w_cols, n, U, perm, dead, bits, group_size, sym ? 1 : 0, block, qweight,
+                         scales, zeros, g_idx, codes, err_sq, ws, d_status, as_stream(stream));
+}
+
+int gptq_quantize_layer(const void* W, int w_dtype, int out, int n, const float* U, const int32_t* perm,
+                        const uint8_t* dead, int bits, int group_size, int sym, int block, int32_t* qweight,
+                        uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq,
+                        void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  return gptq_quantize_layer_padded(W, w_dtype, out, n, n, U, perm, dead, bits, group_size, sym, block, qweight,
+                                    scales, zeros, g_idx, codes, err_sq, ws, ws_bytes, d_status, stream);
 }
 
 int gptq_pack(const uint8_t* codes, int out, int n, int bits, int32_t* qweight, void* stream) {
@@ -122,6 +143,15 @@ int gptq_pack(const uint8_t* codes, int out, int n, int bits, int32_t* qweight, 
   if (!valid_bits(bits)) return GPTQ_ERR_UNSUPPORTED;
   if (((int64_t)n * bits) % 32 != 0) return GPTQ_ERR_UNSUPPORTED;
   return launch_pack(codes, nullptr, out, n, n, bits, qweight, nullptr, as_stream(stream));
+}
+
+int gptq_pack_zeros(const uint16_t* zeros, int groups, int out, int bits, int zero_offset, int32_t* qzeros,
+                    int32_t* d_status, void* stream) {
+  if (zeros == nullptr || qzeros == nullptr || groups <= 0 || out <= 0) return GPTQ_ERR_INVALID_ARG;
+  if (zero_offset != 0 && zero_offset != 1) return GPTQ_ERR_INVALID_ARG;
+  if (!valid_bits(bits)) return GPTQ_ERR_UNSUPPORTED;
+  if (((int64_t)out * bits) % 32 != 0) return GPTQ_ERR_UNSUPPORTED;
+  return launch_pack_zeros(zeros, groups, out, bits, zero_offset, qzeros, d_status, as_stream(stream));
 }
 
 }  // extern "C"

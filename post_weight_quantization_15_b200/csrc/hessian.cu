@@ -263,11 +263,13 @@ int launch_hessian_diag64(double* hdiag, int n, const void* X, int64_t ld_x, int
   return GPTQ_OK;
 }
 
-int launch_hessian(float* H, int n, const void* X, int64_t ld_x, int64_t tokens, int32_t* st,
+int launch_hessian(float* H, int n, const void* X, int x_rows, int64_t ld_x, int64_t tokens, int32_t* st,
                    cudaStream_t s) {
   CUtensorMap map;
   // One map serves both operands: its box is 64 tokens x 128 rows; the B tile is two boxes.
-  int rc = make_tmap_2d(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)tokens, (uint64_t)n,
+  // The map holds X's x_rows rows; tiles reaching rows x_rows .. n-1 (zero padding) load
+  // the map's zero fill, so those rows and columns of H receive nothing.
+  int rc = make_tmap_2d(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)tokens, (uint64_t)x_rows,
                         (uint64_t)ld_x * 2, HKB, HBM_, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != GPTQ_OK) return rc;
   const int TB = (int)cdiv(n, HBN);

@@ -45,9 +45,10 @@ int64_t hessian_host_chunk(int n, size_t staging_bytes) {
   return per_half / 64 * 64;
 }
 
-int launch_hessian_host(float* H, double* hdiag, int n, const void* X_host, int64_t ld_x_host, int64_t tokens,
-                        void* staging, size_t staging_bytes, int32_t* st, cudaStream_t s) {
-  const int64_t chunk = std::min(hessian_host_chunk(n, staging_bytes), (int64_t)align_up((size_t)tokens, 64));
+int launch_hessian_host(float* H, double* hdiag, int n, const void* X_host, int x_rows, int64_t ld_x_host,
+                        int64_t tokens, void* staging, size_t staging_bytes, int32_t* st, cudaStream_t s) {
+  // only X's x_rows rows cross; the rest of H's n rows are zero padding
+  const int64_t chunk = std::min(hessian_host_chunk(x_rows, staging_bytes), (int64_t)align_up((size_t)tokens, 64));
   if (chunk < 64) return GPTQ_ERR_WORKSPACE;
   CopyStream* cs = nullptr;
   int rc = copy_stream(&cs);
@@ -60,14 +61,14 @@ int launch_hessian_host(float* H, double* hdiag, int n, const void* X_host, int6
   for (int64_t t0 = 0; t0 < tokens; t0 += chunk, ++i) {
     const int b = i & 1;
     const int64_t cw = std::min(chunk, tokens - t0);
-    char* dst = static_cast<char*>(staging) + (size_t)b * (size_t)n * (size_t)chunk * 2;
+    char* dst = static_cast<char*>(staging) + (size_t)b * (size_t)x_rows * (size_t)chunk * 2;
     if (i >= 2) GPTQ_CUDA_TRY(cudaStreamWaitEvent(cs->s, cs->consumed[b], 0));   // that half is free again
     GPTQ_CUDA_TRY(cudaMemcpy2DAsync(dst, (size_t)chunk * 2, src + t0 * 2, (size_t)ld_x_host * 2, (size_t)cw * 2,
-                                    (size_t)n, cudaMemcpyHostToDevice, cs->s));
+                                    (size_t)x_rows, cudaMemcpyHostToDevice, cs->s));
     GPTQ_CUDA_TRY(cudaEventRecord(cs->copied[b], cs->s));
     GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, cs->copied[b], 0));
-    rc = launch_hessian(H, n, dst, chunk, cw, st, s);
-    if (rc == GPTQ_OK && hdiag != nullptr) rc = launch_hessian_diag64(hdiag, n, dst, chunk, cw, st, s);
+    rc = launch_hessian(H, n, dst, x_rows, chunk, cw, st, s);
+    if (rc == GPTQ_OK && hdiag != nullptr) rc = launch_hessian_diag64(hdiag, x_rows, dst, chunk, cw, st, s);
     if (rc != GPTQ_OK) return rc;
     GPTQ_CUDA_TRY(cudaEventRecord(cs->consumed[b], s));
   }

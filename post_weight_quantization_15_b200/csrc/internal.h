@@ -7,13 +7,14 @@
 namespace gptq {
 
 // ---- K1: Hessian -----------------------------------------------------------
-int launch_hessian(float* H, int n, const void* X, int64_t ld_x, int64_t tokens, int32_t* st,
+// H [n, n] from X's first x_rows rows (x_rows <= n; the rows after them are zero padding).
+int launch_hessian(float* H, int n, const void* X, int x_rows, int64_t ld_x, int64_t tokens, int32_t* st,
                    cudaStream_t s);
 int launch_hessian_diag64(double* hdiag, int n, const void* X, int64_t ld_x, int64_t tokens,
                           int32_t* st, cudaStream_t s);
 int64_t hessian_host_chunk(int n, size_t staging_bytes);
-int launch_hessian_host(float* H, double* hdiag, int n, const void* X_host, int64_t ld_x_host, int64_t tokens,
-                        void* staging, size_t staging_bytes, int32_t* st, cudaStream_t s);
+int launch_hessian_host(float* H, double* hdiag, int n, const void* X_host, int x_rows, int64_t ld_x_host,
+                        int64_t tokens, void* staging, size_t staging_bytes, int32_t* st, cudaStream_t s);
 
 // ---- K2: prepare -------------------------------------------------------------
 size_t prepare_ws_bytes(int n);
@@ -22,12 +23,15 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
 
 // ---- K0/K3/K4/K5: quantize ---------------------------------------------------
 size_t quantize_ws_bytes(int out, int n, int block);
-int launch_quantize(const void* W, int w_dtype, int out, int n, const float* U, const int32_t* perm,
+// W [out, w_cols] (w_cols <= n; columns w_cols .. n-1 are zero padding).
+int launch_quantize(const void* W, int w_dtype, int out, int w_cols, int n, const float* U, const int32_t* perm,
                     const uint8_t* dead, int bits, int gs, int sym, int block, int32_t* qweight,
                     uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq,
                     void* ws, int32_t* st, cudaStream_t s);
 int launch_pack(const uint8_t* codes, const int32_t* invperm, int out, int n, int ld_codes, int bits,
                 int32_t* qweight, const int32_t* st, cudaStream_t s);
+int launch_pack_zeros(const uint16_t* zeros, int groups, int out, int bits, int zero_offset, int32_t* qzeros,
+                      int32_t* st, cudaStream_t s);
 
 // ---- tensor-core GEMM: C -= A . B^T in 3 x TF32 (operands pre-split) ---------
 // store = false: C -= A.B^T; store = true: C = A.B^T (C may be null then, if Chi/Clo are given).

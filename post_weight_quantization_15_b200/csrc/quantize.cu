@@ -137,10 +137,12 @@ __device__ __forceinline__ float code_from_q(float q, QParams p, int bits, bool 
 // K0: Wf[r][k] = W[r][perm[k]] (0 for dead inputs), invperm, g_idx.
 // ---------------------------------------------------------------------------
 // Four consecutive columns per thread (n % 4 == 0): 16-byte stores, and the loads of a
-// warp cover 128 consecutive columns of a row for the identity order.
+// warp cover 128 consecutive columns of a row for the identity order.  W has w_cols
+// columns (its row stride); columns w_cols .. n-1 are the zero padding of a layer
+// whose width the group size or the packing does not divide.
 template <typename T>
-__global__ void ingest_kernel(const T* W, int out, int n, const int32_t* perm, const uint8_t* dead, int gs,
-                              float* Wf, int32_t* invperm, int32_t* g_idx, int32_t* st) {
+__global__ void ingest_kernel(const T* W, int out, int w_cols, int n, const int32_t* perm, const uint8_t* dead,
+                              int gs, float* Wf, int32_t* invperm, int32_t* g_idx, int32_t* st) {
   if (has_error(st)) return;
   const int k0 = 4 * (blockIdx.x * 32 + threadIdx.x);
   const int r = blockIdx.y * 8 + threadIdx.y;
@@ -156,11 +158,11 @@ __global__ void ingest_kernel(const T* W, int out, int n, const int32_t* perm, c
     }
   }
   if (r >= out) return;
-  const T* row = W + (int64_t)r * n;
+  const T* row = W + (int64_t)r * w_cols;
   float v[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
-    v[u] = load_as_float<T>(row + src[u]);
+    v[u] = src[u] < w_cols ? load_as_float<T>(row + src[u]) : 0.f;
     if (!isfinite(v[u])) set_error(st, GPTQ_ERR_NONFINITE, src[u], STAGE_INGEST);
     if (dead && dead[src[u]]) v[u] = 0.f;
   }
@@ -555,6 +557,34 @@ __global__ void pack_kernel(const uint8_t* codes, const int32_t* invperm, int ou
   }
 }
 
+// Zero points packed along the output dimension: qzeros[g][w] holds the bit stream of
+// (zeros[g][o] - zero_offset) mod 2^bits for o = 0 .. out-1 (column o at stream bits
+// o*bits .., codes straddling words as in qweight).  One thread per output word.  A zero
+// that is not an integer in [0, 2^bits - 1] is reported (GPTQ_ERR_INVALID_ARG, info =
+// group * out + column) and packed masked like the others.
+__global__ void pack_zeros_kernel(const uint16_t* zeros, int groups, int out, int bits, int zero_offset,
+                                  int32_t* qzeros, int32_t* st) {
+  if (has_error(st)) return;
+  const int words = out * bits / 32;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)groups * words) return;
+  const int g = (int)(i / words), wi = (int)(i % words);
+  const int pos0 = wi * 32;
+  const int o_lo = pos0 / bits, o_hi = min((pos0 + 31) / bits, out - 1);
+  const uint32_t mask = (1u << bits) - 1u;
+  const uint16_t* zrow = zeros + (int64_t)g * out;
+  uint64_t acc = 0;
+  for (int o = o_lo; o <= o_hi; ++o) {
+    const float z = __half2float(__ushort_as_half(zrow[o]));
+    if (!(z >= 0.f && z <= (float)mask && z == rintf(z)))
+      set_error(st, GPTQ_ERR_INVALID_ARG, (int)((int64_t)g * out + o), STAGE_PACK);
+    const uint64_t v = (uint32_t)((int)z - zero_offset) & mask;
+    const int sh = o * bits - pos0;  // negative for a code straddling in from the previous word
+    if (sh >= 0) acc |= v << sh; else acc |= v >> (-sh);
+  }
+  qzeros[i] = (int32_t)(uint32_t)(acc & 0xFFFFFFFFull);
+}
+
 // Optional output: codes in the original column order.
 __global__ void codes_out_kernel(const uint8_t* codes_p, const int32_t* invperm, int out, int n, uint8_t* codes,
                                  const int32_t* st) {
@@ -583,7 +613,15 @@ int launch_pack(const uint8_t* codes, const int32_t* invperm, int out, int n, in
   return GPTQ_OK;
 }
 
-int launch_quantize(const void* W, int w_dtype, int out, int n, const float* U, const int32_t* perm,
+int launch_pack_zeros(const uint16_t* zeros, int groups, int out, int bits, int zero_offset, int32_t* qzeros,
+                      int32_t* st, cudaStream_t s) {
+  const int64_t total = (int64_t)groups * (out * bits / 32);
+  pack_zeros_kernel<<<(unsigned)cdiv(total, 256), 256, 0, s>>>(zeros, groups, out, bits, zero_offset, qzeros, st);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
+int launch_quantize(const void* W, int w_dtype, int out, int w_cols, int n, const float* U, const int32_t* perm,
                     const uint8_t* dead, int bits, int gs, int sym, int block, int32_t* qweight,
                     uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq,
                     void* ws, int32_t* st, cudaStream_t s) {
@@ -592,11 +630,11 @@ int launch_quantize(const void* W, int w_dtype, int out, int n, const float* U, 
   {
     dim3 blk(32, 8), grd((unsigned)cdiv(n, 128), (unsigned)cdiv(std::max(out, 1), 8));
     if (w_dtype == GPTQ_F32)
-      ingest_kernel<float><<<grd, blk, 0, s>>>(static_cast<const float*>(W), out, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
+      ingest_kernel<float><<<grd, blk, 0, s>>>(static_cast<const float*>(W), out, w_cols, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
     else if (w_dtype == GPTQ_F16)
-      ingest_kernel<__half><<<grd, blk, 0, s>>>(static_cast<const __half*>(W), out, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
+      ingest_kernel<__half><<<grd, blk, 0, s>>>(static_cast<const __half*>(W), out, w_cols, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
     else
-      ingest_kernel<__nv_bfloat16><<<grd, blk, 0, s>>>(static_cast<const __nv_bfloat16*>(W), out, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
+      ingest_kernel<__nv_bfloat16><<<grd, blk, 0, s>>>(static_cast<const __nv_bfloat16*>(W), out, w_cols, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
     GPTQ_LAUNCH_CHECK();
   }
   if (err_sq) GPTQ_CUDA_TRY(cudaMemsetAsync(err_sq, 0, (size_t)out * 4, s));

@@ -12,7 +12,12 @@ The calls mirror include/gptq.h:
     quantize_layer(W, prep, bits, group_size, sym, block=128)
                                                   -> QuantizedLayer(qweight, scales, zeros, g_idx, ...)
     pack(codes, bits)                             -> qweight
-    gptq_quantize(W, X, ...)                      the whole path for one layer
+    pack_zeros(zeros, bits, zero_offset=0)        -> qzeros
+    gptq_quantize(W, X, ..., pad=False)           the whole path for one layer
+
+Zero padding: H may be wider than X has rows, and U wider than W has columns; the
+calls then go to the *_padded entry points, which read the missing rows / columns
+as zeros (padded_width gives the width to pad to).
 """
 from __future__ import annotations
 
@@ -88,6 +93,14 @@ def lib() -> ctypes.CDLL:
     L.gptq_quantize_layer.argtypes = [P, I, I, I, P, P, P, I, I, I, I, P, P, P, P, P, P, P, SZ, P, P]
     L.gptq_pack.restype = I
     L.gptq_pack.argtypes = [P, I, I, I, P, P]
+    L.gptq_hessian_accumulate_padded.restype = I
+    L.gptq_hessian_accumulate_padded.argtypes = [P, P, I, P, I, I64, I64, P, P]
+    L.gptq_hessian_accumulate_host_padded.restype = I
+    L.gptq_hessian_accumulate_host_padded.argtypes = [P, P, I, P, I, I64, I64, P, SZ, P, P]
+    L.gptq_quantize_layer_padded.restype = I
+    L.gptq_quantize_layer_padded.argtypes = [P, I, I, I, I, P, P, P, I, I, I, I, P, P, P, P, P, P, P, SZ, P, P]
+    L.gptq_pack_zeros.restype = I
+    L.gptq_pack_zeros.argtypes = [P, I, I, I, I, P, P, P]
     L.gptq_quantize_layer_noalloc.restype = I
     L.gptq_quantize_layer_noalloc.argtypes = [P, I, I, I, P, P, P, I, I, I, I, P, P, P, P, P, P, P, P]
     _lib = L
@@ -157,19 +170,40 @@ def raise_on_status(st: torch.Tensor, where: str, stream=None):
 # --------------------------------------------------------------------------- #
 # K1
 # --------------------------------------------------------------------------- #
+def padded_width(n: int, group_size: int) -> int:
+    """The width a layer of n inputs is zero-padded to: the next multiple of
+    max(32, group_size) (32 for group_size -1)."""
+    m = 32 if group_size == -1 else max(32, int(group_size))
+    return (int(n) + m - 1) // m * m
+
+
+def _check_h(H: torch.Tensor, rows: int, hdiag: Optional[torch.Tensor]) -> int:
+    n = H.shape[0] if H.dim() == 2 else -1
+    if H.dtype != torch.float32 or H.dim() != 2 or H.shape[1] != n or n < rows or not H.is_contiguous():
+        raise ValueError("H must be a contiguous fp32 [n, n] tensor with n >= the rows of X")
+    if hdiag is not None and (hdiag.dtype != torch.float64 or hdiag.numel() != n):
+        raise ValueError("hdiag must be fp64 [n]")
+    return n
+
+
 def hessian_accumulate(H: torch.Tensor, X: torch.Tensor, hdiag: Optional[torch.Tensor] = None,
                        status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """H += 2 . X . X^T.  H fp32 [n, n]; X bf16 [n, tokens] (row stride may exceed tokens)."""
+    """H += 2 . X . X^T.  H fp32 [n, n]; X bf16 [rows, tokens] (row stride may exceed tokens).
+
+    rows < n: X is zero-padded to n rows (gptq_hessian_accumulate_padded).
+    """
     _require_cuda(H, X, hdiag, status)
     if X.dtype != torch.bfloat16 or X.dim() != 2 or X.stride(1) != 1:
         raise ValueError("X must be a bf16 [n, tokens] tensor with contiguous rows")
-    n = X.shape[0]
-    if H.dtype != torch.float32 or tuple(H.shape) != (n, n) or not H.is_contiguous():
-        raise ValueError("H must be a contiguous fp32 [n, n] tensor")
-    if hdiag is not None and (hdiag.dtype != torch.float64 or hdiag.numel() != n):
-        raise ValueError("hdiag must be fp64 [n]")
-    _check(lib().gptq_hessian_accumulate(_ptr(H), _ptr(hdiag), n, _ptr(X), X.stride(0), X.shape[1],
-                                         _ptr(status), _stream(stream)), "gptq_hessian_accumulate")
+    rows = X.shape[0]
+    n = _check_h(H, rows, hdiag)
+    if rows == n:
+        rc = lib().gptq_hessian_accumulate(_ptr(H), _ptr(hdiag), n, _ptr(X), X.stride(0), X.shape[1],
+                                           _ptr(status), _stream(stream))
+    else:
+        rc = lib().gptq_hessian_accumulate_padded(_ptr(H), _ptr(hdiag), n, _ptr(X), rows, X.stride(0), X.shape[1],
+                                                  _ptr(status), _stream(stream))
+    _check(rc, "gptq_hessian_accumulate")
     return H
 
 
@@ -185,17 +219,15 @@ def hessian_accumulate_host(H: torch.Tensor, X_host: torch.Tensor, hdiag: Option
     if X_host.device.type != "cpu" or X_host.dtype not in (torch.bfloat16, torch.int16, torch.uint16) \
             or X_host.dim() != 2 or X_host.stride(1) != 1:
         raise ValueError("X_host must be a host [n, tokens] bf16 tensor with contiguous rows")
-    n = X_host.shape[0]
-    if H.dtype != torch.float32 or tuple(H.shape) != (n, n) or not H.is_contiguous():
-        raise ValueError("H must be a contiguous fp32 [n, n] tensor")
-    if hdiag is not None and (hdiag.dtype != torch.float64 or hdiag.numel() != n):
-        raise ValueError("hdiag must be fp64 [n]")
+    rows = X_host.shape[0]
+    n = _check_h(H, rows, hdiag)
     if staging is None:
         chunk = max(64, min(int(chunk_tokens), (X_host.shape[1] + 63) // 64 * 64)) // 64 * 64
-        staging = workspace(2 * n * chunk * 2, H.device)
-    _check(lib().gptq_hessian_accumulate_host(_ptr(H), _ptr(hdiag), n, ctypes.c_void_p(X_host.data_ptr()),
-                                              X_host.stride(0), X_host.shape[1], _ptr(staging), staging.numel(),
-                                              _ptr(status), _stream(stream)), "gptq_hessian_accumulate_host")
+        staging = workspace(2 * rows * chunk * 2, H.device)
+    _check(lib().gptq_hessian_accumulate_host_padded(_ptr(H), _ptr(hdiag), n, ctypes.c_void_p(X_host.data_ptr()),
+                                                     rows, X_host.stride(0), X_host.shape[1], _ptr(staging),
+                                                     staging.numel(), _ptr(status), _stream(stream)),
+           "gptq_hessian_accumulate_host")
     return H
 
 
@@ -275,20 +307,23 @@ def quantize_layer(W: torch.Tensor, prep: Prepared, bits: int = 4, group_size: i
     _require_cuda(W, ws)
     if W.dim() != 2 or not W.is_contiguous() or W.dtype not in _DTYPE_CODE:
         raise ValueError("W must be a contiguous fp32/fp16/bf16 [out, n] tensor")
-    o, n = W.shape
-    if prep.U.shape[0] != n:
-        raise ValueError("W and U disagree on n")
+    o, w_cols = W.shape
+    n = prep.U.shape[0]
+    if w_cols > n:
+        raise ValueError("W has more columns than U")
     dev = W.device
     need = quantize_workspace_size(o, n, block)
     if ws is None or ws.numel() < need:
         ws = workspace(need, dev)
     if out is None:
         out = alloc_quantized(o, n, bits, group_size, sym, dev, want_codes, want_err)
-    _check(lib().gptq_quantize_layer(_ptr(W), _DTYPE_CODE[W.dtype], o, n, _ptr(prep.U), _ptr(prep.perm),
-                                     _ptr(prep.dead), int(bits), int(group_size), int(bool(sym)), int(block),
-                                     _ptr(out.qweight), _ptr(out.scales), _ptr(out.zeros), _ptr(out.g_idx),
-                                     _ptr(out.codes), _ptr(out.err_sq), _ptr(ws), ws.numel(), _ptr(prep.status),
-                                     _stream(stream)), "gptq_quantize_layer")
+    # w_cols < n: W is zero-padded to n columns (gptq_quantize_layer_padded)
+    _check(lib().gptq_quantize_layer_padded(_ptr(W), _DTYPE_CODE[W.dtype], o, w_cols, n, _ptr(prep.U),
+                                            _ptr(prep.perm), _ptr(prep.dead), int(bits), int(group_size),
+                                            int(bool(sym)), int(block), _ptr(out.qweight), _ptr(out.scales),
+                                            _ptr(out.zeros), _ptr(out.g_idx), _ptr(out.codes), _ptr(out.err_sq),
+                                            _ptr(ws), ws.numel(), _ptr(prep.status), _stream(stream)),
+           "gptq_quantize_layer")
     return out
 
 
@@ -303,18 +338,37 @@ def pack(codes: torch.Tensor, bits: int, out: Optional[torch.Tensor] = None, str
     return out
 
 
+def pack_zeros(zeros: torch.Tensor, bits: int, zero_offset: int = 0, status: Optional[torch.Tensor] = None,
+               out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """fp16 zero points [G, out] -> qzeros int32 [G, out*bits/32], packed along the outputs.
+
+    zero_offset 1 stores zero - 1 (the convention of older checkpoints).
+    """
+    _require_cuda(zeros, status, out)
+    if zeros.dtype != torch.float16 or zeros.dim() != 2 or not zeros.is_contiguous():
+        raise ValueError("zeros must be a contiguous fp16 [G, out] tensor")
+    g, o = zeros.shape
+    if out is None:
+        out = torch.empty((g, o * bits // 32), dtype=torch.int32, device=zeros.device)
+    _check(lib().gptq_pack_zeros(_ptr(zeros), g, o, int(bits), int(zero_offset), _ptr(out), _ptr(status),
+                                 _stream(stream)), "gptq_pack_zeros")
+    return out
+
+
 # --------------------------------------------------------------------------- #
 # The whole path for one layer
 # --------------------------------------------------------------------------- #
 def gptq_quantize(W: torch.Tensor, X: torch.Tensor, bits: int = 4, group_size: int = 128, sym: bool = False,
                   desc_act: bool = False, damp_percent: float = 0.01, block: int = 128,
-                  want_codes: bool = False, want_err: bool = False, check: bool = True):
+                  want_codes: bool = False, want_err: bool = False, check: bool = True, pad: bool = False):
     """H = 2.X.X^T, prepare, quantize.  Returns (QuantizedLayer, Prepared, H).
 
     W and X on the device, or both in host memory (pinned for overlap): then X crosses
     to the device in token chunks while the Hessian of the previous chunk is formed.
+    pad: quantize the layer zero-padded to padded_width(in, group_size) inputs (the
+    outputs then describe the padded layer).
     """
-    n = X.shape[0]
+    n = padded_width(X.shape[0], group_size) if pad else X.shape[0]
     host = X.device.type == "cpu"
     dev = torch.device("cuda", torch.cuda.current_device()) if host else X.device
     st = new_status(dev)

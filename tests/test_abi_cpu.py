@@ -72,3 +72,37 @@ def test_bad_arguments_rejected_without_a_gpu(L):
     assert L.gptq_hessian_accumulate_host(fake, None, 64, fake, 100, 100, fake, 2 * 64 * 63 * 2, None, None) == -7
     assert L.gptq_hessian_accumulate_host(fake, None, 64, fake, 100, 100, P(258), 1 << 20, None, None) == -7
     assert L.gptq_hessian_accumulate_host(fake, None, 64, fake, 100, 0, fake, 0, None, None) == 0
+
+
+def test_padded_calls_and_zero_packing_reject_bad_arguments_without_a_gpu(L):
+    P = ctypes.c_void_p
+    fake = P(256)
+    # Hessian of X zero-padded to n rows: x_rows must lie in 1..n; the empty chunk is a no-op
+    assert L.gptq_hessian_accumulate_padded(fake, None, 64, fake, 65, 96, 96, None, None) == -1
+    assert L.gptq_hessian_accumulate_padded(fake, None, 64, fake, 0, 96, 96, None, None) == -1
+    assert L.gptq_hessian_accumulate_padded(fake, None, 64, fake, 60, 100, 100, None, None) == -1   # ld_x % 8
+    assert L.gptq_hessian_accumulate_padded(fake, None, 64, fake, 60, 96, 0, None, None) == 0
+    # host form: the staging halves hold x_rows (not n) rows of at least 64 tokens
+    assert L.gptq_hessian_accumulate_host_padded(fake, None, 64, fake, 65, 100, 100, fake, 1 << 20, None, None) == -1
+    assert L.gptq_hessian_accumulate_host_padded(fake, None, 64, fake, 60, 100, 100, fake, 2 * 60 * 63 * 2,
+                                                 None, None) == -7
+    assert L.gptq_hessian_accumulate_host_padded(fake, None, 64, fake, 60, 100, 0, fake, 0, None, None) == 0
+    # quantize: w_cols in 1..n, and the padded width obeys the packing and group rules
+    args = (None, None, 4, 128, 0, 128, fake, fake, fake, fake, None, None, fake, 1 << 30, fake, None)
+    assert L.gptq_quantize_layer_padded(fake, 0, 8, 129, 128, fake, *args) == -1
+    assert L.gptq_quantize_layer_padded(fake, 0, 8, 0, 128, fake, *args) == -1
+    assert L.gptq_quantize_layer_padded(fake, 0, 8, 90, 100, fake, *args) == -2
+    # zero points: offset 0 or 1, supported widths, out * bits % 32 == 0
+    assert L.gptq_pack_zeros(None, 4, 8, 4, 0, fake, None, None) == -1
+    assert L.gptq_pack_zeros(fake, 4, 8, 4, 2, fake, None, None) == -1
+    assert L.gptq_pack_zeros(fake, 0, 8, 4, 0, fake, None, None) == -1
+    assert L.gptq_pack_zeros(fake, 4, 8, 5, 0, fake, None, None) == -2
+    assert L.gptq_pack_zeros(fake, 4, 12, 4, 0, fake, None, None) == -2
+
+
+def test_padded_width():
+    import post_weight_quantization_15_b200 as G
+    assert G.padded_width(300, 128) == 384 and G.padded_width(300, 64) == 320 and G.padded_width(300, 32) == 320
+    assert G.padded_width(300, -1) == 320 and G.padded_width(4096, 128) == 4096
+    # the page's example of a width that 128 x 8 does not divide
+    assert G.padded_width(29568 // 8, 128) == 3712

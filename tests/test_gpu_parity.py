@@ -391,3 +391,98 @@ def test_rounding_boundaries_are_bit_exact(sym):
     rc, rs, rz = O.rtn(W, 4, gs, sym)
     assert np.array_equal(rs, s0.T)
     assert np.array_equal(q.codes.cpu().numpy(), rc)
+
+
+# --------------------------------------------------------------------------- #
+# Checkpoint variants: zero padding, packed zero points
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("n,bits,gs,sym,act", [
+    (300, 4, 128, False, False),
+    (300, 4, 128, True, True),
+    (300, 3, 64, False, True),
+    (300, 4, -1, False, False),     # one group per row: padded to a multiple of 32
+    (100, 4, 128, True, False),     # fewer rows in X than one tile of the Hessian
+])
+def test_zero_padded_layer(n, bits, gs, sym, act):
+    """W [72, n] and X [n, 1000] zero-padded to the group size through the *_padded
+    entry points, against the oracle on the explicitly padded arrays."""
+    dev = _dev()
+    W, x = S.small_case(72, n, 1000, seed=n + bits, rank=8, frac=0.02, mult=20.0)
+    n_pad = G.padded_width(n, gs)
+    q, prep, Hg = G.gptq_quantize(_w_tensor(W, dev), _to_dev_x(x, dev), bits, gs, sym, act, want_codes=True,
+                                  want_err=True, pad=True)
+    torch.cuda.synchronize()
+    assert tuple(Hg.shape) == (n_pad, n_pad) and q.g_idx.numel() == n_pad and q.codes.shape[1] == n_pad
+    Hu = torch.triu(Hg).cpu().numpy()
+    assert not Hu[n:].any() and not Hu[:, n:].any()        # the padded rows and columns receive nothing
+    assert np.array_equal(np.flatnonzero(prep.dead.cpu().numpy()), np.arange(n, n_pad))
+    Wp, xp = O.pad_layer(W, x, n_pad)
+    H64 = O.hessian(xp)
+    ora = O.gptq_layer(Wp, None, bits, gs, sym, act, H=H64)
+    c = compare_layer(Wp, H64, ora, q.qweight.cpu().numpy(), q.scales.cpu().numpy(), q.zeros.cpu().numpy(),
+                      q.g_idx.cpu().numpy(), q.codes.cpu().numpy(), prep.perm.cpu().numpy(), bits, gs)
+    print(c)
+    assert c.ok(), c
+    What = O.dequantize(q.qweight.cpu().numpy(), q.scales.cpu().numpy(), q.zeros.cpu().numpy(),
+                        q.g_idx.cpu().numpy(), bits, n_pad)
+    assert not What[:, n:].any()
+
+
+def test_zero_padded_layer_from_host_memory():
+    dev = _dev()
+    n = 300
+    W, x = S.small_case(48, n, 2504, seed=6)
+    Wt = torch.from_numpy(np.ascontiguousarray(W))
+    X_host = torch.from_numpy(x.view(np.int16)).pin_memory()
+    # a small staging area: several chunks of 300 rows
+    n_pad = G.padded_width(n, 64)
+    H = torch.zeros((n_pad, n_pad), dtype=torch.float32, device=dev)
+    hd = torch.zeros(n_pad, dtype=torch.float64, device=dev)
+    st = G.new_status(dev)
+    G.hessian_accumulate_host(H, X_host, hd, st, staging=G.workspace(2 * n * 512 * 2, dev))
+    G.raise_on_status(st, "padded host Hessian")
+    H64 = O.hessian(O.pad_layer(W, x, n_pad)[1])
+    Hg = H.cpu().numpy().astype(np.float64)
+    iu = np.triu_indices(n_pad)
+    norm = np.sqrt(np.maximum(np.outer(np.diag(H64), np.diag(H64)), 1e-300))[iu]
+    assert (np.abs(Hg[iu] - H64[iu]) / norm).max() <= 2504 * 2.0 ** -23
+    assert not Hg[iu][H64[iu] == 0].any()
+    assert np.allclose(hd.cpu().numpy(), np.diag(H64), rtol=1e-13, atol=0)
+    # the whole padded path from host tensors gives the device path's result
+    q_h, p_h, _ = G.gptq_quantize(Wt.pin_memory(), X_host, 4, 64, False, True, want_codes=True, pad=True)
+    q_d, p_d, _ = G.gptq_quantize(Wt.to(dev), _to_dev_x(x, dev), 4, 64, False, True, want_codes=True, pad=True)
+    assert np.array_equal(p_h.perm.cpu().numpy(), p_d.perm.cpu().numpy())
+    assert float(np.mean(q_h.codes.cpu().numpy() != q_d.codes.cpu().numpy())) <= CODE_MISMATCH_MAX
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("offset", [0, 1])
+def test_pack_zeros_bit_exact(bits, offset):
+    dev = _dev()
+    rng = np.random.default_rng(10 * bits + offset)
+    z = rng.integers(0, 2 ** bits, (7, 352)).astype(np.float16)
+    st = G.new_status(dev)
+    qz = G.pack_zeros(torch.from_numpy(z).to(dev), bits, offset, st)
+    G.raise_on_status(st, "pack_zeros")
+    assert np.array_equal(qz.cpu().numpy().view(np.uint32), O.pack_zeros(z, bits, offset).view(np.uint32))
+
+
+def test_pack_zeros_of_a_quantized_layer():
+    dev = _dev()
+    W, x = S.small_case(96, 256, 1024, seed=12)
+    q, prep, _ = _run_gpu(W, x, 3, 64, False, True)
+    zg = q.zeros.cpu().numpy()
+    qz = G.pack_zeros(q.zeros, 3, 1, prep.status)
+    G.raise_on_status(prep.status, "pack_zeros")
+    assert np.array_equal(qz.cpu().numpy().view(np.uint32), O.pack_zeros(zg, 3, 1).view(np.uint32))
+    assert np.array_equal(O.unpack_zeros(qz.cpu().numpy(), 3, 96, 1), zg.astype(np.float64))
+
+
+def test_pack_zeros_reports_a_zero_that_is_not_a_code():
+    dev = _dev()
+    z = np.full((3, 64), 5, dtype=np.float16)
+    z[1, 17] = 2.5
+    st = G.new_status(dev)
+    G.pack_zeros(torch.from_numpy(z).to(dev), 4, 0, st)
+    rc, info = G.status_read(st)
+    assert rc == G.gptq.ERR_INVALID_ARG and info == 64 + 17
