@@ -65,6 +65,9 @@ typedef enum {
 
 typedef enum { GPTQ_F32 = 0, GPTQ_F16 = 1, GPTQ_BF16 = 2 } gptq_dtype;
 
+/* Largest number of output rows gptq_quantize_layer accepts (8 x 65535). */
+#define GPTQ_MAX_OUT 524280
+
 /* Library / ABI version (GPTQ_ABI_VERSION). */
 GPTQ_API int gptq_version(void);
 
@@ -179,7 +182,9 @@ GPTQ_API int gptq_prepare(const float* H, const double* hdiag, int n, float damp
  *   U, perm, dead   from gptq_prepare (perm and dead may be NULL: identity / none).
  *   bits       2, 3, 4 or 8.     group_size 32, 64, 128, or -1 (one group per row).
  *   block      128 (the pages' batch); block % group_size == 0 when group_size > 0.
- *   n % 32 == 0, and n % group_size == 0 when group_size > 0.  out >= 1.
+ *   n % 32 == 0, and n % group_size == 0 when group_size > 0.
+ *   1 <= out <= GPTQ_MAX_OUT (GPTQ_ERR_UNSUPPORTED above: the row kernels put
+ *   eight rows per block along the grid's second dimension).
  *   qweight    int32 [n*bits/32, out]: per output row, the codes of the input
  *              columns in original order as a little-endian bit stream (column k
  *              at stream bits k*bits ...), word-major.

@@ -120,6 +120,7 @@ int gptq_quantize_layer_padded(const void* W, int w_dtype, int out, int w_cols, 
       g_idx == nullptr || d_status == nullptr)
     return GPTQ_ERR_INVALID_ARG;
   if (out <= 0 || n <= 0 || w_cols <= 0 || w_cols > n) return GPTQ_ERR_INVALID_ARG;
+  if (out > GPTQ_MAX_OUT) return GPTQ_ERR_UNSUPPORTED;
   if (w_dtype != GPTQ_F32 && w_dtype != GPTQ_F16 && w_dtype != GPTQ_BF16) return GPTQ_ERR_INVALID_ARG;
   if (!valid_bits(bits) || !valid_gs(group_size)) return GPTQ_ERR_UNSUPPORTED;
   if (block != 128) return GPTQ_ERR_UNSUPPORTED;

@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(256) prep_reverse_kernel(const float* H, const
 // inverse accumulates; its diagonal blocks are written whole and nothing reads
 // below them.
 __global__ void zero_upper_blocks_kernel(float* Xt, int n, int ldn) {
-  const int r = blockIdx.y;
+  const int r = blockIdx.x;
   const int c0 = (r / PB + 1) * PB;
   float* row = Xt + (int64_t)r * ldn;
   for (int c = c0 + 4 * (int)threadIdx.x; c < n; c += 4 * (int)blockDim.x)
@@ -927,7 +927,7 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
   GPTQ_LAUNCH_CHECK();
   if (n > PB) {
     // rows above the last block row (which starts at the last multiple of PB below n)
-    zero_upper_blocks_kernel<<<dim3(1, (unsigned)((n - 1) / PB * PB)), 256, 0, s>>>(w.Xt, n, ldn);
+    zero_upper_blocks_kernel<<<(unsigned)((n - 1) / PB * PB), 256, 0, s>>>(w.Xt, n, ldn);
     GPTQ_LAUNCH_CHECK();
   }
 

@@ -92,6 +92,8 @@ def test_padded_calls_and_zero_packing_reject_bad_arguments_without_a_gpu(L):
     assert L.gptq_quantize_layer_padded(fake, 0, 8, 129, 128, fake, *args) == -1
     assert L.gptq_quantize_layer_padded(fake, 0, 8, 0, 128, fake, *args) == -1
     assert L.gptq_quantize_layer_padded(fake, 0, 8, 90, 100, fake, *args) == -2
+    # more output rows than the row kernels' grids hold
+    assert L.gptq_quantize_layer_padded(fake, 0, 524281, 128, 128, fake, *args) == -2
     # zero points: offset 0 or 1, supported widths, out * bits % 32 == 0
     assert L.gptq_pack_zeros(None, 4, 8, 4, 0, fake, None, None) == -1
     assert L.gptq_pack_zeros(fake, 4, 8, 4, 2, fake, None, None) == -1
