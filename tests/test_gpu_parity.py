@@ -486,3 +486,62 @@ def test_pack_zeros_reports_a_zero_that_is_not_a_code():
     G.pack_zeros(torch.from_numpy(z).to(dev), 4, 0, st)
     rc, info = G.status_read(st)
     assert rc == G.gptq.ERR_INVALID_ARG and info == 64 + 17
+
+
+# --------------------------------------------------------------------------- #
+# Ordering: the multi-stream stages are deterministic and calls queue safely
+# --------------------------------------------------------------------------- #
+def test_repeated_and_back_to_back_calls_are_bit_identical():
+    """Every stage computes each element in a fixed order, so repeated runs give the same
+    bits.  prepare() forks onto four library streams and the host Hessian onto a copy
+    stream shared by all calls of a host thread; calls queued back to back without a
+    synchronization must give the bits of calls run one at a time."""
+    dev = _dev()
+    W, x = S.small_case(1024, 1536, 3000, seed=21, rank=16)
+    Wt, X = _w_tensor(W, dev), _to_dev_x(x, dev)
+    X2 = _to_dev_x(S.small_case(8, 1536, 2000, seed=22, rank=16)[1], dev)
+
+    def one(Xa, act):
+        st = G.new_status(dev)
+        H = torch.zeros((1536, 1536), dtype=torch.float32, device=dev)
+        hd = torch.zeros(1536, dtype=torch.float64, device=dev)
+        G.hessian_accumulate(H, Xa, hd, st)
+        p = G.prepare(H, 0.01, act, hd, st)
+        q = G.quantize_layer(Wt, p, 4, 128, False, want_codes=True)
+        return st, H, p, q
+
+    ref = []
+    for Xa, act in [(X, True), (X2, False)]:
+        st, H, p, q = one(Xa, act)
+        torch.cuda.synchronize()
+        G.raise_on_status(st, "reference run")
+        ref.append((H.clone(), p.U.clone(), p.perm.clone(), q.qweight.clone(), q.scales.clone(), q.zeros.clone()))
+    for _ in range(2):
+        runs = [one(X, True), one(X2, False), one(X, True)]      # queued back to back
+        torch.cuda.synchronize()
+        for (st, H, p, q), r in zip(runs, [ref[0], ref[1], ref[0]]):
+            G.raise_on_status(st, "back-to-back run")
+            got = (torch.triu(H), p.U, p.perm, q.qweight, q.scales, q.zeros)
+            exp = (torch.triu(r[0]),) + r[1:]
+            for a, b in zip(got, exp):
+                assert torch.equal(a, b)
+
+
+def test_host_hessian_calls_back_to_back_are_bit_identical():
+    # the copy stream and its events are shared by the calls of a host thread; two calls
+    # sharing one staging area, queued without a synchronization, give the bits of one call
+    dev = _dev()
+    _, x = S.small_case(8, 640, 5000, seed=23, rank=16)
+    X_host = torch.from_numpy(x.view(np.int16)).pin_memory()
+    staging = G.workspace(2 * 640 * 1024 * 2, dev)
+    st = G.new_status(dev)
+    H0 = torch.zeros((640, 640), dtype=torch.float32, device=dev)
+    G.hessian_accumulate_host(H0, X_host, None, st, staging=staging)
+    torch.cuda.synchronize()
+    Hs = [torch.zeros((640, 640), dtype=torch.float32, device=dev) for _ in range(3)]
+    for H in Hs:
+        G.hessian_accumulate_host(H, X_host, None, st, staging=staging)
+    torch.cuda.synchronize()
+    G.raise_on_status(st, "host Hessian back to back")
+    for H in Hs:
+        assert torch.equal(torch.triu(H), torch.triu(H0))
