@@ -304,6 +304,12 @@ def quantize_layer(W: torch.Tensor, prep: Prepared, bits: int = 4, group_size: i
                    block: int = 128, want_codes: bool = False, want_err: bool = False,
                    ws: Optional[torch.Tensor] = None, out: Optional[QuantizedLayer] = None,
                    stream=None) -> QuantizedLayer:
+    """Sweep, lazy trailing update and packing of W [out, in] given ``prep`` (n = U's size).
+
+    in == n is the ordinary call.  in < n quantizes W zero-padded to n columns (the
+    outputs then describe the padded layer: qweight, g_idx and codes have n columns);
+    ``prep`` must then come from the padded Hessian (see hessian_accumulate).
+    """
     _require_cuda(W, ws)
     if W.dim() != 2 or not W.is_contiguous() or W.dtype not in _DTYPE_CODE:
         raise ValueError("W must be a contiguous fp32/fp16/bf16 [out, n] tensor")
