@@ -296,7 +296,7 @@ GPTQ_API int gptq_pack_zeros(const uint16_t* zeros, int groups, int out, int bit
  *   from host threads that do not order them - race on it.
  * - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
  */
-#define GPTQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+#define GPTQ_NOALLOC_SCRATCH_BYTES (32u << 20)
 GPTQ_API int gptq_quantize_layer_noalloc(const void* W, int w_dtype, int out, int n, const float* U,
                                          const int32_t* perm, const uint8_t* dead, int bits, int group_size,
                                          int sym, int block, int32_t* qweight, uint16_t* scales,

@@ -8,7 +8,7 @@
 // capture), or a service that must not grow its footprint after start-up.  They
 // still pass their own inputs and outputs; only the scratch comes from here.
 //
-// The array is GPTQ_NOALLOC_SCRATCH_BYTES (16 MiB).  Every GPU that loads this
+// The array is GPTQ_NOALLOC_SCRATCH_BYTES (32 MiB).  Every GPU that loads this
 // library holds one copy of it until the process exits.  All calls on a device
 // share it and it keeps the last call's contents; every byte a call reads from it
 // is written by that same call first, so nothing needs clearing between calls.

@@ -31,12 +31,14 @@ constexpr int BLK = 128;           // columns per lazy batch
 constexpr int SUPER = 4;           // lazy batches per super-block
 constexpr int SBK = SUPER * BLK;   // columns per super-block
 
+// Super-block s uses the error and operand buffers of parity s & 1: the trailing
+// update of super-block s still reads them while super-block s + 1 is swept.
 struct QuantWs {
   float* Wf;          // [out, n] working weights, processing order
-  float* Ehi;         // [out, SBK] scaled errors of the current super-block, TF32-exact high part
-  float* Elo;         // [out, SBK] and the remainder
-  float* Bhi;         // [n, SBK] U[super-block rows, later columns]^T, high part (K-major operand)
-  float* Blo;         // [n, SBK] and the remainder
+  float* Ehi[2];      // [out, SBK] scaled errors of a super-block, TF32-exact high part
+  float* Elo[2];      // [out, SBK] and the remainder
+  float* Bhi[2];      // [n, SBK] U[super-block rows, later columns]^T, high part (K-major operand)
+  float* Blo[2];      // [n, SBK] and the remainder
   uint8_t* codes_p;   // [out, n] codes, processing order
   int32_t* invperm;   // [n] processing position of every input column
   float* rows;        // [out] row-wide scale, [out] row-wide zero (group_size = -1)
@@ -46,10 +48,12 @@ QuantWs carve(void* ws, int out, int n) {
   char* p = static_cast<char*>(ws);
   QuantWs w;
   w.Wf = reinterpret_cast<float*>(p);        p += align_up((size_t)out * n * 4, 256);
-  w.Ehi = reinterpret_cast<float*>(p);       p += align_up((size_t)out * SBK * 4, 256);
-  w.Elo = reinterpret_cast<float*>(p);       p += align_up((size_t)out * SBK * 4, 256);
-  w.Bhi = reinterpret_cast<float*>(p);       p += align_up((size_t)n * SBK * 4, 256);
-  w.Blo = reinterpret_cast<float*>(p);       p += align_up((size_t)n * SBK * 4, 256);
+  for (int b = 0; b < 2; ++b) {
+    w.Ehi[b] = reinterpret_cast<float*>(p);  p += align_up((size_t)out * SBK * 4, 256);
+    w.Elo[b] = reinterpret_cast<float*>(p);  p += align_up((size_t)out * SBK * 4, 256);
+    w.Bhi[b] = reinterpret_cast<float*>(p);  p += align_up((size_t)n * SBK * 4, 256);
+    w.Blo[b] = reinterpret_cast<float*>(p);  p += align_up((size_t)n * SBK * 4, 256);
+  }
   w.codes_p = reinterpret_cast<uint8_t*>(p); p += align_up((size_t)out * n, 256);
   w.invperm = reinterpret_cast<int32_t*>(p); p += align_up((size_t)n * 4, 256);
   w.rows = reinterpret_cast<float*>(p);
@@ -599,10 +603,46 @@ __global__ void codes_out_kernel(const uint8_t* codes_p, const int32_t* invperm,
 
 size_t quantize_ws_bytes(int out, int n, int block) {
   (void)block;
-  return align_up((size_t)out * n * 4, 256) + 2 * align_up((size_t)out * SBK * 4, 256) +
-         2 * align_up((size_t)n * SBK * 4, 256) + align_up((size_t)out * n, 256) + align_up((size_t)n * 4, 256) +
+  return align_up((size_t)out * n * 4, 256) + 4 * align_up((size_t)out * SBK * 4, 256) +
+         4 * align_up((size_t)n * SBK * 4, 256) + align_up((size_t)out * n, 256) + align_up((size_t)n * 4, 256) +
          align_up((size_t)out * 8, 256);
 }
+
+namespace {
+
+// Two library streams per host thread and device: the sweeps and the update of the
+// next super-block on a high-priority stream (the critical chain), the rest of each
+// trailing update and the U operands of later super-blocks on a low-priority one.
+// Created on first use, kept for the life of the process.
+struct QuantStreams {
+  cudaStream_t hi = nullptr, lo = nullptr;
+  cudaEvent_t fork = nullptr, join_hi = nullptr, join_lo = nullptr;
+  cudaEvent_t swept = nullptr;   // the latest sweep is done: its errors are complete
+  cudaEvent_t near = nullptr;    // the latest next-super-block update is done with its operand buffers
+  cudaEvent_t far = nullptr;     // the latest far update is done with its columns and error buffers
+  cudaEvent_t opnd[2] = {};      // the U operand in buffer b is written
+};
+
+int quant_streams(QuantStreams** out) {
+  thread_local QuantStreams per_dev[64];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GPTQ_ERR_CUDA;
+  QuantStreams& q = per_dev[dev];
+  if (q.hi == nullptr) {
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return GPTQ_ERR_CUDA;
+    if (cudaStreamCreateWithPriority(&q.hi, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&q.lo, cudaStreamNonBlocking, least) != cudaSuccess)
+      return GPTQ_ERR_CUDA;
+    cudaEvent_t* evs[] = {&q.fork, &q.join_hi, &q.join_lo, &q.swept, &q.near, &q.far, &q.opnd[0], &q.opnd[1]};
+    for (cudaEvent_t* e : evs)
+      if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return GPTQ_ERR_CUDA;
+  }
+  *out = &q;
+  return GPTQ_OK;
+}
+
+}  // namespace
 
 int launch_pack(const uint8_t* codes, const int32_t* invperm, int out, int n, int ld_codes, int bits,
                 int32_t* qweight, const int32_t* st, cudaStream_t s) {
@@ -664,25 +704,69 @@ int launch_quantize(const void* W, int w_dtype, int out, int w_cols, int n, cons
   GPTQ_CUDA_TRY(cudaFuncSetAttribute(sweep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   // Two-level lazy batches: blocks of 128 columns inside super-blocks of 512.  A
   // block's sweep also updates the rest of its super-block; the columns after a
-  // super-block absorb its 512 errors at once on the tensor cores.
-  for (int s0 = 0; s0 < n; s0 += SBK) {
-    const int se = std::min(n, s0 + SBK);
-    sweep<<<(unsigned)cdiv(out, rows_per_cta), threads, smem, s>>>(w.Wf, out, n, s0, se, U, w.Ehi, w.Elo, w.codes_p,
-                                                                scales, zeros, w.rows, err_sq, bits, sym, st);
+  // super-block absorb its 512 errors at once on the tensor cores, as
+  // Wf[:, se:] -= Err[:, super-block] . U[super-block, se:] (K = 512, accumulated by
+  // the GEMM in 128-deep chunks summed in fp32 registers: one long tensor-core
+  // accumulation let the codes of a 28,672-column layer drift past 0.5 %).
+  // That update is split in two: the next super-block's columns on the critical
+  // chain (hi), the columns after them (and the U operand of super-block s + 2) on
+  // the low-priority stream, beside the next sweep.  Ordering, for super-block s
+  // with buffers b = s & 1:
+  //   near(s)   waits far(s - 1), which updated the same columns, and operand(s);
+  //   far(s)    waits sweep(s); far(s - 1) precedes it on lo;
+  //   sweep(s + 1) follows near(s) on hi, so it sees both updates of its columns;
+  //   sweep(s + 2) rewrites the errors E[b]: near(s + 1) waited far(s) before it;
+  //   operand(s + 2) rewrites B[b]: it waits near(s) and follows far(s) on lo.
+  QuantStreams* q = nullptr;
+  int rc = quant_streams(&q);
+  if (rc != GPTQ_OK) return rc;
+  GPTQ_CUDA_TRY(cudaEventRecord(q->fork, s));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->hi, q->fork, 0));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->lo, q->fork, 0));
+  const int S = (int)cdiv(n, SBK);
+  // U[super-block sb rows, the columns after it]^T, split, into B[sb & 1] (on lo)
+  auto operand = [&](int sb) -> int {
+    const int b0 = sb * SBK, be = b0 + SBK;   // sb < S - 1: a whole super-block with columns after it
+    dim3 blk(32, 8), grd((unsigned)cdiv(n - be, 32), (unsigned)(SBK / 32));
+    u_block_transpose_split_kernel<<<grd, blk, 0, q->lo>>>(U, n, b0, SBK, be, w.Bhi[sb & 1], w.Blo[sb & 1], SBK, st);
     GPTQ_LAUNCH_CHECK();
-    if (se < n) {
-      const int kw = se - s0;   // == SBK
-      dim3 blk(32, 8), grd((unsigned)cdiv(n - se, 32), (unsigned)(SBK / 32));
-      u_block_transpose_split_kernel<<<grd, blk, 0, s>>>(U, n, s0, kw, se, w.Bhi, w.Blo, SBK, st);
-      GPTQ_LAUNCH_CHECK();
-      // Wf[:, se:] -= Err[:, super-block] . U[super-block, se:] (K = 512, accumulated by
-      // the GEMM in 128-deep chunks summed in fp32 registers: one long tensor-core
-      // accumulation let the codes of a 28,672-column layer drift past 0.5 %)
-      const int rc = launch_gemm3(w.Wf + se, n, out, n - se, kw, w.Ehi, w.Elo, SBK, w.Bhi, w.Blo, SBK, false, st, s);
+    GPTQ_CUDA_TRY(cudaEventRecord(q->opnd[sb & 1], q->lo));
+    return GPTQ_OK;
+  };
+  for (int sb = 0; sb < std::min(2, S - 1); ++sb)
+    if ((rc = operand(sb)) != GPTQ_OK) return rc;
+  for (int sb = 0; sb < S; ++sb) {
+    const int b = sb & 1;
+    const int s0 = sb * SBK, se = std::min(n, s0 + SBK);
+    sweep<<<(unsigned)cdiv(out, rows_per_cta), threads, smem, q->hi>>>(w.Wf, out, n, s0, se, U, w.Ehi[b], w.Elo[b],
+                                                                    w.codes_p, scales, zeros, w.rows, err_sq, bits,
+                                                                    sym, st);
+    GPTQ_LAUNCH_CHECK();
+    if (se >= n) break;
+    const int kn = std::min(SBK, n - se);   // the next super-block's width
+    GPTQ_CUDA_TRY(cudaEventRecord(q->swept, q->hi));
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->hi, q->opnd[b], 0));
+    if (sb > 0) GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->hi, q->far, 0));
+    rc = launch_gemm3(w.Wf + se, n, out, kn, SBK, w.Ehi[b], w.Elo[b], SBK, w.Bhi[b], w.Blo[b], SBK, false, st, q->hi);
+    if (rc != GPTQ_OK) return rc;
+    GPTQ_CUDA_TRY(cudaEventRecord(q->near, q->hi));
+    if (n - se > kn) {
+      GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->lo, q->swept, 0));
+      rc = launch_gemm3(w.Wf + se + kn, n, out, n - se - kn, SBK, w.Ehi[b], w.Elo[b], SBK,
+                        w.Bhi[b] + (size_t)kn * SBK, w.Blo[b] + (size_t)kn * SBK, SBK, false, st, q->lo);
       if (rc != GPTQ_OK) return rc;
     }
+    GPTQ_CUDA_TRY(cudaEventRecord(q->far, q->lo));
+    if (sb + 2 < S - 1) {
+      GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->lo, q->near, 0));
+      if ((rc = operand(sb + 2)) != GPTQ_OK) return rc;
+    }
   }
-  int rc = launch_pack(w.codes_p, w.invperm, out, n, n, bits, qweight, st, s);
+  GPTQ_CUDA_TRY(cudaEventRecord(q->join_hi, q->hi));
+  GPTQ_CUDA_TRY(cudaEventRecord(q->join_lo, q->lo));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, q->join_hi, 0));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, q->join_lo, 0));
+  rc = launch_pack(w.codes_p, w.invperm, out, n, n, bits, qweight, st, s);
   if (rc != GPTQ_OK) return rc;
   if (codes) {
     dim3 blk(32, 8), grd((unsigned)cdiv(n, 32), (unsigned)cdiv(out, 8));

@@ -395,14 +395,14 @@ def gptq_quantize(W: torch.Tensor, X: torch.Tensor, bits: int = 4, group_size: i
 # --------------------------------------------------------------------------- #
 # Static-scratch variant (no workspace)
 # --------------------------------------------------------------------------- #
-NOALLOC_SCRATCH_BYTES = 16 << 20
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 def quantize_layer_noalloc(W: torch.Tensor, prep: Prepared, out: QuantizedLayer, block: int = 128,
                            stream=None) -> QuantizedLayer:
     """quantize_layer for callers that cannot allocate device memory.
 
-    The library takes its scratch from a static 16 MiB device array instead of a
+    The library takes its scratch from a static 32 MiB device array instead of a
     workspace, so this call allocates nothing; the caller passes preallocated
     outputs (see alloc_quantized).  Layers whose workspace would exceed the array
     raise GptqError(ERR_WORKSPACE).  Calls that overlap on the GPU race on the
