@@ -661,6 +661,62 @@ int launch_pack_zeros(const uint16_t* zeros, int groups, int out, int bits, int 
   return GPTQ_OK;
 }
 
+// The super-blocks of one layer on the two library streams (ordering: see launch_quantize).
+template <typename SweepFn>
+int super_block_loop(QuantStreams* q, const QuantWs& w, int out, int n, const float* U, int bits, int sym,
+                     uint16_t* scales, uint16_t* zeros, float* err_sq, int32_t* st, SweepFn sweep, size_t smem,
+                     int rows_per_cta, int threads) {
+  int rc = GPTQ_OK;
+  const int S = (int)cdiv(n, SBK);
+  // U[super-block sb rows, the columns after it]^T, split, into B[sb & 1] (on lo)
+  auto operand = [&](int sb) -> int {
+    const int b0 = sb * SBK, be = b0 + SBK;   // sb < S - 1: a whole super-block with columns after it
+    dim3 blk(32, 8), grd((unsigned)cdiv(n - be, 32), (unsigned)(SBK / 32));
+    u_block_transpose_split_kernel<<<grd, blk, 0, q->lo>>>(U, n, b0, SBK, be, w.Bhi[sb & 1], w.Blo[sb & 1], SBK, st);
+    GPTQ_LAUNCH_CHECK();
+    GPTQ_CUDA_TRY(cudaEventRecord(q->opnd[sb & 1], q->lo));
+    return GPTQ_OK;
+  };
+  for (int sb = 0; sb < std::min(2, S - 1); ++sb)
+    if ((rc = operand(sb)) != GPTQ_OK) return rc;
+  for (int sb = 0; sb < S; ++sb) {
+    const int b = sb & 1;
+    const int s0 = sb * SBK, se = std::min(n, s0 + SBK);
+    sweep<<<(unsigned)cdiv(out, rows_per_cta), threads, smem, q->hi>>>(w.Wf, out, n, s0, se, U, w.Ehi[b], w.Elo[b],
+                                                                    w.codes_p, scales, zeros, w.rows, err_sq, bits,
+                                                                    sym, st);
+    GPTQ_LAUNCH_CHECK();
+    if (se >= n) break;
+    const int kn = std::min(SBK, n - se);   // the next super-block's width
+    GPTQ_CUDA_TRY(cudaEventRecord(q->swept, q->hi));
+    GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->hi, q->opnd[b], 0));
+    if (sb > 0) GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->hi, q->far, 0));
+    rc = launch_gemm3(w.Wf + se, n, out, kn, SBK, w.Ehi[b], w.Elo[b], SBK, w.Bhi[b], w.Blo[b], SBK, false, st, q->hi);
+    if (rc != GPTQ_OK) return rc;
+    GPTQ_CUDA_TRY(cudaEventRecord(q->near, q->hi));
+    if (n - se > kn) {
+      GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->lo, q->swept, 0));
+      rc = launch_gemm3(w.Wf + se + kn, n, out, n - se - kn, SBK, w.Ehi[b], w.Elo[b], SBK,
+                        w.Bhi[b] + (size_t)kn * SBK, w.Blo[b] + (size_t)kn * SBK, SBK, false, st, q->lo);
+      if (rc != GPTQ_OK) return rc;
+    }
+    GPTQ_CUDA_TRY(cudaEventRecord(q->far, q->lo));
+    if (sb + 2 < S - 1) {
+      GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->lo, q->near, 0));
+      if ((rc = operand(sb + 2)) != GPTQ_OK) return rc;
+    }
+  }
+  return GPTQ_OK;
+}
+
+int join_streams(QuantStreams* q, cudaStream_t s) {
+  GPTQ_CUDA_TRY(cudaEventRecord(q->join_hi, q->hi));
+  GPTQ_CUDA_TRY(cudaEventRecord(q->join_lo, q->lo));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, q->join_hi, 0));
+  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, q->join_lo, 0));
+  return GPTQ_OK;
+}
+
 int launch_quantize(const void* W, int w_dtype, int out, int w_cols, int n, const float* U, const int32_t* perm,
                     const uint8_t* dead, int bits, int gs, int sym, int block, int32_t* qweight,
                     uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq,
@@ -723,49 +779,12 @@ int launch_quantize(const void* W, int w_dtype, int out, int w_cols, int n, cons
   GPTQ_CUDA_TRY(cudaEventRecord(q->fork, s));
   GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->hi, q->fork, 0));
   GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->lo, q->fork, 0));
-  const int S = (int)cdiv(n, SBK);
-  // U[super-block sb rows, the columns after it]^T, split, into B[sb & 1] (on lo)
-  auto operand = [&](int sb) -> int {
-    const int b0 = sb * SBK, be = b0 + SBK;   // sb < S - 1: a whole super-block with columns after it
-    dim3 blk(32, 8), grd((unsigned)cdiv(n - be, 32), (unsigned)(SBK / 32));
-    u_block_transpose_split_kernel<<<grd, blk, 0, q->lo>>>(U, n, b0, SBK, be, w.Bhi[sb & 1], w.Blo[sb & 1], SBK, st);
-    GPTQ_LAUNCH_CHECK();
-    GPTQ_CUDA_TRY(cudaEventRecord(q->opnd[sb & 1], q->lo));
-    return GPTQ_OK;
-  };
-  for (int sb = 0; sb < std::min(2, S - 1); ++sb)
-    if ((rc = operand(sb)) != GPTQ_OK) return rc;
-  for (int sb = 0; sb < S; ++sb) {
-    const int b = sb & 1;
-    const int s0 = sb * SBK, se = std::min(n, s0 + SBK);
-    sweep<<<(unsigned)cdiv(out, rows_per_cta), threads, smem, q->hi>>>(w.Wf, out, n, s0, se, U, w.Ehi[b], w.Elo[b],
-                                                                    w.codes_p, scales, zeros, w.rows, err_sq, bits,
-                                                                    sym, st);
-    GPTQ_LAUNCH_CHECK();
-    if (se >= n) break;
-    const int kn = std::min(SBK, n - se);   // the next super-block's width
-    GPTQ_CUDA_TRY(cudaEventRecord(q->swept, q->hi));
-    GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->hi, q->opnd[b], 0));
-    if (sb > 0) GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->hi, q->far, 0));
-    rc = launch_gemm3(w.Wf + se, n, out, kn, SBK, w.Ehi[b], w.Elo[b], SBK, w.Bhi[b], w.Blo[b], SBK, false, st, q->hi);
-    if (rc != GPTQ_OK) return rc;
-    GPTQ_CUDA_TRY(cudaEventRecord(q->near, q->hi));
-    if (n - se > kn) {
-      GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->lo, q->swept, 0));
-      rc = launch_gemm3(w.Wf + se + kn, n, out, n - se - kn, SBK, w.Ehi[b], w.Elo[b], SBK,
-                        w.Bhi[b] + (size_t)kn * SBK, w.Blo[b] + (size_t)kn * SBK, SBK, false, st, q->lo);
-      if (rc != GPTQ_OK) return rc;
-    }
-    GPTQ_CUDA_TRY(cudaEventRecord(q->far, q->lo));
-    if (sb + 2 < S - 1) {
-      GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->lo, q->near, 0));
-      if ((rc = operand(sb + 2)) != GPTQ_OK) return rc;
-    }
-  }
-  GPTQ_CUDA_TRY(cudaEventRecord(q->join_hi, q->hi));
-  GPTQ_CUDA_TRY(cudaEventRecord(q->join_lo, q->lo));
-  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, q->join_hi, 0));
-  GPTQ_CUDA_TRY(cudaStreamWaitEvent(s, q->join_lo, 0));
+  rc = super_block_loop(q, w, out, n, U, bits, sym, scales, zeros, err_sq, st, sweep, smem, rows_per_cta, threads);
+  // both library streams join the caller's stream, after an error too, so that the
+  // caller's stream is ordered after everything this call enqueued
+  const int jrc = join_streams(q, s);
+  if (rc != GPTQ_OK) return rc;
+  if (jrc != GPTQ_OK) return jrc;
   rc = launch_pack(w.codes_p, w.invperm, out, n, n, bits, qweight, st, s);
   if (rc != GPTQ_OK) return rc;
   if (codes) {
