@@ -22,8 +22,13 @@
  *   library allocates nothing: calls that need scratch take a caller-provided
  *   workspace whose size the matching *_workspace_size() call reports.
  * - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
- *   Every call only enqueues work on that stream and returns; calls on one
- *   stream run in order.  Calls on different streams that share buffers race.
+ *   Every call only enqueues work and returns; calls on one stream run in order.
+ *   Calls on different streams that share buffers race.  gptq_prepare,
+ *   gptq_quantize_layer and the host-memory Hessian run parts of their work on
+ *   streams of the library's own (one set per host thread and device, created on
+ *   the first call) that fork from `stream` and join it again before the call
+ *   returns, so `stream` is ordered after all of a call's work, after an error
+ *   too.  Make the first such call on a device outside any stream capture.
  * - Argument errors are returned synchronously (nothing is enqueued).
  *   Errors found on the device (a non-positive Cholesky pivot, non-finite
  *   values, a bounded wait that gave up) are recorded in a caller-provided
