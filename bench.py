@@ -221,6 +221,20 @@ def oracle_sample(layer: S.Layer, st: S.QuantSettings, tokens: int):
     return est, desc
 
 
+def oracle_single_thread(workload: str = "layer-256x512"):
+    """The oracle on the small layer, whole (all its tokens), with one BLAS thread.
+
+    Returns {"value", "unit", "cores": 1, "seconds", "workload"}.
+    """
+    from threadpoolctl import threadpool_limits
+    wl = S.workloads()[workload]
+    layer, st = wl.layers[0], wl.settings[0]
+    with threadpool_limits(limits=1):
+        est, _ = oracle_sample(layer, st, layer.x.tokens)
+    return {"value": layer.w.out * layer.w.n / est / 1e9, "unit": UNIT, "cores": 1, "seconds": est,
+            "workload": workload}
+
+
 # --------------------------------------------------------------------------- #
 # reference arm: the oracle
 # --------------------------------------------------------------------------- #
@@ -406,7 +420,8 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         est, desc = oracle_sample(layer, st, min(N, args.ref_tokens))
-        cpu = {"value": out * n / est / 1e9, "unit": UNIT, "cores": host_cores(), "kind": "oracle", "sample": desc}
+        cpu = {"value": out * n / est / 1e9, "unit": UNIT, "cores": host_cores(), "kind": "oracle", "sample": desc,
+               "single_thread": oracle_single_thread()}
 
     if world > 1:
         dist.barrier()
