@@ -420,8 +420,11 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         est, desc = oracle_sample(layer, st, min(N, args.ref_tokens))
-        cpu = {"value": out * n / est / 1e9, "unit": UNIT, "cores": host_cores(), "kind": "oracle", "sample": desc,
-               "single_thread": oracle_single_thread()}
+        cpu = {"value": out * n / est / 1e9, "unit": UNIT, "cores": host_cores(), "kind": "oracle", "sample": desc}
+        try:
+            cpu["single_thread"] = oracle_single_thread()
+        except Exception as e:  # a side figure: never let it cost the bench line
+            cpu["single_thread"] = {"unavailable": f"{type(e).__name__}: {e}"}
 
     if world > 1:
         dist.barrier()
