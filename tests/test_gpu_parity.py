@@ -545,3 +545,19 @@ def test_host_hessian_calls_back_to_back_are_bit_identical():
     G.raise_on_status(st, "host Hessian back to back")
     for H in Hs:
         assert torch.equal(torch.triu(H), torch.triu(H0))
+
+
+def test_bf16_weights():
+    # W given in bf16: the oracle quantizes exactly the values the library reads
+    dev = _dev()
+    W32, x = S.small_case(96, 1024, 1200, seed=44)
+    Wb = torch.from_numpy(W32).to(torch.bfloat16)
+    W = Wb.float().numpy()
+    q, prep, _ = G.gptq_quantize(Wb.to(dev), _to_dev_x(x, dev), 4, 128, False, True, want_codes=True)
+    torch.cuda.synchronize()
+    H64 = O.hessian(x)
+    ora = O.gptq_layer(W, None, 4, 128, False, True, H=H64)
+    c = compare_layer(W, H64, ora, q.qweight.cpu().numpy(), q.scales.cpu().numpy(), q.zeros.cpu().numpy(),
+                      q.g_idx.cpu().numpy(), q.codes.cpu().numpy(), prep.perm.cpu().numpy(), 4, 128)
+    print(c)
+    assert c.ok(), c

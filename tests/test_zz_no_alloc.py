@@ -47,7 +47,8 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     cases = [(256, 512, 2048, 1, 4, 128, False, False),
-             (200, 384, 1024, 2, 3, 64, True, True)]
+             (200, 384, 1024, 2, 3, 64, True, True),
+             (256, 1536, 3072, 3, 4, 64, False, True)]    # three super-blocks: both library streams
     for out, n, tokens, seed, bits, gs, sym, act in cases:
         G, W, prep = _setup(out, n, tokens, seed, bits, gs, sym, act)
         ref = G.quantize_layer(W, prep, bits, gs, sym, want_codes=True, want_err=True)
