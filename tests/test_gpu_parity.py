@@ -561,3 +561,31 @@ def test_bf16_weights():
                       q.g_idx.cpu().numpy(), q.codes.cpu().numpy(), prep.perm.cpu().numpy(), 4, 128)
     print(c)
     assert c.ok(), c
+
+
+@pytest.mark.parametrize("bits,gs,sym", [(4, 128, False), (4, 128, True), (2, 32, False), (3, -1, True),
+                                         (8, 64, False)])
+def test_degenerate_groups_are_bit_exact_round_to_nearest(bits, gs, sym):
+    """Rows whose groups hit the quantizer's special cases: all zero (asymmetric range
+    taken as [-1, 1], symmetric magnitude 1), constant of either sign (one end of the
+    range at 0), tiny (the scale clamps to fp16's smallest subnormal), huge (the scale
+    clamps to fp16's largest value and codes saturate), one non-zero weight per group.
+    With H = I the method reduces to round-to-nearest, so codes, scales and zeros must
+    equal the oracle's bit for bit."""
+    dev = _dev()
+    n = 512
+    rng = np.random.default_rng(bits * 10 + int(sym))
+    rows = [np.zeros(n), np.full(n, 0.01), np.full(n, -0.03), 1e-9 * rng.standard_normal(n),
+            1e6 * rng.standard_normal(n), 3e-6 * rng.standard_normal(n)]
+    lone = np.zeros(n)
+    lone[::32] = 0.05 * rng.standard_normal(n // 32)
+    rows.append(lone)
+    W = np.stack(rows * 5).astype(np.float32)                 # 35 rows
+    H = torch.eye(n, dtype=torch.float32, device=dev)
+    p = G.prepare(H, 0.01, False)
+    q = G.quantize_layer(_w_tensor(W, dev), p, bits, gs, sym, want_codes=True)
+    G.raise_on_status(p.status, "degenerate groups")
+    rc, rs, rz = O.rtn(W, bits, gs, sym)
+    assert np.array_equal(q.scales.cpu().numpy(), rs.astype(np.float16))
+    assert np.array_equal(q.zeros.cpu().numpy(), rz.astype(np.float16))
+    assert np.array_equal(q.codes.cpu().numpy(), rc)
