@@ -483,3 +483,28 @@ def test_padded_columns_quantize_to_zero_and_carry_no_error(bits, gs, sym, act):
     assert not res.sw.err[:, pos].any()
     # their groups continue the processing order's numbering
     assert np.array_equal(res.g_idx[pad], (pos // gs).astype(np.int32))
+
+
+def test_rows_are_independent_given_u(monkeypatch):
+    # polydesk, "Etape 1": the inverse-Hessian work is shared by all rows, and each row is
+    # quantized on its own; the full-size parity tests compare sampled rows on this basis.
+    W, x = S.small_case(64, 384, 1024, seed=5)
+    prep = O.prepare(O.hessian(x), 0.01, True)
+    rows = np.array([3, 17, 18, 40, 63])
+    sw, codes = O.quantize_layer(W, prep, 4, 128, False, 128)
+    sw_r, codes_r = O.quantize_layer(W[rows], prep, 4, 128, False, 128)
+    assert np.array_equal(codes[rows], codes_r)
+    assert np.array_equal(sw.scales[:, rows], sw_r.scales) and np.array_equal(sw.zeros[:, rows], sw_r.zeros)
+    assert np.allclose(sw.err[rows], sw_r.err, rtol=0, atol=1e-12)
+    # planted mistake: parameters shared by all rows of a group (a per-tensor range) couple
+    # the rows, and the subset no longer reproduces them
+    real = O.group_params
+
+    def shared(wg, bits, sym):
+        s, z = real(np.broadcast_to(np.asarray(wg, np.float32).reshape(1, -1), (wg.shape[0], wg.size)), bits, sym)
+        return s, z
+
+    monkeypatch.setattr(O, "group_params", shared)
+    _, codes_all = O.quantize_layer(W, prep, 4, 128, False, 128)
+    _, codes_sub = O.quantize_layer(W[rows], prep, 4, 128, False, 128)
+    assert not np.array_equal(codes_all[rows], codes_sub)
