@@ -1,4 +1,6 @@
-// K0 ingest, K3 column sweep, K4 lazy trailing update, K5 packing.
+// K0 ingest, K3 column sweep, K4 lazy trailing update, K5 packing; the zero points
+// packed into words; W read as the first columns of a zero-padded layer
+// ("polydesk.ai/glossaire/gptq", "Limites de GPTQ": weights padded with zeros).
 //
 // "polydesk.ai/glossaire/gptq":
 //   "Etape 2" - per column: quantize (rounding + scale), take the error, push it
