@@ -288,13 +288,17 @@ GPTQ_API int gptq_pack_zeros(const uint16_t* zeros, int groups, int out, int bit
  * static device array of GPTQ_NOALLOC_SCRATCH_BYTES inside the library instead
  * of `ws`:
  *
- * - A layer whose gptq_quantize_workspace_size(out, n, block) exceeds
- *   GPTQ_NOALLOC_SCRATCH_BYTES is rejected with GPTQ_ERR_WORKSPACE before
- *   anything is enqueued.
+ * - The arguments are checked first, exactly as gptq_quantize_layer checks them
+ *   (same codes, same order); then a layer whose
+ *   gptq_quantize_workspace_size(out, n, block) exceeds
+ *   GPTQ_NOALLOC_SCRATCH_BYTES is rejected with GPTQ_ERR_WORKSPACE.  Nothing is
+ *   enqueued in either case.
  * - Every GPU that loads the library holds one copy of the array until the
  *   process exits.  The first call on a device looks up the array's device
- *   address (cudaGetSymbolAddress, with that device current) and caches it;
- *   make that first call before any stream capture.
+ *   address (cudaGetSymbolAddress, with that device current) and caches it for
+ *   the life of the process; make that first call before any stream capture,
+ *   and do not use this call across cudaDeviceReset (the cached address would
+ *   belong to the destroyed context).
  * - All calls on a device share the array, which keeps the last call's
  *   contents (every byte a call reads from it is written by the same call
  *   first).  Calls whose work overlaps on the GPU - on different streams, or

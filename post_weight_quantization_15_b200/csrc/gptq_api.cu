@@ -112,10 +112,14 @@ size_t gptq_quantize_workspace_size(int out, int n, int block) {
   return quantize_ws_bytes(out, n, block);
 }
 
-int gptq_quantize_layer_padded(const void* W, int w_dtype, int out, int w_cols, int n, const float* U,
-                               const int32_t* perm, const uint8_t* dead, int bits, int group_size, int sym, int block,
-                               int32_t* qweight, uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes,
-                               float* err_sq, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+}  // extern "C"
+
+namespace gptq {
+// Every check of gptq_quantize_layer_padded except the workspace's, in the order the
+// ABI reports them; shared with the entry point whose scratch is a static array.
+int check_quantize_args(const void* W, int w_dtype, int out, int w_cols, int n, const float* U, int bits,
+                        int group_size, int block, const int32_t* qweight, const uint16_t* scales,
+                        const uint16_t* zeros, const int32_t* g_idx, const int32_t* d_status) {
   if (W == nullptr || U == nullptr || qweight == nullptr || scales == nullptr || zeros == nullptr ||
       g_idx == nullptr || d_status == nullptr)
     return GPTQ_ERR_INVALID_ARG;
@@ -126,6 +130,19 @@ int gptq_quantize_layer_padded(const void* W, int w_dtype, int out, int w_cols, 
   if (block != 128) return GPTQ_ERR_UNSUPPORTED;
   if (n % 32 != 0) return GPTQ_ERR_UNSUPPORTED;
   if (group_size > 0 && (n % group_size != 0 || block % group_size != 0)) return GPTQ_ERR_UNSUPPORTED;
+  return GPTQ_OK;
+}
+}  // namespace gptq
+
+extern "C" {
+
+int gptq_quantize_layer_padded(const void* W, int w_dtype, int out, int w_cols, int n, const float* U,
+                               const int32_t* perm, const uint8_t* dead, int bits, int group_size, int sym, int block,
+                               int32_t* qweight, uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes,
+                               float* err_sq, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  const int arc = check_quantize_args(W, w_dtype, out, w_cols, n, U, bits, group_size, block, qweight, scales, zeros,
+                                      g_idx, d_status);
+  if (arc != GPTQ_OK) return arc;
   if (ws == nullptr || ws_bytes < quantize_ws_bytes(out, n, block) || !aligned(ws, 256)) return GPTQ_ERR_WORKSPACE;
   return launch_quantize(W, w_dtype, out, w_cols, n, U, perm, dead, bits, group_size, sym ? 1 : 0, block, qweight,
                          scales, zeros, g_idx, codes, err_sq, ws, d_status, as_stream(stream));

@@ -23,6 +23,10 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
 
 // ---- K0/K3/K4/K5: quantize ---------------------------------------------------
 size_t quantize_ws_bytes(int out, int n, int block);
+// The argument checks of gptq_quantize_layer_padded, workspace excluded (GPTQ_OK or the error code).
+int check_quantize_args(const void* W, int w_dtype, int out, int w_cols, int n, const float* U, int bits,
+                        int group_size, int block, const int32_t* qweight, const uint16_t* scales,
+                        const uint16_t* zeros, const int32_t* g_idx, const int32_t* d_status);
 // W [out, w_cols] (w_cols <= n; columns w_cols .. n-1 are zero padding).
 int launch_quantize(const void* W, int w_dtype, int out, int w_cols, int n, const float* U, const int32_t* perm,
                     const uint8_t* dead, int bits, int gs, int sym, int block, int32_t* qweight,

@@ -33,7 +33,10 @@ void* g_scratch_addr[kMaxDevices] = {};
 
 // Device address of the array on the current device.  Host code cannot use
 // g_noalloc_scratch itself: on the host that name is a stand-in, not a device
-// address.  Looked up once per device, with that device current.
+// address.  Looked up once per device, with that device current, and kept for the
+// life of the process: after cudaDeviceReset the cached address belongs to a
+// context that no longer exists, so this entry point must not be used across a
+// device reset.
 int scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return GPTQ_ERR_CUDA;
@@ -51,13 +54,18 @@ int scratch_address(void** out) {
 
 }  // namespace
 
+using namespace gptq;
+
 extern "C" int gptq_quantize_layer_noalloc(const void* W, int w_dtype, int out, int n, const float* U,
                                            const int32_t* perm, const uint8_t* dead, int bits, int group_size,
                                            int sym, int block, int32_t* qweight, uint16_t* scales,
                                            uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq,
                                            int32_t* d_status, void* stream) {
-  if (out <= 0 || n <= 0) return GPTQ_ERR_INVALID_ARG;
-  if (gptq_quantize_workspace_size(out, n, block) > kScratchBytes) return GPTQ_ERR_WORKSPACE;
+  // the arguments are checked exactly as gptq_quantize_layer checks them, before the size
+  const int arc = check_quantize_args(W, w_dtype, out, n, n, U, bits, group_size, block, qweight, scales, zeros,
+                                      g_idx, d_status);
+  if (arc != GPTQ_OK) return arc;
+  if (quantize_ws_bytes(out, n, block) > kScratchBytes) return GPTQ_ERR_WORKSPACE;
   void* ws = nullptr;
   const int rc = scratch_address(&ws);
   if (rc != GPTQ_OK) return rc;

@@ -300,6 +300,36 @@ def alloc_quantized(out: int, n: int, bits: int, group_size: int, sym: bool, dev
         bits=bits, group_size=group_size, sym=bool(sym))
 
 
+def _check_shape(t: Optional[torch.Tensor], shape, dtype, what: str):
+    if t is not None and (tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous()):
+        raise ValueError(f"{what} must be a contiguous {dtype} tensor of shape {tuple(shape)}, "
+                         f"got {t.dtype} {tuple(t.shape)}")
+
+
+def _check_prepared(prep: Prepared, n: int):
+    """U fp32 [n, n], perm int32 [n], dead uint8 [n], status int32 [4]."""
+    _check_shape(prep.U, (n, n), torch.float32, "prep.U")
+    _check_shape(prep.perm, (n,), torch.int32, "prep.perm")
+    _check_shape(prep.dead, (n,), torch.uint8, "prep.dead")
+    if prep.status is None:
+        raise ValueError("prep.status must be a status block")
+    _check_shape(prep.status, (4,), torch.int32, "prep.status")
+
+
+def _check_quantized(out: QuantizedLayer, o: int, n: int):
+    """Output buffers sized for an o x n layer at out.bits / out.group_size."""
+    bits, gs = int(out.bits), int(out.group_size)
+    if bits not in (2, 3, 4, 8) or gs not in (-1, 32, 64, 128) or (gs > 0 and n % gs) or (n * bits) % 32:
+        raise ValueError(f"unsupported bits={bits} / group_size={gs} for n={n}")
+    G = 1 if gs == -1 else n // gs
+    _check_shape(out.qweight, (n * bits // 32, o), torch.int32, "qweight")
+    _check_shape(out.scales, (G, o), torch.float16, "scales")
+    _check_shape(out.zeros, (G, o), torch.float16, "zeros")
+    _check_shape(out.g_idx, (n,), torch.int32, "g_idx")
+    _check_shape(out.codes, (o, n), torch.uint8, "codes")
+    _check_shape(out.err_sq, (o,), torch.float32, "err_sq")
+
+
 def quantize_layer(W: torch.Tensor, prep: Prepared, bits: int = 4, group_size: int = 128, sym: bool = False,
                    block: int = 128, want_codes: bool = False, want_err: bool = False,
                    ws: Optional[torch.Tensor] = None, out: Optional[QuantizedLayer] = None,
@@ -323,6 +353,8 @@ def quantize_layer(W: torch.Tensor, prep: Prepared, bits: int = 4, group_size: i
         ws = workspace(need, dev)
     if out is None:
         out = alloc_quantized(o, n, bits, group_size, sym, dev, want_codes, want_err)
+    else:
+        _check_quantized(out, o, n)
     # w_cols < n: W is zero-padded to n columns (gptq_quantize_layer_padded)
     _check(lib().gptq_quantize_layer_padded(_ptr(W), _DTYPE_CODE[W.dtype], o, w_cols, n, _ptr(prep.U),
                                             _ptr(prep.perm), _ptr(prep.dead), int(bits), int(group_size),
@@ -408,10 +440,13 @@ def quantize_layer_noalloc(W: torch.Tensor, prep: Prepared, out: QuantizedLayer,
     raise GptqError(ERR_WORKSPACE).  Calls that overlap on the GPU race on the
     shared array.
     """
-    _require_cuda(W)
     if W.dim() != 2 or not W.is_contiguous() or W.dtype not in _DTYPE_CODE:
         raise ValueError("W must be a contiguous fp32/fp16/bf16 [out, n] tensor")
     o, n = W.shape
+    _check_prepared(prep, n)
+    _check_quantized(out, o, n)
+    _require_cuda(W, prep.U, prep.perm, prep.dead, prep.status, out.qweight, out.scales, out.zeros, out.g_idx,
+                  out.codes, out.err_sq)
     _check(lib().gptq_quantize_layer_noalloc(_ptr(W), _DTYPE_CODE[W.dtype], o, n, _ptr(prep.U), _ptr(prep.perm),
                                              _ptr(prep.dead), int(out.bits), int(out.group_size), int(out.sym),
                                              int(block), _ptr(out.qweight), _ptr(out.scales), _ptr(out.zeros),

@@ -108,3 +108,52 @@ def test_padded_width():
     assert G.padded_width(300, -1) == 320 and G.padded_width(4096, 128) == 4096
     # the page's example of a width that 128 x 8 does not divide
     assert G.padded_width(29568 // 8, 128) == 3712
+
+
+def test_noalloc_checks_arguments_before_the_scratch_size(L):
+    """The no-alloc entry point reports argument errors exactly as gptq_quantize_layer does,
+    even for a layer whose workspace would not fit its static scratch (4096 x 4096)."""
+    P = ctypes.c_void_p
+    fake = P(256)
+    big = (4096, 4096)
+    tail = (fake, fake, fake, fake, None, None, fake, None)
+    assert L.gptq_quantize_layer_noalloc(None, 0, *big, fake, None, None, 4, 128, 0, 128, *tail) == -1
+    assert L.gptq_quantize_layer_noalloc(fake, 0, *big, fake, None, None, 4, 128, 0, 64, *tail) == -2   # block
+    assert L.gptq_quantize_layer_noalloc(fake, 0, *big, fake, None, None, 5, 128, 0, 128, *tail) == -2  # bits
+    assert L.gptq_quantize_layer_noalloc(fake, 0, 524281, 128, fake, None, None, 4, 128, 0, 128, *tail) == -2
+    assert L.gptq_quantize_layer_noalloc(fake, 7, *big, fake, None, None, 4, 128, 0, 128, *tail) == -1  # dtype
+    # valid arguments: only now does the size decide
+    assert L.gptq_quantize_layer_noalloc(fake, 0, *big, fake, None, None, 4, 128, 0, 128, *tail) == -7
+
+
+def test_noalloc_binding_rejects_mismatched_buffers_without_launching():
+    """Outputs sized for another layer or bit width, or a U of another size, raise
+    ValueError in the binding before anything reaches the library."""
+    import torch
+
+    import post_weight_quantization_15_b200 as G
+    o, n = 64, 256
+    W = torch.zeros((o, n), dtype=torch.float16)
+
+    def prep(m):
+        return G.Prepared(U=torch.zeros((m, m)), perm=torch.zeros(m, dtype=torch.int32),
+                          dead=torch.zeros(m, dtype=torch.uint8), status=torch.zeros(4, dtype=torch.int32),
+                          desc_act=False)
+
+    good = G.alloc_quantized(o, n, 4, 128, False, "cpu", want_codes=True, want_err=True)
+    wrong_bits = G.alloc_quantized(o, n, 3, 128, False, "cpu")
+    wrong_bits.bits = 4                                   # qweight sized for 3 bits
+    cases = [(prep(n + 128), good, "prep.U"),             # a padded preparation
+             (prep(n), G.alloc_quantized(o + 1, n, 4, 128, False, "cpu"), "qweight"),
+             (prep(n), wrong_bits, "qweight"),
+             (prep(n), G.alloc_quantized(o, n, 4, 64, False, "cpu"), "bits"),
+             (prep(n), G.QuantizedLayer(good.qweight, good.scales, good.zeros, good.g_idx,
+                                        torch.zeros((o, n + 1), dtype=torch.uint8), None, 4, 128, False), "codes")]
+    cases[3][1].group_size = 128                          # scales / zeros sized for g64
+    for p, out, what in cases:
+        with pytest.raises(ValueError) as e:
+            G.quantize_layer_noalloc(W, p, out)
+        assert what in str(e.value) or "scales" in str(e.value), (what, str(e.value))
+    # well-shaped host tensors still never reach the library
+    with pytest.raises(ValueError, match="CUDA"):
+        G.quantize_layer_noalloc(W, prep(n), good)
