@@ -42,7 +42,8 @@ import scipy.linalg
 import scipy.linalg.lapack
 
 __all__ = [
-    "bf16_bits_to_f64", "hessian", "act_order", "prepare", "prepare_trailing", "Prepared",
+    "bf16_bits_to_f64", "hessian", "hessian_chunked", "hessian_diag", "hessian_matvec", "damped_matvec",
+    "act_order", "prepare", "prepare_trailing", "prepare_trailing_x", "Prepared",
     "group_params", "quantize_codes", "dequant_value", "sweep", "SweepResult",
     "g_idx", "unpermute_codes", "pack", "unpack", "dequantize", "layer_error",
     "rtn", "quantize_layer", "LayerResult", "gptq_layer", "pad_layer", "pack_zeros", "unpack_zeros",
@@ -68,6 +69,49 @@ def hessian(x_bits: np.ndarray) -> np.ndarray:
     """
     x = bf16_bits_to_f64(x_bits)
     return 2.0 * (x @ x.T)
+
+
+def hessian_chunked(x_bits: np.ndarray, chunk: int = 8192) -> np.ndarray:
+    """``hessian`` summed over token chunks, so that a wide X never has to exist in
+    fp64 all at once (the same fp64 sum, taken in another order)."""
+    n, N = x_bits.shape
+    H = np.zeros((n, n))
+    for t0 in range(0, N, chunk):
+        H += hessian(x_bits[:, t0:t0 + chunk])
+    return H
+
+
+def hessian_diag(x_bits: np.ndarray, chunk: int = 8192) -> np.ndarray:
+    """diag(H) = 2 . sum_t x_it^2 in fp64 (every bf16 square is exact in fp64)."""
+    n, N = x_bits.shape
+    d = np.zeros(n)
+    for t0 in range(0, N, chunk):
+        x = bf16_bits_to_f64(x_bits[:, t0:t0 + chunk])
+        d += 2.0 * np.einsum("ij,ij->i", x, x)
+    return d
+
+
+def hessian_matvec(x_bits: np.ndarray, V: np.ndarray, chunk: int = 4096) -> np.ndarray:
+    """H . V = 2 . X . (X^T . V) in fp64 without forming H (V is [n, k]).
+
+    For layers whose H the oracle cannot form in seconds: O(n.N.k) instead of O(n^2.N).
+    """
+    n, N = x_bits.shape
+    V = np.asarray(V, np.float64)
+    out = np.zeros_like(V)
+    for t0 in range(0, N, chunk):
+        x = bf16_bits_to_f64(x_bits[:, t0:t0 + chunk])
+        out += x @ (x.T @ V)
+    return 2.0 * out
+
+
+def damped_matvec(x_bits: np.ndarray, perm: np.ndarray, lam: float, V: np.ndarray) -> np.ndarray:
+    """H_d . V for the permuted, damped Hessian of ``prepare`` (no dead inputs), without
+    forming it: (H_d . V)[k] = (H . V')[perm[k]] + lam . V[k], V'[perm[k]] = V[k]."""
+    V = np.asarray(V, np.float64)
+    Vp = np.zeros_like(V)
+    Vp[perm] = V
+    return hessian_matvec(x_bits, Vp)[perm] + lam * V
 
 
 # --------------------------------------------------------------------------- #
@@ -148,8 +192,24 @@ def prepare_trailing(H: np.ndarray, damp_percent: float, desc_act: bool, m: int,
     factor of that block's inverse, the last m rows and columns of U.
     """
     H = np.asarray(H)
-    n = H.shape[0]
-    d = np.diag(H).astype(np.float64).copy()
+    return _trailing(np.diag(H).astype(np.float64), lambda idx: np.array(H[np.ix_(idx, idx)], np.float64),
+                     damp_percent, desc_act, m, order_key)
+
+
+def prepare_trailing_x(x_bits: np.ndarray, damp_percent: float, desc_act: bool, m: int,
+                       order_key: Optional[np.ndarray] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """``prepare_trailing`` of H = 2.X.X^T formed from X itself: only the exact
+    diagonal and the trailing m x m block of H are computed (for layers whose whole H
+    the oracle cannot form in seconds)."""
+    return _trailing(hessian_diag(x_bits), lambda idx: hessian_chunked(x_bits[idx]), damp_percent, desc_act, m,
+                     order_key)
+
+
+def _trailing(d: np.ndarray, block, damp_percent: float, desc_act: bool, m: int,
+              order_key: Optional[np.ndarray]) -> Tuple[np.ndarray, np.ndarray]:
+    """Steps 1-3 of ``prepare`` from diag(H) ``d``; step 4 on ``block(tail)`` = H[tail, tail]."""
+    n = d.shape[0]
+    d = d.copy()
     dead = d == 0.0
     d[dead] = 1.0
     if desc_act:
@@ -161,7 +221,7 @@ def prepare_trailing(H: np.ndarray, damp_percent: float, desc_act: bool, m: int,
         perm = np.arange(n, dtype=np.int64)
     lam = float(damp_percent) * float(np.mean(d))
     tail = perm[n - m:]
-    Hs = np.array(H[np.ix_(tail, tail)], dtype=np.float64)
+    Hs = block(tail)
     Hs[np.arange(m), np.arange(m)] = d[tail] + lam
     L = np.linalg.cholesky(Hs)
     Linv, info = scipy.linalg.lapack.dtrtri(L, lower=1)

@@ -20,6 +20,48 @@ CODE_MISMATCH_MAX = 0.005
 REL_ERR_TOL = 0.02
 SCALE_TOL = 1e-3
 
+# The Hessian kernel's summation, which the Hessian bound below follows: every
+# 16-token tensor-core instruction adds 16 exact bf16 products to its fp32
+# accumulator; an accumulator starts from zero every 256 tokens (a chunk); the
+# finished chunks are added into fp32 registers with round-to-nearest; at the end
+# of a call H_ij += 2 . sum (one more rounding).
+HESS_MMA_K = 16
+HESS_CHUNK = 256
+
+
+def hessian_bound(token_counts) -> float:
+    """c such that |H_gpu[i, j] - H[i, j]| <= c . sqrt(H_ii . H_jj), H the exact 2.X.X^T.
+
+    ``token_counts``: the tokens of each accumulate call (kernel launch) that formed H.
+    Derivation, with S = sum_t |x_it x_jt| and u = 2^-23 (one fp32 ulp, relative):
+    * inside a chunk, each instruction sums 17 terms (16 products and the accumulator),
+      each at most sum-so-far <= S_chunk in magnitude; whether the tensor core rounds or
+      truncates after aligning them, each term loses at most one ulp: <= 17 u S_chunk per
+      instruction, 16 instructions per 256-token chunk: 272 u S_chunk;
+    * each addition of a chunk into the fp32 register sum rounds to nearest: <= u/2 S
+      each, one per chunk, plus the final H += 2 . sum, one per call;
+    * 2 S <= sqrt(H_ii H_jj) (Cauchy-Schwarz), the factor 2 being exact.
+    So c = 17 . 16 . u + (chunks + calls) . u/2.  At 65,536 tokens in one call,
+    c = 4.8e-5: a kernel that dropped one 256-token chunk (0.4 % of the sum) fails.
+    """
+    counts = [int(t) for t in token_counts if int(t) > 0]
+    chunks = sum((t + HESS_CHUNK - 1) // HESS_CHUNK for t in counts)
+    per_chunk = (HESS_MMA_K + 1) * (HESS_CHUNK // HESS_MMA_K)
+    return per_chunk * 2.0 ** -23 + (chunks + len(counts)) * 2.0 ** -24
+
+
+def u_residual_bound(n: int) -> float:
+    """Bound on ||U . H_d . U^T . v - v|| / ||v|| for the GPU's U and the exact H_d.
+
+    U H_d U^T = I exactly (H_d^-1 = U^T U); a computed U = (I + F) U_exact gives
+    U H_d U^T - I = F + F^T + O(F^2), with F the factor's backward error, which does
+    not carry H_d's condition number.  Rounding errors of a length-n fp32 chain grow
+    like sqrt(n) times the unit roundoff (fp32 LAPACK factors measured 0.07-0.08 .
+    sqrt(n) . 2^-23 for n = 2048 and 4096); the tensor-core products keep operands to
+    2^-21 (the TF32 low parts), so the bound is 8 . sqrt(n) . 2^-21.
+    """
+    return 8.0 * float(np.sqrt(n)) * 2.0 ** -21
+
 
 @dataclasses.dataclass
 class Comparison:

@@ -7,7 +7,7 @@ import pytest
 
 import synthetic as S
 from oracle import gptq_oracle as O
-from tests.parity import CODE_MISMATCH_MAX, REL_ERR_TOL, compare_layer
+from tests.parity import CODE_MISMATCH_MAX, REL_ERR_TOL, compare_layer, hessian_bound
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -92,11 +92,9 @@ def test_hessian_and_diag_against_oracle():
     H64 = O.hessian(x)
     Hg = H.cpu().numpy().astype(np.float64)
     iu = np.triu_indices(300)
-    # fp32 accumulation of N exact products, each addition off by at most one ulp
-    # (the tensor cores need not round to nearest): |error| <= N . 2^-23 .
-    # sum_t |x_it x_jt| <= N . 2^-23 . sqrt(H_ii H_jj) (Cauchy-Schwarz).
+    # the bound derived from the kernel's chunked summation (tests/parity.py), two calls
     rel = np.abs(Hg[iu] - H64[iu]) / np.sqrt(np.outer(np.diag(H64), np.diag(H64)))[iu]
-    assert rel.max() <= 2504 * 2.0 ** -23, rel.max()
+    assert rel.max() <= hessian_bound([1200, 1304]), rel.max()
     print("hessian max normalised error", rel.max())
     assert np.allclose(hd.cpu().numpy(), np.diag(H64), rtol=1e-13, atol=0)
 
@@ -116,7 +114,8 @@ def test_hessian_from_host_memory_in_chunks():
     Hg = H.cpu().numpy().astype(np.float64)
     iu = np.triu_indices(300)
     rel = np.abs(Hg[iu] - H64[iu]) / np.sqrt(np.outer(np.diag(H64), np.diag(H64)))[iu]
-    assert rel.max() <= 2504 * 2.0 ** -23, rel.max()
+    # one launch per staged chunk of 512 tokens (the staging area's halves)
+    assert rel.max() <= hessian_bound([512] * 4 + [2504 - 4 * 512]), rel.max()
     assert np.allclose(hd.cpu().numpy(), np.diag(H64), rtol=1e-13, atol=0)
     # the whole path from host tensors gives the device path's result
     W, x = S.small_case(48, 320, 2504, seed=4)
@@ -192,7 +191,9 @@ def test_err_sq_matches_loss_identity():
     d = W.astype(np.float64)[:, ora.perm] - What
     rhs = np.einsum("ij,jk,ik->i", d, ora.prep.Hd, d)
     lhs = q.err_sq.cpu().numpy().astype(np.float64)
-    assert np.allclose(lhs, rhs, rtol=2e-2)
+    # the identity holds to rounding: fp32 sums of 256 squares on the GPU (~1e-7), the
+    # GPU's U and compensation in 3xTF32 against the oracle's fp64 H_d (~1e-6)
+    assert np.allclose(lhs, rhs, rtol=1e-4), np.max(np.abs(lhs / rhs - 1))
 
 
 # --------------------------------------------------------------------------- #
@@ -262,76 +263,7 @@ def test_worked_example_layer_full_size():
     assert c.ok(), c
 
 
-# --------------------------------------------------------------------------- #
-# Llama-shaped layers, act-order, symmetric and low-bit settings.  Rows are
-# independent given U, so the oracle sweeps a sample of rows against its own
-# (full) preparation; calibration tokens are reduced so its fp64 Hessian
-# finishes in seconds.
-# --------------------------------------------------------------------------- #
-def _sampled_compare(W, x, bits, gs, sym, act, rows, H64=None, prep_o=None):
-    import tests.parity as P
-    q, prep, Hg = _run_gpu(W, x, bits, gs, sym, act)
-    if H64 is None:
-        H64 = O.hessian(x)
-    if prep_o is None:
-        prep_o = O.prepare(H64, 0.01, act, order_key=np.diag(H64))
-    perm_g = prep.perm.cpu().numpy().astype(np.int64)
-    assert np.array_equal(perm_g, prep_o.perm)
-    sw, codes_o = O.quantize_layer(W[rows], prep_o, bits, gs, sym, 128)
-    codes_g = q.codes.cpu().numpy()
-    qw = q.qweight.cpu().numpy()
-    assert np.array_equal(O.pack(codes_g, bits).view(np.uint32), qw.view(np.uint32))
-    assert np.array_equal(O.g_idx(perm_g, gs), q.g_idx.cpu().numpy())
-    mism = float(np.mean(codes_g[rows] != codes_o))
-    sc_g = q.scales.cpu().numpy()[:, rows]
-    zr_g = q.zeros.cpu().numpy()[:, rows]
-    n = W.shape[1]
-    What_g = O.dequantize(qw[:, rows], sc_g, zr_g, q.g_idx.cpu().numpy(), bits, n)
-    What_o = O.dequantize(O.pack(codes_o, bits), sw.scales.astype(np.float16), sw.zeros.astype(np.float16),
-                          O.g_idx(prep_o.perm, gs), bits, n)
-    rel_g = O.layer_error(W[rows], What_g, H64)
-    rel_o = O.layer_error(W[rows], What_o, H64)
-    G = sc_g.shape[0]
-    gsz = n if gs == -1 else gs
-    cp_g, cp_o = codes_g[rows][:, prep_o.perm], codes_o[:, prep_o.perm]
-    same = np.logical_and.accumulate((cp_g == cp_o).reshape(len(rows), G, gsz).all(axis=2), axis=1).T
-    s_rel = np.max(np.abs(sc_g[same].astype(float) - sw.scales[same]) / sw.scales[same]) if same.any() else 0.0
-    z_eq = np.array_equal(zr_g[same].astype(float), sw.zeros[same].astype(float))
-    print(f"mismatch {mism:.5f} rel_err gpu {rel_g:.6g} oracle {rel_o:.6g} scale_rel {s_rel:.3g} zeros_eq {z_eq}")
-    assert mism <= P.CODE_MISMATCH_MAX
-    assert abs(rel_g / rel_o - 1) <= P.REL_ERR_TOL
-    assert s_rel <= P.SCALE_TOL and z_eq
-    return q, prep
-
-
-def test_llama7b_down_shape_act_order_symmetric():
-    wl = S.workloads()["llama2-7b-block"]
-    down = [l for l in wl.layers if l.name == "down"][0]
-    st = wl.settings[0]
-    import dataclasses
-    x = S.make_x(dataclasses.replace(down.x, tokens=8192))
-    W = S.make_w(down.w)
-    rows = np.random.default_rng(0).choice(W.shape[0], 48, replace=False)
-    _sampled_compare(W, x, st.bits, st.group_size, st.sym, st.desc_act, np.sort(rows))
-
-
-@pytest.fixture(scope="module")
-def gate_lowbit():
-    wl = S.workloads()["llama2-7b-mlp-lowbit"]
-    gate = [l for l in wl.layers if l.name == "gate"][0]
-    import dataclasses
-    x = S.make_x(dataclasses.replace(gate.x, tokens=8192))
-    W = S.make_w(gate.w)
-    H64 = O.hessian(x)
-    prep_o = O.prepare(H64, 0.01, True, order_key=np.diag(H64))
-    rows = np.sort(np.random.default_rng(1).choice(W.shape[0], 64, replace=False))
-    return W, x, H64, prep_o, rows
-
-
-@pytest.mark.parametrize("bits,gs", [(3, 128), (3, 64), (2, 128), (2, 64)])
-def test_llama7b_gate_shape_low_bit_sweep(gate_lowbit, bits, gs):
-    W, x, H64, prep_o, rows = gate_lowbit
-    _sampled_compare(W, x, bits, gs, False, True, rows, H64=H64, prep_o=prep_o)
+# The Llama-shaped layers at their own token counts, every setting: test_gpu_full_shapes.py.
 
 
 def test_bounded_wait_reports_timeout_and_the_context_survives(monkeypatch):
@@ -445,7 +377,8 @@ def test_zero_padded_layer_from_host_memory():
     Hg = H.cpu().numpy().astype(np.float64)
     iu = np.triu_indices(n_pad)
     norm = np.sqrt(np.maximum(np.outer(np.diag(H64), np.diag(H64)), 1e-300))[iu]
-    assert (np.abs(Hg[iu] - H64[iu]) / norm).max() <= 2504 * 2.0 ** -23
+    # one launch per staged chunk of at least 64 tokens: at most ceil(2504 / 64) launches
+    assert (np.abs(Hg[iu] - H64[iu]) / norm).max() <= hessian_bound([64] * 39 + [8])
     assert not Hg[iu][H64[iu] == 0].any()
     assert np.allclose(hd.cpu().numpy(), np.diag(H64), rtol=1e-13, atol=0)
     # the whole padded path from host tensors gives the device path's result

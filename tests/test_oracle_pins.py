@@ -42,6 +42,53 @@ def test_hessian_brute_force_and_symmetry():
     assert np.array_equal(H, H.T)
 
 
+def test_hessian_without_forming_it_brute_force():
+    # The matrix-free forms the large-layer parity tests use: chunked H, exact diagonal,
+    # H . V and H_d . V, each against pure-Python sums over tokens on a tiny X.
+    n, N = 6, 11
+    x = S.make_x(S.XSpec(n, N, 2, 0.2, 4.0, 5, 1))
+    xf = S.bf16_bits_to_f32(x).astype(float).tolist()
+    rng = np.random.default_rng(2)
+    V = rng.standard_normal((n, 2))
+    Hc = O.hessian_chunked(x, chunk=4)          # three chunks, the last ragged
+    d = O.hessian_diag(x, chunk=4)
+    HV = O.hessian_matvec(x, V, chunk=3)
+    for i in range(n):
+        assert d[i] == pytest.approx(2.0 * sum(v * v for v in xf[i]), rel=1e-15)
+        for j in range(n):
+            hij = 2.0 * sum(xf[i][t] * xf[j][t] for t in range(N))
+            assert Hc[i, j] == pytest.approx(hij, rel=1e-14, abs=1e-14)
+        for c in range(2):
+            hv = 2.0 * sum(xf[i][t] * sum(xf[j][t] * V[j, c] for j in range(n)) for t in range(N))
+            assert HV[i, c] == pytest.approx(hv, rel=1e-12, abs=1e-12)
+    # H_d . V with an order and a damping: (H_d V)[k] = sum_l H[perm k, perm l] V[l] + lam V[k]
+    perm = np.array([3, 0, 5, 1, 4, 2])
+    lam = 0.37
+    HdV = O.damped_matvec(x, perm, lam, V)
+    for k in range(n):
+        for c in range(2):
+            ref = lam * V[k, c] + sum(2.0 * sum(xf[perm[k]][t] * xf[perm[l]][t] for t in range(N)) * V[l, c]
+                                      for l in range(n))
+            assert HdV[k, c] == pytest.approx(ref, rel=1e-12, abs=1e-12)
+    # a planted mistake: the order applied the wrong way round
+    assert not np.allclose(O.damped_matvec(x, np.argsort(perm), lam, V), HdV)
+
+
+@pytest.mark.parametrize("act", [False, True])
+def test_trailing_factor_from_x_inverts_the_trailing_block(act):
+    # U's trailing block formed from X alone (exact diagonal + the block of H) is the
+    # upper factor of the inverse of H_d's trailing block: U_t^T U_t H_d[t, t] = I, with
+    # H_d from the full preparation; and it equals the full factor's block.
+    n, m = 48, 20
+    x = S.make_x(S.XSpec(n, 400, 3, 0.2, 10.0, 9, 7))
+    full = O.prepare(O.hessian(x), 0.02, act)
+    Ut, perm = O.prepare_trailing_x(x, 0.02, act, m)
+    assert np.array_equal(perm, full.perm)
+    assert np.all(np.tril(Ut, -1) == 0) and np.all(np.diag(Ut) > 0)
+    assert np.allclose(Ut.T @ Ut @ full.Hd[n - m:, n - m:], np.eye(m), atol=1e-9)
+    assert np.allclose(Ut, full.U[n - m:, n - m:], rtol=1e-10, atol=1e-12 * np.abs(full.U).max())
+
+
 def test_bf16_generator_matches_torch_rounding():
     torch = pytest.importorskip("torch")
     rng = np.random.default_rng(5)
