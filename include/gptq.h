@@ -277,6 +277,48 @@ GPTQ_API int gptq_pack_zeros(const uint16_t* zeros, int groups, int out, int bit
                              int32_t* qzeros, int32_t* d_status, void* stream);
 
 /*
+ * Kernel timing trace.  The GPTQ pages have no counterpart to these calls: they
+ * are a measurement aid.  While the trace is on, every kernel the library launches
+ * is bracketed by two CUDA events recorded on the stream it is launched on (the
+ * caller's or one of the library's own), so that each kernel's device time can be
+ * read inside a whole call, where several library streams overlap.
+ *
+ *   gptq_trace_enable(on)   1: record from now on; 0: stop recording (what was
+ *                           recorded stays until read).  Process-wide, all devices.
+ *   gptq_trace_read(rows, max_rows, n_rows)
+ *                           synchronizes every recorded event, aggregates them per
+ *                           kernel (first-launch order) into rows[0 .. *n_rows),
+ *                           and clears the record (rows beyond max_rows are
+ *                           dropped).  Per row: kernel name, the unit of `work`
+ *                           ("flop": useful floating-point operations of the
+ *                           algorithm; "byte": algorithmic HBM bytes; "" none),
+ *                           launches, summed device milliseconds and summed work.
+ *                           Returns GPTQ_ERR_CUDA if an event could not be read.
+ * Recording costs two event records per launch; the events are created per
+ * launch and destroyed when read.  Make no call with the trace on inside a stream
+ * capture.
+ */
+typedef struct {
+  const char* kernel;
+  const char* work_unit;
+  uint64_t launches;
+  double ms;
+  double work;
+} gptq_trace_row;
+GPTQ_API int gptq_trace_enable(int on);
+GPTQ_API int gptq_trace_read(gptq_trace_row* rows, int max_rows, int* n_rows);
+
+/*
+ * gptq_probe_fp32_peak - measurement aid (no counterpart on the pages): launches
+ * `blocks` blocks of 256 threads, each thread running 8 independent chains of
+ * iters x 16 fp32 FMAs (2 . blocks . 256 . iters . 128 flop in all) on `stream`;
+ * timed by the caller, it gives the FP32 CUDA-core peak that bounds the library's
+ * non-tensor kernels.  `out` is device memory of blocks . 256 floats that the
+ * kernel may write (it normally writes nothing).
+ */
+GPTQ_API int gptq_probe_fp32_peak(float* out, int blocks, int iters, void* stream);
+
+/*
  * gptq_quantize_layer_noalloc - gptq_quantize_layer without a caller workspace.
  *
  * The GPTQ pages have no counterpart to this call: it exists for callers that

@@ -2,7 +2,7 @@
 from .gptq import (  # noqa: F401
     GptqError, Prepared, QuantizedLayer, alloc_quantized, gptq_quantize, hessian_accumulate, hessian_accumulate_host, kernel_launches, lib, library_path,
     new_status, pack, pack_zeros, padded_width, prepare, quantize_layer, quantize_layer_noalloc, quantize_workspace_size, raise_on_status, status_read, status_reset,
-    status_string, workspace,
+    status_string, trace_enable, trace_read, workspace,
 )
 
 __version__ = "0.1.0"

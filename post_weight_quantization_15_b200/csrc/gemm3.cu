@@ -368,9 +368,12 @@ int launch_split_tf32(const float* X, int rows, int cols, int ldx, float* hi, fl
 
 int launch_gemm3(float* C, int ldc, int M, int N, int K, const float* Ahi, const float* Alo, int lda,
                  const float* Bhi, const float* Blo, int ldb, bool lower, int32_t* st, cudaStream_t s,
-                 bool store, float* Chi, float* Clo, int ldh) {
+                 bool store, float* Chi, float* Clo, int ldh, const char* trace) {
   if (M <= 0 || N <= 0 || K <= 0) return GPTQ_OK;
   GemmOut out{C, ldc, store ? 1 : 0, Chi, Clo, ldh};
+  // useful flops of the product (lower: about the tiles that reach the lower triangle)
+  const double flop = 2.0 * M * N * K * (lower ? 0.5 : 1.0);
+  TraceScope ts(trace ? trace : "gemm3", "flop", flop, s);
   // the widest tile that still gives about one CTA per SM; K beyond one chunk takes
   // the chunked (<= 128-wide) tiles
   const int64_t tm = (int64_t)cdiv(M, GM);

@@ -257,6 +257,7 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap tmap, float* H, int n, int
 
 int launch_hessian_diag64(double* hdiag, int n, const void* X, int64_t ld_x, int64_t tokens,
                           int32_t* st, cudaStream_t s) {
+  TraceScope ts("hessian_diag64", "byte", 2.0 * n * (double)tokens, s);
   hessian_diag64_kernel<<<n, DIAG_THREADS, 0, s>>>(hdiag, n, static_cast<const __nv_bfloat16*>(X), ld_x,
                                                    tokens, st);
   GPTQ_LAUNCH_CHECK();
@@ -284,6 +285,8 @@ int launch_hessian(float* H, int n, const void* X, int x_rows, int64_t ld_x, int
   const int stall = (fi != nullptr && strcmp(fi, "hessian_stall") == 0) ? 1 : 0;
   const uint64_t wait_ns = stall ? 200000000ull : tc::kWaitLimitNs;
   GPTQ_CUDA_TRY(cudaFuncSetAttribute(hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)HESS_SMEM));
+  // the algorithm's flops: the upper triangle (diagonal included) of the x_rows real rows
+  TraceScope ts("hessian_tc", "flop", (double)x_rows * (x_rows + 1) * (double)tokens, s);
   hessian_tc_kernel<<<tiles, HESS_THREADS, HESS_SMEM, s>>>(map, H, n, kblocks, st, stall, wait_ns);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;

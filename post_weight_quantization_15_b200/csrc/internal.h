@@ -6,6 +6,23 @@
 
 namespace gptq {
 
+// ---- timing trace (gptq_trace_enable): events around one launch on its stream ----
+class TraceScope {
+ public:
+  // kernel and unit are string literals; work is the launch's algorithmic work in unit
+  TraceScope(const char* kernel, const char* unit, double work, cudaStream_t s);
+  ~TraceScope();
+  TraceScope(const TraceScope&) = delete;
+  TraceScope& operator=(const TraceScope&) = delete;
+
+ private:
+  const char* kernel_;
+  const char* unit_;
+  double work_;
+  cudaStream_t s_;
+  void* a_;
+};
+
 // ---- K1: Hessian -----------------------------------------------------------
 // H [n, n] from X's first x_rows rows (x_rows <= n; the rows after them are zero padding).
 int launch_hessian(float* H, int n, const void* X, int x_rows, int64_t ld_x, int64_t tokens, int32_t* st,
@@ -41,9 +58,11 @@ int launch_pack_zeros(const uint16_t* zeros, int groups, int out, int bits, int 
 // store = false: C -= A.B^T; store = true: C = A.B^T (C may be null then, if Chi/Clo are given).
 // Chi/Clo (optional, leading dimension ldh) receive the TF32 split of the result.
 // lower: only tiles reaching the lower triangle of square C.
+// trace: the kernel name the timing trace records this launch under (nullptr: not traced).
 int launch_gemm3(float* C, int ldc, int M, int N, int K, const float* Ahi, const float* Alo, int lda,
                  const float* Bhi, const float* Blo, int ldb, bool lower, int32_t* st, cudaStream_t s,
-                 bool store = false, float* Chi = nullptr, float* Clo = nullptr, int ldh = 0);
+                 bool store = false, float* Chi = nullptr, float* Clo = nullptr, int ldh = 0,
+                 const char* trace = nullptr);
 int launch_split_tf32(const float* X, int rows, int cols, int ldx, float* hi, float* lo, int ldo,
                       const int32_t* st, cudaStream_t s);
 

@@ -832,6 +832,9 @@ int panel_loop(const PrepWs& w, int n, int ldn, AuxStream* aux, int32_t* st) {
       GPTQ_CUDA_TRY(cudaStreamWaitEvent(c, aux->trail[b2], 0));
     }
     if (panel >= NBUF) GPTQ_CUDA_TRY(cudaStreamWaitEvent(c, aux->done[b], 0));   // LI[b] is free again
+    // useful flops: the previous panel's two 128-deep products (when there is one), the
+    // block's Cholesky factorization and its triangular inverse
+    TraceScope ts_d("potrf_inv", "flop", (panel > 0 ? 4.0 * nb * nb * PB : 0.0) + 2.0 / 3.0 * nb * nb * nb, c);
     potrf_inv_kernel<<<1, DT, POTRF_SMEM, c>>>(w.A, ldn, k0, nb, n, w.LIhi[b1], w.LIlo[b1],
                                                panel > 0 ? k0 - PB : -1, w.LIhi[b], w.LIlo[b], st);
     GPTQ_LAUNCH_CHECK();
@@ -848,7 +851,7 @@ int panel_loop(const PrepWs& w, int n, int ldn, AuxStream* aux, int32_t* st) {
       if (panel == 0) rc = launch_split_tf32(w.A + (int64_t)nb * ldn, rest, nb, ldn, w.Phi, w.Plo, PB, st, o);
       if (rc == GPTQ_OK)
         rc = launch_gemm3(nullptr, 0, rest, nb, nb, w.Phi, w.Plo, PB, w.LIhi[b], w.LIlo[b], PB, false, st, o, true,
-                          w.Lhi[b], w.Llo[b], PB);
+                          w.Lhi[b], w.Llo[b], PB, "prepare_gemm3");
       if (rc != GPTQ_OK) return rc;
       GPTQ_CUDA_TRY(cudaEventRecord(aux->l21[b], o));
       const int nb2 = std::min(PB, rest);
@@ -857,14 +860,15 @@ int panel_loop(const PrepWs& w, int n, int ldn, AuxStream* aux, int32_t* st) {
         if (panel >= 1) GPTQ_CUDA_TRY(cudaStreamWaitEvent(o, aux->trail[b1], 0));
         float* Anext = w.A + (int64_t)(k0 + nb + nb2) * ldn + (k0 + nb);
         rc = launch_gemm3(Anext, ldn, rest - nb2, nb2, nb, w.Lhi[b] + (int64_t)nb2 * PB, w.Llo[b] + (int64_t)nb2 * PB,
-                          PB, w.Lhi[b], w.Llo[b], PB, false, st, o, false, w.Phi, w.Plo, PB);
+                          PB, w.Lhi[b], w.Llo[b], PB, false, st, o, false, w.Phi, w.Plo, PB, "prepare_gemm3");
         if (rc != GPTQ_OK) return rc;
         GPTQ_CUDA_TRY(cudaEventRecord(aux->next[b], o));
         // ---- the trailing update of blocks >= k + 2 ----
         GPTQ_CUDA_TRY(cudaStreamWaitEvent(t, aux->l21[b], 0));
         const float* Lh2 = w.Lhi[b] + (int64_t)nb2 * PB;
         const float* Ll2 = w.Llo[b] + (int64_t)nb2 * PB;
-        rc = launch_gemm3(Anext + nb2, ldn, rest - nb2, rest - nb2, nb, Lh2, Ll2, PB, Lh2, Ll2, PB, true, st, t);
+        rc = launch_gemm3(Anext + nb2, ldn, rest - nb2, rest - nb2, nb, Lh2, Ll2, PB, Lh2, Ll2, PB, true, st, t, false, nullptr, nullptr, 0,
+                          "prepare_gemm3");
         if (rc != GPTQ_OK) return rc;
         GPTQ_CUDA_TRY(cudaEventRecord(aux->trail[b], t));
       }
@@ -882,14 +886,14 @@ int panel_loop(const PrepWs& w, int n, int ldn, AuxStream* aux, int32_t* st) {
       rc = launch_split_tf32(Xk, k0, nb, ldn, w.XPhi, w.XPlo, PB, st, s2);
       if (rc == GPTQ_OK)
         rc = launch_gemm3(Xk, ldn, k0, nb, nb, w.XPhi, w.XPlo, PB, w.LIhi[b], w.LIlo[b], PB, false, st, s2, true,
-                          w.XQhi, w.XQlo, PB);
+                          w.XQhi, w.XQlo, PB, "prepare_gemm3");
       if (rc != GPTQ_OK) return rc;
     }
     if (rest > 0) {
       // Xt[:k0+nb, later] -= Xt[:k0+nb, k] . L21^T
       GPTQ_CUDA_TRY(cudaStreamWaitEvent(s2, aux->l21[b], 0));
       rc = launch_gemm3(w.Xt + (k0 + nb), ldn, k0 + nb, rest, nb, w.XQhi, w.XQlo, PB, w.Lhi[b], w.Llo[b], PB, false,
-                        st, s2);
+                        st, s2, false, nullptr, nullptr, 0, "prepare_gemm3");
       if (rc != GPTQ_OK) return rc;
     }
     GPTQ_CUDA_TRY(cudaEventRecord(aux->done[b], s2));

@@ -650,6 +650,7 @@ int launch_pack(const uint8_t* codes, const int32_t* invperm, int out, int n, in
                 int32_t* qweight, const int32_t* st, cudaStream_t s) {
   const int words = n * bits / 32;
   dim3 blk(32, 8), grd((unsigned)cdiv(out, 32), (unsigned)cdiv(words, 32));
+  TraceScope ts("pack", "byte", (double)out * n * (1.0 + bits / 8.0) + 4.0 * n, s);
   pack_kernel<<<grd, blk, 0, s>>>(codes, invperm, out, n, ld_codes, bits, qweight, st);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
@@ -674,6 +675,7 @@ int super_block_loop(QuantStreams* q, const QuantWs& w, int out, int n, const fl
   auto operand = [&](int sb) -> int {
     const int b0 = sb * SBK, be = b0 + SBK;   // sb < S - 1: a whole super-block with columns after it
     dim3 blk(32, 8), grd((unsigned)cdiv(n - be, 32), (unsigned)(SBK / 32));
+    TraceScope ts_t("u_operand", "byte", 12.0 * SBK * (double)(n - be), q->lo);
     u_block_transpose_split_kernel<<<grd, blk, 0, q->lo>>>(U, n, b0, SBK, be, w.Bhi[sb & 1], w.Blo[sb & 1], SBK, st);
     GPTQ_LAUNCH_CHECK();
     GPTQ_CUDA_TRY(cudaEventRecord(q->opnd[sb & 1], q->lo));
@@ -684,6 +686,8 @@ int super_block_loop(QuantStreams* q, const QuantWs& w, int out, int n, const fl
   for (int sb = 0; sb < S; ++sb) {
     const int b = sb & 1;
     const int s0 = sb * SBK, se = std::min(n, s0 + SBK);
+    // bytes of the section's work: W in, both error halves and the codes out, U's block
+    TraceScope ts_s("sweep", "byte", (double)out * (se - s0) * 13.0 + 4.0 * (se - s0) * (se - s0), q->hi);
     sweep<<<(unsigned)cdiv(out, rows_per_cta), threads, smem, q->hi>>>(w.Wf, out, n, s0, se, U, w.Ehi[b], w.Elo[b],
                                                                     w.codes_p, scales, zeros, w.rows, err_sq, bits,
                                                                     sym, st);
@@ -693,13 +697,15 @@ int super_block_loop(QuantStreams* q, const QuantWs& w, int out, int n, const fl
     GPTQ_CUDA_TRY(cudaEventRecord(q->swept, q->hi));
     GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->hi, q->opnd[b], 0));
     if (sb > 0) GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->hi, q->far, 0));
-    rc = launch_gemm3(w.Wf + se, n, out, kn, SBK, w.Ehi[b], w.Elo[b], SBK, w.Bhi[b], w.Blo[b], SBK, false, st, q->hi);
+    rc = launch_gemm3(w.Wf + se, n, out, kn, SBK, w.Ehi[b], w.Elo[b], SBK, w.Bhi[b], w.Blo[b], SBK, false, st, q->hi,
+                      false, nullptr, nullptr, 0, "trailing_update");
     if (rc != GPTQ_OK) return rc;
     GPTQ_CUDA_TRY(cudaEventRecord(q->near, q->hi));
     if (n - se > kn) {
       GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->lo, q->swept, 0));
       rc = launch_gemm3(w.Wf + se + kn, n, out, n - se - kn, SBK, w.Ehi[b], w.Elo[b], SBK,
-                        w.Bhi[b] + (size_t)kn * SBK, w.Blo[b] + (size_t)kn * SBK, SBK, false, st, q->lo);
+                        w.Bhi[b] + (size_t)kn * SBK, w.Blo[b] + (size_t)kn * SBK, SBK, false, st, q->lo,
+                        false, nullptr, nullptr, 0, "trailing_update");
       if (rc != GPTQ_OK) return rc;
     }
     GPTQ_CUDA_TRY(cudaEventRecord(q->far, q->lo));
@@ -727,6 +733,8 @@ int launch_quantize(const void* W, int w_dtype, int out, int w_cols, int n, cons
   QuantWs w = carve(ws, out, n);
   {
     dim3 blk(32, 8), grd((unsigned)cdiv(n, 128), (unsigned)cdiv(std::max(out, 1), 8));
+    const double esz = w_dtype == GPTQ_F32 ? 4.0 : 2.0;
+    TraceScope ts("ingest", "byte", (double)out * w_cols * esz + (double)out * n * 4.0, s);
     if (w_dtype == GPTQ_F32)
       ingest_kernel<float><<<grd, blk, 0, s>>>(static_cast<const float*>(W), out, w_cols, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
     else if (w_dtype == GPTQ_F16)

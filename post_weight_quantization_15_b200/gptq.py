@@ -45,6 +45,11 @@ _DTYPE_CODE = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
 _lib = None
 
 
+class _TraceRow(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_char_p), ("work_unit", ctypes.c_char_p), ("launches", ctypes.c_uint64),
+                ("ms", ctypes.c_double), ("work", ctypes.c_double)]
+
+
 class GptqError(RuntimeError):
     def __init__(self, code: int, where: str, info: Optional[int] = None):
         self.code = code
@@ -101,6 +106,12 @@ def lib() -> ctypes.CDLL:
     L.gptq_quantize_layer_padded.argtypes = [P, I, I, I, I, P, P, P, I, I, I, I, P, P, P, P, P, P, P, SZ, P, P]
     L.gptq_pack_zeros.restype = I
     L.gptq_pack_zeros.argtypes = [P, I, I, I, I, P, P, P]
+    L.gptq_trace_enable.restype = I
+    L.gptq_trace_enable.argtypes = [I]
+    L.gptq_trace_read.restype = I
+    L.gptq_trace_read.argtypes = [ctypes.POINTER(_TraceRow), I, ctypes.POINTER(ctypes.c_int)]
+    L.gptq_probe_fp32_peak.restype = I
+    L.gptq_probe_fp32_peak.argtypes = [P, I, I, P]
     L.gptq_quantize_layer_noalloc.restype = I
     L.gptq_quantize_layer_noalloc.argtypes = [P, I, I, I, P, P, P, I, I, I, I, P, P, P, P, P, P, P, P]
     _lib = L
@@ -110,6 +121,30 @@ def lib() -> ctypes.CDLL:
 def kernel_launches() -> int:
     """Kernels enqueued by the library since it was loaded (host-side counter)."""
     return int(lib().gptq_kernel_launches())
+
+
+def trace_enable(on: bool = True):
+    """Start (or stop) recording CUDA events around every kernel the library launches."""
+    _check(lib().gptq_trace_enable(1 if on else 0), "gptq_trace_enable")
+
+
+def trace_read(max_rows: int = 64) -> dict:
+    """Synchronize the recorded events and return {kernel: {launches, ms, work, unit}}; clears the record."""
+    rows = (_TraceRow * max_rows)()
+    n = ctypes.c_int(0)
+    _check(lib().gptq_trace_read(rows, max_rows, ctypes.byref(n)), "gptq_trace_read")
+    return {rows[i].kernel.decode(): {"launches": int(rows[i].launches), "ms": float(rows[i].ms),
+                                      "work": float(rows[i].work), "unit": rows[i].work_unit.decode()}
+            for i in range(n.value)}
+
+
+def probe_fp32_peak(blocks: int, iters: int, out: torch.Tensor, stream=None) -> float:
+    """Enqueue the FP32 FMA probe; returns the flops it performs (time it with events)."""
+    _require_cuda(out)
+    if out.dtype != torch.float32 or out.numel() < blocks * 256:
+        raise ValueError("out must be fp32 with at least blocks * 256 elements")
+    _check(lib().gptq_probe_fp32_peak(_ptr(out), int(blocks), int(iters), _stream(stream)), "gptq_probe_fp32_peak")
+    return 2.0 * blocks * 256 * iters * 128
 
 
 def status_string(code: int) -> str:

@@ -168,6 +168,47 @@ def make_w(spec: WSpec) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------- #
+# The same recipe drawn on the device (benchmarks)
+# --------------------------------------------------------------------------- #
+def make_x_device(spec: XSpec, device, chunk: int = 8192):
+    """X [n, tokens] as a torch bf16 tensor drawn on ``device`` with torch's generator.
+
+    Same recipe as ``make_x`` (the per-feature scales and the low-rank factor are
+    make_x's own; Z is drawn by torch), so the values differ from make_x's but the
+    distribution does not.  For benchmarks of large workloads, where generating X on
+    the host would take longer than the work itself; parity tests use make_x.
+    """
+    import torch
+    s, G = _x_feature_terms(spec)
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(int(spec.seed) * 1000003 + int(spec.stream) * 7919 + 17)
+    s32 = torch.from_numpy(s.astype(np.float32)).to(dev)[:, None]
+    G32 = torch.from_numpy(G.astype(np.float32)).to(dev)
+    ld = (spec.tokens + 7) // 8 * 8
+    out = torch.empty((spec.n, ld), dtype=torch.bfloat16, device=dev)
+    for a in range(0, spec.tokens, chunk):
+        w = min(chunk, spec.tokens - a)
+        zr = torch.randn((G32.shape[1], w), generator=gen, device=dev, dtype=torch.float32)
+        blk = torch.randn((spec.n, w), generator=gen, device=dev, dtype=torch.float32)
+        blk.addmm_(G32, zr)
+        blk.mul_(s32)
+        out[:, a:a + w] = blk.to(torch.bfloat16)       # round to nearest even
+    return out[:, :spec.tokens]
+
+
+def make_w_device(spec: WSpec, device):
+    """W [out, n] drawn on ``device`` with torch's generator (make_w's recipe; other values)."""
+    import torch
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(int(spec.seed) * 1000003 + int(spec.stream) * 7919 + 29)
+    w = torch.randn((spec.out, spec.n), generator=gen, device=dev, dtype=torch.float32)
+    w.mul_(float(spec.sigma))
+    return w.half() if spec.dtype == "f16" else w
+
+
+# --------------------------------------------------------------------------- #
 # Workloads
 # --------------------------------------------------------------------------- #
 @dataclasses.dataclass(frozen=True)
@@ -265,5 +306,5 @@ def small_case(out: int, n: int, tokens: int, seed: int, rank: int = 8, frac: fl
 
 __all__: List[str] = [
     "X_CHUNK", "XSpec", "WSpec", "QuantSettings", "Layer", "Workload",
-    "make_x", "make_w", "workloads", "small_case", "f32_to_bf16_bits", "bf16_bits_to_f32",
+    "make_x", "make_w", "make_x_device", "make_w_device", "workloads", "small_case", "f32_to_bf16_bits", "bf16_bits_to_f32",
 ]
