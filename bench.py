@@ -15,8 +15,13 @@ independently seeded layer: layers are independent problems, so there is no
 data-path collective and scaling is weak; the process group only carries the
 barrier and the max-over-ranks of the timings.
 
+The default line also carries the two decoder blocks (Llama-2-70B- and 7B-shaped:
+seconds per block, per-input stage times, Hessian and kernel roofline fractions),
+per-kernel roofline entries from the library's timing trace, and the tf32 and FP32
+peaks measured in the same run.
+
 `--impl reference` times the fp64 CPU oracle on rank 0 (the other ranks exit),
-each step on a bounded token sample of the same workload.
+each step the whole layer with all of its tokens, nothing extrapolated.
 """
 from __future__ import annotations
 
@@ -216,8 +221,12 @@ def oracle_sample(layer: S.Layer, st: S.QuantSettings, tokens: int):
     t2 = time.perf_counter()
     scale = layer.x.tokens / tokens
     est = (t1 - t0) * scale + (t2 - t1)
-    desc = (f"full layer {layer.w.out}x{layer.w.n} (prepare, sweep, pack run in full); Hessian on the first "
-            f"{tokens} of {layer.x.tokens} tokens, its time scaled x{scale:g}; measured {t2 - t0:.1f} s")
+    if tokens == layer.x.tokens:
+        desc = (f"full layer {layer.w.out}x{layer.w.n} with all {tokens} tokens, every stage measured "
+                f"(nothing extrapolated): {t2 - t0:.1f} s")
+    else:
+        desc = (f"full layer {layer.w.out}x{layer.w.n} (prepare, sweep, pack run in full); Hessian on the first "
+                f"{tokens} of {layer.x.tokens} tokens, its time extrapolated x{scale:g}; measured {t2 - t0:.1f} s")
     return est, desc
 
 
@@ -244,7 +253,9 @@ def run_reference(args):
         return 0
     wl = S.workloads()[args.workload]
     layer, st = wl.layers[0], wl.settings[0]
-    tokens = min(layer.x.tokens, args.ref_tokens)
+    # every step is the whole layer with all of its calibration tokens: nothing is
+    # extrapolated, so the line's ms_per_step is the oracle's measured time
+    tokens = layer.x.tokens
     times = []
     desc = ""
     for i in range(args.warmup + args.steps):
@@ -286,6 +297,81 @@ def hessian_traffic(n: int, tokens: int):
         except OSError:
             return None
     return HESSIAN_TRAFFIC["bytes"]
+
+
+def measure_peaks(G, torch, dev):
+    """Denominators the driver does not measure: the dense tf32 tensor-core peak
+    (torch.matmul on fp32 with TF32 allowed, 8192^3, best of 10 — the method of the
+    measured bf16 peak) and the FP32 CUDA-core peak (the library's FMA probe, best of 5)."""
+    out = {}
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = True
+    try:
+        a = torch.randn((8192, 8192), device=dev)
+        b = torch.randn((8192, 8192), device=dev)
+        best = float("inf")
+        for _ in range(12):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch.matmul(a, b)
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        out["tf32_tflops"] = 2.0 * 8192 ** 3 / (best * 1e-3) / 1e12
+        del a, b
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev
+    blocks, iters = 148 * 8, 4096
+    buf = torch.empty(blocks * 256, dtype=torch.float32, device=dev)
+    best = float("inf")
+    flop = 0.0
+    for _ in range(6):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        flop = G.gptq.probe_fp32_peak(blocks, iters, buf)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    out["fp32_tflops"] = flop / (best * 1e-3) / 1e12
+    out["how"] = ("tf32: torch.matmul fp32 8192^3 with TF32 allowed, best of 12; fp32: the library's FMA probe "
+                  f"({blocks} x 256 threads, 8 chains), best of 6; CUDA events")
+    return out
+
+
+def kernel_rooflines(trace, peaks, measured, prepare_ms=None, n=None):
+    """Per-kernel roofline entries from a traced pass (device time on each launch's stream)."""
+    hbm = float(peaks["hbm_gbs"])
+    tf32 = measured.get("tf32_tflops")
+    fp32 = measured.get("fp32_tflops")
+    bf16 = float(peaks["bf16_tflops"])
+    res = {}
+    for name, r in trace.items():
+        if r["ms"] <= 0:
+            continue
+        rate = r["work"] / (r["ms"] * 1e-3)
+        e = {"launches": r["launches"], "ms_total": r["ms"], "ms_per_launch": r["ms"] / r["launches"]}
+        if name == "hessian_tc":
+            e.update(bound="tensor", unit="TFLOP/s", achieved=rate / 1e12, peak=bf16, frac=rate / 1e12 / bf16,
+                     peak_source=f"{peaks['_source']} bf16 burst", work="n(n+1)N flop")
+        elif name in ("trailing_update", "prepare_gemm3") and tf32:
+            e.update(bound="tensor", unit="TFLOP/s", achieved=3 * rate / 1e12, peak=tf32, frac=3 * rate / 1e12 / tf32,
+                     useful_tflops=rate / 1e12, frac_useful=rate / 1e12 / tf32, peak_source="measured tf32 (in this run)",
+                     work="3 x 2MNK flop (3xTF32: three tensor passes per product)")
+        elif name == "potrf_inv" and fp32:
+            e.update(bound="alu", unit="TFLOP/s", achieved=rate / 1e12, peak=fp32, frac=rate / 1e12 / fp32,
+                     peak_source="measured fp32 FMA probe (in this run)",
+                     work="per panel: the previous panel's two 128-deep products + Cholesky + inverse of the block")
+        elif r["unit"] == "byte":
+            e.update(bound="hbm", unit="GB/s", achieved=rate / 1e9, peak=hbm, frac=rate / 1e9 / hbm,
+                     peak_source=f"{peaks['_source']} HBM copy", work="algorithmic bytes")
+        res[name] = e
+    if prepare_ms and n and tf32:
+        useful = 2.0 / 3.0 * float(n) ** 3 / (prepare_ms * 1e-3) / 1e12
+        res["prepare (stage)"] = {"bound": "tensor", "unit": "TFLOP/s", "achieved": 3 * useful, "peak": tf32,
+                                  "frac": 3 * useful / tf32, "useful_tflops": useful, "frac_useful": useful / tf32,
+                                  "ms": prepare_ms, "peak_source": "measured tf32 (in this run)",
+                                  "work": "(2/3) n^3 flop (Cholesky n^3/3 + triangular inverse n^3/3), x3 for 3xTF32"}
+    return res
 
 
 def config_dict(name, layer, st):
@@ -386,6 +472,19 @@ def run_ours(args):
     clk = clocks.stop()
     G.raise_on_status(status, "timed steps")
 
+    # A second pass of the same steps with the library's timing trace on: events around
+    # every kernel on the stream it runs on, for the per-kernel roofline entries (kept out
+    # of the headline timing above, whose events bracket whole steps on this stream).
+    G.trace_read()
+    G.trace_enable(True)
+    for i in range(args.steps):
+        step()
+        flush.fill_(1.0)
+    torch.cuda.synchronize()
+    G.trace_enable(False)
+    trace = G.trace_read()
+    G.raise_on_status(status, "traced steps")
+
     step_ms = [e[0].elapsed_time(e[3]) for e in ev]
     hess_ms = [e[4].elapsed_time(e[1]) for e in ev]        # the Hessian launch(es) alone
     clear_ms = [e[0].elapsed_time(e[4]) for e in ev]
@@ -417,6 +516,20 @@ def run_ours(args):
         e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], world, dev)
         e2e["value"] = job_gparams_per_s(world, out, n, e2e["ms_per_step"])
 
+    measured = measure_peaks(G, torch, dev)
+    kernels = kernel_rooflines(trace, peaks, measured, prepare_ms=statistics.mean(prep_ms), n=n)
+    kernels["note"] = (f"device time of each kernel on the stream it runs on, from the library's timing trace over a "
+                       f"second pass of the same {args.steps} steps (the K4 and prepare products run on library "
+                       "streams beside other kernels, so their times include sharing the SMs)")
+
+    blocks = None
+    if world == 1 and not args.no_blocks:
+        del X, H, prep_ws, q_ws, prep, qout
+        torch.cuda.empty_cache()
+        blocks = {}
+        for name in ("llama2-70b-block", "llama2-7b-block"):
+            blocks[name] = time_block(G, torch, name, dev, steps=2, warmup=1, peaks=peaks, measured=measured)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         est, desc = oracle_sample(layer, st, min(N, args.ref_tokens))
@@ -442,6 +555,9 @@ def run_ours(args):
                       "prepare": statistics.mean(prep_ms), "quantize": statistics.mean(quant_ms)},
         "wall_ms_per_step_incl_flush": (t_wall1 - t_wall0) * 1e3 / args.steps,
         "roofline": roofline,
+        "kernel_rooflines": kernels,
+        "peaks_measured_here": measured,
+        "blocks": blocks,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches,
@@ -490,31 +606,27 @@ def run_e2e(G, torch, W_host, X_host, st, n, out, dev, steps, flush):
 BLOCK_INPUTS = (("q", "k", "v"), ("o",), ("gate", "up"), ("down",))
 
 
-def run_block(args):
-    """Time every layer of a decoder block on one GPU (Hessian and preparation once per
-    input, quantization once per layer); prints its own JSON line."""
-    import torch
+def time_block(G, torch, name, dev, steps, warmup, peaks, measured):
+    """One decoder block on one GPU: H and U once per input, then the layers of that input.
 
-    import post_weight_quantization_15_b200 as G
-
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py --block needs a CUDA device")
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    wl = S.workloads()[args.block]
+    Inputs are drawn on the device (synthetic.make_x_device / make_w_device: the same
+    recipe as the parity tests' inputs, torch's generator).  Timed with CUDA events on
+    this stream per input stage; a traced pass after the timed passes gives the
+    per-kernel device times.  Returns a dict for the bench line.
+    """
+    wl = S.workloads()[name]
     st = wl.settings[0]
     by = {l.name: l for l in wl.layers}
     groups = [[by[nm] for nm in g if nm in by] for g in BLOCK_INPUTS]
     groups = [g for g in groups if g]
     xs = {}
-    work = []     # (n, X, [W...], tokens) per input
+    work = []     # (n, X, [W...], tokens, names) per input
     for g in groups:
         xspec = g[0].x
-        key = (xspec.n, xspec.tokens)
-        if key not in xs:   # the synthetic activations of equal shape are the same array
-            xs[key] = torch.from_numpy(S.make_x(xspec).view(np.int16)).to(dev).view(torch.bfloat16)
-        Ws = [torch.from_numpy(S.make_w(l.w)).to(dev) for l in g]
-        work.append((xspec.n, xs[key], Ws, xspec.tokens, [l.name for l in g]))
+        if xspec.stream not in xs:
+            xs[xspec.stream] = S.make_x_device(xspec, dev)
+        Ws = [S.make_w_device(l.w, dev) for l in g]
+        work.append((xspec.n, xs[xspec.stream], Ws, xspec.tokens, [l.name for l in g]))
     status = G.new_status(dev)
     stream = torch.cuda.current_stream()
     bufs = []
@@ -525,8 +637,9 @@ def run_block(args):
         prep = G.Prepared(U=torch.empty((n, n), dtype=torch.float32, device=dev),
                           perm=torch.empty(n, dtype=torch.int32, device=dev),
                           dead=torch.empty(n, dtype=torch.uint8, device=dev), status=status, desc_act=st.desc_act)
-        qws = G.workspace(max(G.quantize_workspace_size(W.shape[0], n, st.block) for W in Ws), dev)
-        outs = [G.alloc_quantized(W.shape[0], n, st.bits, st.group_size, st.sym, dev) for W in Ws]
+        rows = sum(int(W.shape[0]) for W in Ws)      # the layers of one input, stacked in one call
+        qws = G.workspace(G.quantize_workspace_size(rows, n, st.block), dev)
+        outs = G.alloc_quantized(rows, n, st.bits, st.group_size, st.sym, dev)
         bufs.append((H, hd, ws, prep, qws, outs))
 
     def once(ev=None):
@@ -545,51 +658,99 @@ def run_block(args):
             G.prepare(H, st.damp_percent, st.desc_act, hd, status, ws=ws, out=prep)
             if ev is not None:
                 ev[gi][2].record(stream)
-            for W, q in zip(Ws, outs):
-                G.quantize_layer(W, prep, st.bits, st.group_size, st.sym, st.block, ws=qws, out=q)
+            G.quantize_layers(Ws, prep, st.bits, st.group_size, st.sym, st.block, ws=qws, out=outs)
             if ev is not None:
                 ev[gi][3].record(stream)
 
-    for _ in range(max(1, min(args.warmup, 2))):
+    for _ in range(max(1, warmup)):
         once()
     torch.cuda.synchronize()
     G.raise_on_status(status, "block warm-up")
-    steps = max(1, min(args.steps, 3))
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in work] for _ in range(steps)]
-    clocks = ClockSampler(0)
+    clocks = ClockSampler(dev.index or 0)
     clocks.start()
     for i in range(steps):
         once(evs[i])
     torch.cuda.synchronize()
     clk = clocks.stop()
     G.raise_on_status(status, "block")
+    G.trace_read()
+    G.trace_enable(True)
+    once()
+    torch.cuda.synchronize()
+    G.trace_enable(False)
+    trace = G.trace_read()
+    # for comparison: the same layers quantized one call per layer (same U, same outputs' sizes)
+    separate = []
+    for (n, X, Ws, N, names), (H, hd, ws, prep, qws, outs) in zip(work, bufs):
+        if len(Ws) == 1:
+            separate.append(None)
+            continue
+        qs = [G.alloc_quantized(int(W.shape[0]), n, st.bits, st.group_size, st.sym, dev) for W in Ws]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for W, q in zip(Ws, qs):
+            G.quantize_layer(W, prep, st.bits, st.group_size, st.sym, st.block, ws=qws, out=q)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        separate.append(e0.elapsed_time(e1))
+        del qs
+    G.raise_on_status(status, "block, separate calls")
     per_input = []
-    hess_flop, hess_s, total = 0.0, 0.0, 0.0
+    hess_flop, hess_s = 0.0, 0.0
     for gi, (n, X, Ws, N, names) in enumerate(work):
         h = statistics.mean(evs[i][gi][0].elapsed_time(evs[i][gi][1]) for i in range(steps))
         pr = statistics.mean(evs[i][gi][1].elapsed_time(evs[i][gi][2]) for i in range(steps))
         qu = statistics.mean(evs[i][gi][2].elapsed_time(evs[i][gi][3]) for i in range(steps))
-        per_input.append({"layers": names, "in": n, "out": [int(W.shape[0]) for W in Ws], "hessian_ms": h,
-                          "prepare_ms": pr, "quantize_ms": qu})
+        per_input.append({"layers": names, "in": n, "out": [int(W.shape[0]) for W in Ws], "tokens": N,
+                          "hessian_ms": h, "prepare_ms": pr, "quantize_ms": qu,
+                          "quantize_ms_one_call_per_layer": separate[gi],
+                          "hessian_tflops": float(n) * (n + 1) * N / (h * 1e-3) / 1e12})
         hess_flop += float(n) * (n + 1) * N
         hess_s += h * 1e-3
-        total += h + pr + qu
     block_ms = statistics.mean(evs[i][0][4].elapsed_time(evs[i][-1][3]) for i in range(steps))   # clears included
     weights = sum(int(W.numel()) for _, _, Ws, _, _ in work for W in Ws)
-    peaks = load_peaks()
     achieved = hess_flop / hess_s / 1e12
-    line = {
-        "metric": f"GPTQ decoder block ({args.block}): seconds per block, 1 B200", "value": block_ms * 1e-3,
-        "unit": "s", "higher_is_better": False, "steps": steps, "n_gpus": 1, "data": "synthetic",
-        "config": {"workload": args.block, "bits": st.bits, "group_size": st.group_size, "sym": st.sym,
-                   "desc_act": st.desc_act, "inputs": "H and U once per input: q/k/v, o, gate/up, down"},
-        "gparam_per_s": weights / (block_ms * 1e-3) / 1e9,
+    kr = kernel_rooflines(trace, peaks, measured)
+    res = {
+        "seconds_per_block": block_ms * 1e-3, "gparam_per_s": weights / (block_ms * 1e-3) / 1e9,
+        "weights": weights, "steps": steps, "warmup": warmup,
+        "config": {"workload": name, "bits": st.bits, "group_size": st.group_size, "sym": st.sym,
+                   "desc_act": st.desc_act, "damp_percent": st.damp_percent,
+                   "inputs": "H and U once per input: q/k/v, o, gate/up, down; the layers of one input "
+                             "quantized in one call (gptq_quantize_layers)",
+                   "data": "synthetic, drawn on the device (same recipe as the tests' inputs)"},
         "per_input": per_input,
-        "roofline": {"kernel": "hessian (K1), all inputs", "bound": "tensor", "achieved": achieved,
-                     "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
-                     "frac": achieved / float(peaks["bf16_tflops"]), "peak_source": f"{peaks['_source']} bf16 burst"},
+        "hessian_roofline": {"bound": "tensor", "unit": "TFLOP/s", "achieved": achieved,
+                             "peak": float(peaks["bf16_tflops"]), "frac": achieved / float(peaks["bf16_tflops"]),
+                             "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained",
+                                                                             peaks["bf16_tflops"])),
+                             "peak_source": f"{peaks['_source']} bf16 burst (and sustained)"},
+        "kernel_rooflines": kr,
         "clocks": clk,
     }
+    del work, bufs, xs
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_block(args):
+    """Time every layer of a decoder block on one GPU; prints its own JSON line."""
+    import torch
+
+    import post_weight_quantization_15_b200 as G
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --block needs a CUDA device")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    measured = measure_peaks(G, torch, dev)
+    r = time_block(G, torch, args.block, dev, max(1, min(args.steps, 3)), max(1, min(args.warmup, 2)), peaks,
+                   measured)
+    line = {"metric": f"GPTQ decoder block ({args.block}): seconds per block, 1 B200",
+            "value": r["seconds_per_block"], "unit": "s", "higher_is_better": False, "n_gpus": 1,
+            "data": "synthetic", **r, "peaks_measured_here": measured}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -607,6 +768,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--block", default=None, choices=["llama2-7b-block", "llama2-70b-block"],
                     help="time every layer of a decoder block instead (its own JSON line)")
+    ap.add_argument("--no-blocks", action="store_true",
+                    help="leave the two decoder blocks out of the default line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

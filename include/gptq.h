@@ -208,6 +208,35 @@ GPTQ_API int gptq_quantize_layer(const void* W, int w_dtype, int out, int n, con
                         int32_t* d_status, void* stream);
 
 /*
+ * gptq_quantize_layers - gptq_quantize_layer for several layers that read the same
+ * input (a decoder block's q, k and v; its gate and up), in one call.
+ *
+ * "polydesk.ai/glossaire/gptq", "Etape 1": the order of the columns, and with it the
+ * inverse-Hessian work, is shared by every row, and rows are independent given U.
+ * So the rows of layers that share H (and U) are quantized as the rows of one layer
+ * whose weights are the layers' weights stacked along the outputs: the results are
+ * exactly those of one gptq_quantize_layer call per layer, and the row kernels get
+ * more rows per launch.
+ *
+ *   W          HOST array of `count` DEVICE pointers; W[i] is [outs[i], n] row-major,
+ *              all of dtype w_dtype.  1 <= count <= GPTQ_MAX_LAYERS.
+ *   outs       HOST array of the layers' row counts (each >= 1, sum <= GPTQ_MAX_OUT).
+ *   outputs    those of gptq_quantize_layer for the stacked layer, out = sum(outs):
+ *              qweight [n*bits/32, out], scales / zeros [G, out], codes [out, n],
+ *              err_sq [out]; layer i owns output columns (qweight, scales, zeros) and
+ *              rows (codes, err_sq) row0 .. row0 + outs[i] - 1, row0 = outs[0] + ... +
+ *              outs[i-1]; g_idx [n] is shared.
+ *   ws         >= gptq_quantize_workspace_size(out, n, block) bytes.
+ * Everything else, errors included, as gptq_quantize_layer.
+ */
+#define GPTQ_MAX_LAYERS 8
+GPTQ_API int gptq_quantize_layers(const void* const* W, const int* outs, int count, int w_dtype, int n,
+                                  const float* U, const int32_t* perm, const uint8_t* dead, int bits,
+                                  int group_size, int sym, int block, int32_t* qweight, uint16_t* scales,
+                                  uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq, void* ws,
+                                  size_t ws_bytes, int32_t* d_status, void* stream);
+
+/*
  * gptq_pack - bit-packing on its own: codes uint8 [out, n] (original order)
  * -> qweight int32 [n*bits/32, out], the layout gptq_quantize_layer writes.
  * bits in {2, 3, 4, 8}; n*bits % 32 == 0; codes must be < 2^bits.

@@ -144,7 +144,12 @@ int gptq_quantize_layer_padded(const void* W, int w_dtype, int out, int w_cols, 
                                       g_idx, d_status);
   if (arc != GPTQ_OK) return arc;
   if (ws == nullptr || ws_bytes < quantize_ws_bytes(out, n, block) || !aligned(ws, 256)) return GPTQ_ERR_WORKSPACE;
-  return launch_quantize(W, w_dtype, out, w_cols, n, U, perm, dead, bits, group_size, sym ? 1 : 0, block, qweight,
+  WRows rows{};
+  rows.W[0] = W;
+  rows.row0[0] = 0;
+  rows.row0[1] = out;
+  rows.count = 1;
+  return launch_quantize(rows, w_dtype, out, w_cols, n, U, perm, dead, bits, group_size, sym ? 1 : 0, block, qweight,
                          scales, zeros, g_idx, codes, err_sq, ws, d_status, as_stream(stream));
 }
 
@@ -154,6 +159,31 @@ int gptq_quantize_layer(const void* W, int w_dtype, int out, int n, const float*
                         void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
   return gptq_quantize_layer_padded(W, w_dtype, out, n, n, U, perm, dead, bits, group_size, sym, block, qweight,
                                     scales, zeros, g_idx, codes, err_sq, ws, ws_bytes, d_status, stream);
+}
+
+int gptq_quantize_layers(const void* const* W, const int* outs, int count, int w_dtype, int n, const float* U,
+                         const int32_t* perm, const uint8_t* dead, int bits, int group_size, int sym, int block,
+                         int32_t* qweight, uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes,
+                         float* err_sq, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (W == nullptr || outs == nullptr || count < 1 || count > GPTQ_MAX_LAYERS) return GPTQ_ERR_INVALID_ARG;
+  WRows rows{};
+  int64_t total = 0;
+  rows.row0[0] = 0;
+  for (int i = 0; i < count; ++i) {
+    if (W[i] == nullptr || outs[i] <= 0) return GPTQ_ERR_INVALID_ARG;
+    total += outs[i];
+    if (total > GPTQ_MAX_OUT) return GPTQ_ERR_UNSUPPORTED;
+    rows.W[i] = W[i];
+    rows.row0[i + 1] = (int)total;
+  }
+  rows.count = count;
+  const int out = (int)total;
+  const int arc = check_quantize_args(W[0], w_dtype, out, n, n, U, bits, group_size, block, qweight, scales, zeros,
+                                      g_idx, d_status);
+  if (arc != GPTQ_OK) return arc;
+  if (ws == nullptr || ws_bytes < quantize_ws_bytes(out, n, block) || !aligned(ws, 256)) return GPTQ_ERR_WORKSPACE;
+  return launch_quantize(rows, w_dtype, out, n, n, U, perm, dead, bits, group_size, sym ? 1 : 0, block, qweight,
+                         scales, zeros, g_idx, codes, err_sq, ws, d_status, as_stream(stream));
 }
 
 int gptq_pack(const uint8_t* codes, int out, int n, int bits, int32_t* qweight, void* stream) {

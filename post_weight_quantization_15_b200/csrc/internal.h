@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/gptq.h"
+
 namespace gptq {
 
 // ---- timing trace (gptq_trace_enable): events around one launch on its stream ----
@@ -44,8 +46,16 @@ size_t quantize_ws_bytes(int out, int n, int block);
 int check_quantize_args(const void* W, int w_dtype, int out, int w_cols, int n, const float* U, int bits,
                         int group_size, int block, const int32_t* qweight, const uint16_t* scales,
                         const uint16_t* zeros, const int32_t* g_idx, const int32_t* d_status);
+// The weights of the rows of one quantize call: up to kMaxLayers layers of one input,
+// their rows concatenated (layer i holds rows row0[i] .. row0[i+1]-1).
+constexpr int kMaxLayers = GPTQ_MAX_LAYERS;
+struct WRows {
+  const void* W[kMaxLayers];
+  int row0[kMaxLayers + 1];
+  int count;
+};
 // W [out, w_cols] (w_cols <= n; columns w_cols .. n-1 are zero padding).
-int launch_quantize(const void* W, int w_dtype, int out, int w_cols, int n, const float* U, const int32_t* perm,
+int launch_quantize(const WRows& W, int w_dtype, int out, int w_cols, int n, const float* U, const int32_t* perm,
                     const uint8_t* dead, int bits, int gs, int sym, int block, int32_t* qweight,
                     uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq,
                     void* ws, int32_t* st, cudaStream_t s);

@@ -146,9 +146,11 @@ __device__ __forceinline__ float code_from_q(float q, QParams p, int bits, bool 
 // warp cover 128 consecutive columns of a row for the identity order.  W has w_cols
 // columns (its row stride); columns w_cols .. n-1 are the zero padding of a layer
 // whose width the group size or the packing does not divide.
+// Rows may come from several layers of one input (WRows: row r belongs to the layer
+// whose range holds it).
 template <typename T>
-__global__ void ingest_kernel(const T* W, int out, int w_cols, int n, const int32_t* perm, const uint8_t* dead,
-                              int gs, float* Wf, int32_t* invperm, int32_t* g_idx, int32_t* st) {
+__global__ void ingest_kernel(const __grid_constant__ WRows W, int out, int w_cols, int n, const int32_t* perm,
+                              const uint8_t* dead, int gs, float* Wf, int32_t* invperm, int32_t* g_idx, int32_t* st) {
   if (has_error(st)) return;
   const int k0 = 4 * (blockIdx.x * 32 + threadIdx.x);
   const int r = blockIdx.y * 8 + threadIdx.y;
@@ -164,7 +166,9 @@ __global__ void ingest_kernel(const T* W, int out, int w_cols, int n, const int3
     }
   }
   if (r >= out) return;
-  const T* row = W + (int64_t)r * w_cols;
+  int li = 0;
+  while (li + 1 < W.count && r >= W.row0[li + 1]) ++li;
+  const T* row = static_cast<const T*>(W.W[li]) + (int64_t)(r - W.row0[li]) * w_cols;
   float v[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
@@ -725,7 +729,7 @@ int join_streams(QuantStreams* q, cudaStream_t s) {
   return GPTQ_OK;
 }
 
-int launch_quantize(const void* W, int w_dtype, int out, int w_cols, int n, const float* U, const int32_t* perm,
+int launch_quantize(const WRows& W, int w_dtype, int out, int w_cols, int n, const float* U, const int32_t* perm,
                     const uint8_t* dead, int bits, int gs, int sym, int block, int32_t* qweight,
                     uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq,
                     void* ws, int32_t* st, cudaStream_t s) {
@@ -736,11 +740,11 @@ int launch_quantize(const void* W, int w_dtype, int out, int w_cols, int n, cons
     const double esz = w_dtype == GPTQ_F32 ? 4.0 : 2.0;
     TraceScope ts("ingest", "byte", (double)out * w_cols * esz + (double)out * n * 4.0, s);
     if (w_dtype == GPTQ_F32)
-      ingest_kernel<float><<<grd, blk, 0, s>>>(static_cast<const float*>(W), out, w_cols, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
+      ingest_kernel<float><<<grd, blk, 0, s>>>(W, out, w_cols, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
     else if (w_dtype == GPTQ_F16)
-      ingest_kernel<__half><<<grd, blk, 0, s>>>(static_cast<const __half*>(W), out, w_cols, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
+      ingest_kernel<__half><<<grd, blk, 0, s>>>(W, out, w_cols, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
     else
-      ingest_kernel<__nv_bfloat16><<<grd, blk, 0, s>>>(static_cast<const __nv_bfloat16*>(W), out, w_cols, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
+      ingest_kernel<__nv_bfloat16><<<grd, blk, 0, s>>>(W, out, w_cols, n, perm, dead, gs, w.Wf, w.invperm, g_idx, st);
     GPTQ_LAUNCH_CHECK();
   }
   if (err_sq) GPTQ_CUDA_TRY(cudaMemsetAsync(err_sq, 0, (size_t)out * 4, s));

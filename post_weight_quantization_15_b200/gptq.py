@@ -96,6 +96,8 @@ def lib() -> ctypes.CDLL:
     L.gptq_quantize_workspace_size.argtypes = [I, I, I]
     L.gptq_quantize_layer.restype = I
     L.gptq_quantize_layer.argtypes = [P, I, I, I, P, P, P, I, I, I, I, P, P, P, P, P, P, P, SZ, P, P]
+    L.gptq_quantize_layers.restype = I
+    L.gptq_quantize_layers.argtypes = [P, P, I, I, I, P, P, P, I, I, I, I, P, P, P, P, P, P, P, SZ, P, P]
     L.gptq_pack.restype = I
     L.gptq_pack.argtypes = [P, I, I, I, P, P]
     L.gptq_hessian_accumulate_padded.restype = I
@@ -398,6 +400,56 @@ def quantize_layer(W: torch.Tensor, prep: Prepared, bits: int = 4, group_size: i
                                             _ptr(ws), ws.numel(), _ptr(prep.status), _stream(stream)),
            "gptq_quantize_layer")
     return out
+
+
+MAX_LAYERS = 8
+
+
+def quantize_layers(Ws, prep: Prepared, bits: int = 4, group_size: int = 128, sym: bool = False,
+                    block: int = 128, want_codes: bool = False, want_err: bool = False,
+                    ws: Optional[torch.Tensor] = None, out: Optional[QuantizedLayer] = None, stream=None):
+    """Several layers that read the same input (share ``prep``), in one call.
+
+    Returns (stacked, views): ``stacked`` is the QuantizedLayer of the layers stacked
+    along the outputs, ``views`` one QuantizedLayer per layer whose tensors are views of
+    it (qweight / scales / zeros: column ranges, not contiguous; codes / err_sq: row
+    ranges).  Bit-identical to one quantize_layer call per layer.
+    """
+    Ws = list(Ws)
+    if not 1 <= len(Ws) <= MAX_LAYERS:
+        raise ValueError(f"1 to {MAX_LAYERS} layers per call")
+    n = prep.U.shape[0]
+    dt = Ws[0].dtype
+    for W in Ws:
+        if W.dim() != 2 or not W.is_contiguous() or W.dtype != dt or dt not in _DTYPE_CODE or W.shape[1] != n:
+            raise ValueError("every W must be a contiguous [out_i, n] tensor of one dtype (fp32/fp16/bf16)")
+    _require_cuda(*Ws, ws)
+    outs = [int(W.shape[0]) for W in Ws]
+    o = sum(outs)
+    dev = Ws[0].device
+    need = quantize_workspace_size(o, n, block)
+    if ws is None or ws.numel() < need:
+        ws = workspace(need, dev)
+    if out is None:
+        out = alloc_quantized(o, n, bits, group_size, sym, dev, want_codes, want_err)
+    else:
+        _check_quantized(out, o, n)
+    ptrs = (ctypes.c_void_p * len(Ws))(*[W.data_ptr() for W in Ws])
+    rows = (ctypes.c_int * len(Ws))(*outs)
+    _check(lib().gptq_quantize_layers(ptrs, rows, len(Ws), _DTYPE_CODE[dt], n, _ptr(prep.U), _ptr(prep.perm),
+                                      _ptr(prep.dead), int(bits), int(group_size), int(bool(sym)), int(block),
+                                      _ptr(out.qweight), _ptr(out.scales), _ptr(out.zeros), _ptr(out.g_idx),
+                                      _ptr(out.codes), _ptr(out.err_sq), _ptr(ws), ws.numel(), _ptr(prep.status),
+                                      _stream(stream)), "gptq_quantize_layers")
+    views, r0 = [], 0
+    for k in outs:
+        sl = slice(r0, r0 + k)
+        views.append(QuantizedLayer(out.qweight[:, sl], out.scales[:, sl], out.zeros[:, sl], out.g_idx,
+                                    None if out.codes is None else out.codes[sl],
+                                    None if out.err_sq is None else out.err_sq[sl], out.bits, out.group_size,
+                                    out.sym))
+        r0 += k
+    return out, views
 
 
 def pack(codes: torch.Tensor, bits: int, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

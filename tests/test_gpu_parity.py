@@ -522,3 +522,50 @@ def test_degenerate_groups_are_bit_exact_round_to_nearest(bits, gs, sym):
     assert np.array_equal(q.scales.cpu().numpy(), rs.astype(np.float16))
     assert np.array_equal(q.zeros.cpu().numpy(), rz.astype(np.float16))
     assert np.array_equal(q.codes.cpu().numpy(), rc)
+
+
+# --------------------------------------------------------------------------- #
+# Layers that share an input, stacked in one call
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("outs,n,bits,gs,sym,act,wdtype", [
+    ((300, 64, 64), 512, 4, 128, True, True, "f16"),       # q / k / v-like: one wide, two narrow
+    ((2000, 600), 384, 3, 64, False, True, "f16"),         # the stacked rows change the lanes per row
+    ((5000, 200, 77), 256, 2, 32, False, False, "f32"),
+])
+def test_stacked_layers_equal_separate_calls_bit_for_bit(outs, n, bits, gs, sym, act, wdtype):
+    """Rows are independent given U ("Etape 1"): quantizing layers of one input stacked
+    along the outputs gives exactly the per-layer results."""
+    dev = _dev()
+    _, x = S.small_case(8, n, 3 * n, seed=n + len(outs))
+    X = _to_dev_x(x, dev)
+    st = G.new_status(dev)
+    H = torch.zeros((n, n), dtype=torch.float32, device=dev)
+    hd = torch.zeros(n, dtype=torch.float64, device=dev)
+    G.hessian_accumulate(H, X, hd, st)
+    prep = G.prepare(H, 0.01, act, hd, st)
+    Ws = [_w_tensor(S.make_w(S.WSpec(o, n, 0.02, wdtype, 5, 100 + i)), dev) for i, o in enumerate(outs)]
+    sep = [G.quantize_layer(W, prep, bits, gs, sym, want_codes=True, want_err=True) for W in Ws]
+    stacked, views = G.quantize_layers(Ws, prep, bits, gs, sym, want_codes=True, want_err=True)
+    G.raise_on_status(st, "stacked layers")
+    for a, b in zip(views, sep):
+        for name in ("qweight", "scales", "zeros", "g_idx", "codes", "err_sq"):
+            x_, y_ = getattr(a, name).contiguous().cpu().numpy(), getattr(b, name).cpu().numpy()
+            assert np.array_equal(x_.view(np.uint8), y_.view(np.uint8)), name
+
+
+def test_timing_trace_records_every_stage_on_its_stream():
+    dev = _dev()
+    W, x = S.small_case(256, 1536, 2048, seed=9)
+    G.trace_read()
+    G.trace_enable(True)
+    q, prep, H = _run_gpu(W, x, 4, 128, False, True)
+    G.trace_enable(False)
+    tr = G.trace_read()
+    for k in ("hessian_tc", "hessian_diag64", "potrf_inv", "prepare_gemm3", "ingest", "sweep", "trailing_update",
+              "u_operand", "pack"):
+        assert k in tr and tr[k]["launches"] > 0 and tr[k]["ms"] > 0, k
+    assert tr["sweep"]["launches"] == 3 and tr["potrf_inv"]["launches"] == 12
+    assert tr["hessian_tc"]["work"] == pytest.approx(1536 * 1537 * 2048)
+    # with the trace off nothing is recorded
+    _run_gpu(W, x, 4, 128, False, True)
+    assert G.trace_read() == {}
