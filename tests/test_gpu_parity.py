@@ -569,3 +569,49 @@ def test_timing_trace_records_every_stage_on_its_stream():
     # with the trace off nothing is recorded
     _run_gpu(W, x, 4, 128, False, True)
     assert G.trace_read() == {}
+
+
+def test_layer_split_over_two_ranks_on_one_device():
+    """The two-rank split of sharded.py, both ranks' kernels on one device (no
+    collective: the all-reduce of two partial H is their sum, one fp32 addition per
+    entry, and the gather is the concatenation of the row shards).  H from the two
+    token halves stays within the derived bound of the oracle's H; the rows quantized
+    in two shards equal the unsplit call bit for bit."""
+    from post_weight_quantization_15_b200 import sharded as SH
+    dev = _dev()
+    out, n, N = 333, 512, 3000
+    W, x = S.small_case(out, n, N, seed=21)
+    X = _to_dev_x(x, dev)
+    st = G.new_status(dev)
+    Hs, ds, spans = [], [], []
+    for r in range(2):
+        t0, t1 = SH.split_range(N, 2, r, align=8)
+        spans.append(t1 - t0)
+        H = torch.zeros((n, n), dtype=torch.float32, device=dev)
+        hd = torch.zeros(n, dtype=torch.float64, device=dev)
+        G.hessian_accumulate(H, X[:, t0:t1], hd, st)
+        Hs.append(H)
+        ds.append(hd)
+    H = Hs[0] + Hs[1]
+    hd = ds[0] + ds[1]
+    H64 = O.hessian(x)
+    iu = np.triu_indices(n)
+    rel = np.abs(H.cpu().numpy().astype(np.float64)[iu] - H64[iu]) / np.sqrt(np.outer(np.diag(H64), np.diag(H64)))[iu]
+    # each rank's own summation, and one more addition (counted as one more call)
+    assert rel.max() <= hessian_bound(spans + [1]), rel.max()
+    assert np.allclose(hd.cpu().numpy(), np.diag(H64), rtol=1e-13, atol=0)
+    prep = G.prepare(H, 0.01, True, hd, st)
+    Wt = _w_tensor(W, dev)
+    whole = G.quantize_layer(Wt, prep, 4, 128, True, want_codes=True, want_err=True)
+    parts = []
+    for r in range(2):
+        o0, o1 = SH.split_range(out, 2, r)
+        parts.append(G.quantize_layer(Wt[o0:o1].contiguous(), prep, 4, 128, True, want_codes=True, want_err=True))
+    G.raise_on_status(st, "split layer")
+    for name, dim in (("qweight", 1), ("scales", 1), ("zeros", 1), ("codes", 0), ("err_sq", 0)):
+        cat = torch.cat([getattr(p, name) for p in parts], dim=dim).cpu().numpy()
+        assert np.array_equal(cat.view(np.uint8), getattr(whole, name).cpu().numpy().view(np.uint8)), name
+    c = compare_layer(W, H64, O.gptq_layer(W, None, 4, 128, True, True, H=H64), whole.qweight.cpu().numpy(),
+                      whole.scales.cpu().numpy(), whole.zeros.cpu().numpy(), whole.g_idx.cpu().numpy(),
+                      whole.codes.cpu().numpy(), prep.perm.cpu().numpy(), 4, 128)
+    assert c.ok(), c
