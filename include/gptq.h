@@ -214,9 +214,10 @@ GPTQ_API int gptq_quantize_layer(const void* W, int w_dtype, int out, int n, con
  * "polydesk.ai/glossaire/gptq", "Etape 1": the order of the columns, and with it the
  * inverse-Hessian work, is shared by every row, and rows are independent given U.
  * So the rows of layers that share H (and U) are quantized as the rows of one layer
- * whose weights are the layers' weights stacked along the outputs: the results are
- * exactly those of one gptq_quantize_layer call per layer, and the row kernels get
- * more rows per launch.
+ * whose weights are the layers' weights stacked along the outputs: qweight, scales,
+ * zeros, g_idx and codes are bit for bit those of one gptq_quantize_layer call per
+ * layer (err_sq up to the order of its per-row sum, which depends on the rows per
+ * launch), and the row kernels get more rows per launch.
  *
  *   W          HOST array of `count` DEVICE pointers; W[i] is [outs[i], n] row-major,
  *              all of dtype w_dtype.  1 <= count <= GPTQ_MAX_LAYERS.

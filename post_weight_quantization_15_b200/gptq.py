@@ -413,7 +413,8 @@ def quantize_layers(Ws, prep: Prepared, bits: int = 4, group_size: int = 128, sy
     Returns (stacked, views): ``stacked`` is the QuantizedLayer of the layers stacked
     along the outputs, ``views`` one QuantizedLayer per layer whose tensors are views of
     it (qweight / scales / zeros: column ranges, not contiguous; codes / err_sq: row
-    ranges).  Bit-identical to one quantize_layer call per layer.
+    ranges).  Bit-identical to one quantize_layer call per layer (err_sq up to the order
+    of its per-row sum).
     """
     Ws = list(Ws)
     if not 1 <= len(Ws) <= MAX_LAYERS:
