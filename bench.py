@@ -374,6 +374,57 @@ def kernel_rooflines(trace, peaks, measured, prepare_ms=None, n=None):
     return res
 
 
+# Decode shapes for the consumer of the stored format (out, in): the 70B block's gate/up
+# and down, the 7B block's gate/up, 4-bit g128 with an act-order g_idx.
+DECODE_SHAPES = ((28672, 8192), (8192, 28672), (11008, 4096))
+
+
+def time_qmatvec(G, torch, dev, peaks, flush, iters=20):
+    """gptq_qmatvec at decode shapes (1 and 16 activation rows): device time per call (CUDA
+    events on this stream, L2 flushed before every call) against the HBM roofline on the
+    bytes the call must move (packed weights, scales and zeros, g_idx, X in, Y out)."""
+    res = []
+    stream = torch.cuda.current_stream()
+    for out, n in DECODE_SHAPES:
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(out + n)
+        G_ = n // 128
+        q = G.QuantizedLayer(
+            qweight=torch.randint(-2 ** 31, 2 ** 31 - 1, (n * 4 // 32, out), generator=gen, device=dev,
+                                  dtype=torch.int64).to(torch.int32),
+            scales=(torch.rand((G_, out), generator=gen, device=dev) * 0.01 + 1e-4).half(),
+            zeros=torch.randint(0, 16, (G_, out), generator=gen, device=dev).half(),
+            g_idx=(torch.randperm(n, generator=gen, device=dev) // 128).to(torch.int32),
+            codes=None, err_sq=None, bits=4, group_size=128, sym=False)
+        for M in (1, 16):
+            X = torch.randn((M, n), generator=gen, device=dev).half()
+            Y = torch.empty((M, out), dtype=torch.float32, device=dev)
+            ws = G.workspace(G.lib().gptq_qmatvec_workspace_size(M, n, out), dev)
+            st = G.new_status(dev)
+            times = []
+            for i in range(iters + 3):
+                flush.fill_(1.0)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                G.qmatvec(q, X, st, ws=ws, out=Y)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                if i >= 3:
+                    times.append(e0.elapsed_time(e1))
+            G.raise_on_status(st, "qmatvec bench")
+            ms = statistics.median(times)
+            nbytes = out * n * 4 / 8 + 4.0 * G_ * out + 4.0 * n + 2.0 * M * n + 4.0 * M * out
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            res.append({"out": out, "in": n, "tokens": M, "bits": 4, "group_size": 128, "act_order_g_idx": True,
+                        "us_per_call": ms * 1e3, "bytes": nbytes, "achieved_gbs": gbs,
+                        "frac": gbs / float(peaks["hbm_gbs"]),
+                        "flop": 2.0 * M * out * n, "tflops": 2.0 * M * out * n / (ms * 1e-3) / 1e12})
+    return {"kernel": "qmatvec (+ its k-split reduction)", "bound": "hbm", "peak": float(peaks["hbm_gbs"]),
+            "unit": "GB/s", "peak_source": f"{peaks['_source']} HBM copy",
+            "timing": f"CUDA events around each call, L2 flushed before each, median of {iters}",
+            "shapes": res}
+
+
 def config_dict(name, layer, st):
     return {"workload": name, "out": layer.w.out, "in": layer.w.n, "tokens": layer.x.tokens,
             "w_dtype": layer.w.dtype, "bits": st.bits, "group_size": st.group_size, "sym": st.sym,
@@ -522,6 +573,8 @@ def run_ours(args):
                        f"second pass of the same {args.steps} steps (the K4 and prepare products run on library "
                        "streams beside other kernels, so their times include sharing the SMs)")
 
+    decode = time_qmatvec(G, torch, dev, peaks, flush) if world == 1 else None
+
     blocks = None
     if world == 1 and not args.no_blocks:
         del X, H, prep_ws, q_ws, prep, qout
@@ -558,6 +611,7 @@ def run_ours(args):
         "kernel_rooflines": kernels,
         "peaks_measured_here": measured,
         "blocks": blocks,
+        "decode_qmatvec": decode,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches,

@@ -307,6 +307,39 @@ GPTQ_API int gptq_pack_zeros(const uint16_t* zeros, int groups, int out, int bit
                              int32_t* qzeros, int32_t* d_status, void* stream);
 
 /*
+ * The consumer side of the stored format.  The pages name the inference kernels
+ * that read GPTQ's packed weights (Marlin, ExLlama: "skillmd.com/skills/artubss/gptq",
+ * "Backends de inferencia") and store scale and zero point in FP16 ("dev.ayinedjimi-
+ * consultants.fr ... ia-quantization-gptq-gguf-awq", "Calibration et dataset").  Both
+ * calls read what gptq_quantize_layer writes: qweight int32 [n*bits/32, out], scales
+ * and zeros fp16 [groups, out], g_idx int32 [n] (any order, act-order included).
+ * bits in {2, 4, 8} (3-bit codes straddle words: GPTQ_ERR_UNSUPPORTED).  A g_idx
+ * entry outside [0, groups) is recorded in d_status (GPTQ_ERR_INVALID_ARG, info = its
+ * column) and read as group 0.  qweight 16-byte aligned; out % 4 == 0 for the
+ * vectorised path (any out works).
+ *
+ * gptq_dequantize - What[o][k] = scales[g_idx[k]][o] . (code(o, k) - zeros[g_idx[k]][o])
+ *   into What [out, n] row-major of dtype out_dtype (GPTQ_F32: exact, the product of an
+ *   fp16 scale and a small integer being exact in fp32; GPTQ_F16 / GPTQ_BF16: rounded
+ *   once to nearest even).
+ *
+ * gptq_qmatvec - Y[M, out] = X[M, n] . What^T for 1 <= M <= 16 activation rows (the
+ *   decode shapes), the weights dequantized in registers and never written: the call
+ *   reads qweight once, so HBM bandwidth bounds it.  X of dtype x_dtype (F16, BF16 or
+ *   F32), row stride ld_x; Y fp32, row stride ld_y (>= out).  Sums in fp32, in an order
+ *   fixed by the shapes (deterministic).  ws: >= gptq_qmatvec_workspace_size(M, n, out)
+ *   bytes, 256-byte aligned (the partial sums of the k splits).
+ */
+GPTQ_API int gptq_dequantize(const int32_t* qweight, const uint16_t* scales, const uint16_t* zeros,
+                             const int32_t* g_idx, int bits, int n, int out, int groups, int out_dtype, void* What,
+                             int32_t* d_status, void* stream);
+GPTQ_API size_t gptq_qmatvec_workspace_size(int M, int n, int out);
+GPTQ_API int gptq_qmatvec(const int32_t* qweight, const uint16_t* scales, const uint16_t* zeros,
+                          const int32_t* g_idx, int bits, int n, int out, int groups, const void* X, int x_dtype,
+                          int M, int64_t ld_x, float* Y, int64_t ld_y, void* ws, size_t ws_bytes,
+                          int32_t* d_status, void* stream);
+
+/*
  * Kernel timing trace.  The GPTQ pages have no counterpart to these calls: they
  * are a measurement aid.  While the trace is on, every kernel the library launches
  * is bracketed by two CUDA events recorded on the stream it is launched on (the

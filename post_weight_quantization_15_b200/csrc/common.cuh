@@ -16,7 +16,8 @@ enum { ST_CODE = 0, ST_INFO = 1, ST_STAGE = 2 };
 // Stage ids recorded in d_status[ST_STAGE] next to an error.
 enum {
   STAGE_HESSIAN = 1, STAGE_PREP_DIAG = 2, STAGE_POTRF = 3, STAGE_TRINV = 4,
-  STAGE_INGEST = 5, STAGE_SWEEP = 6, STAGE_TRAILING = 7, STAGE_PACK = 8
+  STAGE_INGEST = 5, STAGE_SWEEP = 6, STAGE_TRAILING = 7, STAGE_PACK = 8, STAGE_DEQUANT = 9,
+  STAGE_LINEAR = 10
 };
 
 // First error wins; later kernels see a non-zero code and skip their work.

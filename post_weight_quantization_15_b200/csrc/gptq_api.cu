@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <climits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -184,6 +185,49 @@ int gptq_quantize_layers(const void* const* W, const int* outs, int count, int w
   if (ws == nullptr || ws_bytes < quantize_ws_bytes(out, n, block) || !aligned(ws, 256)) return GPTQ_ERR_WORKSPACE;
   return launch_quantize(rows, w_dtype, out, n, n, U, perm, dead, bits, group_size, sym ? 1 : 0, block, qweight,
                          scales, zeros, g_idx, codes, err_sq, ws, d_status, as_stream(stream));
+}
+
+namespace {
+int check_stored(const int32_t* qweight, const uint16_t* scales, const uint16_t* zeros, const int32_t* g_idx,
+                 int bits, int n, int out, int groups) {
+  if (qweight == nullptr || scales == nullptr || zeros == nullptr || g_idx == nullptr) return GPTQ_ERR_INVALID_ARG;
+  if (n <= 0 || out <= 0 || groups <= 0 || !aligned(qweight, 16)) return GPTQ_ERR_INVALID_ARG;
+  if (bits != 2 && bits != 4 && bits != 8) return GPTQ_ERR_UNSUPPORTED;
+  if ((n * bits) % 32 != 0) return GPTQ_ERR_UNSUPPORTED;
+  if ((int64_t)out * 4 > (int64_t)65535 * 128 * 4) return GPTQ_ERR_UNSUPPORTED;
+  return GPTQ_OK;
+}
+}  // namespace
+
+int gptq_dequantize(const int32_t* qweight, const uint16_t* scales, const uint16_t* zeros, const int32_t* g_idx,
+                    int bits, int n, int out, int groups, int out_dtype, void* What, int32_t* d_status,
+                    void* stream) {
+  const int rc = check_stored(qweight, scales, zeros, g_idx, bits, n, out, groups);
+  if (rc != GPTQ_OK) return rc;
+  if (What == nullptr) return GPTQ_ERR_INVALID_ARG;
+  if (out_dtype != GPTQ_F32 && out_dtype != GPTQ_F16 && out_dtype != GPTQ_BF16) return GPTQ_ERR_INVALID_ARG;
+  if ((int64_t)n * bits / 32 > (int64_t)65535 * 8) return GPTQ_ERR_UNSUPPORTED;
+  return launch_dequant(qweight, scales, zeros, g_idx, bits, n, out, groups, out_dtype, What, d_status,
+                        as_stream(stream));
+}
+
+size_t gptq_qmatvec_workspace_size(int M, int n, int out) {
+  if (M <= 0 || n <= 0 || out <= 0) return 0;
+  return qmatvec_ws_bytes(M, n, out);
+}
+
+int gptq_qmatvec(const int32_t* qweight, const uint16_t* scales, const uint16_t* zeros, const int32_t* g_idx,
+                 int bits, int n, int out, int groups, const void* X, int x_dtype, int M, int64_t ld_x, float* Y,
+                 int64_t ld_y, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  const int rc = check_stored(qweight, scales, zeros, g_idx, bits, n, out, groups);
+  if (rc != GPTQ_OK) return rc;
+  if (X == nullptr || Y == nullptr || M < 1 || ld_x < n || ld_y < out || ld_x > INT32_MAX || ld_y > INT32_MAX)
+    return GPTQ_ERR_INVALID_ARG;
+  if (M > 16) return GPTQ_ERR_UNSUPPORTED;
+  if (x_dtype != GPTQ_F32 && x_dtype != GPTQ_F16 && x_dtype != GPTQ_BF16) return GPTQ_ERR_INVALID_ARG;
+  if (ws == nullptr || ws_bytes < qmatvec_ws_bytes(M, n, out) || !aligned(ws, 256)) return GPTQ_ERR_WORKSPACE;
+  return launch_qmatvec(qweight, scales, zeros, g_idx, bits, n, out, groups, X, x_dtype, M, (int)ld_x, Y, (int)ld_y,
+                        ws, d_status, as_stream(stream));
 }
 
 int gptq_pack(const uint8_t* codes, int out, int n, int bits, int32_t* qweight, void* stream) {

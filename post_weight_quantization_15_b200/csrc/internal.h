@@ -64,6 +64,14 @@ int launch_pack(const uint8_t* codes, const int32_t* invperm, int out, int n, in
 int launch_pack_zeros(const uint16_t* zeros, int groups, int out, int bits, int zero_offset, int32_t* qzeros,
                       int32_t* st, cudaStream_t s);
 
+// ---- the consumer of the stored format (dequant.cu) -----------------------------
+int launch_dequant(const int32_t* qweight, const uint16_t* scales, const uint16_t* zeros, const int32_t* g_idx,
+                   int bits, int n, int out, int groups, int dtype, void* What, int32_t* st, cudaStream_t s);
+size_t qmatvec_ws_bytes(int M, int n, int out);
+int launch_qmatvec(const int32_t* qweight, const uint16_t* scales, const uint16_t* zeros, const int32_t* g_idx,
+                   int bits, int n, int out, int groups, const void* X, int x_dtype, int M, int ldx, float* Y, int ldy,
+                   void* ws, int32_t* st, cudaStream_t s);
+
 // ---- tensor-core GEMM: C -= A . B^T in 3 x TF32 (operands pre-split) ---------
 // store = false: C -= A.B^T; store = true: C = A.B^T (C may be null then, if Chi/Clo are given).
 // Chi/Clo (optional, leading dimension ldh) receive the TF32 split of the result.

@@ -112,6 +112,12 @@ def lib() -> ctypes.CDLL:
     L.gptq_trace_enable.argtypes = [I]
     L.gptq_trace_read.restype = I
     L.gptq_trace_read.argtypes = [ctypes.POINTER(_TraceRow), I, ctypes.POINTER(ctypes.c_int)]
+    L.gptq_dequantize.restype = I
+    L.gptq_dequantize.argtypes = [P, P, P, P, I, I, I, I, I, P, P, P]
+    L.gptq_qmatvec_workspace_size.restype = SZ
+    L.gptq_qmatvec_workspace_size.argtypes = [I, I, I]
+    L.gptq_qmatvec.restype = I
+    L.gptq_qmatvec.argtypes = [P, P, P, P, I, I, I, I, P, I, I, I64, P, I64, P, SZ, P, P]
     L.gptq_probe_fp32_peak.restype = I
     L.gptq_probe_fp32_peak.argtypes = [P, I, I, P]
     L.gptq_quantize_layer_noalloc.restype = I
@@ -451,6 +457,50 @@ def quantize_layers(Ws, prep: Prepared, bits: int = 4, group_size: int = 128, sy
                                     out.sym))
         r0 += k
     return out, views
+
+
+def _stored(q: QuantizedLayer):
+    n = q.g_idx.numel()
+    out = q.qweight.shape[1]
+    if q.qweight.shape[0] * 32 != n * q.bits or not q.qweight.is_contiguous() or not q.scales.is_contiguous() \
+            or not q.zeros.is_contiguous() or q.scales.shape != q.zeros.shape or q.scales.shape[1] != out:
+        raise ValueError("a contiguous stored layer (qweight [n*bits/32, out], scales / zeros [G, out]) is needed")
+    _require_cuda(q.qweight, q.scales, q.zeros, q.g_idx)
+    return n, out, q.scales.shape[0]
+
+
+def dequantize(q: QuantizedLayer, dtype=torch.float16, status: Optional[torch.Tensor] = None,
+               out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """What [out, n] = scales[g_idx] . (codes - zeros[g_idx]) from the stored format."""
+    n, o, groups = _stored(q)
+    if out is None:
+        out = torch.empty((o, n), dtype=dtype, device=q.qweight.device)
+    _check_shape(out, (o, n), dtype, "What")
+    _check(lib().gptq_dequantize(_ptr(q.qweight), _ptr(q.scales), _ptr(q.zeros), _ptr(q.g_idx), int(q.bits), n, o,
+                                 groups, _DTYPE_CODE[dtype], _ptr(out), _ptr(status), _stream(stream)),
+           "gptq_dequantize")
+    return out
+
+
+def qmatvec(q: QuantizedLayer, X: torch.Tensor, status: Optional[torch.Tensor] = None,
+            ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Y [M, out] (fp32) = X [M, n] . What^T for M <= 16, the weights dequantized in registers."""
+    n, o, groups = _stored(q)
+    _require_cuda(X, ws, out)
+    if X.dim() != 2 or X.shape[1] != n or X.stride(1) != 1 or X.dtype not in _DTYPE_CODE:
+        raise ValueError("X must be an fp16/bf16/fp32 [M, n] tensor with contiguous rows")
+    M = X.shape[0]
+    need = int(lib().gptq_qmatvec_workspace_size(M, n, o))
+    if ws is None or ws.numel() < need:
+        ws = workspace(need, X.device)
+    if out is None:
+        out = torch.empty((M, o), dtype=torch.float32, device=X.device)
+    if out.dtype != torch.float32 or out.dim() != 2 or out.shape[0] != M or out.shape[1] != o or out.stride(1) != 1:
+        raise ValueError("out must be an fp32 [M, out] tensor with contiguous rows")
+    _check(lib().gptq_qmatvec(_ptr(q.qweight), _ptr(q.scales), _ptr(q.zeros), _ptr(q.g_idx), int(q.bits), n, o,
+                              groups, _ptr(X), _DTYPE_CODE[X.dtype], M, X.stride(0), _ptr(out), out.stride(0),
+                              _ptr(ws), ws.numel(), _ptr(status), _stream(stream)), "gptq_qmatvec")
+    return out
 
 
 def pack(codes: torch.Tensor, bits: int, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

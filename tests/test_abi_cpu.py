@@ -157,3 +157,22 @@ def test_noalloc_binding_rejects_mismatched_buffers_without_launching():
     # well-shaped host tensors still never reach the library
     with pytest.raises(ValueError, match="CUDA"):
         G.quantize_layer_noalloc(W, prep(n), good)
+
+
+def test_stored_format_consumers_reject_bad_arguments_without_a_gpu(L):
+    P = ctypes.c_void_p
+    fake = P(256)
+    # dequantize: 3-bit codes straddle words, unaligned qweight, a bad output dtype
+    assert L.gptq_dequantize(fake, fake, fake, fake, 3, 128, 64, 1, 1, fake, None, None) == -2
+    assert L.gptq_dequantize(P(260), fake, fake, fake, 4, 128, 64, 1, 1, fake, None, None) == -1
+    assert L.gptq_dequantize(fake, fake, fake, fake, 4, 128, 64, 1, 9, fake, None, None) == -1
+    assert L.gptq_dequantize(fake, fake, fake, fake, 4, 128, 64, 0, 1, fake, None, None) == -1
+    # matvec: at most 16 rows, a workspace of the reported size, ld_x >= n
+    need = L.gptq_qmatvec_workspace_size(4, 1024, 256)
+    assert need >= 2 * 4 * 256 * 4
+    assert L.gptq_qmatvec(fake, fake, fake, fake, 4, 1024, 256, 8, fake, 1, 17, 1024, fake, 256, fake, need,
+                          None, None) == -2
+    assert L.gptq_qmatvec(fake, fake, fake, fake, 4, 1024, 256, 8, fake, 1, 4, 1024, fake, 256, fake, need - 1,
+                          None, None) == -7
+    assert L.gptq_qmatvec(fake, fake, fake, fake, 4, 1024, 256, 8, fake, 1, 4, 1000, fake, 256, fake, need,
+                          None, None) == -1
