@@ -396,29 +396,33 @@ def time_qmatvec(G, torch, dev, peaks, flush, iters=20):
             zeros=torch.randint(0, 16, (G_, out), generator=gen, device=dev).half(),
             g_idx=(torch.randperm(n, generator=gen, device=dev) // 128).to(torch.int32),
             codes=None, err_sq=None, bits=4, group_size=128, sym=False)
-        for M in (1, 16):
-            X = torch.randn((M, n), generator=gen, device=dev).half()
-            Y = torch.empty((M, out), dtype=torch.float32, device=dev)
-            ws = G.workspace(G.lib().gptq_qmatvec_workspace_size(M, n, out), dev)
-            st = G.new_status(dev)
-            times = []
-            for i in range(iters + 3):
-                flush.fill_(1.0)
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                G.qmatvec(q, X, st, ws=ws, out=Y)
-                e1.record(stream)
-                torch.cuda.synchronize()
-                if i >= 3:
-                    times.append(e0.elapsed_time(e1))
-            G.raise_on_status(st, "qmatvec bench")
-            ms = statistics.median(times)
-            nbytes = out * n * 4 / 8 + 4.0 * G_ * out + 4.0 * n + 2.0 * M * n + 4.0 * M * out
-            gbs = nbytes / (ms * 1e-3) / 1e9
-            res.append({"out": out, "in": n, "tokens": M, "bits": 4, "group_size": 128, "act_order_g_idx": True,
-                        "us_per_call": ms * 1e3, "bytes": nbytes, "achieved_gbs": gbs,
-                        "frac": gbs / float(peaks["hbm_gbs"]),
-                        "flop": 2.0 * M * out * n, "tflops": 2.0 * M * out * n / (ms * 1e-3) / 1e12})
+        st = G.new_status(dev)
+        qg, xperm = G.reorder_groups(q, st)       # once per layer: the columns sorted by group
+        G.raise_on_status(st, "reorder")
+        for layout, lay, xp in (("act-order, as stored", q, None), ("act-order, reordered once", qg, xperm)):
+            for M in (1, 16):
+                X = torch.randn((M, n), generator=gen, device=dev).half()
+                Y = torch.empty((M, out), dtype=torch.float32, device=dev)
+                ws = G.workspace(G.lib().gptq_qmatvec_workspace_size(M, n, out), dev)
+                times = []
+                for i in range(iters + 3):
+                    flush.fill_(1.0)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    G.qmatvec(lay, X, st, ws=ws, out=Y, xperm=xp)
+                    e1.record(stream)
+                    torch.cuda.synchronize()
+                    if i >= 3:
+                        times.append(e0.elapsed_time(e1))
+                G.raise_on_status(st, "qmatvec bench")
+                ms = statistics.median(times)
+                nbytes = out * n * 4 / 8 + 4.0 * G_ * out + 4.0 * n + 2.0 * M * n + 4.0 * M * out + \
+                    (4.0 * n if xp is not None else 0.0)
+                gbs = nbytes / (ms * 1e-3) / 1e9
+                res.append({"out": out, "in": n, "tokens": M, "bits": 4, "group_size": 128, "layout": layout,
+                            "us_per_call": ms * 1e3, "bytes": nbytes, "achieved_gbs": gbs,
+                            "frac": gbs / float(peaks["hbm_gbs"]),
+                            "flop": 2.0 * M * out * n, "tflops": 2.0 * M * out * n / (ms * 1e-3) / 1e12})
     return {"kernel": "qmatvec (+ its k-split reduction)", "bound": "hbm", "peak": float(peaks["hbm_gbs"]),
             "unit": "GB/s", "peak_source": f"{peaks['_source']} HBM copy",
             "timing": f"CUDA events around each call, L2 flushed before each, median of {iters}",

@@ -326,18 +326,35 @@ GPTQ_API int gptq_pack_zeros(const uint16_t* zeros, int groups, int out, int bit
  * gptq_qmatvec - Y[M, out] = X[M, n] . What^T for 1 <= M <= 16 activation rows (the
  *   decode shapes), the weights dequantized in registers and never written: the call
  *   reads qweight once, so HBM bandwidth bounds it.  X of dtype x_dtype (F16, BF16 or
- *   F32), row stride ld_x; Y fp32, row stride ld_y (>= out).  Sums in fp32, in an order
- *   fixed by the shapes (deterministic).  ws: >= gptq_qmatvec_workspace_size(M, n, out)
- *   bytes, 256-byte aligned (the partial sums of the k splits).
+ *   F32), row stride ld_x; Y fp32, row stride ld_y (>= out).  xperm: NULL, or int32 [n]
+ *   (column k of the packed layer multiplies column xperm[k] of X: the form that
+ *   gptq_reorder_groups writes).  Sums in fp32, in an order fixed by the shapes
+ *   (deterministic).  ws: >= gptq_qmatvec_workspace_size(M, n, out) bytes, 256-byte
+ *   aligned (the partial sums of the k splits).  Fastest when the groups of nearby
+ *   columns are contiguous (no act-order, or a reordered layer): their scales and zero
+ *   points are then staged once per block of columns.
+ *
+ * gptq_reorder_groups - once per layer, for act-order layers (whose g_idx scatters the
+ *   groups over the columns): xperm = the columns sorted by group (ties in column
+ *   order), g_idx_g[k] = g_idx[xperm[k]] (non-decreasing), and qweight_g [n*bits/32,
+ *   out] holding the codes of columns xperm[k] at position k.  The sum over columns does
+ *   not depend on their order, so gptq_qmatvec(qweight_g, scales, zeros, g_idx_g,
+ *   xperm, ...) is the same product as on the original layer (up to the order of the
+ *   fp32 additions).  ws >= gptq_reorder_groups_workspace_size(groups) bytes.
+ *   n * bits / 32 <= 65535.
  */
 GPTQ_API int gptq_dequantize(const int32_t* qweight, const uint16_t* scales, const uint16_t* zeros,
                              const int32_t* g_idx, int bits, int n, int out, int groups, int out_dtype, void* What,
                              int32_t* d_status, void* stream);
 GPTQ_API size_t gptq_qmatvec_workspace_size(int M, int n, int out);
 GPTQ_API int gptq_qmatvec(const int32_t* qweight, const uint16_t* scales, const uint16_t* zeros,
-                          const int32_t* g_idx, int bits, int n, int out, int groups, const void* X, int x_dtype,
-                          int M, int64_t ld_x, float* Y, int64_t ld_y, void* ws, size_t ws_bytes,
-                          int32_t* d_status, void* stream);
+                          const int32_t* g_idx, const int32_t* xperm, int bits, int n, int out, int groups,
+                          const void* X, int x_dtype, int M, int64_t ld_x, float* Y, int64_t ld_y, void* ws,
+                          size_t ws_bytes, int32_t* d_status, void* stream);
+GPTQ_API size_t gptq_reorder_groups_workspace_size(int groups);
+GPTQ_API int gptq_reorder_groups(const int32_t* qweight, const int32_t* g_idx, int bits, int n, int out, int groups,
+                                 int32_t* qweight_g, int32_t* g_idx_g, int32_t* xperm, void* ws, size_t ws_bytes,
+                                 int32_t* d_status, void* stream);
 
 /*
  * Kernel timing trace.  The GPTQ pages have no counterpart to these calls: they

@@ -16,6 +16,9 @@
 //                    partial sums reduced in a fixed order (deterministic).
 // Both take any g_idx (act-order included).  Codes of 2, 4 or 8 bits (a word holds
 // 32 / bits whole codes).
+#include <algorithm>
+#include <climits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -78,44 +81,75 @@ __global__ void __launch_bounds__(256) dequant_kernel(const int32_t* qweight, co
 // M = 1, 2, 4, 8, 16 rows; rows m .. M-1 are staged as zeros and never written).
 // Block: 8 warps over the same 128 outputs (lane: four outputs, one uint4 of a
 // qweight row); the block's k range [k0, k0 + kc) is split between the warps word by
-// word, four words in flight per thread; X's columns of the range sit in shared
-// memory as fp32, g_idx beside them.  Per word and output the code of each of its
-// 32/bits columns is dequantized once and multiplies all rows.  The 8 warps' sums
-// are added in warp order into part[split][m][out] (fp32); qmatvec_reduce_kernel
-// adds the splits in order.
+// word, four words in flight per thread.  Staged in shared memory first: X's columns
+// of the range as fp32 (column k of the packed layer multiplies X column xperm[k],
+// or k), the range's group indices, and - when the range's groups span at most
+// QMV_MAXG consecutive groups (groups contiguous in k: no act-order, or a layer
+// reordered by gptq_reorder_groups) - their scales and zero points for the block's
+// 128 outputs; otherwise the inner loop reads those from global memory.  Per word and
+// output the code of each of its 32/bits columns is dequantized once and multiplies
+// all rows.  The 8 warps' sums are added in warp order into part[split][m][out]
+// (fp32); qmatvec_reduce_kernel adds the splits in order.
 // ---------------------------------------------------------------------------
 constexpr int QMV_MAXM = 16;
-constexpr int QMV_KC = 512;           // input columns per block
+constexpr int QMV_KC = 512;           // input columns per block (256 for 16 rows: shared memory)
+__host__ __device__ constexpr int qmv_kc(int M) { return M > 8 ? QMV_KC / 2 : QMV_KC; }
 constexpr int QMV_UNROLL = 4;         // words in flight per thread
+constexpr int QMV_MAXG = 17;          // staged groups: 512 / 32 + 1
 
 template <typename TX, int BITS, int M>
 __global__ void __launch_bounds__(256) qmatvec_kernel(const int32_t* qweight, const uint16_t* scales,
                                                       const uint16_t* zeros, const int32_t* g_idx, int n, int out,
-                                                      int groups, const TX* X, int m_real, int ldx, float* part,
-                                                      int32_t* st) {
+                                                      int groups, const TX* X, const int32_t* xperm, int m_real,
+                                                      int ldx, float* part, int32_t* st) {
   if (has_error(st)) return;
   constexpr int PER = 32 / BITS;
-  constexpr int kc = QMV_KC;
+  constexpr int kc = qmv_kc(M);
   __shared__ float xs[M * kc];
   __shared__ int gsm[kc];
   __shared__ float red[8 * 128];
+  __shared__ float2 szs[QMV_MAXG * 128];      // (scale, zero) of staged group g_lo + i for output o0 + j
+  __shared__ int grange[2];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int o0 = blockIdx.x * 128;
   const int k0 = blockIdx.y * kc;
   const int k1 = min(n, k0 + kc);
-  for (int i = threadIdx.x; i < M * kc; i += blockDim.x) {
-    const int m = i / kc, k = k0 + i % kc;
-    xs[i] = (k < k1 && m < m_real) ? load_as_float<TX>(X + (int64_t)m * ldx + k) : 0.f;
-  }
+  if (threadIdx.x == 0) { grange[0] = INT_MAX; grange[1] = -1; }
+  __syncthreads();
+  int gmin = INT_MAX, gmax = -1;
   for (int i = threadIdx.x; i < kc; i += blockDim.x) {
-    int g = k0 + i < k1 ? g_idx[k0 + i] : 0;
-    if ((unsigned)g >= (unsigned)groups) {          // a group index the scales do not have
+    int g = k0 + i < k1 ? g_idx[k0 + i] : -1;
+    if (g >= groups || (g < 0 && k0 + i < k1)) {     // a group index the scales do not have
       set_error(st, GPTQ_ERR_INVALID_ARG, k0 + i, STAGE_DEQUANT);
       g = 0;
     }
-    gsm[i] = g;
+    if (k0 + i < k1) { gmin = min(gmin, g); gmax = max(gmax, g); }
+    gsm[i] = g < 0 ? 0 : g;
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, o));
+    gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
+  }
+  if (lane == 0) { atomicMin(&grange[0], gmin); atomicMax(&grange[1], gmax); }
+  for (int i = threadIdx.x; i < M * kc; i += blockDim.x) {
+    const int m = i / kc, k = k0 + i % kc;
+    const int xk = k < k1 ? (xperm ? xperm[k] : k) : 0;
+    xs[i] = (k < k1 && m < m_real) ? load_as_float<TX>(X + (int64_t)m * ldx + xk) : 0.f;
   }
   __syncthreads();
+  const int g_lo = grange[0];
+  const bool staged = grange[1] - g_lo < QMV_MAXG;
+  if (staged) {
+    for (int i = threadIdx.x; i < (grange[1] - g_lo + 1) * 128; i += blockDim.x) {
+      const int gi = i / 128, oo = o0 + i % 128;
+      float2 v = make_float2(0.f, 0.f);
+      if (oo < out)
+        v = make_float2(__half2float(__ushort_as_half(scales[(int64_t)(g_lo + gi) * out + oo])),
+                        __half2float(__ushort_as_half(zeros[(int64_t)(g_lo + gi) * out + oo])));
+      szs[i] = v;
+    }
+    __syncthreads();
+  }
   const int o = o0 + 4 * lane;
   float acc[M][4];
 #pragma unroll
@@ -151,7 +185,14 @@ __global__ void __launch_bounds__(256) qmatvec_kernel(const int32_t* qweight, co
       for (int i = 0; i < PER; ++i) {
         const int kl = w * PER + i - k0;
         const int g = gsm[kl];
-        if (g != g_prev) {             // a new group: its scales and zero points for the four outputs
+        if (staged) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 v = szs[(g - g_lo) * 128 + 4 * lane + j];
+            s[j] = v.x;
+            z[j] = v.y;
+          }
+        } else if (g != g_prev) {      // a new group: its scales and zero points for the four outputs
           g_prev = g;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -215,29 +256,114 @@ int dequant_t(const int32_t* qweight, const uint16_t* scales, const uint16_t* ze
 
 template <typename TX, int BITS, int M>
 int qmv_launch(const int32_t* qweight, const uint16_t* scales, const uint16_t* zeros, const int32_t* g_idx, int n,
-               int out, int groups, const void* X, int m_real, int ldx, float* part, int splits, int32_t* st,
-               cudaStream_t s) {
-  dim3 grd((unsigned)cdiv(out, 128), (unsigned)splits);
+               int out, int groups, const void* X, const int32_t* xperm, int m_real, int ldx, float* part,
+               int splits, int32_t* st, cudaStream_t s) {
+  (void)splits;
+  dim3 grd((unsigned)cdiv(out, 128), (unsigned)cdiv(n, qmv_kc(M)));
   qmatvec_kernel<TX, BITS, M><<<grd, 256, 0, s>>>(qweight, scales, zeros, g_idx, n, out, groups,
-                                                   static_cast<const TX*>(X), m_real, ldx, part, st);
+                                                   static_cast<const TX*>(X), xperm, m_real, ldx, part, st);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }
 
 template <typename TX, int BITS>
 int qmv_m(int M, const int32_t* qweight, const uint16_t* scales, const uint16_t* zeros, const int32_t* g_idx, int n,
-          int out, int groups, const void* X, int ldx, float* part, int splits, int32_t* st, cudaStream_t s) {
-  if (M <= 1) return qmv_launch<TX, BITS, 1>(qweight, scales, zeros, g_idx, n, out, groups, X, M, ldx, part, splits, st, s);
-  if (M <= 2) return qmv_launch<TX, BITS, 2>(qweight, scales, zeros, g_idx, n, out, groups, X, M, ldx, part, splits, st, s);
-  if (M <= 4) return qmv_launch<TX, BITS, 4>(qweight, scales, zeros, g_idx, n, out, groups, X, M, ldx, part, splits, st, s);
-  if (M <= 8) return qmv_launch<TX, BITS, 8>(qweight, scales, zeros, g_idx, n, out, groups, X, M, ldx, part, splits, st, s);
-  return qmv_launch<TX, BITS, 16>(qweight, scales, zeros, g_idx, n, out, groups, X, M, ldx, part, splits, st, s);
+          int out, int groups, const void* X, const int32_t* xperm, int ldx, float* part, int splits, int32_t* st,
+          cudaStream_t s) {
+  if (M <= 1) return qmv_launch<TX, BITS, 1>(qweight, scales, zeros, g_idx, n, out, groups, X, xperm, M, ldx, part, splits, st, s);
+  if (M <= 2) return qmv_launch<TX, BITS, 2>(qweight, scales, zeros, g_idx, n, out, groups, X, xperm, M, ldx, part, splits, st, s);
+  if (M <= 4) return qmv_launch<TX, BITS, 4>(qweight, scales, zeros, g_idx, n, out, groups, X, xperm, M, ldx, part, splits, st, s);
+  if (M <= 8) return qmv_launch<TX, BITS, 8>(qweight, scales, zeros, g_idx, n, out, groups, X, xperm, M, ldx, part, splits, st, s);
+  return qmv_launch<TX, BITS, 16>(qweight, scales, zeros, g_idx, n, out, groups, X, xperm, M, ldx, part, splits, st, s);
+}
+
+// ---------------------------------------------------------------------------
+// Reordering a layer so that its groups are contiguous: xperm = the columns sorted by
+// group, ties in column order (stable).  One thread per group scans g_idx (staged in
+// shared memory in slabs, every thread reading the same word: a broadcast) and writes
+// the positions of its group's columns in order, after the counts of the groups
+// before it.
+// ---------------------------------------------------------------------------
+constexpr int RG_SLAB = 8192;
+
+__global__ void __launch_bounds__(1024) group_count_kernel(const int32_t* g_idx, int n, int groups, int* counts,
+                                                           int32_t* st) {
+  if (has_error(st)) return;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int g = g_idx[i];
+    if ((unsigned)g >= (unsigned)groups) { set_error(st, GPTQ_ERR_INVALID_ARG, i, STAGE_DEQUANT); continue; }
+    atomicAdd(counts + g, 1);
+  }
+}
+
+__global__ void __launch_bounds__(1024) group_scatter_kernel(const int32_t* g_idx, int n, int groups,
+                                                             const int* counts, int32_t* xperm, int32_t* g_sorted,
+                                                             const int32_t* st) {
+  if (has_error(st)) return;
+  __shared__ int slab[RG_SLAB];
+  const int g = blockIdx.x * blockDim.x + threadIdx.x;
+  int pos = 0;                                       // the first position of group g
+  if (g < groups)
+    for (int h = 0; h < g; ++h) pos += counts[h];
+  for (int base = 0; base < n; base += RG_SLAB) {
+    const int len = min(RG_SLAB, n - base);
+    __syncthreads();
+    for (int i = threadIdx.x; i < len; i += blockDim.x) slab[i] = g_idx[base + i];
+    __syncthreads();
+    if (g < groups) {
+      for (int i = 0; i < len; ++i) {
+        if (slab[i] == g) {
+          xperm[pos] = base + i;
+          g_sorted[pos] = g;
+          ++pos;
+        }
+      }
+    }
+  }
+}
+
+// qweight_g[w][o]: the codes of columns xperm[w.PER .. w.PER + PER - 1] for output o.
+template <int BITS>
+__global__ void repack_kernel(const int32_t* qweight, const int32_t* xperm, int n, int out, int32_t* qweight_g,
+                              const int32_t* st) {
+  if (has_error(st)) return;
+  constexpr int PER = 32 / BITS;
+  const int o = blockIdx.x * blockDim.x + threadIdx.x;
+  const int w = blockIdx.y;
+  if (o >= out || w >= n / PER) return;
+  uint32_t word = 0u;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int k = xperm[w * PER + i];
+    const uint32_t src = (uint32_t)qweight[(int64_t)(k / PER) * out + o];
+    word |= ((src >> ((k % PER) * BITS)) & ((1u << BITS) - 1u)) << (i * BITS);
+  }
+  qweight_g[(int64_t)w * out + o] = (int32_t)word;
 }
 
 }  // namespace
 
+size_t reorder_ws_bytes(int groups) { return align_up((size_t)groups * 4, 256); }
+
+int launch_reorder_groups(const int32_t* qweight, const int32_t* g_idx, int bits, int n, int out, int groups,
+                          int32_t* qweight_g, int32_t* g_sorted, int32_t* xperm, void* ws, int32_t* st,
+                          cudaStream_t s) {
+  int* counts = static_cast<int*>(ws);
+  GPTQ_CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)groups * 4, s));
+  group_count_kernel<<<(unsigned)std::min<int64_t>(cdiv(n, 1024), 148), 1024, 0, s>>>(g_idx, n, groups, counts, st);
+  GPTQ_LAUNCH_CHECK();
+  group_scatter_kernel<<<(unsigned)cdiv(groups, 1024), 1024, 0, s>>>(g_idx, n, groups, counts, xperm, g_sorted, st);
+  GPTQ_LAUNCH_CHECK();
+  dim3 grd((unsigned)cdiv(out, 256), (unsigned)(n * bits / 32));
+  if (bits == 2) repack_kernel<2><<<grd, 256, 0, s>>>(qweight, xperm, n, out, qweight_g, st);
+  else if (bits == 4) repack_kernel<4><<<grd, 256, 0, s>>>(qweight, xperm, n, out, qweight_g, st);
+  else repack_kernel<8><<<grd, 256, 0, s>>>(qweight, xperm, n, out, qweight_g, st);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
 size_t qmatvec_ws_bytes(int M, int n, int out) {
-  const int splits = (int)cdiv(n, QMV_KC);
+  const int splits = (int)cdiv(n, qmv_kc(M <= 8 ? M : 16));
   return align_up((size_t)splits * M * out * 4, 256);
 }
 
@@ -251,9 +377,9 @@ int launch_dequant(const int32_t* qweight, const uint16_t* scales, const uint16_
 }
 
 int launch_qmatvec(const int32_t* qweight, const uint16_t* scales, const uint16_t* zeros, const int32_t* g_idx,
-                   int bits, int n, int out, int groups, const void* X, int x_dtype, int M, int ldx, float* Y, int ldy,
-                   void* ws, int32_t* st, cudaStream_t s) {
-  const int splits = (int)cdiv(n, QMV_KC);
+                   int bits, int n, int out, int groups, const void* X, const int32_t* xperm, int x_dtype, int M,
+                   int ldx, float* Y, int ldy, void* ws, int32_t* st, cudaStream_t s) {
+  const int splits = (int)cdiv(n, qmv_kc(M <= 8 ? M : 16));
   float* part = static_cast<float*>(ws);
   // bytes read once: packed weights, scales and zeros, g_idx, X; Y written
   TraceScope ts("qmatvec", "byte",
@@ -261,9 +387,9 @@ int launch_qmatvec(const int32_t* qweight, const uint16_t* scales, const uint16_
   int rc = GPTQ_ERR_UNSUPPORTED;
   auto go = [&](auto tx_tag) {
     using TX = decltype(tx_tag);
-    if (bits == 2) return qmv_m<TX, 2>(M, qweight, scales, zeros, g_idx, n, out, groups, X, ldx, part, splits, st, s);
-    if (bits == 4) return qmv_m<TX, 4>(M, qweight, scales, zeros, g_idx, n, out, groups, X, ldx, part, splits, st, s);
-    return qmv_m<TX, 8>(M, qweight, scales, zeros, g_idx, n, out, groups, X, ldx, part, splits, st, s);
+    if (bits == 2) return qmv_m<TX, 2>(M, qweight, scales, zeros, g_idx, n, out, groups, X, xperm, ldx, part, splits, st, s);
+    if (bits == 4) return qmv_m<TX, 4>(M, qweight, scales, zeros, g_idx, n, out, groups, X, xperm, ldx, part, splits, st, s);
+    return qmv_m<TX, 8>(M, qweight, scales, zeros, g_idx, n, out, groups, X, xperm, ldx, part, splits, st, s);
   };
   if (x_dtype == GPTQ_F16) rc = go(__half{});
   else if (x_dtype == GPTQ_BF16) rc = go(__nv_bfloat16{});

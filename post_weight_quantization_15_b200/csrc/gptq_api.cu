@@ -217,8 +217,8 @@ size_t gptq_qmatvec_workspace_size(int M, int n, int out) {
 }
 
 int gptq_qmatvec(const int32_t* qweight, const uint16_t* scales, const uint16_t* zeros, const int32_t* g_idx,
-                 int bits, int n, int out, int groups, const void* X, int x_dtype, int M, int64_t ld_x, float* Y,
-                 int64_t ld_y, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+                 const int32_t* xperm, int bits, int n, int out, int groups, const void* X, int x_dtype, int M,
+                 int64_t ld_x, float* Y, int64_t ld_y, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
   const int rc = check_stored(qweight, scales, zeros, g_idx, bits, n, out, groups);
   if (rc != GPTQ_OK) return rc;
   if (X == nullptr || Y == nullptr || M < 1 || ld_x < n || ld_y < out || ld_x > INT32_MAX || ld_y > INT32_MAX)
@@ -226,8 +226,23 @@ int gptq_qmatvec(const int32_t* qweight, const uint16_t* scales, const uint16_t*
   if (M > 16) return GPTQ_ERR_UNSUPPORTED;
   if (x_dtype != GPTQ_F32 && x_dtype != GPTQ_F16 && x_dtype != GPTQ_BF16) return GPTQ_ERR_INVALID_ARG;
   if (ws == nullptr || ws_bytes < qmatvec_ws_bytes(M, n, out) || !aligned(ws, 256)) return GPTQ_ERR_WORKSPACE;
-  return launch_qmatvec(qweight, scales, zeros, g_idx, bits, n, out, groups, X, x_dtype, M, (int)ld_x, Y, (int)ld_y,
-                        ws, d_status, as_stream(stream));
+  return launch_qmatvec(qweight, scales, zeros, g_idx, bits, n, out, groups, X, xperm, x_dtype, M, (int)ld_x, Y,
+                        (int)ld_y, ws, d_status, as_stream(stream));
+}
+
+size_t gptq_reorder_groups_workspace_size(int groups) { return groups > 0 ? reorder_ws_bytes(groups) : 0; }
+
+int gptq_reorder_groups(const int32_t* qweight, const int32_t* g_idx, int bits, int n, int out, int groups,
+                        int32_t* qweight_g, int32_t* g_idx_g, int32_t* xperm, void* ws, size_t ws_bytes,
+                        int32_t* d_status, void* stream) {
+  if (qweight == nullptr || g_idx == nullptr || qweight_g == nullptr || g_idx_g == nullptr || xperm == nullptr ||
+      d_status == nullptr || n <= 0 || out <= 0 || groups <= 0 || groups > n)
+    return GPTQ_ERR_INVALID_ARG;
+  if (bits != 2 && bits != 4 && bits != 8) return GPTQ_ERR_UNSUPPORTED;
+  if ((n * bits) % 32 != 0 || (int64_t)n * bits / 32 > 65535) return GPTQ_ERR_UNSUPPORTED;
+  if (ws == nullptr || ws_bytes < reorder_ws_bytes(groups) || !aligned(ws, 256)) return GPTQ_ERR_WORKSPACE;
+  return launch_reorder_groups(qweight, g_idx, bits, n, out, groups, qweight_g, g_idx_g, xperm, ws, d_status,
+                               as_stream(stream));
 }
 
 int gptq_pack(const uint8_t* codes, int out, int n, int bits, int32_t* qweight, void* stream) {

@@ -69,8 +69,12 @@ int launch_dequant(const int32_t* qweight, const uint16_t* scales, const uint16_
                    int bits, int n, int out, int groups, int dtype, void* What, int32_t* st, cudaStream_t s);
 size_t qmatvec_ws_bytes(int M, int n, int out);
 int launch_qmatvec(const int32_t* qweight, const uint16_t* scales, const uint16_t* zeros, const int32_t* g_idx,
-                   int bits, int n, int out, int groups, const void* X, int x_dtype, int M, int ldx, float* Y, int ldy,
-                   void* ws, int32_t* st, cudaStream_t s);
+                   int bits, int n, int out, int groups, const void* X, const int32_t* xperm, int x_dtype, int M,
+                   int ldx, float* Y, int ldy, void* ws, int32_t* st, cudaStream_t s);
+size_t reorder_ws_bytes(int groups);
+int launch_reorder_groups(const int32_t* qweight, const int32_t* g_idx, int bits, int n, int out, int groups,
+                          int32_t* qweight_g, int32_t* g_sorted, int32_t* xperm, void* ws, int32_t* st,
+                          cudaStream_t s);
 
 // ---- tensor-core GEMM: C -= A . B^T in 3 x TF32 (operands pre-split) ---------
 // store = false: C -= A.B^T; store = true: C = A.B^T (C may be null then, if Chi/Clo are given).

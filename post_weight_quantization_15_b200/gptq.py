@@ -117,7 +117,11 @@ def lib() -> ctypes.CDLL:
     L.gptq_qmatvec_workspace_size.restype = SZ
     L.gptq_qmatvec_workspace_size.argtypes = [I, I, I]
     L.gptq_qmatvec.restype = I
-    L.gptq_qmatvec.argtypes = [P, P, P, P, I, I, I, I, P, I, I, I64, P, I64, P, SZ, P, P]
+    L.gptq_qmatvec.argtypes = [P, P, P, P, P, I, I, I, I, P, I, I, I64, P, I64, P, SZ, P, P]
+    L.gptq_reorder_groups_workspace_size.restype = SZ
+    L.gptq_reorder_groups_workspace_size.argtypes = [I]
+    L.gptq_reorder_groups.restype = I
+    L.gptq_reorder_groups.argtypes = [P, P, I, I, I, I, P, P, P, P, SZ, P, P]
     L.gptq_probe_fp32_peak.restype = I
     L.gptq_probe_fp32_peak.argtypes = [P, I, I, P]
     L.gptq_quantize_layer_noalloc.restype = I
@@ -482,11 +486,31 @@ def dequantize(q: QuantizedLayer, dtype=torch.float16, status: Optional[torch.Te
     return out
 
 
-def qmatvec(q: QuantizedLayer, X: torch.Tensor, status: Optional[torch.Tensor] = None,
-            ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """Y [M, out] (fp32) = X [M, n] . What^T for M <= 16, the weights dequantized in registers."""
+def reorder_groups(q: QuantizedLayer, status: Optional[torch.Tensor] = None, stream=None):
+    """Once per act-order layer: (layer with its columns sorted by group, xperm) for qmatvec."""
     n, o, groups = _stored(q)
-    _require_cuda(X, ws, out)
+    dev = q.qweight.device
+    st = status if status is not None else new_status(dev)
+    qg = torch.empty_like(q.qweight)
+    gg = torch.empty_like(q.g_idx)
+    xperm = torch.empty_like(q.g_idx)
+    ws = workspace(int(lib().gptq_reorder_groups_workspace_size(groups)), dev)
+    _check(lib().gptq_reorder_groups(_ptr(q.qweight), _ptr(q.g_idx), int(q.bits), n, o, groups, _ptr(qg), _ptr(gg),
+                                     _ptr(xperm), _ptr(ws), ws.numel(), _ptr(st), _stream(stream)),
+           "gptq_reorder_groups")
+    return QuantizedLayer(qg, q.scales, q.zeros, gg, None, None, q.bits, q.group_size, q.sym), xperm
+
+
+def qmatvec(q: QuantizedLayer, X: torch.Tensor, status: Optional[torch.Tensor] = None,
+            ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+            xperm: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Y [M, out] (fp32) = X [M, n] . What^T for M <= 16, the weights dequantized in registers.
+
+    xperm: for a layer from reorder_groups, its column permutation."""
+    n, o, groups = _stored(q)
+    _require_cuda(X, ws, out, xperm)
+    if xperm is not None and (xperm.dtype != torch.int32 or xperm.numel() != n):
+        raise ValueError("xperm must be int32 [n]")
     if X.dim() != 2 or X.shape[1] != n or X.stride(1) != 1 or X.dtype not in _DTYPE_CODE:
         raise ValueError("X must be an fp16/bf16/fp32 [M, n] tensor with contiguous rows")
     M = X.shape[0]
@@ -497,7 +521,8 @@ def qmatvec(q: QuantizedLayer, X: torch.Tensor, status: Optional[torch.Tensor] =
         out = torch.empty((M, o), dtype=torch.float32, device=X.device)
     if out.dtype != torch.float32 or out.dim() != 2 or out.shape[0] != M or out.shape[1] != o or out.stride(1) != 1:
         raise ValueError("out must be an fp32 [M, out] tensor with contiguous rows")
-    _check(lib().gptq_qmatvec(_ptr(q.qweight), _ptr(q.scales), _ptr(q.zeros), _ptr(q.g_idx), int(q.bits), n, o,
+    _check(lib().gptq_qmatvec(_ptr(q.qweight), _ptr(q.scales), _ptr(q.zeros), _ptr(q.g_idx), _ptr(xperm),
+                              int(q.bits), n, o,
                               groups, _ptr(X), _DTYPE_CODE[X.dtype], M, X.stride(0), _ptr(out), out.stride(0),
                               _ptr(ws), ws.numel(), _ptr(status), _stream(stream)), "gptq_qmatvec")
     return out

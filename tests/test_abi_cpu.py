@@ -170,9 +170,14 @@ def test_stored_format_consumers_reject_bad_arguments_without_a_gpu(L):
     # matvec: at most 16 rows, a workspace of the reported size, ld_x >= n
     need = L.gptq_qmatvec_workspace_size(4, 1024, 256)
     assert need >= 2 * 4 * 256 * 4
-    assert L.gptq_qmatvec(fake, fake, fake, fake, 4, 1024, 256, 8, fake, 1, 17, 1024, fake, 256, fake, need,
+    assert L.gptq_qmatvec(fake, fake, fake, fake, None, 4, 1024, 256, 8, fake, 1, 17, 1024, fake, 256, fake, need,
                           None, None) == -2
-    assert L.gptq_qmatvec(fake, fake, fake, fake, 4, 1024, 256, 8, fake, 1, 4, 1024, fake, 256, fake, need - 1,
-                          None, None) == -7
-    assert L.gptq_qmatvec(fake, fake, fake, fake, 4, 1024, 256, 8, fake, 1, 4, 1000, fake, 256, fake, need,
+    assert L.gptq_qmatvec(fake, fake, fake, fake, None, 4, 1024, 256, 8, fake, 1, 4, 1024, fake, 256, fake,
+                          need - 1, None, None) == -7
+    assert L.gptq_qmatvec(fake, fake, fake, fake, None, 4, 1024, 256, 8, fake, 1, 4, 1000, fake, 256, fake, need,
                           None, None) == -1
+    # reordering: 3-bit, too many groups, a small workspace
+    wsz = L.gptq_reorder_groups_workspace_size(8)
+    assert L.gptq_reorder_groups(fake, fake, 3, 1024, 256, 8, fake, fake, fake, fake, wsz, fake, None) == -2
+    assert L.gptq_reorder_groups(fake, fake, 4, 1024, 256, 2048, fake, fake, fake, fake, wsz, fake, None) == -1
+    assert L.gptq_reorder_groups(fake, fake, 4, 1024, 256, 8, fake, fake, fake, fake, 0, fake, None) == -7

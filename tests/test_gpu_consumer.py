@@ -132,3 +132,28 @@ def test_group_index_outside_the_scales_is_reported():
     G.qmatvec(bad, torch.zeros((2, 256), dtype=torch.float16, device=q.qweight.device), st)
     rc, info = G.status_read(st)
     assert rc == G.gptq.ERR_INVALID_ARG and info == 77
+
+
+@pytest.mark.parametrize("bits,gs,M", [(4, 128, 1), (4, 32, 16), (2, 64, 5), (8, 128, 8)])
+def test_reordered_act_order_layer(bits, gs, M):
+    """gptq_reorder_groups on an act-order layer: xperm is a permutation sorting the columns by
+    group (stable), the reordered layer dequantizes to the original's columns in that order
+    bit for bit, and its product (with xperm) is the oracle's within the summation bound."""
+    q = _stored_layer(260, 1024, 2048, bits, gs, False, True, seed=bits + gs + M)
+    st = G.new_status(q.qweight.device)
+    qg, xperm = G.reorder_groups(q, st)
+    G.raise_on_status(st, "reorder")
+    g = q.g_idx.cpu().numpy()
+    xp = xperm.cpu().numpy()
+    assert np.array_equal(np.sort(xp), np.arange(1024))
+    assert np.array_equal(xp, np.argsort(g, kind="stable"))
+    assert np.array_equal(qg.g_idx.cpu().numpy(), g[xp])
+    What = _oracle_what(q)
+    assert np.array_equal(G.dequantize(qg, torch.float32, st).cpu().numpy(), What[:, xp].astype(np.float32))
+    X = torch.from_numpy(np.random.default_rng(M).standard_normal((M, 1024)).astype(np.float32)).to(
+        q.qweight.device).half()
+    Y = G.qmatvec(qg, X, st, xperm=xperm)
+    G.raise_on_status(st, "reordered qmatvec")
+    X64 = X.float().cpu().numpy().astype(np.float64)
+    err = np.abs(Y.cpu().numpy().astype(np.float64) - X64 @ What.T)
+    assert np.all(err <= _matvec_bound(X64, What))

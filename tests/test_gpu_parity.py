@@ -266,14 +266,15 @@ def test_worked_example_layer_full_size():
 # The Llama-shaped layers at their own token counts, every setting: test_gpu_full_shapes.py.
 
 
-def test_bounded_wait_reports_timeout_and_the_context_survives(monkeypatch):
-    """The Hessian producer withholds its loads (host-side test switch); the MMA
-    side's bounded wait runs out, the kernel drains, frees TMEM and reports
+@pytest.mark.parametrize("n", [200, 256, 520])     # the single-CTA kernel; CTA pairs (one tile; ragged tiles)
+def test_bounded_wait_reports_timeout_and_the_context_survives(monkeypatch, n):
+    """The Hessian producers withhold their loads (host-side test switch); the MMA
+    side's bounded waits run out, the kernel drains, frees TMEM and reports
     GPTQ_ERR_TIMEOUT; the next call on the same context works."""
     dev = _dev()
-    _, x = S.small_case(8, 256, 1024, seed=9)
+    _, x = S.small_case(8, n, 1024, seed=9)
     X = _to_dev_x(x, dev)
-    H = torch.zeros((256, 256), dtype=torch.float32, device=dev)
+    H = torch.zeros((n, n), dtype=torch.float32, device=dev)
     st = G.new_status(dev)
     monkeypatch.setenv("GPTQ_FAULT_INJECT", "hessian_stall")
     G.hessian_accumulate(H, X, None, st)
@@ -286,8 +287,26 @@ def test_bounded_wait_reports_timeout_and_the_context_survives(monkeypatch):
     rc, _ = G.status_read(st)
     assert rc == G.gptq.OK
     H64 = O.hessian(x)
-    iu = np.triu_indices(256)
-    assert np.allclose(H.cpu().numpy().astype(np.float64)[iu], H64[iu], rtol=1e-4, atol=1e-3)
+    iu = np.triu_indices(n)
+    rel = np.abs(H.cpu().numpy().astype(np.float64)[iu] - H64[iu]) / np.sqrt(np.outer(np.diag(H64), np.diag(H64)))[iu]
+    assert rel.max() <= hessian_bound([1024])
+
+
+@pytest.mark.parametrize("n,tokens", [(256, 64), (384, 1000), (768, 4096), (1300, 777)])
+def test_hessian_tile_pairs_against_oracle(n, tokens):
+    """The CTA-pair kernel (n >= 256): whole tiles, ragged tiles, one stage, ragged tokens."""
+    dev = _dev()
+    _, x = S.small_case(8, n, tokens, seed=n + tokens)
+    H = torch.zeros((n, n), dtype=torch.float32, device=dev)
+    hd = torch.zeros(n, dtype=torch.float64, device=dev)
+    st = G.new_status(dev)
+    G.hessian_accumulate(H, _to_dev_x(x, dev), hd, st)
+    G.raise_on_status(st, "pair Hessian")
+    H64 = O.hessian(x)
+    iu = np.triu_indices(n)
+    rel = np.abs(H.cpu().numpy().astype(np.float64)[iu] - H64[iu]) / np.sqrt(np.outer(np.diag(H64), np.diag(H64)))[iu]
+    assert rel.max() <= hessian_bound([tokens]), rel.max()
+    assert np.allclose(hd.cpu().numpy(), np.diag(H64), rtol=1e-13, atol=0)
 
 
 @pytest.mark.parametrize("sym", [True, False])
