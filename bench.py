@@ -26,6 +26,7 @@ each step the whole layer with all of its tokens, nothing extrapolated.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -429,6 +430,32 @@ def time_qmatvec(G, torch, dev, peaks, flush, iters=20):
             "shapes": res}
 
 
+def time_pipeline(G, torch, dev, blocks=2, warmup=1):
+    """The sequential pipeline (pipeline.quantize_mlp_blocks) over the MLP halves of
+    Llama-2-7B-shaped blocks: d 4096, d_ff 11008, 65,536 tokens, 4-bit symmetric g128
+    act-order; inputs drawn on the device.  Device time per block and per stage."""
+    from post_weight_quantization_15_b200 import pipeline as PL
+    wl = S.workloads()["llama2-7b-block"]
+    st = wl.settings[0]
+    by = {l.name: l for l in wl.layers}
+    X0 = S.make_x_device(by["gate"].x, dev)
+    X0 = X0.contiguous() if X0.stride(0) != X0.shape[1] else X0
+    weights = []
+    for b in range(blocks):
+        weights.append(tuple(S.make_w_device(dataclasses.replace(by[nm].w, stream=by[nm].w.stream + 1000 * b), dev)
+                             for nm in ("gate", "up", "down")))
+    for _ in range(warmup):
+        PL.quantize_mlp_blocks(X0, weights[:1], st.bits, st.group_size, st.sym, st.desc_act, st.damp_percent)
+    res, _ = PL.quantize_mlp_blocks(X0, weights, st.bits, st.group_size, st.sym, st.desc_act, st.damp_percent)
+    per = [r.ms for r in res]
+    ms = statistics.mean(p["block"] for p in per)
+    n_w = sum(int(w.numel()) for w in weights[0])
+    return {"workload": "llama2-7b MLP blocks (gate, up, down), 65,536 tokens, each block calibrated on the "
+                        "previous quantized block's output", "blocks": blocks,
+            "ms_per_block": ms, "gparam_per_s": n_w / (ms * 1e-3) / 1e9, "per_block_stages_ms": per,
+            "timing": "CUDA events on the calling stream around each stage"}
+
+
 def config_dict(name, layer, st):
     return {"workload": name, "out": layer.w.out, "in": layer.w.n, "tokens": layer.x.tokens,
             "w_dtype": layer.w.dtype, "bits": st.bits, "group_size": st.group_size, "sym": st.sym,
@@ -571,13 +598,14 @@ def run_ours(args):
         e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], world, dev)
         e2e["value"] = job_gparams_per_s(world, out, n, e2e["ms_per_step"])
 
-    measured = measure_peaks(G, torch, dev)
+    measured = measure_peaks(G, torch, dev) if not args.no_peaks else {}
     kernels = kernel_rooflines(trace, peaks, measured, prepare_ms=statistics.mean(prep_ms), n=n)
     kernels["note"] = (f"device time of each kernel on the stream it runs on, from the library's timing trace over a "
                        f"second pass of the same {args.steps} steps (the K4 and prepare products run on library "
                        "streams beside other kernels, so their times include sharing the SMs)")
 
-    decode = time_qmatvec(G, torch, dev, peaks, flush) if world == 1 else None
+    decode = time_qmatvec(G, torch, dev, peaks, flush) if world == 1 and not args.no_decode else None
+    pipeline = time_pipeline(G, torch, dev) if world == 1 and not args.no_pipeline else None
 
     blocks = None
     if world == 1 and not args.no_blocks:
@@ -616,6 +644,7 @@ def run_ours(args):
         "peaks_measured_here": measured,
         "blocks": blocks,
         "decode_qmatvec": decode,
+        "pipeline": pipeline,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches,
@@ -828,6 +857,9 @@ def main():
                     help="time every layer of a decoder block instead (its own JSON line)")
     ap.add_argument("--no-blocks", action="store_true",
                     help="leave the two decoder blocks out of the default line")
+    ap.add_argument("--no-decode", action="store_true", help="leave the decode-shape qmatvec leg out")
+    ap.add_argument("--no-pipeline", action="store_true", help="leave the sequential-pipeline leg out")
+    ap.add_argument("--no-peaks", action="store_true", help="do not measure the tf32 / fp32 peaks here")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -357,6 +357,33 @@ GPTQ_API int gptq_reorder_groups(const int32_t* qweight, const int32_t* g_idx, i
                                  int32_t* d_status, void* stream);
 
 /*
+ * A quantized block's forward pass, for the sequential pipeline: the pages quantize
+ * layer by layer ("polydesk.ai/glossaire/gptq"; "wikiprompt.org", "GPTQ"), each
+ * layer calibrated on the activations the layers quantized before it produce.
+ * Activations keep the layout of gptq_hessian_accumulate's X: [features, tokens] bf16,
+ * tokens contiguous.
+ *
+ * gptq_linear_bf16 - C[M, N] = A[M, K] . B[N, K]^T on the tensor cores (bf16 in, fp32
+ *   accumulate in chunks of 256 added in fp32 registers, fp32 out).  A and B row-major,
+ *   K contiguous (lda, ldb >= K, multiples of 8, 16-byte aligned); C fp32, row stride
+ *   ldc >= N.  With A = the dequantized weights [out, in] and B = the activations
+ *   transposed [tokens, in], C is the layer's output [out, tokens].
+ * gptq_transpose_bf16 - Xt[c][r] = X[r][c] for X [rows, cols] (row strides ldx, ldt).
+ * gptq_silu_mul - h = bf16(silu(G) . U) elementwise over count fp32 values (G, U
+ *   16-byte aligned, h 8-byte aligned), silu(g) = g / (1 + exp(-g)): the gated MLP.
+ * gptq_residual_add - Xn = bf16(X + Y) elementwise, X bf16, Y fp32.
+ * d_status may be NULL; a bounded wait of the product that gives up reports
+ * GPTQ_ERR_TIMEOUT there.
+ */
+GPTQ_API int gptq_linear_bf16(const void* A, int M, int64_t lda, const void* B, int N, int64_t ldb, int K, float* C,
+                              int64_t ldc, int32_t* d_status, void* stream);
+GPTQ_API int gptq_transpose_bf16(const void* X, int rows, int cols, int64_t ldx, void* Xt, int64_t ldt,
+                                 int32_t* d_status, void* stream);
+GPTQ_API int gptq_silu_mul(const float* G, const float* U, int64_t count, void* h, int32_t* d_status, void* stream);
+GPTQ_API int gptq_residual_add(const void* X, const float* Y, int64_t count, void* Xn, int32_t* d_status,
+                               void* stream);
+
+/*
  * Kernel timing trace.  The GPTQ pages have no counterpart to these calls: they
  * are a measurement aid.  While the trace is on, every kernel the library launches
  * is bracketed by two CUDA events recorded on the stream it is launched on (the

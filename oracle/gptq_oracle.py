@@ -47,6 +47,7 @@ __all__ = [
     "group_params", "quantize_codes", "dequant_value", "sweep", "SweepResult",
     "g_idx", "unpermute_codes", "pack", "unpack", "dequantize", "layer_error",
     "rtn", "quantize_layer", "LayerResult", "gptq_layer", "pad_layer", "pack_zeros", "unpack_zeros",
+    "silu", "mlp_hidden", "mlp_residual",
 ]
 
 F16_MIN_SUBNORMAL = np.float32(2.0 ** -24)
@@ -608,3 +609,27 @@ def unpack_zeros(qzeros: np.ndarray, bits: int, out: int, zero_offset: int = 0) 
             v |= q[:, wi + 1] << np.uint64(32 - off)
         z[:, o] = ((v & mask).astype(np.int64) + zero_offset) % (2 ** bits)
     return z
+
+
+# --------------------------------------------------------------------------- #
+# The forward pass of a quantized MLP block (the sequential pipeline)
+# --------------------------------------------------------------------------- #
+# Reading: the pages quantize layer by layer, each layer calibrated on the outputs of
+# the layers quantized before it (polydesk, GPTQ works layer by layer); the blocks are
+# Llama-shaped (the workloads'), whose MLP is down(silu(gate x) . up x) with a
+# residual connection around it.  In fp64 from the dequantized weights.
+def silu(g: np.ndarray) -> np.ndarray:
+    """silu(g) = g / (1 + exp(-g))."""
+    g = np.asarray(g, np.float64)
+    return g / (1.0 + np.exp(-g))
+
+
+def mlp_hidden(x_bits: np.ndarray, What_gate: np.ndarray, What_up: np.ndarray) -> np.ndarray:
+    """h = silu(What_gate . X) * (What_up . X), X [d, tokens] as bf16 bits, h [d_ff, tokens]."""
+    x = bf16_bits_to_f64(x_bits)
+    return silu(np.asarray(What_gate, np.float64) @ x) * (np.asarray(What_up, np.float64) @ x)
+
+
+def mlp_residual(x_bits: np.ndarray, What_down: np.ndarray, h: np.ndarray) -> np.ndarray:
+    """The block's output X + What_down . h (fp64)."""
+    return bf16_bits_to_f64(x_bits) + np.asarray(What_down, np.float64) @ np.asarray(h, np.float64)

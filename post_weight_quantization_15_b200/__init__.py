@@ -1,6 +1,7 @@
 """B200-native GPTQ layer solver: a C-ABI CUDA library (libgptq.so) and its binding."""
 from .gptq import (  # noqa: F401
-    GptqError, Prepared, QuantizedLayer, alloc_quantized, dequantize, qmatvec, gptq_quantize, hessian_accumulate, hessian_accumulate_host, kernel_launches, lib, library_path,
+    GptqError, Prepared, QuantizedLayer, alloc_quantized, dequantize, linear_bf16, qmatvec, residual_add, silu_mul,
+    transpose_bf16, gptq_quantize, hessian_accumulate, hessian_accumulate_host, kernel_launches, lib, library_path,
     new_status, pack, pack_zeros, padded_width, prepare, quantize_layer, quantize_layer_noalloc, quantize_layers, reorder_groups, quantize_workspace_size, raise_on_status, status_read, status_reset,
     status_string, trace_enable, trace_read, workspace,
 )

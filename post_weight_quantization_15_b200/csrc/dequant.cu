@@ -108,13 +108,15 @@ __global__ void __launch_bounds__(256) qmatvec_kernel(const int32_t* qweight, co
   __shared__ float xs[M * kc];
   __shared__ int gsm[kc];
   __shared__ float red[8 * 128];
-  __shared__ float2 szs[QMV_MAXG * 128];      // (scale, zero) of staged group g_lo + i for output o0 + j
-  __shared__ int grange[2];
+  // scales, then zero points, of staged group g_lo + gi for the four outputs of lane l:
+  // szs[gi][l] = (s0, s1, s2, s3), szs[gi][32 + l] = (z0, z1, z2, z3)
+  __shared__ float4 szs[QMV_MAXG * 64];
+  __shared__ int grange[3];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int o0 = blockIdx.x * 128;
   const int k0 = blockIdx.y * kc;
   const int k1 = min(n, k0 + kc);
-  if (threadIdx.x == 0) { grange[0] = INT_MAX; grange[1] = -1; }
+  if (threadIdx.x == 0) { grange[0] = INT_MAX; grange[1] = -1; grange[2] = 0; }
   __syncthreads();
   int gmin = INT_MAX, gmax = -1;
   for (int i = threadIdx.x; i < kc; i += blockDim.x) {
@@ -126,6 +128,13 @@ __global__ void __launch_bounds__(256) qmatvec_kernel(const int32_t* qweight, co
     if (k0 + i < k1) { gmin = min(gmin, g); gmax = max(gmax, g); }
     gsm[i] = g < 0 ? 0 : g;
   }
+  __syncthreads();
+  // does every packed word of the range hold columns of one group?  (k0 is a multiple of
+  // PER, so the words start at multiples of PER within the range)
+  int split_word = 0;
+  for (int i = threadIdx.x; i < k1 - k0; i += blockDim.x)
+    if (gsm[i] != gsm[i - i % PER]) split_word = 1;
+  if (__any_sync(0xffffffffu, split_word) && lane == 0) atomicOr(&grange[2], 1);
   for (int o = 16; o > 0; o >>= 1) {
     gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, o));
     gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
@@ -139,14 +148,16 @@ __global__ void __launch_bounds__(256) qmatvec_kernel(const int32_t* qweight, co
   __syncthreads();
   const int g_lo = grange[0];
   const bool staged = grange[1] - g_lo < QMV_MAXG;
+  const bool uniform = grange[2] == 0;
   if (staged) {
+    float* szf = reinterpret_cast<float*>(szs);
     for (int i = threadIdx.x; i < (grange[1] - g_lo + 1) * 128; i += blockDim.x) {
-      const int gi = i / 128, oo = o0 + i % 128;
-      float2 v = make_float2(0.f, 0.f);
-      if (oo < out)
-        v = make_float2(__half2float(__ushort_as_half(scales[(int64_t)(g_lo + gi) * out + oo])),
-                        __half2float(__ushort_as_half(zeros[(int64_t)(g_lo + gi) * out + oo])));
-      szs[i] = v;
+      const int gi = i / 128, oi = i % 128, oo = o0 + oi;
+      const bool in = oo < out;
+      szf[(gi * 64 + oi / 4) * 4 + oi % 4] =
+          in ? __half2float(__ushort_as_half(scales[(int64_t)(g_lo + gi) * out + oo])) : 0.f;
+      szf[(gi * 64 + 32 + oi / 4) * 4 + oi % 4] =
+          in ? __half2float(__ushort_as_half(zeros[(int64_t)(g_lo + gi) * out + oo])) : 0.f;
     }
     __syncthreads();
   }
@@ -181,17 +192,41 @@ __global__ void __launch_bounds__(256) qmatvec_kernel(const int32_t* qweight, co
     for (int u = 0; u < QMV_UNROLL; ++u) {
       const int w = wb + 8 * u;
       if (w >= w1) break;
+      if (staged && uniform) {
+        // the word's columns share one group: its scales and zero points once, the
+        // activations of its PER columns as 16-byte loads
+        const int kl0 = w * PER - k0;
+        const int gi = gsm[kl0] - g_lo;
+        const float4 sv = szs[gi * 64 + lane], zv = szs[gi * 64 + 32 + lane];
+        const float s4[4] = {sv.x, sv.y, sv.z, sv.w}, z4[4] = {zv.x, zv.y, zv.z, zv.w};
+#pragma unroll
+        for (int i0 = 0; i0 < PER; i0 += 4) {
+          float wv[4][4];
+#pragma unroll
+          for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              wv[ii][j] = s4[j] * ((float)((q[u][j] >> ((i0 + ii) * BITS)) & ((1u << BITS) - 1u)) - z4[j]);
+#pragma unroll
+          for (int m = 0; m < M; ++m) {
+            const float4 x4 = *reinterpret_cast<const float4*>(xs + m * kc + kl0 + i0);
+            const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+              for (int j = 0; j < 4; ++j) acc[m][j] = fmaf(xv[ii], wv[ii][j], acc[m][j]);
+          }
+        }
+        continue;
+      }
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
         const int kl = w * PER + i - k0;
         const int g = gsm[kl];
         if (staged) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 v = szs[(g - g_lo) * 128 + 4 * lane + j];
-            s[j] = v.x;
-            z[j] = v.y;
-          }
+          const float4 sv = szs[(g - g_lo) * 64 + lane], zv = szs[(g - g_lo) * 64 + 32 + lane];
+          s[0] = sv.x; s[1] = sv.y; s[2] = sv.z; s[3] = sv.w;
+          z[0] = zv.x; z[1] = zv.y; z[2] = zv.z; z[3] = zv.w;
         } else if (g != g_prev) {      // a new group: its scales and zero points for the four outputs
           g_prev = g;
 #pragma unroll

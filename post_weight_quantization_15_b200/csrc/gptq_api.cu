@@ -245,6 +245,36 @@ int gptq_reorder_groups(const int32_t* qweight, const int32_t* g_idx, int bits, 
                                as_stream(stream));
 }
 
+int gptq_linear_bf16(const void* A, int M, int64_t lda, const void* B, int N, int64_t ldb, int K, float* C,
+                     int64_t ldc, int32_t* d_status, void* stream) {
+  if (A == nullptr || B == nullptr || C == nullptr || M <= 0 || N <= 0 || K <= 0) return GPTQ_ERR_INVALID_ARG;
+  if (lda < K || ldb < K || ldc < N || lda % 8 != 0 || ldb % 8 != 0 || !aligned(A, 16) || !aligned(B, 16))
+    return GPTQ_ERR_INVALID_ARG;
+  if (cdiv(M, 128) * cdiv(N, 256) > INT32_MAX) return GPTQ_ERR_UNSUPPORTED;
+  return launch_linear(A, M, lda, B, N, ldb, K, C, ldc, d_status, as_stream(stream));
+}
+
+int gptq_transpose_bf16(const void* X, int rows, int cols, int64_t ldx, void* Xt, int64_t ldt, int32_t* d_status,
+                        void* stream) {
+  if (X == nullptr || Xt == nullptr || rows <= 0 || cols <= 0 || ldx < cols || ldt < rows) return GPTQ_ERR_INVALID_ARG;
+  if (cdiv(rows, 64) > 65535) return GPTQ_ERR_UNSUPPORTED;
+  return launch_transpose_bf16(X, rows, cols, ldx, Xt, ldt, d_status, as_stream(stream));
+}
+
+int gptq_silu_mul(const float* G, const float* U, int64_t count, void* h, int32_t* d_status, void* stream) {
+  if (G == nullptr || U == nullptr || h == nullptr || count < 0) return GPTQ_ERR_INVALID_ARG;
+  if (!aligned(G, 16) || !aligned(U, 16) || !aligned(h, 8)) return GPTQ_ERR_INVALID_ARG;
+  if (count == 0) return GPTQ_OK;
+  return launch_silu_mul(G, U, count, h, d_status, as_stream(stream));
+}
+
+int gptq_residual_add(const void* X, const float* Y, int64_t count, void* Xn, int32_t* d_status, void* stream) {
+  if (X == nullptr || Y == nullptr || Xn == nullptr || count < 0) return GPTQ_ERR_INVALID_ARG;
+  if (!aligned(X, 8) || !aligned(Y, 16) || !aligned(Xn, 8)) return GPTQ_ERR_INVALID_ARG;
+  if (count == 0) return GPTQ_OK;
+  return launch_residual_add(X, Y, count, Xn, d_status, as_stream(stream));
+}
+
 int gptq_pack(const uint8_t* codes, int out, int n, int bits, int32_t* qweight, void* stream) {
   if (codes == nullptr || qweight == nullptr || out <= 0 || n <= 0) return GPTQ_ERR_INVALID_ARG;
   if (!valid_bits(bits)) return GPTQ_ERR_UNSUPPORTED;

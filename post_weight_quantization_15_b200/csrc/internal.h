@@ -76,6 +76,14 @@ int launch_reorder_groups(const int32_t* qweight, const int32_t* g_idx, int bits
                           int32_t* qweight_g, int32_t* g_sorted, int32_t* xperm, void* ws, int32_t* st,
                           cudaStream_t s);
 
+// ---- a quantized block's forward pass (linear.cu, forward.cu) -----------------------
+int launch_linear(const void* A, int M, int64_t lda, const void* B, int N, int64_t ldb, int K, float* C, int64_t ldc,
+                  int32_t* st, cudaStream_t s);
+int launch_transpose_bf16(const void* X, int rows, int cols, int64_t ldx, void* Xt, int64_t ldt, const int32_t* st,
+                          cudaStream_t s);
+int launch_silu_mul(const float* G, const float* U, int64_t count, void* h, const int32_t* st, cudaStream_t s);
+int launch_residual_add(const void* X, const float* Y, int64_t count, void* Xn, const int32_t* st, cudaStream_t s);
+
 // ---- tensor-core GEMM: C -= A . B^T in 3 x TF32 (operands pre-split) ---------
 // store = false: C -= A.B^T; store = true: C = A.B^T (C may be null then, if Chi/Clo are given).
 // Chi/Clo (optional, leading dimension ldh) receive the TF32 split of the result.

@@ -122,6 +122,14 @@ def lib() -> ctypes.CDLL:
     L.gptq_reorder_groups_workspace_size.argtypes = [I]
     L.gptq_reorder_groups.restype = I
     L.gptq_reorder_groups.argtypes = [P, P, I, I, I, I, P, P, P, P, SZ, P, P]
+    L.gptq_linear_bf16.restype = I
+    L.gptq_linear_bf16.argtypes = [P, I, I64, P, I, I64, I, P, I64, P, P]
+    L.gptq_transpose_bf16.restype = I
+    L.gptq_transpose_bf16.argtypes = [P, I, I, I64, P, I64, P, P]
+    L.gptq_silu_mul.restype = I
+    L.gptq_silu_mul.argtypes = [P, P, I64, P, P, P]
+    L.gptq_residual_add.restype = I
+    L.gptq_residual_add.argtypes = [P, P, I64, P, P, P]
     L.gptq_probe_fp32_peak.restype = I
     L.gptq_probe_fp32_peak.argtypes = [P, I, I, P]
     L.gptq_quantize_layer_noalloc.restype = I
@@ -526,6 +534,64 @@ def qmatvec(q: QuantizedLayer, X: torch.Tensor, status: Optional[torch.Tensor] =
                               groups, _ptr(X), _DTYPE_CODE[X.dtype], M, X.stride(0), _ptr(out), out.stride(0),
                               _ptr(ws), ws.numel(), _ptr(status), _stream(stream)), "gptq_qmatvec")
     return out
+
+
+# --------------------------------------------------------------------------- #
+# A quantized block's forward pass (the sequential pipeline)
+# --------------------------------------------------------------------------- #
+def linear_bf16(A: torch.Tensor, B: torch.Tensor, status: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """C [M, N] fp32 = A [M, K] . B [N, K]^T, bf16 operands with contiguous rows."""
+    _require_cuda(A, B, status, out)
+    for t in (A, B):
+        if t.dtype != torch.bfloat16 or t.dim() != 2 or t.stride(1) != 1:
+            raise ValueError("A and B must be bf16 2-D tensors with contiguous rows")
+    M, K = A.shape
+    N = B.shape[0]
+    if B.shape[1] != K:
+        raise ValueError("A and B must share K")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=A.device)
+    if out.dtype != torch.float32 or tuple(out.shape) != (M, N) or out.stride(1) != 1:
+        raise ValueError("out must be fp32 [M, N] with contiguous rows")
+    _check(lib().gptq_linear_bf16(_ptr(A), M, A.stride(0), _ptr(B), N, B.stride(0), K, _ptr(out), out.stride(0),
+                                  _ptr(status), _stream(stream)), "gptq_linear_bf16")
+    return out
+
+
+def transpose_bf16(X: torch.Tensor, status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    _require_cuda(X, status)
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.stride(1) != 1:
+        raise ValueError("X must be a bf16 2-D tensor with contiguous rows")
+    r, c = X.shape
+    Xt = torch.empty((c, r), dtype=torch.bfloat16, device=X.device)
+    _check(lib().gptq_transpose_bf16(_ptr(X), r, c, X.stride(0), _ptr(Xt), r, _ptr(status), _stream(stream)),
+           "gptq_transpose_bf16")
+    return Xt
+
+
+def silu_mul(G: torch.Tensor, U: torch.Tensor, status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """bf16(silu(G) . U) for contiguous fp32 G, U of one shape."""
+    _require_cuda(G, U, status)
+    if G.dtype != torch.float32 or U.dtype != torch.float32 or G.shape != U.shape or not G.is_contiguous() \
+            or not U.is_contiguous():
+        raise ValueError("G and U must be contiguous fp32 tensors of one shape")
+    h = torch.empty(G.shape, dtype=torch.bfloat16, device=G.device)
+    _check(lib().gptq_silu_mul(_ptr(G), _ptr(U), G.numel(), _ptr(h), _ptr(status), _stream(stream)), "gptq_silu_mul")
+    return h
+
+
+def residual_add(X: torch.Tensor, Y: torch.Tensor, status: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """bf16(X + Y) for contiguous X bf16 and Y fp32 of one shape."""
+    _require_cuda(X, Y, status)
+    if X.dtype != torch.bfloat16 or Y.dtype != torch.float32 or X.shape != Y.shape or not X.is_contiguous() \
+            or not Y.is_contiguous():
+        raise ValueError("X (bf16) and Y (fp32) must be contiguous tensors of one shape")
+    Xn = torch.empty(X.shape, dtype=torch.bfloat16, device=X.device)
+    _check(lib().gptq_residual_add(_ptr(X), _ptr(Y), X.numel(), _ptr(Xn), _ptr(status), _stream(stream)),
+           "gptq_residual_add")
+    return Xn
 
 
 def pack(codes: torch.Tensor, bits: int, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

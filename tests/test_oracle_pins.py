@@ -555,3 +555,30 @@ def test_rows_are_independent_given_u(monkeypatch):
     _, codes_all = O.quantize_layer(W, prep, 4, 128, False, 128)
     _, codes_sub = O.quantize_layer(W[rows], prep, 4, 128, False, 128)
     assert not np.array_equal(codes_all[rows], codes_sub)
+
+
+def test_mlp_forward_closed_forms_and_brute_force():
+    # silu: 0 at 0, g . sigmoid(g), odd part g/2, tends to g and to 0
+    assert O.silu(np.array([0.0]))[0] == 0.0
+    assert O.silu(np.array([1.0]))[0] == pytest.approx(1.0 / (1.0 + np.exp(-1.0)), rel=1e-15)
+    g = np.array([-3.0, -0.5, 0.25, 2.0])
+    assert np.allclose(O.silu(g) - O.silu(-g), g, rtol=1e-14)
+    assert O.silu(np.array([40.0]))[0] == pytest.approx(40.0, rel=1e-15) and abs(O.silu(np.array([-40.0]))[0]) < 1e-15
+    # the hidden activations and the residual output, against loops over a tiny block
+    rng = np.random.default_rng(4)
+    x = S.f32_to_bf16_bits(rng.standard_normal((3, 5)).astype(np.float32))
+    xf = S.bf16_bits_to_f32(x).astype(float)
+    Wg, Wu, Wd = rng.standard_normal((4, 3)), rng.standard_normal((4, 3)), rng.standard_normal((3, 4))
+    h = O.mlp_hidden(x, Wg, Wu)
+    out = O.mlp_residual(x, Wd, h)
+    for i in range(4):
+        for t in range(5):
+            gv = sum(Wg[i, k] * xf[k, t] for k in range(3))
+            uv = sum(Wu[i, k] * xf[k, t] for k in range(3))
+            assert h[i, t] == pytest.approx(gv / (1 + np.exp(-gv)) * uv, rel=1e-12, abs=1e-14)
+    for r in range(3):
+        for t in range(5):
+            assert out[r, t] == pytest.approx(xf[r, t] + sum(Wd[r, i] * h[i, t] for i in range(4)), rel=1e-12,
+                                              abs=1e-14)
+    # a planted mistake (the gate and up roles swapped) changes the result
+    assert not np.allclose(O.mlp_hidden(x, Wu, Wg), h)
