@@ -199,8 +199,10 @@ __device__ __forceinline__ uint32_t map_to_cta(uint32_t local, uint32_t rank) {
   return r;
 }
 
+// Arrival on a barrier of another CTA of the cluster (default semantics: the ordering
+// the accumulator hand-off needs comes from tcgen05.wait::ld and the tcgen05 fences).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // 2-D TMA load into this CTA's shared memory completing on the LEADER's barrier at the

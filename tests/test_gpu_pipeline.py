@@ -30,7 +30,7 @@ def _dev():
 
 
 def _linear_bound(K, absprod):
-    """The product's summation, as the Hessian kernel's (tests/parity.py, hessian_bound):
+    """The product's summation (linear_kernel, the structure of tests/parity.py's hessian_bound):
     16-deep tensor-core steps in chunks of 256 from zero (272 ulps of the chunk's sum of
     |terms|), chunks added in fp32 with round to nearest, one store: relative to
     sum_k |a_k b_k|."""
@@ -40,6 +40,13 @@ def _linear_bound(K, absprod):
 
 def _bits(t):
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _as_bf16(What):
+    """The dequantized weights as the forward uses them: in bf16, the activations' type (one
+    tensor-core product takes one operand type).  What is exact in fp32 (an fp16 scale times
+    a small integer), so this is one round to nearest even of the exact value."""
+    return O.bf16_bits_to_f64(S.f32_to_bf16_bits(np.asarray(What, np.float64).astype(np.float32)))
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 520, 1000), (1100, 300, 4104)])
@@ -107,7 +114,7 @@ def test_two_block_pipeline_stage_by_stage():
         # h from the stored gate and up
         What = O.dequantize(q.qweight.cpu().numpy(), q.scales.cpu().numpy(), q.zeros.cpu().numpy(),
                             q.g_idx.cpu().numpy(), 4, d)
-        Wg_hat, Wu_hat = What[:d_ff], What[d_ff:]
+        Wg_hat, Wu_hat = _as_bf16(What[:d_ff]), _as_bf16(What[d_ff:])
         x64 = O.bf16_bits_to_f64(xb)
         g64, u64 = Wg_hat @ x64, Wu_hat @ x64
         h_ref = O.mlp_hidden(xb, Wg_hat, Wu_hat)
@@ -129,8 +136,8 @@ def test_two_block_pipeline_stage_by_stage():
         print(f"block {b} down:", cd)
         assert cd.ok(), cd
         # the block's output from the stored down
-        Wd_hat = O.dequantize(qd.qweight.cpu().numpy(), qd.scales.cpu().numpy(), qd.zeros.cpu().numpy(),
-                              qd.g_idx.cpu().numpy(), 4, d_ff)
+        Wd_hat = _as_bf16(O.dequantize(qd.qweight.cpu().numpy(), qd.scales.cpu().numpy(), qd.zeros.cpu().numpy(),
+                                       qd.g_idx.cpu().numpy(), 4, d_ff))
         x_ref = O.mlp_residual(xb, Wd_hat, h_gpu)
         tol = _linear_bound(d_ff, np.abs(Wd_hat) @ np.abs(h_gpu)) + 2.0 ** -8 * np.abs(x_ref)
         x_gpu = O.bf16_bits_to_f64(_bits(xs[b + 1]))
