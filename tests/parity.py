@@ -22,11 +22,11 @@ SCALE_TOL = 1e-3
 
 # The Hessian kernel's summation, which the Hessian bound below follows: every
 # 16-token tensor-core instruction adds 16 exact bf16 products to its fp32
-# accumulator; an accumulator starts from zero every 512 tokens (a chunk); the
+# accumulator; an accumulator starts from zero every 1024 tokens (a chunk); the
 # finished chunks are added into fp32 registers with round-to-nearest; at the end
 # of a call H_ij += 2 . sum (one more rounding).
 HESS_MMA_K = 16
-HESS_CHUNK = 512
+HESS_CHUNK = 1024
 
 
 def hessian_bound(token_counts) -> float:
@@ -37,12 +37,12 @@ def hessian_bound(token_counts) -> float:
     * inside a chunk, each instruction sums 17 terms (16 products and the accumulator),
       each at most sum-so-far <= S_chunk in magnitude; whether the tensor core rounds or
       truncates after aligning them, each term loses at most one ulp: <= 17 u S_chunk per
-      instruction, 32 instructions per 512-token chunk: 544 u S_chunk;
+      instruction, 64 instructions per 1024-token chunk: 1088 u S_chunk;
     * each addition of a chunk into the fp32 register sum rounds to nearest: <= u/2 S
       each, one per chunk, plus the final H += 2 . sum, one per call;
     * 2 S <= sqrt(H_ii H_jj) (Cauchy-Schwarz), the factor 2 being exact.
-    So c = 17 . 32 . u + (chunks + calls) . u/2.  At 65,536 tokens in one call,
-    c = 7.3e-5: a kernel that dropped one 512-token chunk (0.8 % of the sum) fails.
+    So c = 17 . 64 . u + (chunks + calls) . u/2.  At 65,536 tokens in one call,
+    c = 1.3e-4: a kernel that dropped one 1024-token chunk (1.6 % of the sum) fails.
     """
     counts = [int(t) for t in token_counts if int(t) > 0]
     chunks = sum((t + HESS_CHUNK - 1) // HESS_CHUNK for t in counts)

@@ -264,4 +264,4 @@ def test_llama70b_down_28672_input():
     """down [8192 x 28672]: H and U are 28,672 x 28,672; 65,536 tokens."""
     (down,), (st,) = _layers("llama2-70b-block", ["down"])
     x = S.make_x(down.x)
-    _input_check(x, st.damp_percent, st.desc_act, [Job(S.make_w(down.w), st, 8)], seed=71)
+    _input_check(x, st.damp_percent, st.desc_act, [Job(S.make_w(down.w), st, 16)], seed=71)
