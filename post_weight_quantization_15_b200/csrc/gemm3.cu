@@ -21,6 +21,8 @@
 // All operands are row-major with K contiguous (K-major).  `lower` skips tiles
 // that lie entirely above the diagonal of a square C.
 // Every wait is bounded (GPTQ_ERR_TIMEOUT).
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
@@ -313,6 +315,242 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
   }
 }
 
+// ---------------------------------------------------------------------------
+// The persistent form for products at least 256 columns wide: one CTA per SM walks
+// its share of the 128 x 256 output tiles (t = blockIdx.x, blockIdx.x + gridDim.x,
+// ...).  The stage ring, the chunk counter and the two TMEM accumulators run on
+// across tiles, so the producer loads the next tile's operands and the MMAs start
+// it while the epilogue warps still update C with the previous one.
+//   warp 0      TMA producer: 32-wide K slices of A hi / lo (128 rows) and B hi / lo
+//               (256 rows), 2-stage ring of 96 KB stages;
+//   warp 1      allocates 512 TMEM columns (two 128 x 256 accumulators); one thread
+//               issues tcgen05.mma kind::tf32 (M = 128, N = 256, K = 8), three per
+//               K step (lo.hi + hi.lo + hi.hi);
+//   warps 2..9  epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 32 (its rows) and
+//               columns 128 ((w - 2) / 4) .. + 128, adds each 128-deep chunk into fp32
+//               registers, releases the accumulator, and at a tile's last chunk
+//               updates its rows of C (C -= acc or C = acc; optionally the split of
+//               the result) straight from registers, 16 bytes at a time.
+// K is accumulated in chunks of 128 (as in gemm3_kernel), each from zero.  Every
+// wait is bounded (GPTQ_ERR_TIMEOUT).
+// ---------------------------------------------------------------------------
+constexpr int PN = 256;
+constexpr int PST = 2;
+constexpr int P_BTILE = PN * GK * 4;             // 32 KB
+constexpr int P_EPI = 8;
+constexpr int P_THREADS = 64 + P_EPI * 32;
+constexpr uint32_t P_IDESC = tc::idesc_f32acc(2, GM, PN);
+
+struct GemmPSmem {
+  uint8_t bhi[PST][P_BTILE];
+  uint8_t blo[PST][P_BTILE];
+  uint8_t ahi[PST][A_TILE];
+  uint8_t alo[PST][A_TILE];
+  uint64_t full[PST];
+  uint64_t empty[PST];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int skip;
+};
+constexpr size_t GEMMP_SMEM = sizeof(GemmPSmem) + 1024;
+
+// Tile t of the walk -> (ti, tj).  lower: only tiles that reach the lower triangle of
+// square C, tj . 256 <= ti . 128 + 127, i.e. tj <= ti / 2, row by row.
+__device__ __forceinline__ void gemmp_tile(int t, int tiles_n, bool lower, int& ti, int& tj) {
+  if (!lower) { ti = t / tiles_n; tj = t % tiles_n; return; }
+  ti = 0;
+  for (;;) {
+    const int cnt = min(ti / 2 + 1, tiles_n);
+    if (t < cnt) break;
+    t -= cnt;
+    ++ti;
+  }
+  tj = t;
+}
+
+__global__ void __launch_bounds__(P_THREADS, 1)
+gemm3p_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, int K, int lower, int tiles,
+              int tiles_n, int32_t* st) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // offset arithmetic on the shared array keeps every access a shared-memory one
+  GemmPSmem& S = *reinterpret_cast<GemmPSmem*>(smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kblocks = (int)cdiv(K, GK);
+  const int nchunks = (int)cdiv(kblocks, CHUNK_KB);        // chunks per tile
+
+  if (threadIdx.x == 0) {
+    S.skip = has_error(st) ? 1 : 0;
+    S.abort = 0;
+    for (int s2 = 0; s2 < PST; ++s2) { tc::mbar_init(&S.full[s2], 1); tc::mbar_init(&S.empty[s2], 1); }
+    for (int b = 0; b < 2; ++b) { tc::mbar_init(&S.acc_full[b], 1); tc::mbar_init(&S.acc_empty[b], P_EPI); }
+    tc::mbar_init(&S.drain, 1);
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) tc::tmem_alloc<512>(&S.tmem_base);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t taddr = S.tmem_base;
+  const bool skip = S.skip != 0;
+  volatile int* abort_flag = &S.abort;
+  int armed[PST] = {};
+  bool mma_committed = false;
+
+  if (!skip) {
+    if (warp == 0 && lane == 0) {
+      // ---------------- producer ----------------
+      int q = 0;                                           // stage counter over all tiles
+      for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+        int ti, tj;
+        gemmp_tile(t, tiles_n, lower != 0, ti, tj);
+        for (int kb = 0; kb < kblocks; ++kb, ++q) {
+          const int s2 = q % PST;
+          const uint32_t ph = (uint32_t)(q / PST) & 1u;
+          if (!tc::mbar_wait(&S.empty[s2], ph ^ 1u, abort_flag)) break;
+          tc::mbar_arrive_expect_tx(&S.full[s2], 2 * (A_TILE + P_BTILE));
+          tc::tma_load_2d(S.ahi[s2], &maps.ahi, &S.full[s2], kb * GK, ti * GM);
+          tc::tma_load_2d(S.alo[s2], &maps.alo, &S.full[s2], kb * GK, ti * GM);
+          tc::tma_load_2d(S.bhi[s2], &maps.bhi, &S.full[s2], kb * GK, tj * PN);
+          tc::tma_load_2d(S.blo[s2], &maps.blo, &S.full[s2], kb * GK, tj * PN);
+          ++armed[s2];
+        }
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ---------------- MMA issuer ----------------
+      int q = 0, g = 0;                                    // stage and chunk counters over all tiles
+      for (int t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+        int kb = 0;
+        for (int c = 0; c < nchunks && !*abort_flag; ++c, ++g) {
+          const int buf = g & 1;
+          if (!tc::mbar_wait(&S.acc_empty[buf], ((uint32_t)(g >> 1) & 1u) ^ 1u, abort_flag)) break;
+          tc::tc_fence_after();
+          const uint32_t dacc = taddr + buf * PN;
+          const int kb_end = min(kblocks, (c + 1) * CHUNK_KB);
+          bool first = true;
+          for (; kb < kb_end; ++kb, ++q) {
+            const int s2 = q % PST;
+            const uint32_t ph = (uint32_t)(q / PST) & 1u;
+            if (!tc::mbar_wait(&S.full[s2], ph, abort_flag)) break;
+            tc::tc_fence_after();
+            const uint32_t ah = tc::smem_u32(S.ahi[s2]), al = tc::smem_u32(S.alo[s2]);
+            const uint32_t bh = tc::smem_u32(S.bhi[s2]), bl = tc::smem_u32(S.blo[s2]);
+#pragma unroll
+            for (int kk = 0; kk < GK / 8; ++kk) {
+              const uint32_t o = kk * 32;
+              tc::mma_tf32(dacc, tc::sdesc_k_sw128(al + o), tc::sdesc_k_sw128(bh + o), P_IDESC, !first);
+              tc::mma_tf32(dacc, tc::sdesc_k_sw128(ah + o), tc::sdesc_k_sw128(bl + o), P_IDESC, true);
+              tc::mma_tf32(dacc, tc::sdesc_k_sw128(ah + o), tc::sdesc_k_sw128(bh + o), P_IDESC, true);
+              first = false;
+            }
+            tc::mma_commit(&S.empty[s2]);
+          }
+          if (*abort_flag) break;
+          tc::mma_commit(&S.acc_full[buf]);
+        }
+      }
+      tc::mma_commit(&S.drain);
+      mma_committed = true;
+      if (!*abort_flag) drain_wait(&S.drain, 0);
+    } else if (warp >= 2) {
+      // ---------------- epilogue ----------------
+      const int qq = warp & 3;                   // TMEM lane quarter this warp may access
+      const int hc = (warp - 2) >> 2;            // which 128 of the 256 columns
+      const uint32_t lane_base = (uint32_t)(qq * 32) << 16;
+      const bool vec = out.C == nullptr || ((out.ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(out.C) & 15) == 0);
+      const bool vech = out.Chi == nullptr || (out.ldh & 3) == 0;
+      int g = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        int ti, tj;
+        gemmp_tile(t, tiles_n, lower != 0, ti, tj);
+        float acc[128];
+#pragma unroll
+        for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+        for (int c = 0; c < nchunks; ++c, ++g) {
+          const int buf = g & 1;
+          int ready = 0;
+          if (lane == 0) ready = tc::mbar_wait(&S.acc_full[buf], (uint32_t)(g >> 1) & 1u, abort_flag) && !*abort_flag;
+          ready = __shfl_sync(0xffffffffu, ready, 0);
+          if (!ready) { ok = false; break; }
+          tc::tc_fence_after();
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            float v[32];
+            tc::tmem_ld_32x32b_x32(taddr + lane_base + buf * PN + hc * 128 + c4 * 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[c4 * 32 + i] += v[i];
+          }
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&S.acc_empty[buf]);   // the MMAs may reuse it now
+        }
+        if (!ok) break;
+        const int r = ti * GM + qq * 32 + lane;
+        const int col0 = tj * PN + hc * 128;
+        if (r >= M || col0 >= N) continue;
+        const bool whole = col0 + 128 <= N;
+        float* crow = out.C ? out.C + (int64_t)r * out.ldc + col0 : nullptr;
+#pragma unroll
+        for (int i = 0; i < 128; i += 4) {
+          float x[4];
+          if (whole && vec) {
+            if (out.store) {
+              x[0] = acc[i]; x[1] = acc[i + 1]; x[2] = acc[i + 2]; x[3] = acc[i + 3];
+            } else {
+              const float4 o = *reinterpret_cast<const float4*>(crow + i);
+              x[0] = o.x - acc[i]; x[1] = o.y - acc[i + 1]; x[2] = o.z - acc[i + 2]; x[3] = o.w - acc[i + 3];
+            }
+            if (crow) *reinterpret_cast<float4*>(crow + i) = make_float4(x[0], x[1], x[2], x[3]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              x[e] = 0.f;
+              if (col0 + i + e < N) {
+                x[e] = out.store ? acc[i + e] : crow[i + e] - acc[i + e];
+                if (crow) crow[i + e] = x[e];
+              }
+            }
+          }
+          if (out.Chi != nullptr) {
+            float hs[4], ls[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) { hs[e] = tf32_hi(x[e]); ls[e] = x[e] - hs[e]; }
+            float* hrow = out.Chi + (int64_t)r * out.ldh + col0 + i;
+            float* lrow = out.Clo + (int64_t)r * out.ldh + col0 + i;
+            if (whole && vech) {
+              *reinterpret_cast<float4*>(hrow) = make_float4(hs[0], hs[1], hs[2], hs[3]);
+              *reinterpret_cast<float4*>(lrow) = make_float4(ls[0], ls[1], ls[2], ls[3]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (col0 + i + e < N) { hrow[e] = hs[e]; lrow[e] = ls[e]; }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    if (warp == 0 && lane == 0) {
+      for (int s2 = 0; s2 < PST; ++s2)
+        if (armed[s2] > 0) drain_wait(&S.full[s2], (uint32_t)(armed[s2] - 1) & 1u);
+    }
+    if (warp == 1 && lane == 0 && mma_committed) drain_wait(&S.drain, 0);
+    if (threadIdx.x == 0) set_error(st, GPTQ_ERR_TIMEOUT, blockIdx.x, STAGE_TRAILING);
+    __syncthreads();
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tc::tmem_dealloc<512>(taddr);
+  }
+}
+
 // hi = x with the low 13 mantissa bits cleared, lo = x - hi.
 __global__ void split_tf32_kernel(const float* X, int rows, int cols, int ldx, float* hi, float* lo, int ldo,
                                   const int32_t* st) {
@@ -359,6 +597,42 @@ int launch_gemm3_t(const GemmOut& out, int M, int N, int K, const float* Ahi, co
   return GPTQ_OK;
 }
 
+int launch_gemm3p(const GemmOut& out, int M, int N, int K, const float* Ahi, const float* Alo, int lda,
+                  const float* Bhi, const float* Blo, int ldb, bool lower, int32_t* st, cudaStream_t s) {
+  GemmMaps maps;
+  int rc = make_tmap_2d(&maps.ahi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Ahi, (uint64_t)K, (uint64_t)M,
+                        (uint64_t)lda * 4, GK, GM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc == GPTQ_OK)
+    rc = make_tmap_2d(&maps.alo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Alo, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 4,
+                      GK, GM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc == GPTQ_OK)
+    rc = make_tmap_2d(&maps.bhi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Bhi, (uint64_t)K, (uint64_t)N, (uint64_t)ldb * 4,
+                      GK, PN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc == GPTQ_OK)
+    rc = make_tmap_2d(&maps.blo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Blo, (uint64_t)K, (uint64_t)N, (uint64_t)ldb * 4,
+                      GK, PN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != GPTQ_OK) return rc;
+  const int tm = (int)cdiv(M, GM), tn = (int)cdiv(N, PN);
+  int tiles = 0;
+  if (lower) {
+    for (int ti = 0; ti < tm; ++ti) tiles += std::min(ti / 2 + 1, tn);
+  } else {
+    tiles = tm * tn;
+  }
+  if (tiles == 0) return GPTQ_OK;
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                 cudaSuccess)
+      return GPTQ_ERR_CUDA;
+  }
+  GPTQ_CUDA_TRY(cudaFuncSetAttribute(gemm3p_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GEMMP_SMEM));
+  gemm3p_kernel<<<std::min(tiles, sms), P_THREADS, GEMMP_SMEM, s>>>(maps, out, M, N, K, lower ? 1 : 0, tiles, tn, st);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
 }  // namespace
 
 int launch_split_tf32(const float* X, int rows, int cols, int ldx, float* hi, float* lo, int ldo,
@@ -377,6 +651,12 @@ int launch_gemm3(float* C, int ldc, int M, int N, int K, const float* Ahi, const
   // the widest tile that still gives about one CTA per SM; K beyond one chunk takes
   // the chunked (<= 128-wide) tiles
   const int64_t tm = (int64_t)cdiv(M, GM);
+  // Products with at least two waves of 128 x 256 tiles (296 on 148 SMs): the persistent
+  // form.  Below that, the 128-wide tiles of gemm3_kernel give more CTAs, which the
+  // measured layers preferred (1024-row far updates, the trailing updates at n = 4096).
+  const int64_t wide_tiles = lower ? tm * (tm / 4 + 1) : tm * (int64_t)cdiv(N, PN);
+  if (N >= PN && wide_tiles >= 296)
+    return launch_gemm3p(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, st, s);
   if (K > CHUNK_KB * GK) return launch_gemm3_t<128>(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, st, s);
   if (N <= 128 && tm * (int64_t)cdiv(N, 64) < 148)
     return launch_gemm3_t<32>(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, st, s);
