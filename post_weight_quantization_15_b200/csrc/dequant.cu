@@ -92,10 +92,15 @@ __global__ void __launch_bounds__(256) dequant_kernel(const int32_t* qweight, co
 // (fp32); qmatvec_reduce_kernel adds the splits in order.
 // ---------------------------------------------------------------------------
 constexpr int QMV_MAXM = 16;
-constexpr int QMV_KC = 512;           // input columns per block (256 for 16 rows: shared memory)
-__host__ __device__ constexpr int qmv_kc(int M) { return M > 8 ? QMV_KC / 2 : QMV_KC; }
+// input columns per block: as many as the staged activations allow (the staging's
+// latency is paid once per block, so longer ranges amortise it)
+__host__ __device__ constexpr int qmv_kc(int M) { return M <= 2 ? 2048 : M <= 4 ? 1024 : M <= 8 ? 512 : 256; }
 constexpr int QMV_UNROLL = 4;         // words in flight per thread
-constexpr int QMV_MAXG = 17;          // staged groups: 512 / 32 + 1
+// staged groups: the range's groups when groups of 64 or more columns are contiguous
+__host__ __device__ constexpr int qmv_maxg(int M) { return qmv_kc(M) / 64 + 1; }
+__host__ __device__ constexpr size_t qmv_smem(int M) {
+  return (size_t)M * qmv_kc(M) * 4 + (size_t)qmv_kc(M) * 4 + 8 * 128 * 4 + (size_t)qmv_maxg(M) * 64 * 16;
+}
 
 template <typename TX, int BITS, int M>
 __global__ void __launch_bounds__(256) qmatvec_kernel(const int32_t* qweight, const uint16_t* scales,
@@ -105,12 +110,14 @@ __global__ void __launch_bounds__(256) qmatvec_kernel(const int32_t* qweight, co
   if (has_error(st)) return;
   constexpr int PER = 32 / BITS;
   constexpr int kc = qmv_kc(M);
-  __shared__ float xs[M * kc];
-  __shared__ int gsm[kc];
-  __shared__ float red[8 * 128];
+  constexpr int QMV_MAXG = qmv_maxg(M);
+  extern __shared__ __align__(16) uint8_t qsm[];
+  float* xs = reinterpret_cast<float*>(qsm);                          // [M][kc]
+  int* gsm = reinterpret_cast<int*>(xs + M * kc);                     // [kc]
+  float* red = reinterpret_cast<float*>(gsm + kc);                    // [8][128]
   // scales, then zero points, of staged group g_lo + gi for the four outputs of lane l:
   // szs[gi][l] = (s0, s1, s2, s3), szs[gi][32 + l] = (z0, z1, z2, z3)
-  __shared__ float4 szs[QMV_MAXG * 64];
+  float4* szs = reinterpret_cast<float4*>(red + 8 * 128);             // [QMV_MAXG][64]
   __shared__ int grange[3];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int o0 = blockIdx.x * 128;
@@ -198,7 +205,10 @@ __global__ void __launch_bounds__(256) qmatvec_kernel(const int32_t* qweight, co
         const int kl0 = w * PER - k0;
         const int gi = gsm[kl0] - g_lo;
         const float4 sv = szs[gi * 64 + lane], zv = szs[gi * 64 + 32 + lane];
-        const float s4[4] = {sv.x, sv.y, sv.z, sv.w}, z4[4] = {zv.x, zv.y, zv.z, zv.w};
+        // code c as a float without a conversion instruction: the bits of 2^23 + c are
+        // 0x4B000000 | c, and (2^23 + c) - 2^23 = c exactly (c < 2^23)
+        const float s4[4] = {sv.x, sv.y, sv.z, sv.w};
+        const float z4[4] = {zv.x, zv.y, zv.z, zv.w};
 #pragma unroll
         for (int i0 = 0; i0 < PER; i0 += 4) {
           float wv[4][4];
@@ -206,7 +216,8 @@ __global__ void __launch_bounds__(256) qmatvec_kernel(const int32_t* qweight, co
           for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              wv[ii][j] = s4[j] * ((float)((q[u][j] >> ((i0 + ii) * BITS)) & ((1u << BITS) - 1u)) - z4[j]);
+              wv[ii][j] = s4[j] * ((__uint_as_float(((q[u][j] >> ((i0 + ii) * BITS)) & ((1u << BITS) - 1u)) |
+                                                    0x4B000000u) - 8388608.f) - z4[j]);
 #pragma unroll
           for (int m = 0; m < M; ++m) {
             const float4 x4 = *reinterpret_cast<const float4*>(xs + m * kc + kl0 + i0);
@@ -295,7 +306,10 @@ int qmv_launch(const int32_t* qweight, const uint16_t* scales, const uint16_t* z
                int splits, int32_t* st, cudaStream_t s) {
   (void)splits;
   dim3 grd((unsigned)cdiv(out, 128), (unsigned)cdiv(n, qmv_kc(M)));
-  qmatvec_kernel<TX, BITS, M><<<grd, 256, 0, s>>>(qweight, scales, zeros, g_idx, n, out, groups,
+  const size_t smem = qmv_smem(M);
+  GPTQ_CUDA_TRY(cudaFuncSetAttribute(qmatvec_kernel<TX, BITS, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem));
+  qmatvec_kernel<TX, BITS, M><<<grd, 256, smem, s>>>(qweight, scales, zeros, g_idx, n, out, groups,
                                                    static_cast<const TX*>(X), xperm, m_real, ldx, part, st);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
@@ -398,7 +412,7 @@ int launch_reorder_groups(const int32_t* qweight, const int32_t* g_idx, int bits
 }
 
 size_t qmatvec_ws_bytes(int M, int n, int out) {
-  const int splits = (int)cdiv(n, qmv_kc(M <= 8 ? M : 16));
+  const int splits = (int)cdiv(n, qmv_kc(M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16));
   return align_up((size_t)splits * M * out * 4, 256);
 }
 
@@ -414,7 +428,7 @@ int launch_dequant(const int32_t* qweight, const uint16_t* scales, const uint16_
 int launch_qmatvec(const int32_t* qweight, const uint16_t* scales, const uint16_t* zeros, const int32_t* g_idx,
                    int bits, int n, int out, int groups, const void* X, const int32_t* xperm, int x_dtype, int M,
                    int ldx, float* Y, int ldy, void* ws, int32_t* st, cudaStream_t s) {
-  const int splits = (int)cdiv(n, qmv_kc(M <= 8 ? M : 16));
+  const int splits = (int)cdiv(n, qmv_kc(M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16));
   float* part = static_cast<float*>(ws);
   // bytes read once: packed weights, scales and zeros, g_idx, X; Y written
   TraceScope ts("qmatvec", "byte",
