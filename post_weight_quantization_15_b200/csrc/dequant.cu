@@ -205,19 +205,28 @@ __global__ void __launch_bounds__(256) qmatvec_kernel(const int32_t* qweight, co
         const int kl0 = w * PER - k0;
         const int gi = gsm[kl0] - g_lo;
         const float4 sv = szs[gi * 64 + lane], zv = szs[gi * 64 + 32 + lane];
-        // code c as a float without a conversion instruction: the bits of 2^23 + c are
-        // 0x4B000000 | c, and (2^23 + c) - 2^23 = c exactly (c < 2^23)
-        const float s4[4] = {sv.x, sv.y, sv.z, sv.w};
-        const float z4[4] = {zv.x, zv.y, zv.z, zv.w};
+        // s (c - z) in one exact fma: the code c placed in the top mantissa bits of 1.0 gives
+        // f = 1 + c / 2^BITS without a conversion instruction (a shift and a mask-or), and
+        // s (c - z) = (2^BITS s) f - s (2^BITS + z): every product has at most 20 significant
+        // bits (an fp16 scale, integers below 2^9), so the fma's one rounding is exact
+        const float s4[4] = {sv.x * (float)(1 << BITS), sv.y * (float)(1 << BITS), sv.z * (float)(1 << BITS),
+                             sv.w * (float)(1 << BITS)};
+        const float n4[4] = {-sv.x * ((float)(1 << BITS) + zv.x), -sv.y * ((float)(1 << BITS) + zv.y),
+                             -sv.z * ((float)(1 << BITS) + zv.z), -sv.w * ((float)(1 << BITS) + zv.w)};
+        constexpr int POS = 23 - BITS;                 // where the code goes in the mantissa
 #pragma unroll
         for (int i0 = 0; i0 < PER; i0 += 4) {
           float wv[4][4];
 #pragma unroll
-          for (int ii = 0; ii < 4; ++ii)
+          for (int ii = 0; ii < 4; ++ii) {
+            constexpr uint32_t MASK = ((1u << BITS) - 1u) << POS;
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              wv[ii][j] = s4[j] * ((__uint_as_float(((q[u][j] >> ((i0 + ii) * BITS)) & ((1u << BITS) - 1u)) |
-                                                    0x4B000000u) - 8388608.f) - z4[j]);
+            for (int j = 0; j < 4; ++j) {
+              const int sh = POS - (i0 + ii) * BITS;   // a compile-time shift after unrolling
+              const uint32_t bitsf = (sh >= 0 ? (q[u][j] << sh) : (q[u][j] >> -sh)) & MASK;
+              wv[ii][j] = fmaf(s4[j], __uint_as_float(bitsf | 0x3F800000u), n4[j]);
+            }
+          }
 #pragma unroll
           for (int m = 0; m < M; ++m) {
             const float4 x4 = *reinterpret_cast<const float4*>(xs + m * kc + kl0 + i0);

@@ -330,7 +330,8 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
 //               columns 128 ((w - 2) / 4) .. + 128, adds each 128-deep chunk into fp32
 //               registers, releases the accumulator, and at a tile's last chunk
 //               updates its rows of C (C -= acc or C = acc; optionally the split of
-//               the result) straight from registers, 16 bytes at a time.
+//               the result), 32 columns at a time turned through a 32 x 32 staging
+//               tile so that each access is one coalesced 128-byte row.
 // K is accumulated in chunks of 128 (as in gemm3_kernel), each from zero.  Every
 // wait is bounded (GPTQ_ERR_TIMEOUT).
 // ---------------------------------------------------------------------------
@@ -341,11 +342,14 @@ constexpr int P_EPI = 8;
 constexpr int P_THREADS = 64 + P_EPI * 32;
 constexpr uint32_t P_IDESC = tc::idesc_f32acc(2, GM, PN);
 
+constexpr int P_LDT = 33;                       // row stride of an epilogue warp's 32 x 32 staging tile
+
 struct GemmPSmem {
   uint8_t bhi[PST][P_BTILE];
   uint8_t blo[PST][P_BTILE];
   uint8_t ahi[PST][A_TILE];
   uint8_t alo[PST][A_TILE];
+  float tr[P_EPI][32 * P_LDT];                  // per epilogue warp: 32 rows x 32 columns, turned
   uint64_t full[PST];
   uint64_t empty[PST];
   uint64_t acc_full[2];
@@ -459,8 +463,6 @@ gemm3p_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, 
       const int qq = warp & 3;                   // TMEM lane quarter this warp may access
       const int hc = (warp - 2) >> 2;            // which 128 of the 256 columns
       const uint32_t lane_base = (uint32_t)(qq * 32) << 16;
-      const bool vec = out.C == nullptr || ((out.ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(out.C) & 15) == 0);
-      const bool vech = out.Chi == nullptr || (out.ldh & 3) == 0;
       int g = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
@@ -488,45 +490,38 @@ gemm3p_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, 
           if (lane == 0) tc::mbar_arrive(&S.acc_empty[buf]);   // the MMAs may reuse it now
         }
         if (!ok) break;
-        const int r = ti * GM + qq * 32 + lane;
+        // C's rows [row0, row0 + 32) and columns [col0, col0 + 128): the registers hold one
+        // row per lane; each 32-column slice turns through the warp's staging tile so that
+        // every access to C (and to its split) is one row of 32 consecutive floats
+        const int row0 = ti * GM + qq * 32;
         const int col0 = tj * PN + hc * 128;
-        if (r >= M || col0 >= N) continue;
-        const bool whole = col0 + 128 <= N;
-        float* crow = out.C ? out.C + (int64_t)r * out.ldc + col0 : nullptr;
+        float* tile = S.tr[warp - 2];
 #pragma unroll
-        for (int i = 0; i < 128; i += 4) {
-          float x[4];
-          if (whole && vec) {
-            if (out.store) {
-              x[0] = acc[i]; x[1] = acc[i + 1]; x[2] = acc[i + 2]; x[3] = acc[i + 3];
-            } else {
-              const float4 o = *reinterpret_cast<const float4*>(crow + i);
-              x[0] = o.x - acc[i]; x[1] = o.y - acc[i + 1]; x[2] = o.z - acc[i + 2]; x[3] = o.w - acc[i + 3];
-            }
-            if (crow) *reinterpret_cast<float4*>(crow + i) = make_float4(x[0], x[1], x[2], x[3]);
-          } else {
+        for (int c4 = 0; c4 < 4; ++c4) {
+          __syncwarp();
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              x[e] = 0.f;
-              if (col0 + i + e < N) {
-                x[e] = out.store ? acc[i + e] : crow[i + e] - acc[i + e];
-                if (crow) crow[i + e] = x[e];
+          for (int i = 0; i < 32; ++i) tile[lane * P_LDT + i] = acc[c4 * 32 + i];
+          __syncwarp();
+          const int col = col0 + c4 * 32 + lane;
+          if (col < N) {
+            for (int rr = 0; rr < 32; ++rr) {
+              const int r = row0 + rr;
+              if (r >= M) break;
+              const float a = tile[rr * P_LDT + lane];
+              float x;
+              if (out.store) {
+                x = a;
+                if (out.C) out.C[(int64_t)r * out.ldc + col] = x;
+              } else {
+                float* cp = out.C + (int64_t)r * out.ldc + col;
+                x = *cp - a;
+                *cp = x;
               }
-            }
-          }
-          if (out.Chi != nullptr) {
-            float hs[4], ls[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) { hs[e] = tf32_hi(x[e]); ls[e] = x[e] - hs[e]; }
-            float* hrow = out.Chi + (int64_t)r * out.ldh + col0 + i;
-            float* lrow = out.Clo + (int64_t)r * out.ldh + col0 + i;
-            if (whole && vech) {
-              *reinterpret_cast<float4*>(hrow) = make_float4(hs[0], hs[1], hs[2], hs[3]);
-              *reinterpret_cast<float4*>(lrow) = make_float4(ls[0], ls[1], ls[2], ls[3]);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                if (col0 + i + e < N) { hrow[e] = hs[e]; lrow[e] = ls[e]; }
+              if (out.Chi != nullptr) {
+                const float h = tf32_hi(x);
+                out.Chi[(int64_t)r * out.ldh + col] = h;
+                out.Clo[(int64_t)r * out.ldh + col] = x - h;
+              }
             }
           }
         }
