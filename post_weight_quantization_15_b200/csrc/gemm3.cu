@@ -497,26 +497,37 @@ gemm3p_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, 
         const int col0 = tj * PN + hc * 128;
         float* tile = S.tr[warp - 2];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          __syncwarp();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) tile[lane * P_LDT + i] = acc[c4 * 32 + i];
-          __syncwarp();
+        for (int c4 = 0; c4 < 4; ++c4) {          // unrolled: acc stays in registers
           const int col = col0 + c4 * 32 + lane;
+          __syncwarp();
+          if (!out.store) {
+            // C's 32 x 32 slice into the tile: lane l copies column col of every row, all
+            // the copies in flight at once, no registers
+#pragma unroll 1
+            for (int rr = 0; rr < 32; ++rr) {
+              const int r = row0 + rr;
+              if (r < M && col < N)
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(tc::smem_u32(tile + rr * P_LDT + lane)),
+                             "l"(out.C + (int64_t)r * out.ldc + col)
+                             : "memory");
+            }
+            asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+          }
+          __syncwarp();
+          // the row owner combines its 32 values
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float* e = tile + lane * P_LDT + i;
+            *e = out.store ? acc[c4 * 32 + i] : *e - acc[c4 * 32 + i];
+          }
+          __syncwarp();
           if (col < N) {
+#pragma unroll 1
             for (int rr = 0; rr < 32; ++rr) {
               const int r = row0 + rr;
               if (r >= M) break;
-              const float a = tile[rr * P_LDT + lane];
-              float x;
-              if (out.store) {
-                x = a;
-                if (out.C) out.C[(int64_t)r * out.ldc + col] = x;
-              } else {
-                float* cp = out.C + (int64_t)r * out.ldc + col;
-                x = *cp - a;
-                *cp = x;
-              }
+              const float x = tile[rr * P_LDT + lane];
+              if (out.C) out.C[(int64_t)r * out.ldc + col] = x;
               if (out.Chi != nullptr) {
                 const float h = tf32_hi(x);
                 out.Chi[(int64_t)r * out.ldh + col] = h;
