@@ -321,8 +321,8 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
 // ...).  The stage ring, the chunk counter and the two TMEM accumulators run on
 // across tiles, so the producer loads the next tile's operands and the MMAs start
 // it while the epilogue warps still update C with the previous one.
-//   warp 0      TMA producer: 32-wide K slices of A hi / lo (128 rows) and B hi / lo
-//               (256 rows), 2-stage ring of 96 KB stages;
+//   warp 0      TMA producer: 16-wide K slices of A hi / lo (128 rows) and B hi / lo
+//               (256 rows), 64-byte swizzled, 4-stage ring of 48 KB stages;
 //   warp 1      allocates 512 TMEM columns (two 128 x 256 accumulators); one thread
 //               issues tcgen05.mma kind::tf32 (M = 128, N = 256, K = 8), three per
 //               K step (lo.hi + hi.lo + hi.hi);
@@ -336,8 +336,11 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
 // wait is bounded (GPTQ_ERR_TIMEOUT).
 // ---------------------------------------------------------------------------
 constexpr int PN = 256;
-constexpr int PST = 2;
-constexpr int P_BTILE = PN * GK * 4;             // 32 KB
+constexpr int PK = 16;                           // fp32 per 64-byte row: 16-deep K slices
+constexpr int PST = 4;
+constexpr int P_ATILE = GM * PK * 4;             // 8 KB
+constexpr int P_BTILE = PN * PK * 4;             // 16 KB
+constexpr int P_CHUNK_KB = CHUNK_KB * GK / PK;   // slices per 128-deep accumulation chunk
 constexpr int P_EPI = 8;
 constexpr int P_THREADS = 64 + P_EPI * 32;
 constexpr uint32_t P_IDESC = tc::idesc_f32acc(2, GM, PN);
@@ -347,8 +350,8 @@ constexpr int P_LDT = 33;                       // row stride of an epilogue war
 struct GemmPSmem {
   uint8_t bhi[PST][P_BTILE];
   uint8_t blo[PST][P_BTILE];
-  uint8_t ahi[PST][A_TILE];
-  uint8_t alo[PST][A_TILE];
+  uint8_t ahi[PST][P_ATILE];
+  uint8_t alo[PST][P_ATILE];
   float tr[P_EPI][32 * P_LDT];                  // per epilogue warp: 32 rows x 32 columns, turned
   uint64_t full[PST];
   uint64_t empty[PST];
@@ -382,8 +385,8 @@ gemm3p_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, 
   // offset arithmetic on the shared array keeps every access a shared-memory one
   GemmPSmem& S = *reinterpret_cast<GemmPSmem*>(smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kblocks = (int)cdiv(K, GK);
-  const int nchunks = (int)cdiv(kblocks, CHUNK_KB);        // chunks per tile
+  const int kblocks = (int)cdiv(K, PK);
+  const int nchunks = (int)cdiv(kblocks, P_CHUNK_KB);      // 128-deep chunks per tile
 
   if (threadIdx.x == 0) {
     S.skip = has_error(st) ? 1 : 0;
@@ -414,11 +417,11 @@ gemm3p_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, 
           const int s2 = q % PST;
           const uint32_t ph = (uint32_t)(q / PST) & 1u;
           if (!tc::mbar_wait(&S.empty[s2], ph ^ 1u, abort_flag)) break;
-          tc::mbar_arrive_expect_tx(&S.full[s2], 2 * (A_TILE + P_BTILE));
-          tc::tma_load_2d(S.ahi[s2], &maps.ahi, &S.full[s2], kb * GK, ti * GM);
-          tc::tma_load_2d(S.alo[s2], &maps.alo, &S.full[s2], kb * GK, ti * GM);
-          tc::tma_load_2d(S.bhi[s2], &maps.bhi, &S.full[s2], kb * GK, tj * PN);
-          tc::tma_load_2d(S.blo[s2], &maps.blo, &S.full[s2], kb * GK, tj * PN);
+          tc::mbar_arrive_expect_tx(&S.full[s2], 2 * (P_ATILE + P_BTILE));
+          tc::tma_load_2d(S.ahi[s2], &maps.ahi, &S.full[s2], kb * PK, ti * GM);
+          tc::tma_load_2d(S.alo[s2], &maps.alo, &S.full[s2], kb * PK, ti * GM);
+          tc::tma_load_2d(S.bhi[s2], &maps.bhi, &S.full[s2], kb * PK, tj * PN);
+          tc::tma_load_2d(S.blo[s2], &maps.blo, &S.full[s2], kb * PK, tj * PN);
           ++armed[s2];
         }
       }
@@ -432,7 +435,7 @@ gemm3p_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, 
           if (!tc::mbar_wait(&S.acc_empty[buf], ((uint32_t)(g >> 1) & 1u) ^ 1u, abort_flag)) break;
           tc::tc_fence_after();
           const uint32_t dacc = taddr + buf * PN;
-          const int kb_end = min(kblocks, (c + 1) * CHUNK_KB);
+          const int kb_end = min(kblocks, (c + 1) * P_CHUNK_KB);
           bool first = true;
           for (; kb < kb_end; ++kb, ++q) {
             const int s2 = q % PST;
@@ -442,11 +445,11 @@ gemm3p_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, 
             const uint32_t ah = tc::smem_u32(S.ahi[s2]), al = tc::smem_u32(S.alo[s2]);
             const uint32_t bh = tc::smem_u32(S.bhi[s2]), bl = tc::smem_u32(S.blo[s2]);
 #pragma unroll
-            for (int kk = 0; kk < GK / 8; ++kk) {
+            for (int kk = 0; kk < PK / 8; ++kk) {
               const uint32_t o = kk * 32;
-              tc::mma_tf32(dacc, tc::sdesc_k_sw128(al + o), tc::sdesc_k_sw128(bh + o), P_IDESC, !first);
-              tc::mma_tf32(dacc, tc::sdesc_k_sw128(ah + o), tc::sdesc_k_sw128(bl + o), P_IDESC, true);
-              tc::mma_tf32(dacc, tc::sdesc_k_sw128(ah + o), tc::sdesc_k_sw128(bh + o), P_IDESC, true);
+              tc::mma_tf32(dacc, tc::sdesc_k_sw64(al + o), tc::sdesc_k_sw64(bh + o), P_IDESC, !first);
+              tc::mma_tf32(dacc, tc::sdesc_k_sw64(ah + o), tc::sdesc_k_sw64(bl + o), P_IDESC, true);
+              tc::mma_tf32(dacc, tc::sdesc_k_sw64(ah + o), tc::sdesc_k_sw64(bh + o), P_IDESC, true);
               first = false;
             }
             tc::mma_commit(&S.empty[s2]);
@@ -607,16 +610,16 @@ int launch_gemm3p(const GemmOut& out, int M, int N, int K, const float* Ahi, con
                   const float* Bhi, const float* Blo, int ldb, bool lower, int32_t* st, cudaStream_t s) {
   GemmMaps maps;
   int rc = make_tmap_2d(&maps.ahi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Ahi, (uint64_t)K, (uint64_t)M,
-                        (uint64_t)lda * 4, GK, GM, CU_TENSOR_MAP_SWIZZLE_128B);
+                        (uint64_t)lda * 4, PK, GM, CU_TENSOR_MAP_SWIZZLE_64B);
   if (rc == GPTQ_OK)
     rc = make_tmap_2d(&maps.alo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Alo, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 4,
-                      GK, GM, CU_TENSOR_MAP_SWIZZLE_128B);
+                      PK, GM, CU_TENSOR_MAP_SWIZZLE_64B);
   if (rc == GPTQ_OK)
     rc = make_tmap_2d(&maps.bhi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Bhi, (uint64_t)K, (uint64_t)N, (uint64_t)ldb * 4,
-                      GK, PN, CU_TENSOR_MAP_SWIZZLE_128B);
+                      PK, PN, CU_TENSOR_MAP_SWIZZLE_64B);
   if (rc == GPTQ_OK)
     rc = make_tmap_2d(&maps.blo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Blo, (uint64_t)K, (uint64_t)N, (uint64_t)ldb * 4,
-                      GK, PN, CU_TENSOR_MAP_SWIZZLE_128B);
+                      PK, PN, CU_TENSOR_MAP_SWIZZLE_64B);
   if (rc != GPTQ_OK) return rc;
   const int tm = (int)cdiv(M, GM), tn = (int)cdiv(N, PN);
   int tiles = 0;

@@ -168,6 +168,18 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t addr) {
   return d;
 }
 
+// The same for 64-byte rows with the 64-byte swizzle (8-row atoms of 512 bytes; the
+// address must be the tile base, 512-byte aligned, plus a k offset of 32 bytes or 0).
+__device__ __forceinline__ uint64_t sdesc_k_sw64(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);        // start address  [0,14)
+  d |= (uint64_t)1u << 16;                       // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(512u >> 4) << 32;              // stride byte offset: 8 rows x 64 B
+  d |= (uint64_t)1u << 46;                       // descriptor version (sm_100)
+  d |= (uint64_t)4u << 61;                       // layout: 64-byte swizzle
+  return d;
+}
+
 // Instruction descriptor: fp32 accumulate, both operands K-major, shape M x N.
 // ab_format: 1 = bf16 (kind::f16), 2 = tf32 (kind::tf32).
 __host__ __device__ constexpr uint32_t idesc_f32acc(int ab_format, int M, int N) {
