@@ -172,6 +172,20 @@ GPTQ_API int gptq_prepare(const float* H, const double* hdiag, int n, float damp
                  int32_t* d_status, void* stream);
 
 /*
+ * gptq_prepare_set_deferred_min_n - how gptq_prepare groups its bulk updates.
+ *
+ * gptq_prepare factors H in 128-wide panels.  For n >= min_n (default 8192) four
+ * panels form a 512-wide outer panel whose trailing and inverse updates are
+ * applied once, as rank-512 products, instead of once per panel as rank-128
+ * products: the same terms, a quarter of the passes over the trailing matrices.
+ * The two forms differ only in the order in which those terms are summed.
+ *   min_n    the new threshold; min_n <= 0 only queries.
+ * Returns the previous threshold.  Process-wide; a call that races a
+ * gptq_prepare on another thread may or may not apply to it.
+ */
+GPTQ_API int gptq_prepare_set_deferred_min_n(int min_n);
+
+/*
  * gptq_quantize_layer - the column sweep, the lazy trailing update and packing.
  *
  * For every column j in processing order ("polydesk.ai/glossaire/gptq",

@@ -663,7 +663,12 @@ int launch_gemm3(float* C, int ldc, int M, int N, int K, const float* Ahi, const
   // Products with at least two waves of 128 x 256 tiles (296 on 148 SMs): the persistent
   // form.  Below that, the 128-wide tiles of gemm3_kernel give more CTAs, which the
   // measured layers preferred (1024-row far updates, the trailing updates at n = 4096).
-  const int64_t wide_tiles = lower ? tm * (tm / 4 + 1) : tm * (int64_t)cdiv(N, PN);
+  const int64_t tnw = (int64_t)cdiv(N, PN);
+  int64_t wide_tiles = tm * tnw;
+  if (lower) {   // the 128 x 256 tiles that reach the lower triangle (tall C: the diagonal starts top left)
+    wide_tiles = 0;
+    for (int64_t ti = 0; ti < tm; ++ti) wide_tiles += std::min(ti / 2 + 1, tnw);
+  }
   if (N >= PN && wide_tiles >= 296)
     return launch_gemm3p(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, st, s);
   if (K > CHUNK_KB * GK) return launch_gemm3_t<128>(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, st, s);

@@ -108,6 +108,8 @@ int gptq_prepare(const float* H, const double* hdiag, int n, float damp_percent,
                         as_stream(stream));
 }
 
+int gptq_prepare_set_deferred_min_n(int min_n) { return prepare_set_deferred_min_n(min_n); }
+
 size_t gptq_quantize_workspace_size(int out, int n, int block) {
   if (out <= 0 || n <= 0) return 0;
   return quantize_ws_bytes(out, n, block);

@@ -37,6 +37,7 @@ int launch_hessian_host(float* H, double* hdiag, int n, const void* X_host, int 
 
 // ---- K2: prepare -------------------------------------------------------------
 size_t prepare_ws_bytes(int n);
+int prepare_set_deferred_min_n(int min_n);
 int launch_prepare(const float* H, const double* hdiag, int n, float damp, int desc_act, float* U,
                    int32_t* perm, uint8_t* dead, void* ws, int32_t* st, cudaStream_t s);
 

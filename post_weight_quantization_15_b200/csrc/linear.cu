@@ -5,7 +5,11 @@
 // proceeds layer by layer).
 //
 // One CTA computes one 128 x 256 tile of C (rows [128 bi, +128) of A, rows
-// [256 bj, +256) of B) over all of K, with the structure of the Hessian kernel:
+// [256 bj, +256) of B) over all of K.  Tiles are walked in bands of `band` row
+// tiles, column by column inside a band, so that the CTAs running at once share
+// their B tiles and the band's rows of A stay in L2: B is read from HBM once per
+// band instead of once per row tile (B, the activations, is the large operand).
+// The kernel has the structure of the Hessian kernel:
 //   warp 0      TMA producer: 64-wide K slices of the 128 A rows and 256 B rows,
 //               128-byte swizzled, 4-stage ring;
 //   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32 accumulators); one
@@ -15,6 +19,8 @@
 // and the epilogue warps add each finished chunk into fp32 registers (the tensor
 // cores' accumulation is not rounded to nearest; its error grows with its length).
 // C = acc is stored (fp32, row stride ldc).  Every wait is bounded (GPTQ_ERR_TIMEOUT).
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
@@ -58,12 +64,16 @@ __device__ __forceinline__ bool lin_drain(uint64_t* bar, uint32_t parity) {
 
 __global__ void __launch_bounds__(LTHREADS, 1)
 linear_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb, float* C, int M, int N,
-              int64_t ldc, int tiles_n, int kblocks, int32_t* st) {
+              int64_t ldc, int tiles_m, int tiles_n, int band, int kblocks, int32_t* st) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // offset arithmetic on the shared array keeps every access a shared-memory one
   LinSmem& S = *reinterpret_cast<LinSmem*>(smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bi = blockIdx.x / tiles_n, bj = blockIdx.x % tiles_n;
+  const int per_band = band * tiles_n;
+  const int b0 = (int)blockIdx.x / per_band * band;          // the band's first row tile
+  const int rows = min(band, tiles_m - b0);                   // row tiles in this band
+  const int r = (int)blockIdx.x % per_band;
+  const int bi = b0 + r % rows, bj = r / rows;
   const int nchunks = (int)cdiv(kblocks, LCHUNK);
 
   if (threadIdx.x == 0) {
@@ -201,9 +211,11 @@ int launch_linear(const void* A, int M, int64_t lda, const void* B, int N, int64
   if (rc != GPTQ_OK) return rc;
   const int tm = (int)cdiv(M, LM), tn = (int)cdiv(N, LN);
   const int kblocks = (int)cdiv(K, LKB);
+  // a band's rows of A: about 32 MB (a quarter of L2)
+  const int band = (int)std::max<int64_t>(1, std::min<int64_t>(tm, (32ll << 20) / ((int64_t)LM * K * 2)));
   TraceScope ts("linear_bf16", "flop", 2.0 * M * (double)N * K, s);
   GPTQ_CUDA_TRY(cudaFuncSetAttribute(linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LIN_SMEM));
-  linear_kernel<<<tm * tn, LTHREADS, LIN_SMEM, s>>>(ta, tb, C, M, N, ldc, tn, kblocks, st);
+  linear_kernel<<<tm * tn, LTHREADS, LIN_SMEM, s>>>(ta, tb, C, M, N, ldc, tm, tn, band, kblocks, st);
   GPTQ_LAUNCH_CHECK();
   return GPTQ_OK;
 }

@@ -21,6 +21,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "internal.h"
@@ -36,7 +37,10 @@ namespace gptq {
 namespace {
 
 constexpr int PB = 128;          // panel width
-constexpr int NBUF = 3;          // panels in flight: per-panel buffers and events form a ring
+constexpr int NBUF = 3;          // panels in flight (per-panel loop): per-panel buffers form a ring
+constexpr int SPB = 4 * PB;      // super-panel width (deferred loop)
+constexpr int NSUP = 3;          // super-panels in flight (deferred loop)
+constexpr int NLI = 3 * (SPB / PB);   // ring of L_kk^-1 splits and per-panel events
 
 int ld_of(int n) { return (int)align_up((size_t)n, 32); }
 
@@ -44,10 +48,14 @@ struct PrepWs {
   float* A;        // [n, ldn] lower triangle: the reversed, permuted, damped H, then L
   float* Xt;       // [n, ldn] upper triangle: (L^-1)^T
   float* Phi; float* Plo;     // [n, PB] split of the panel A21 before the solve
-  float* Lhi[NBUF]; float* Llo[NBUF];     // [n, PB] split of L21 (a ring of panels in flight)
   float* XPhi; float* XPlo;   // [n, PB] split of Xt[:k0, k] before the solve
-  float* XQhi; float* XQlo;   // [n, PB] split of the finished Xt[:, k]
-  float* LIhi[NBUF]; float* LIlo[NBUF];   // [PB, PB] split of L_kk^-1 (the same ring)
+  // per-panel loop: a ring of L21 splits and the finished Xt[:, k]
+  float* Lhi[NBUF]; float* Llo[NBUF];     // [n, PB]
+  float* XQhi; float* XQlo;               // [n, PB]
+  // deferred loop (the same memory): a super-panel's L21 and finished Xt columns
+  float* Shi[NSUP]; float* Slo[NSUP];     // [n, SPB], row r holds L(r, super-panel columns)
+  float* SXhi; float* SXlo;               // [n, SPB], row r holds Xt(r, super-panel columns)
+  float* LIhi[NLI]; float* LIlo[NLI];     // [PB, PB] split of L_kk^-1 (a ring)
   double* key;     // [n] act-order key
   float* dfix;     // [n] diag(H) with dead inputs set to 1
   double* scal;    // [0] sum of dfix, [1] lambda
@@ -57,24 +65,38 @@ PrepWs carve(void* ws, int n) {
   const int ldn = ld_of(n);
   char* p = static_cast<char*>(ws);
   auto take = [&](size_t bytes) { char* q = p; p += align_up(bytes, 256); return q; };
+  auto f = [](char* q) { return reinterpret_cast<float*>(q); };
   PrepWs w;
   const size_t nn = (size_t)n * ldn * sizeof(float);
   const size_t panel = (size_t)n * PB * sizeof(float);
-  w.A = reinterpret_cast<float*>(take(nn));
-  w.Xt = reinterpret_cast<float*>(take(nn));
-  w.Phi = reinterpret_cast<float*>(take(panel));  w.Plo = reinterpret_cast<float*>(take(panel));
-  for (int b = 0; b < NBUF; ++b) {
-    w.Lhi[b] = reinterpret_cast<float*>(take(panel));
-    w.Llo[b] = reinterpret_cast<float*>(take(panel));
+  const size_t sup = (size_t)n * SPB * sizeof(float);
+  w.A = f(take(nn));
+  w.Xt = f(take(nn));
+  w.Phi = f(take(panel));  w.Plo = f(take(panel));
+  w.XPhi = f(take(panel)); w.XPlo = f(take(panel));
+  // the two loops' buffers share one region
+  static_assert((2 * NBUF + 2) * PB <= (2 * NSUP + 2) * SPB, "the per-panel buffers fit in the shared region");
+  char* shared = take((2 * NSUP + 2) * align_up(sup, 256));
+  char* q = shared;
+  for (int b = 0; b < NSUP; ++b) {
+    w.Shi[b] = f(q); q += align_up(sup, 256);
+    w.Slo[b] = f(q); q += align_up(sup, 256);
   }
-  w.XPhi = reinterpret_cast<float*>(take(panel)); w.XPlo = reinterpret_cast<float*>(take(panel));
-  w.XQhi = reinterpret_cast<float*>(take(panel)); w.XQlo = reinterpret_cast<float*>(take(panel));
+  w.SXhi = f(q); q += align_up(sup, 256);
+  w.SXlo = f(q);
+  q = shared;
   for (int b = 0; b < NBUF; ++b) {
-    w.LIhi[b] = reinterpret_cast<float*>(take((size_t)PB * PB * 4));
-    w.LIlo[b] = reinterpret_cast<float*>(take((size_t)PB * PB * 4));
+    w.Lhi[b] = f(q); q += align_up(panel, 256);
+    w.Llo[b] = f(q); q += align_up(panel, 256);
+  }
+  w.XQhi = f(q); q += align_up(panel, 256);
+  w.XQlo = f(q);
+  for (int b = 0; b < NLI; ++b) {
+    w.LIhi[b] = f(take((size_t)PB * PB * 4));
+    w.LIlo[b] = f(take((size_t)PB * PB * 4));
   }
   w.key = reinterpret_cast<double*>(take((size_t)n * 8));
-  w.dfix = reinterpret_cast<float*>(take((size_t)n * 4));
+  w.dfix = f(take((size_t)n * 4));
   w.scal = reinterpret_cast<double*>(take(256));
   return w;
 }
@@ -706,9 +728,9 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tp
 
 // (5b) The diagonal block of Xt = (L^-1)^T and the last nb rows of its split XQ,
 // from the split of T = L_kk^-1: Xt[k0 + k][k0 + i] = T[i][k] (hi + lo is exact),
-// XQ[k0 + k][i] = (hi, lo)(T[i][k]).  32 x 32 tiles through shared memory.
+// XQ[k0 + k][i] = (hi, lo)(T[i][k]) (row stride ldq).  32 x 32 tiles through shared memory.
 __global__ void xt_diag_kernel(const float* LIhi, const float* LIlo, int k0, int nb, float* Xt, int ldx, float* XQhi,
-                               float* XQlo, const int32_t* st) {
+                               float* XQlo, int ldq, const int32_t* st) {
   if (has_error(st)) return;
   __shared__ float th[32][33], tl[32][33];
   const int i0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
@@ -722,8 +744,8 @@ __global__ void xt_diag_kernel(const float* LIhi, const float* LIlo, int k0, int
     if (k >= nb) continue;
     const float h = th[threadIdx.x][yy], l = tl[threadIdx.x][yy];
     if (i < nb) Xt[(int64_t)(k0 + k) * ldx + k0 + i] = h + l;
-    XQhi[(int64_t)(k0 + k) * PB + i] = h;
-    XQlo[(int64_t)(k0 + k) * PB + i] = l;
+    XQhi[(int64_t)(k0 + k) * ldq + i] = h;
+    XQlo[(int64_t)(k0 + k) * ldq + i] = l;
   }
 }
 
@@ -772,7 +794,10 @@ struct AuxStream {
   cudaEvent_t fork = nullptr, join[4] = {};
   // per panel (ring slot): diagonal block done, L21 split ready, next block column
   // updated, trailing update done, inverse done with the panel's buffers
-  cudaEvent_t diag[NBUF] = {}, l21[NBUF] = {}, next[NBUF] = {}, trail[NBUF] = {}, done[NBUF] = {};
+  cudaEvent_t diag[NLI] = {}, l21[NLI] = {}, next[NLI] = {}, trail[NLI] = {}, done[NLI] = {};
+  // per super-panel (deferred loop): its L21 complete, the next super-panel's block
+  // column updated, the bulk trailing update done, the bulk inverse update done
+  cudaEvent_t lsup[NSUP] = {}, col[NSUP] = {}, bulk[NSUP] = {}, inv[NSUP] = {};
 };
 
 int aux_stream(AuxStream** out) {
@@ -793,8 +818,13 @@ int aux_stream(AuxStream** out) {
     if (cudaEventCreateWithFlags(&a.fork, f) != cudaSuccess) return GPTQ_ERR_CUDA;
     for (cudaEvent_t& e : a.join)
       if (cudaEventCreateWithFlags(&e, f) != cudaSuccess) return GPTQ_ERR_CUDA;
-    for (int b = 0; b < NBUF; ++b) {
+    for (int b = 0; b < NLI; ++b) {
       cudaEvent_t* evs[] = {&a.diag[b], &a.l21[b], &a.next[b], &a.trail[b], &a.done[b]};
+      for (cudaEvent_t* e : evs)
+        if (cudaEventCreateWithFlags(e, f) != cudaSuccess) return GPTQ_ERR_CUDA;
+    }
+    for (int b = 0; b < NSUP; ++b) {
+      cudaEvent_t* evs[] = {&a.lsup[b], &a.col[b], &a.bulk[b], &a.inv[b]};
       for (cudaEvent_t* e : evs)
         if (cudaEventCreateWithFlags(e, f) != cudaSuccess) return GPTQ_ERR_CUDA;
     }
@@ -877,7 +907,7 @@ int panel_loop(const PrepWs& w, int n, int ldn, AuxStream* aux, int32_t* st) {
     GPTQ_CUDA_TRY(cudaStreamWaitEvent(s2, aux->diag[b], 0));
     {
       dim3 blk(32, 8), grd(PB / 32, PB / 32);
-      xt_diag_kernel<<<grd, blk, 0, s2>>>(w.LIhi[b], w.LIlo[b], k0, nb, w.Xt, ldn, w.XQhi, w.XQlo, st);
+      xt_diag_kernel<<<grd, blk, 0, s2>>>(w.LIhi[b], w.LIlo[b], k0, nb, w.Xt, ldn, w.XQhi, w.XQlo, PB, st);
       GPTQ_LAUNCH_CHECK();
     }
     if (k0 > 0) {
@@ -901,13 +931,185 @@ int panel_loop(const PrepWs& w, int n, int ldn, AuxStream* aux, int32_t* st) {
   return GPTQ_OK;
 }
 
+// The same factorization and inverse with their bulk updates deferred to
+// super-panels of SPB = 4 panels (for large n, where the per-panel loop is set by
+// the bulk: each K = 128 rank update reads and writes its whole trailing matrix).
+// Super-panel S (columns s0 .. se), buffers of parity sb = S % NSUP:
+//   per panel p = s0 / PB + j, j = 0 .. 3, as in the per-panel loop but confined
+//   to the super-panel's columns:
+//     c  the diagonal block (panel p - 1's term formed in the kernel when p - 1
+//        lies in the super-panel; earlier panels' terms are already in A);
+//     o  L21 of all rows below into the super-panel's L (columns PB j), then the
+//        next block column when it lies in the super-panel (its split: Phi/Plo);
+//     t  the super-panel's columns beyond the next block column, all rows below
+//        (lower, K = PB);
+//     s  the inverse's block column p (Xt[:k0, p] and its split into the
+//        super-panel's Xt split), then Xt[:k0+nb, later columns of the
+//        super-panel] -= Xt[:, p] . L(later, p)^T.
+//   then, once for the super-panel (K = se - s0):
+//     o  the next super-panel's block column: A[se:, se:se2] -= L(se:, S) L(se:se2, S)^T
+//        (lower), and the split of its first panel's A21;
+//     t  the rest of the trailing matrix: A[se2:, se2:] -= L(se2:, S) L(se2:, S)^T;
+//     s  the inverse beyond: Xt[:se, se:] -= Xt[:se, S] . L(se:, S)^T.
+// Every product is the same 3 x TF32 tensor-core GEMM; only the grouping of the
+// rank updates changes (four K = 128 updates of the trailing matrix become one
+// K = 512 update), which is the blocked algorithm with 512-wide outer panels.
+int panel_loop_deferred(const PrepWs& w, int n, int ldn, AuxStream* aux, int32_t* st) {
+  cudaStream_t c = aux->c, o = aux->o, t = aux->t, s2 = aux->s;
+  auto wait = [](cudaStream_t strm, cudaEvent_t ev) { return cudaStreamWaitEvent(strm, ev, 0); };
+  int rc = GPTQ_OK;
+  for (int s0 = 0, S = 0; s0 < n; s0 += SPB, ++S) {
+    const int se = std::min(n, s0 + SPB);
+    const int sb = S % NSUP;
+    float* const Lh = w.Shi[sb];
+    float* const Ll = w.Slo[sb];
+    for (int k0 = s0; k0 < se; k0 += PB) {
+      const int panel = k0 / PB, j = (k0 - s0) / PB;
+      const int nb = std::min(PB, n - k0);
+      const int rest = n - k0 - nb;
+      const int b = panel % NLI, b1 = (panel + NLI - 1) % NLI, b2 = (panel + NLI - 2) % NLI;
+      const int64_t cj = (int64_t)PB * j;   // the panel's columns in the super-panel buffers
+      // ---- the diagonal block ----
+      if (j == 0 && S > 0) GPTQ_CUDA_TRY(wait(c, aux->col[sb]));   // the super-panel's block column
+      if (j >= 2) {   // panel p - 2's next-column and in-super-panel trailing updates
+        GPTQ_CUDA_TRY(wait(c, aux->next[b2]));
+        GPTQ_CUDA_TRY(wait(c, aux->trail[b2]));
+      }
+      if (panel >= NLI) GPTQ_CUDA_TRY(wait(c, aux->done[b]));   // LI[b] is free again
+      TraceScope ts_d("potrf_inv", "flop", (j > 0 ? 4.0 * nb * nb * PB : 0.0) + 2.0 / 3.0 * nb * nb * nb, c);
+      potrf_inv_kernel<<<1, DT, POTRF_SMEM, c>>>(w.A, ldn, k0, nb, n, w.LIhi[b1], w.LIlo[b1], j > 0 ? k0 - PB : -1,
+                                                 w.LIhi[b], w.LIlo[b], st);
+      GPTQ_LAUNCH_CHECK();
+      GPTQ_CUDA_TRY(cudaEventRecord(aux->diag[b], c));
+      if (rest > 0) {
+        // ---- L21 and the next block column ----
+        GPTQ_CUDA_TRY(wait(o, aux->diag[b]));
+        if (j == 0 && S >= NSUP) {   // the super-panel buffers' previous readers are done
+          GPTQ_CUDA_TRY(wait(o, aux->bulk[sb]));
+          GPTQ_CUDA_TRY(wait(o, aux->inv[sb]));
+        }
+        if (panel == 0) rc = launch_split_tf32(w.A + (int64_t)nb * ldn, rest, nb, ldn, w.Phi, w.Plo, PB, st, o);
+        if (rc == GPTQ_OK)
+          rc = launch_gemm3(nullptr, 0, rest, nb, nb, w.Phi, w.Plo, PB, w.LIhi[b], w.LIlo[b], PB, false, st, o, true,
+                            Lh + (int64_t)(k0 + nb) * SPB + cj, Ll + (int64_t)(k0 + nb) * SPB + cj, SPB,
+                            "prepare_gemm3");
+        if (rc != GPTQ_OK) return rc;
+        GPTQ_CUDA_TRY(cudaEventRecord(aux->l21[b], o));
+        const int nb2 = std::min(PB, rest);
+        if (k0 + nb < se && rest > nb2) {
+          // A(i, p+1) for i >= p + 2; panel p - 1's in-super-panel update reached it first
+          if (j >= 1) GPTQ_CUDA_TRY(wait(o, aux->trail[b1]));
+          const int r2 = k0 + nb + nb2;
+          rc = launch_gemm3(w.A + (int64_t)r2 * ldn + (k0 + nb), ldn, n - r2, nb2, nb, Lh + (int64_t)r2 * SPB + cj,
+                            Ll + (int64_t)r2 * SPB + cj, SPB, Lh + (int64_t)(k0 + nb) * SPB + cj,
+                            Ll + (int64_t)(k0 + nb) * SPB + cj, SPB, false, st, o, false, w.Phi, w.Plo, PB,
+                            "prepare_gemm3");
+          if (rc != GPTQ_OK) return rc;
+        }
+        GPTQ_CUDA_TRY(cudaEventRecord(aux->next[b], o));
+        // ---- the super-panel's columns beyond the next block column ----
+        const int c0 = k0 + 2 * PB;
+        if (c0 < se) {
+          GPTQ_CUDA_TRY(wait(t, aux->l21[b]));
+          rc = launch_gemm3(w.A + (int64_t)c0 * ldn + c0, ldn, n - c0, se - c0, nb, Lh + (int64_t)c0 * SPB + cj,
+                            Ll + (int64_t)c0 * SPB + cj, SPB, Lh + (int64_t)c0 * SPB + cj, Ll + (int64_t)c0 * SPB + cj,
+                            SPB, true, st, t, false, nullptr, nullptr, 0, "prepare_gemm3");
+          if (rc != GPTQ_OK) return rc;
+        }
+        GPTQ_CUDA_TRY(cudaEventRecord(aux->trail[b], t));
+      }
+      // ---- the inverse's block column p ----
+      GPTQ_CUDA_TRY(wait(s2, aux->diag[b]));
+      {
+        dim3 blk(32, 8), grd(PB / 32, PB / 32);
+        xt_diag_kernel<<<grd, blk, 0, s2>>>(w.LIhi[b], w.LIlo[b], k0, nb, w.Xt, ldn, w.SXhi + cj, w.SXlo + cj, SPB,
+                                            st);
+        GPTQ_LAUNCH_CHECK();
+      }
+      if (k0 > 0) {
+        float* Xk = w.Xt + k0;
+        rc = launch_split_tf32(Xk, k0, nb, ldn, w.XPhi, w.XPlo, PB, st, s2);
+        if (rc == GPTQ_OK)
+          rc = launch_gemm3(Xk, ldn, k0, nb, nb, w.XPhi, w.XPlo, PB, w.LIhi[b], w.LIlo[b], PB, false, st, s2, true,
+                            w.SXhi + cj, w.SXlo + cj, SPB, "prepare_gemm3");
+        if (rc != GPTQ_OK) return rc;
+      }
+      if (se > k0 + nb) {
+        // rows of the split below this panel's diagonal block inside the super-panel: Xt
+        // is upper triangular there, and the bulk inverse update reads them
+        GPTQ_CUDA_TRY(cudaMemset2DAsync(w.SXhi + (int64_t)(k0 + nb) * SPB + cj, SPB * sizeof(float), 0,
+                                        PB * sizeof(float), se - k0 - nb, s2));
+        GPTQ_CUDA_TRY(cudaMemset2DAsync(w.SXlo + (int64_t)(k0 + nb) * SPB + cj, SPB * sizeof(float), 0,
+                                        PB * sizeof(float), se - k0 - nb, s2));
+      }
+      if (rest > 0) {
+        GPTQ_CUDA_TRY(wait(s2, aux->l21[b]));
+        const int c1 = k0 + nb;
+        if (c1 < se) {   // Xt[:k0+nb, later columns of the super-panel] -= Xt[:, p] . L(later, p)^T
+          rc = launch_gemm3(w.Xt + c1, ldn, k0 + nb, se - c1, nb, w.SXhi + cj, w.SXlo + cj, SPB,
+                            Lh + (int64_t)c1 * SPB + cj, Ll + (int64_t)c1 * SPB + cj, SPB, false, st, s2, false,
+                            nullptr, nullptr, 0, "prepare_gemm3");
+          if (rc != GPTQ_OK) return rc;
+        }
+      }
+      GPTQ_CUDA_TRY(cudaEventRecord(aux->done[b], s2));
+    }
+    if (se >= n) break;
+    // ---- the super-panel's bulk updates (K = se - s0) ----
+    const int se2 = std::min(n, se + SPB);
+    const int K = se - s0;
+    const int sn = (S + 1) % NSUP;
+    GPTQ_CUDA_TRY(cudaEventRecord(aux->lsup[sb], o));
+    // the next super-panel's block column; the previous super-panel's bulk update reached it first
+    if (S >= 1) GPTQ_CUDA_TRY(wait(o, aux->bulk[(S + NSUP - 1) % NSUP]));
+    const float* Lse_h = Lh + (int64_t)se * SPB;
+    const float* Lse_l = Ll + (int64_t)se * SPB;
+    rc = launch_gemm3(w.A + (int64_t)se * ldn + se, ldn, n - se, se2 - se, K, Lse_h, Lse_l, SPB, Lse_h, Lse_l, SPB,
+                      true, st, o, false, nullptr, nullptr, 0, "prepare_gemm3");
+    if (rc != GPTQ_OK) return rc;
+    {
+      const int nbn = std::min(PB, n - se);
+      if (n - se - nbn > 0)
+        rc = launch_split_tf32(w.A + (int64_t)(se + nbn) * ldn + se, n - se - nbn, nbn, ldn, w.Phi, w.Plo, PB, st, o);
+      if (rc != GPTQ_OK) return rc;
+    }
+    GPTQ_CUDA_TRY(cudaEventRecord(aux->col[sn], o));
+    // the rest of the trailing matrix
+    GPTQ_CUDA_TRY(wait(t, aux->lsup[sb]));
+    if (se2 < n) {
+      const float* L2h = Lh + (int64_t)se2 * SPB;
+      const float* L2l = Ll + (int64_t)se2 * SPB;
+      rc = launch_gemm3(w.A + (int64_t)se2 * ldn + se2, ldn, n - se2, n - se2, K, L2h, L2l, SPB, L2h, L2l, SPB, true,
+                        st, t, false, nullptr, nullptr, 0, "prepare_gemm3");
+      if (rc != GPTQ_OK) return rc;
+    }
+    GPTQ_CUDA_TRY(cudaEventRecord(aux->bulk[sb], t));
+    // the inverse beyond the super-panel
+    GPTQ_CUDA_TRY(wait(s2, aux->lsup[sb]));
+    rc = launch_gemm3(w.Xt + se, ldn, se, n - se, K, w.SXhi, w.SXlo, SPB, Lse_h, Lse_l, SPB, false, st, s2, false,
+                      nullptr, nullptr, 0, "prepare_gemm3");
+    if (rc != GPTQ_OK) return rc;
+    GPTQ_CUDA_TRY(cudaEventRecord(aux->inv[sb], s2));
+  }
+  return GPTQ_OK;
+}
+
 }  // namespace
+
+namespace {
+std::atomic<int> g_deferred_min_n{8192};
+}  // namespace
+
+int prepare_set_deferred_min_n(int min_n) {
+  return min_n > 0 ? g_deferred_min_n.exchange(min_n) : g_deferred_min_n.load();
+}
 
 size_t prepare_ws_bytes(int n) {
   const int ldn = ld_of(n);
   const size_t nn = align_up((size_t)n * ldn * sizeof(float), 256);
   const size_t panel = align_up((size_t)n * PB * sizeof(float), 256);
-  return 2 * nn + (6 + 2 * NBUF) * panel + 2 * NBUF * align_up((size_t)PB * PB * 4, 256) +
+  const size_t sup = align_up((size_t)n * SPB * sizeof(float), 256);
+  return 2 * nn + 4 * panel + (2 * NSUP + 2) * sup + 2 * NLI * align_up((size_t)PB * PB * 4, 256) +
          align_up((size_t)n * 8, 256) + align_up((size_t)n * 4, 256) + 256;
 }
 
@@ -942,7 +1144,7 @@ int launch_prepare(const float* H, const double* hdiag, int n, float damp, int d
   cudaStream_t loop_streams[4] = {aux->c, aux->o, aux->t, aux->s};
   GPTQ_CUDA_TRY(cudaEventRecord(aux->fork, s));
   for (cudaStream_t ls : loop_streams) GPTQ_CUDA_TRY(cudaStreamWaitEvent(ls, aux->fork, 0));
-  rc = panel_loop(w, n, ldn, aux, st);
+  rc = n >= g_deferred_min_n.load() ? panel_loop_deferred(w, n, ldn, aux, st) : panel_loop(w, n, ldn, aux, st);
   // the loop's streams join the caller's stream, after an error too
   for (int i = 0; i < 4; ++i) {
     GPTQ_CUDA_TRY(cudaEventRecord(aux->join[i], loop_streams[i]));

@@ -92,6 +92,8 @@ def lib() -> ctypes.CDLL:
     L.gptq_prepare_workspace_size.argtypes = [I]
     L.gptq_prepare.restype = I
     L.gptq_prepare.argtypes = [P, P, I, F, I, P, P, P, P, SZ, P, P]
+    L.gptq_prepare_set_deferred_min_n.restype = I
+    L.gptq_prepare_set_deferred_min_n.argtypes = [I]
     L.gptq_quantize_workspace_size.restype = SZ
     L.gptq_quantize_workspace_size.argtypes = [I, I, I]
     L.gptq_quantize_layer.restype = I
@@ -320,6 +322,12 @@ def prepare(H: torch.Tensor, damp_percent: float = 0.01, desc_act: bool = False,
                               _ptr(out.perm), _ptr(out.dead), _ptr(ws), ws.numel(), _ptr(status), _stream(stream)),
            "gptq_prepare")
     return out
+
+
+def prepare_set_deferred_min_n(min_n: int) -> int:
+    """gptq_prepare_set_deferred_min_n: prepare groups its bulk updates by 512-wide outer
+    panels for n >= min_n (default 8192).  min_n <= 0 only queries.  Returns the previous value."""
+    return int(lib().gptq_prepare_set_deferred_min_n(int(min_n)))
 
 
 # --------------------------------------------------------------------------- #

@@ -144,6 +144,40 @@ def test_prepare_u_and_perm():
     assert np.abs(U - ora.U).max() / np.abs(ora.U).max() < 1e-4
 
 
+@pytest.mark.parametrize("n,act", [(1600, True), (2048, False), (2600, True)])
+def test_prepare_outer_panels_against_the_oracle(n, act):
+    """The deferred form of the preparation (bulk updates grouped by 512-wide outer panels,
+    the form large layers take) forced at sizes the oracle factors in seconds: several outer
+    panels, a partial last one (1600 = 3 x 512 + 64; 2600 = 5 x 512 + 40), the rings of
+    buffers reused.  U element by element against the oracle's own U (fp32 chains of length
+    n: n 2^-23 relative), and against the per-panel form."""
+    dev = _dev()
+    _, x = S.small_case(8, n, 2 * n, seed=n)
+    H64 = O.hessian(x)
+    Ht = torch.from_numpy(H64.astype(np.float32)).to(dev)
+    hd = torch.from_numpy(np.diag(H64).copy()).to(dev)
+    ora = O.prepare(H64, 0.01, act)
+    old = G.prepare_set_deferred_min_n(1)
+    try:
+        pd = G.prepare(Ht, 0.01, act, hd)
+        torch.cuda.synchronize()
+    finally:
+        G.prepare_set_deferred_min_n(old)
+    pp = G.prepare(Ht, 0.01, act, hd)       # the per-panel form (n below the default threshold)
+    G.raise_on_status(pd.status, "prepare (outer panels)")
+    G.raise_on_status(pp.status, "prepare (panels)")
+    assert np.array_equal(pd.perm.cpu().numpy(), ora.perm)
+    Ud = pd.U.cpu().numpy().astype(np.float64)
+    Up = pp.U.cpu().numpy().astype(np.float64)
+    assert np.all(np.tril(Ud, -1) == 0) and np.all(np.diag(Ud) > 0)
+    scale = np.abs(ora.U).max()
+    err_d = np.abs(Ud - ora.U).max() / scale
+    err_p = np.abs(Up - ora.U).max() / scale
+    print(f"n={n}: |U - U_oracle| / max|U|: outer panels {err_d:.3g}, panels {err_p:.3g} (bound {n * 2.0 ** -23:.3g})")
+    assert err_d <= n * 2.0 ** -23
+    assert np.abs(Ud - Up).max() / scale <= n * 2.0 ** -23
+
+
 @pytest.mark.parametrize("act", [False, True])
 def test_dead_inputs(act):
     # features whose activations are all zero: H_ii = 0, so the column is dead (unit
