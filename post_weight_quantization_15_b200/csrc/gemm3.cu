@@ -560,6 +560,262 @@ gemm3p_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, 
   }
 }
 
+// ---------------------------------------------------------------------------
+// The persistent form on CTA pairs (cta_group::2): a cluster of two CTAs on two SMs
+// computes 256 x 256 tiles.  Each CTA loads its own 128 rows of A and its half (128
+// rows) of B; the even CTA (the leader) issues tcgen05.mma.cta_group::2 kind::tf32
+// M = 256, N = 256, K = 8, which reads both CTAs' shared memory at the same offsets
+// and leaves each CTA's 128 rows of the accumulator in its own TMEM.  Per flop each
+// CTA loads two thirds of the operand bytes of the 128 x 256 form.  Otherwise as
+// gemm3p_kernel: the stage ring (five 32 KB stages of 16-deep K slices), the chunk
+// counter and the two TMEM accumulators run on across tiles, and each CTA's eight
+// epilogue warps update its 128 rows of C.
+// Protocol (that of the Hessian's pair kernel; every wait bounded):
+//   full[s]      leader only: the leader's producer arrives with both CTAs' bytes;
+//                both producers' loads complete on it.
+//   empty[s]     both CTAs, count 1: the leader's commit reaches both.
+//   acc_full[b]  both CTAs, count 1: a commit to both after a chunk's MMAs.
+//   acc_empty[b] leader only, 2 x P_EPI arrivals (the peer's through the cluster address).
+//   drain        leader: every MMA complete before teardown.
+// A cluster barrier after the barriers' initialisation and another before TMEM is
+// freed.  No load uses cluster multicast.
+// ---------------------------------------------------------------------------
+constexpr int Q_ST = 5;
+constexpr int Q_ATILE = GM * PK * 4;             // 8 KB: this CTA's 128 rows of A (hi or lo)
+constexpr int Q_BTILE = (PN / 2) * PK * 4;       // 8 KB: this CTA's 128 rows of B (hi or lo)
+constexpr uint32_t Q_IDESC = tc::idesc_f32acc(2, 2 * GM, PN);
+
+struct GemmQSmem {
+  uint8_t ahi[Q_ST][Q_ATILE];
+  uint8_t alo[Q_ST][Q_ATILE];
+  uint8_t bhi[Q_ST][Q_BTILE];
+  uint8_t blo[Q_ST][Q_BTILE];
+  float tr[P_EPI][32 * P_LDT];
+  uint64_t full[Q_ST];
+  uint64_t empty[Q_ST];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int skip;
+};
+constexpr size_t GEMMQ_SMEM = sizeof(GemmQSmem) + 1024;
+
+// Pair tile t -> (ti, tj) over 256 x 256 tiles.  lower: only tiles that reach the lower
+// triangle (the diagonal starts top left), tj <= ti, row by row.
+__device__ __forceinline__ void gemmq_tile(int t, int tiles_n, bool lower, int& ti, int& tj) {
+  if (!lower) { ti = t / tiles_n; tj = t % tiles_n; return; }
+  ti = 0;
+  for (;;) {
+    const int cnt = min(ti + 1, tiles_n);
+    if (t < cnt) break;
+    t -= cnt;
+    ++ti;
+  }
+  tj = t;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
+gemm3pp_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, int K, int lower, int tiles,
+               int tiles_n, int32_t* st) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // offset arithmetic on the shared array keeps every access a shared-memory one (and
+  // gives both CTAs the same offsets)
+  GemmQSmem& S = *reinterpret_cast<GemmQSmem*>(smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = tc::cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
+  const int kblocks = (int)cdiv(K, PK);
+  const int nchunks = (int)cdiv(kblocks, P_CHUNK_KB);      // 128-deep chunks per tile
+  const uint32_t stage_tx = 2u * 2u * (uint32_t)(Q_ATILE + Q_BTILE);   // both CTAs, hi and lo
+
+  if (threadIdx.x == 0) {
+    S.skip = has_error(st) ? 1 : 0;
+    S.abort = 0;
+    for (int s2 = 0; s2 < Q_ST; ++s2) { tc::mbar_init(&S.full[s2], 1); tc::mbar_init(&S.empty[s2], 1); }
+    for (int b = 0; b < 2; ++b) { tc::mbar_init(&S.acc_full[b], 1); tc::mbar_init(&S.acc_empty[b], 2 * P_EPI); }
+    tc::mbar_init(&S.drain, 1);
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) tc::tmem_alloc_pair<512>(&S.tmem_base);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::cluster_sync();                            // both CTAs' barriers exist before any remote signal
+  tc::tc_fence_after();
+  const uint32_t taddr = S.tmem_base;
+  // (if the two CTAs disagree here, the waiting side's bounded waits run out)
+  const bool skip = S.skip != 0;
+  volatile int* abort_flag = &S.abort;
+  int armed[Q_ST] = {};
+  bool mma_committed = false;
+
+  if (!skip) {
+    if (warp == 0 && lane == 0) {
+      // ---------------- producer (both CTAs) ----------------
+      int q = 0;                                           // stage counter over all tiles
+      for (int t = pair; t < tiles && !*abort_flag; t += npairs) {
+        int ti, tj;
+        gemmq_tile(t, tiles_n, lower != 0, ti, tj);
+        const int a_row = ti * 2 * GM + (int)rank * GM;
+        const int b_row = tj * PN + (int)rank * (PN / 2);
+        for (int kb = 0; kb < kblocks; ++kb, ++q) {
+          const int s2 = q % Q_ST;
+          const uint32_t ph = (uint32_t)(q / Q_ST) & 1u;
+          if (!tc::mbar_wait(&S.empty[s2], ph ^ 1u, abort_flag)) break;
+          if (leader) tc::mbar_arrive_expect_tx(&S.full[s2], stage_tx);
+          tc::tma_load_2d_pair(S.ahi[s2], &maps.ahi, &S.full[s2], kb * PK, a_row);
+          tc::tma_load_2d_pair(S.alo[s2], &maps.alo, &S.full[s2], kb * PK, a_row);
+          tc::tma_load_2d_pair(S.bhi[s2], &maps.bhi, &S.full[s2], kb * PK, b_row);
+          tc::tma_load_2d_pair(S.blo[s2], &maps.blo, &S.full[s2], kb * PK, b_row);
+          ++armed[s2];
+        }
+      }
+    } else if (warp == 1 && lane == 0 && leader) {
+      // ---------------- MMA issuer (leader) ----------------
+      int q = 0, g = 0;                                    // stage and chunk counters over all tiles
+      for (int t = pair; t < tiles && !*abort_flag; t += npairs) {
+        int kb = 0;
+        for (int c = 0; c < nchunks && !*abort_flag; ++c, ++g) {
+          const int buf = g & 1;
+          if (!tc::mbar_wait(&S.acc_empty[buf], ((uint32_t)(g >> 1) & 1u) ^ 1u, abort_flag)) break;
+          tc::tc_fence_after();
+          const uint32_t dacc = taddr + buf * PN;
+          const int kb_end = min(kblocks, (c + 1) * P_CHUNK_KB);
+          bool first = true;
+          for (; kb < kb_end; ++kb, ++q) {
+            const int s2 = q % Q_ST;
+            const uint32_t ph = (uint32_t)(q / Q_ST) & 1u;
+            if (!tc::mbar_wait(&S.full[s2], ph, abort_flag)) break;
+            tc::tc_fence_after();
+            const uint32_t ah = tc::smem_u32(S.ahi[s2]), al = tc::smem_u32(S.alo[s2]);
+            const uint32_t bh = tc::smem_u32(S.bhi[s2]), bl = tc::smem_u32(S.blo[s2]);
+#pragma unroll
+            for (int kk = 0; kk < PK / 8; ++kk) {
+              const uint32_t o = kk * 32;
+              tc::mma_tf32_pair(dacc, tc::sdesc_k_sw64(al + o), tc::sdesc_k_sw64(bh + o), Q_IDESC, !first);
+              tc::mma_tf32_pair(dacc, tc::sdesc_k_sw64(ah + o), tc::sdesc_k_sw64(bl + o), Q_IDESC, true);
+              tc::mma_tf32_pair(dacc, tc::sdesc_k_sw64(ah + o), tc::sdesc_k_sw64(bh + o), Q_IDESC, true);
+              first = false;
+            }
+            tc::mma_commit_pair_both(&S.empty[s2]);
+          }
+          if (*abort_flag) break;
+          tc::mma_commit_pair_both(&S.acc_full[buf]);
+        }
+      }
+      tc::mma_commit_pair_local(&S.drain);
+      mma_committed = true;
+      if (!*abort_flag) drain_wait(&S.drain, 0);
+    } else if (warp >= 2) {
+      // ---------------- epilogue (both CTAs) ----------------
+      const int qq = warp & 3;                   // TMEM lane quarter this warp may access
+      const int hc = (warp - 2) >> 2;            // which 128 of the 256 columns
+      const uint32_t lane_base = (uint32_t)(qq * 32) << 16;
+      const uint32_t acc_empty_leader[2] = {tc::map_to_cta(tc::smem_u32(&S.acc_empty[0]), 0),
+                                            tc::map_to_cta(tc::smem_u32(&S.acc_empty[1]), 0)};
+      int g = 0;
+      bool ok = true;
+      for (int t = pair; t < tiles && ok; t += npairs) {
+        int ti, tj;
+        gemmq_tile(t, tiles_n, lower != 0, ti, tj);
+        float acc[128];
+#pragma unroll
+        for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+        for (int c = 0; c < nchunks; ++c, ++g) {
+          const int buf = g & 1;
+          int ready = 0;
+          if (lane == 0) ready = tc::mbar_wait(&S.acc_full[buf], (uint32_t)(g >> 1) & 1u, abort_flag) && !*abort_flag;
+          ready = __shfl_sync(0xffffffffu, ready, 0);
+          if (!ready) { ok = false; break; }
+          tc::tc_fence_after();
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            float v[32];
+            tc::tmem_ld_32x32b_x32(taddr + lane_base + buf * PN + hc * 128 + c4 * 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[c4 * 32 + i] += v[i];
+          }
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive_cluster(acc_empty_leader[buf]);   // the MMAs may reuse it now
+        }
+        if (!ok) break;
+        // this CTA's rows [row0, row0 + 32) and columns [col0, col0 + 128), turned through
+        // the warp's staging tile 32 columns at a time (as in gemm3p_kernel)
+        const int row0 = ti * 2 * GM + (int)rank * GM + qq * 32;
+        const int col0 = tj * PN + hc * 128;
+        float* tile = S.tr[warp - 2];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int col = col0 + c4 * 32 + lane;
+          __syncwarp();
+          if (!out.store) {
+#pragma unroll 1
+            for (int rr = 0; rr < 32; ++rr) {
+              const int r = row0 + rr;
+              if (r < M && col < N)
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(tc::smem_u32(tile + rr * P_LDT + lane)),
+                             "l"(out.C + (int64_t)r * out.ldc + col)
+                             : "memory");
+            }
+            asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+          }
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float* e = tile + lane * P_LDT + i;
+            *e = out.store ? acc[c4 * 32 + i] : *e - acc[c4 * 32 + i];
+          }
+          __syncwarp();
+          if (col < N) {
+#pragma unroll 1
+            for (int rr = 0; rr < 32; ++rr) {
+              const int r = row0 + rr;
+              if (r >= M) break;
+              const float x = tile[rr * P_LDT + lane];
+              if (out.C) out.C[(int64_t)r * out.ldc + col] = x;
+              if (out.Chi != nullptr) {
+                const float h = tf32_hi(x);
+                out.Chi[(int64_t)r * out.ldh + col] = h;
+                out.Clo[(int64_t)r * out.ldh + col] = x - h;
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // ---------------- teardown ----------------
+  tc::tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    if (leader && warp == 0 && lane == 0) {
+      // the leader's full barriers count both CTAs' bytes: bounded drain of its armed phases
+      for (int s2 = 0; s2 < Q_ST; ++s2)
+        if (armed[s2] > 0) drain_wait(&S.full[s2], (uint32_t)(armed[s2] - 1) & 1u);
+    }
+    if (warp == 1 && lane == 0 && mma_committed) drain_wait(&S.drain, 0);
+    if (threadIdx.x == 0) set_error(st, GPTQ_ERR_TIMEOUT, blockIdx.x, STAGE_TRAILING);
+    // the peer's loads complete on the leader's barriers, which the peer cannot wait on:
+    // give copies in flight a fixed, bounded time before either CTA leaves
+    if (threadIdx.x == 0) {
+      const uint64_t t0 = tc::globaltimer();
+      while (tc::globaltimer() - t0 < 20000000ull) {
+      }
+    }
+    __syncthreads();
+  }
+  tc::cluster_sync();                            // neither CTA leaves while the other may touch its memory
+  tc::tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tc::tmem_dealloc_pair<512>(taddr);
+  }
+}
+
 // hi = x with the low 13 mantissa bits cleared, lo = x - hi.
 __global__ void split_tf32_kernel(const float* X, int rows, int cols, int ldx, float* hi, float* lo, int ldo,
                                   const int32_t* st) {
@@ -642,6 +898,37 @@ int launch_gemm3p(const GemmOut& out, int M, int N, int K, const float* Ahi, con
   return GPTQ_OK;
 }
 
+int launch_gemm3pp(const GemmOut& out, int M, int N, int K, const float* Ahi, const float* Alo, int lda,
+                   const float* Bhi, const float* Blo, int ldb, bool lower, int64_t tiles, int32_t* st,
+                   cudaStream_t s) {
+  GemmMaps maps;
+  int rc = make_tmap_2d(&maps.ahi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Ahi, (uint64_t)K, (uint64_t)M,
+                        (uint64_t)lda * 4, PK, GM, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (rc == GPTQ_OK)
+    rc = make_tmap_2d(&maps.alo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Alo, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 4,
+                      PK, GM, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (rc == GPTQ_OK)
+    rc = make_tmap_2d(&maps.bhi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Bhi, (uint64_t)K, (uint64_t)N, (uint64_t)ldb * 4,
+                      PK, PN / 2, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (rc == GPTQ_OK)
+    rc = make_tmap_2d(&maps.blo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Blo, (uint64_t)K, (uint64_t)N, (uint64_t)ldb * 4,
+                      PK, PN / 2, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (rc != GPTQ_OK) return rc;
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                 cudaSuccess)
+      return GPTQ_ERR_CUDA;
+  }
+  const int pairs = (int)std::min<int64_t>(tiles, sms / 2);
+  GPTQ_CUDA_TRY(cudaFuncSetAttribute(gemm3pp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GEMMQ_SMEM));
+  gemm3pp_kernel<<<2 * pairs, P_THREADS, GEMMQ_SMEM, s>>>(maps, out, M, N, K, lower ? 1 : 0, (int)tiles,
+                                                           (int)cdiv(N, PN), st);
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
 }  // namespace
 
 int launch_split_tf32(const float* X, int rows, int cols, int ldx, float* hi, float* lo, int ldo,
@@ -669,6 +956,15 @@ int launch_gemm3(float* C, int ldc, int M, int N, int K, const float* Ahi, const
     wide_tiles = 0;
     for (int64_t ti = 0; ti < tm; ++ti) wide_tiles += std::min(ti / 2 + 1, tnw);
   }
+  // Two waves of 256 x 256 tiles on the CTA pairs (148 on 74 pairs): the pair form
+  const int64_t tqm = (int64_t)cdiv(M, 2 * GM);
+  int64_t pair_tiles = tqm * tnw;
+  if (lower) {
+    pair_tiles = 0;
+    for (int64_t ti = 0; ti < tqm; ++ti) pair_tiles += std::min(ti + 1, tnw);
+  }
+  if (N >= PN && pair_tiles >= 148)
+    return launch_gemm3pp(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, pair_tiles, st, s);
   if (N >= PN && wide_tiles >= 296)
     return launch_gemm3p(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, st, s);
   if (K > CHUNK_KB * GK) return launch_gemm3_t<128>(out, M, N, K, Ahi, Alo, lda, Bhi, Blo, ldb, lower, st, s);
