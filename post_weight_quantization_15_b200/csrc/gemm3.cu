@@ -185,6 +185,13 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
     } else if (warp >= 2) {
       const int q = warp & 3;
       const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+      if (!out.store && warp < 6) {   // this warp's rows of C into L2 while the product runs
+        const int r = ti * GM + q * 32 + lane;
+        if (r < M)
+#pragma unroll
+          for (int j = 0; j < GN / 32; ++j)
+            if (tj * GN + 32 * j < N) asm volatile("prefetch.global.L2 [%0];" ::"l"(out.C + (int64_t)r * out.ldc + tj * GN + 32 * j));
+      }
       // chunked: this thread's row of the tile (TMEM lane) in registers
       float acc[Cfg::CHUNKED ? GN : 1];
       int ready = 1;
@@ -331,7 +338,8 @@ gemm3_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, i
 //               registers, releases the accumulator, and at a tile's last chunk
 //               updates its rows of C (C -= acc or C = acc; optionally the split of
 //               the result), 32 columns at a time turned through a 32 x 32 staging
-//               tile so that each access is one coalesced 128-byte row.
+//               tile in 16-byte pieces (update_c_rows); the tile's rows of C are
+//               requested into L2 when the tile starts.
 // K is accumulated in chunks of 128 (as in gemm3_kernel), each from zero.  Every
 // wait is bounded (GPTQ_ERR_TIMEOUT).
 // ---------------------------------------------------------------------------
@@ -345,7 +353,96 @@ constexpr int P_EPI = 8;
 constexpr int P_THREADS = 64 + P_EPI * 32;
 constexpr uint32_t P_IDESC = tc::idesc_f32acc(2, GM, PN);
 
-constexpr int P_LDT = 33;                       // row stride of an epilogue warp's 32 x 32 staging tile
+constexpr int P_LDT = 33;                       // an epilogue warp's staging tile: 32 x 33 floats
+
+// The L2 lines of this warp's rows of C for the tile, requested when the tile starts so
+// that its update at the tile's end reads L2 rather than DRAM.
+__device__ __forceinline__ void prefetch_c_rows(const GemmOut& out, int M, int N, int row0, int col0, int lane) {
+  const int r = row0 + lane;
+  if (out.store || r >= M) return;
+  const float* base = out.C + (int64_t)r * out.ldc + col0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    if (col0 + 32 * j < N) asm volatile("prefetch.global.L2 [%0];" ::"l"(base + 32 * j));
+}
+
+// C -= acc (or C = acc; optionally the TF32 split of the result) for this warp's 32 rows
+// [row0, +32) and 128 columns [col0, +128), acc holding one row per lane.  32 columns at a
+// time go through the warp's 32 x 32 staging tile in 16-byte pieces, piece p of row rr at
+// slot p ^ (rr & 7), so that the global accesses are 16-byte and coalesced (lane = piece)
+// and the combine (lane = row) shares banks at most 4 ways.
+__device__ __forceinline__ void update_c_rows(const GemmOut& out, int M, int N, int row0, int col0,
+                                              const float (&acc)[128], float* tile, int lane) {
+  auto slot = [](int rr, int p) { return rr * 32 + ((p ^ (rr & 7)) << 2); };
+  const bool vec_c = out.C != nullptr && (out.ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(out.C) & 15) == 0;
+  const bool vec_h = out.Chi != nullptr && (out.ldh & 3) == 0 && (reinterpret_cast<uintptr_t>(out.Chi) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(out.Clo) & 15) == 0;
+  const int pr = lane & 7;                     // this lane's piece in the coalesced passes
+#pragma unroll
+  for (int c4 = 0; c4 < 4; ++c4) {             // unrolled: acc stays in registers
+    const int colb = col0 + c4 * 32;
+    __syncwarp();
+    if (!out.store) {
+#pragma unroll 1
+      for (int it = 0; it < 8; ++it) {
+        const int rr = it * 4 + (lane >> 3);
+        const int r = row0 + rr, col = colb + 4 * pr;
+        float* dst = tile + slot(rr, pr);
+        if (vec_c && r < M && col + 3 < N) {
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)),
+                       "l"(out.C + (int64_t)r * out.ldc + col)
+                       : "memory");
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = (r < M && col + e < N) ? out.C[(int64_t)r * out.ldc + col + e] : 0.f;
+        }
+      }
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    }
+    __syncwarp();
+    // the row owner combines its 32 values
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      float4* e = reinterpret_cast<float4*>(tile + slot(lane, p));
+      const float* a = acc + c4 * 32 + 4 * p;
+      float4 x = *e;
+      if (out.store) x = make_float4(a[0], a[1], a[2], a[3]);
+      else x = make_float4(x.x - a[0], x.y - a[1], x.z - a[2], x.w - a[3]);
+      *e = x;
+    }
+    __syncwarp();
+#pragma unroll 1
+    for (int it = 0; it < 8; ++it) {
+      const int rr = it * 4 + (lane >> 3);
+      const int r = row0 + rr, col = colb + 4 * pr;
+      if (r >= M || col >= N) continue;
+      const float4 x = *reinterpret_cast<const float4*>(tile + slot(rr, pr));
+      const float xe[4] = {x.x, x.y, x.z, x.w};
+      if (out.C) {
+        float* d = out.C + (int64_t)r * out.ldc + col;
+        if (vec_c && col + 3 < N) *reinterpret_cast<float4*>(d) = x;
+        else
+#pragma unroll
+          for (int e = 0; e < 4; ++e) if (col + e < N) d[e] = xe[e];
+      }
+      if (out.Chi != nullptr) {
+        float h[4], l[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) { h[e] = tf32_hi(xe[e]); l[e] = xe[e] - h[e]; }
+        float* dh = out.Chi + (int64_t)r * out.ldh + col;
+        float* dl = out.Clo + (int64_t)r * out.ldh + col;
+        if (vec_h && col + 3 < N) {
+          *reinterpret_cast<float4*>(dh) = make_float4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<float4*>(dl) = make_float4(l[0], l[1], l[2], l[3]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (col + e < N) { dh[e] = h[e]; dl[e] = l[e]; }
+        }
+      }
+    }
+  }
+}
 
 struct GemmPSmem {
   uint8_t bhi[PST][P_BTILE];
@@ -471,6 +568,10 @@ gemm3p_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, 
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
         int ti, tj;
         gemmp_tile(t, tiles_n, lower != 0, ti, tj);
+        // this warp's rows [row0, row0 + 32) and columns [col0, col0 + 128) of C
+        const int row0 = ti * GM + qq * 32;
+        const int col0 = tj * PN + hc * 128;
+        prefetch_c_rows(out, M, N, row0, col0, lane);
         float acc[128];
 #pragma unroll
         for (int i = 0; i < 128; ++i) acc[i] = 0.f;
@@ -493,52 +594,7 @@ gemm3p_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N, 
           if (lane == 0) tc::mbar_arrive(&S.acc_empty[buf]);   // the MMAs may reuse it now
         }
         if (!ok) break;
-        // C's rows [row0, row0 + 32) and columns [col0, col0 + 128): the registers hold one
-        // row per lane; each 32-column slice turns through the warp's staging tile so that
-        // every access to C (and to its split) is one row of 32 consecutive floats
-        const int row0 = ti * GM + qq * 32;
-        const int col0 = tj * PN + hc * 128;
-        float* tile = S.tr[warp - 2];
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {          // unrolled: acc stays in registers
-          const int col = col0 + c4 * 32 + lane;
-          __syncwarp();
-          if (!out.store) {
-            // C's 32 x 32 slice into the tile: lane l copies column col of every row, all
-            // the copies in flight at once, no registers
-#pragma unroll 1
-            for (int rr = 0; rr < 32; ++rr) {
-              const int r = row0 + rr;
-              if (r < M && col < N)
-                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(tc::smem_u32(tile + rr * P_LDT + lane)),
-                             "l"(out.C + (int64_t)r * out.ldc + col)
-                             : "memory");
-            }
-            asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-          }
-          __syncwarp();
-          // the row owner combines its 32 values
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float* e = tile + lane * P_LDT + i;
-            *e = out.store ? acc[c4 * 32 + i] : *e - acc[c4 * 32 + i];
-          }
-          __syncwarp();
-          if (col < N) {
-#pragma unroll 1
-            for (int rr = 0; rr < 32; ++rr) {
-              const int r = row0 + rr;
-              if (r >= M) break;
-              const float x = tile[rr * P_LDT + lane];
-              if (out.C) out.C[(int64_t)r * out.ldc + col] = x;
-              if (out.Chi != nullptr) {
-                const float h = tf32_hi(x);
-                out.Chi[(int64_t)r * out.ldh + col] = h;
-                out.Clo[(int64_t)r * out.ldh + col] = x - h;
-              }
-            }
-          }
-        }
+        update_c_rows(out, M, N, row0, col0, acc, S.tr[warp - 2], lane);
       }
     }
   }
@@ -720,6 +776,10 @@ gemm3pp_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N,
       for (int t = pair; t < tiles && ok; t += npairs) {
         int ti, tj;
         gemmq_tile(t, tiles_n, lower != 0, ti, tj);
+        // this CTA's and warp's rows [row0, row0 + 32) and columns [col0, col0 + 128) of C
+        const int row0 = ti * 2 * GM + (int)rank * GM + qq * 32;
+        const int col0 = tj * PN + hc * 128;
+        prefetch_c_rows(out, M, N, row0, col0, lane);
         float acc[128];
 #pragma unroll
         for (int i = 0; i < 128; ++i) acc[i] = 0.f;
@@ -742,48 +802,7 @@ gemm3pp_kernel(const __grid_constant__ GemmMaps maps, GemmOut out, int M, int N,
           if (lane == 0) tc::mbar_arrive_cluster(acc_empty_leader[buf]);   // the MMAs may reuse it now
         }
         if (!ok) break;
-        // this CTA's rows [row0, row0 + 32) and columns [col0, col0 + 128), turned through
-        // the warp's staging tile 32 columns at a time (as in gemm3p_kernel)
-        const int row0 = ti * 2 * GM + (int)rank * GM + qq * 32;
-        const int col0 = tj * PN + hc * 128;
-        float* tile = S.tr[warp - 2];
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const int col = col0 + c4 * 32 + lane;
-          __syncwarp();
-          if (!out.store) {
-#pragma unroll 1
-            for (int rr = 0; rr < 32; ++rr) {
-              const int r = row0 + rr;
-              if (r < M && col < N)
-                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(tc::smem_u32(tile + rr * P_LDT + lane)),
-                             "l"(out.C + (int64_t)r * out.ldc + col)
-                             : "memory");
-            }
-            asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-          }
-          __syncwarp();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float* e = tile + lane * P_LDT + i;
-            *e = out.store ? acc[c4 * 32 + i] : *e - acc[c4 * 32 + i];
-          }
-          __syncwarp();
-          if (col < N) {
-#pragma unroll 1
-            for (int rr = 0; rr < 32; ++rr) {
-              const int r = row0 + rr;
-              if (r >= M) break;
-              const float x = tile[rr * P_LDT + lane];
-              if (out.C) out.C[(int64_t)r * out.ldc + col] = x;
-              if (out.Chi != nullptr) {
-                const float h = tf32_hi(x);
-                out.Chi[(int64_t)r * out.ldh + col] = h;
-                out.Clo[(int64_t)r * out.ldh + col] = x - h;
-              }
-            }
-          }
-        }
+        update_c_rows(out, M, N, row0, col0, acc, S.tr[warp - 2], lane);
       }
     }
   }
