@@ -478,7 +478,23 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tp
     }
   };
   if (kp >= 0) fetch(0);
-  load_diag_block(A, lda, k0, nb, Ls, tid);
+  // The diagonal block: for a full panel, 16-byte asynchronous copies that land while the
+  // prologue's products run (the block is first read after them).  Its upper triangle is
+  // copied as it lies in A (never written there): every reader of the block masks or
+  // skips it (the Cholesky keeps k <= row; the solves and products read the lower part).
+  // A partial last panel takes the masked load with the identity past nb.
+  const bool async_diag = nb == PB && (lda & 3) == 0;
+  if (async_diag) {
+    for (int idx = tid; idx < PB * PB / 4; idx += DT) {
+      const int r = idx / (PB / 4), c = 4 * (idx % (PB / 4));
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(Ls + r * LDL + c)),
+                   "l"(A + (int64_t)(k0 + r) * lda + k0 + c)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  } else {
+    load_diag_block(A, lda, k0, nb, Ls, tid);
+  }
   if (kp >= 0) {
     if (tid == 0) {
       for (int i = 0; i < 6; ++i) tc::mbar_init(&pbar[i], 1);
@@ -569,6 +585,7 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tp
       if (!*fail) tc::mma_commit(&pbar[4]);
       wait_bar(&pbar[4], done_parity);
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");   // this thread's copies of the diagonal block
     __syncthreads();
     tc::tc_fence_after();
     if (warp < 4 && !*fail) {
@@ -603,6 +620,7 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tp
     }
     if (*fail) return;
   }
+  asm volatile("cp.async.wait_all;" ::: "memory");     // (the first panel's block: no prologue)
   // T starts at zero
   for (int idx = tid; idx < PB * PB / 4; idx += DT) {
     const int r = idx / (PB / 4), c = 4 * (idx % (PB / 4));
