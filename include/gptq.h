@@ -186,6 +186,24 @@ GPTQ_API int gptq_prepare(const float* H, const double* hdiag, int n, float damp
 GPTQ_API int gptq_prepare_set_deferred_min_n(int min_n);
 
 /*
+ * gptq_set_graph_replay - whether gptq_prepare and gptq_quantize_layer(s) replay CUDA
+ * graphs.
+ *
+ * Each of those calls enqueues a chain of small dependent launches on several
+ * streams.  When replay is on (the default), the second call with exactly the same
+ * arguments (every pointer, size and setting, on the same device) captures the call's
+ * launches as a CUDA graph (a one-time host cost of milliseconds), and later calls
+ * with those arguments replay it: the same kernels on the same data, their
+ * cross-stream dependencies turned into graph edges, the same results bit for bit.
+ * The data behind the pointers is read when the graph runs.  Calls enqueue launch by
+ * launch the first time, while the timing trace is on, while the caller's stream is
+ * being captured, and once 32 graphs exist (the library keeps them until unload).
+ *   on       1: on; 0: off; < 0: only query.
+ * Returns the previous setting.  Process-wide.
+ */
+GPTQ_API int gptq_set_graph_replay(int on);
+
+/*
  * gptq_quantize_layer - the column sweep, the lazy trailing update and packing.
  *
  * For every column j in processing order ("polydesk.ai/glossaire/gptq",
@@ -428,6 +446,25 @@ typedef struct {
 } gptq_trace_row;
 GPTQ_API int gptq_trace_enable(int on);
 GPTQ_API int gptq_trace_read(gptq_trace_row* rows, int max_rows, int* n_rows);
+
+/*
+ * gptq_trace_read_timeline - the same record, launch by launch instead of aggregated:
+ * per recorded launch (in the order the launches were enqueued) the kernel name, the
+ * stream it went to (an opaque id: launches with equal ids ran in order on one
+ * stream) and its start and end in milliseconds from the earliest recorded start
+ * (records of the first record's device only).  Start and end are events recorded
+ * on the launch's stream just before and after it, so a launch that waited for
+ * another stream starts once that wait is over.  Synchronizes every recorded event
+ * and clears the record, like gptq_trace_read (launches beyond max_events are
+ * dropped).  Returns GPTQ_ERR_CUDA if an event could not be read.
+ */
+typedef struct {
+  const char* kernel;
+  uint64_t stream;
+  double start_ms;
+  double end_ms;
+} gptq_trace_event;
+GPTQ_API int gptq_trace_read_timeline(gptq_trace_event* events, int max_events, int* n_events);
 
 /*
  * gptq_probe_fp32_peak - measurement aid (no counterpart on the pages): launches

@@ -50,6 +50,7 @@ __host__ __device__ constexpr size_t align_up(size_t v, size_t a) { return (v + 
 namespace gptq {
 // Host-side count of enqueued kernels (see gptq_kernel_launches).
 void count_launch();
+void count_launches(int64_t delta);   // a replayed graph's kernels (or, negative, a captured graph's)
 }  // namespace gptq
 
 // Host-side: turn a CUDA launch/runtime failure into GPTQ_ERR_CUDA.

@@ -15,6 +15,7 @@ namespace {
 std::atomic<uint64_t> g_launches{0};
 }
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+void count_launches(int64_t delta) { g_launches.fetch_add((uint64_t)delta, std::memory_order_relaxed); }
 }  // namespace gptq
 
 namespace {

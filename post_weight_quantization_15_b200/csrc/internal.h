@@ -2,6 +2,9 @@
 #pragma once
 
 #include <cuda_runtime.h>
+
+#include <cstring>
+#include <functional>
 #include <stdint.h>
 
 #include "../../include/gptq.h"
@@ -9,6 +12,40 @@
 namespace gptq {
 
 // ---- timing trace (gptq_trace_enable): events around one launch on its stream ----
+// ---- Graph replay of a whole stage (graph.cu) ----------------------------------
+// The arguments a stage's launches hold by value, as words.
+struct GraphKey {
+  static constexpr int kWords = 40;
+  uint64_t w[kWords] = {};
+  int len = 0;
+  bool ok = true;   // false: too many words (the stage then runs launch by launch)
+  template <typename T>
+  GraphKey& add(T v) {
+    uint64_t x = 0;
+    static_assert(sizeof(T) <= sizeof(uint64_t), "one word per value");
+    memcpy(&x, &v, sizeof(T));
+    if (len < kWords) w[len++] = x;
+    else ok = false;
+    return *this;
+  }
+  bool operator==(const GraphKey& o) const {
+    if (len != o.len) return false;
+    for (int i = 0; i < len; ++i)
+      if (w[i] != o.w[i]) return false;
+    return true;
+  }
+};
+// Runs enqueue(stream) so that its work is ordered after stream s's and s continues
+// after it.  The second time the same key (and device) comes, the work is captured as
+// a CUDA graph, which later calls with that key replay on a stream of the library:
+// launches that wait on one another across streams become graph edges.  Runs
+// enqueue(s) directly the first time, with the timing trace on, when s is being
+// captured by the caller, when the key does not fit, when the graph cache is full, and
+// when a capture fails.
+int run_graph_cached(const GraphKey& key, cudaStream_t s, const std::function<int(cudaStream_t)>& enqueue);
+
+bool trace_enabled();   // the kernel timing trace is recording
+
 class TraceScope {
  public:
   // kernel and unit are string literals; work is the launch's algorithmic work in unit

@@ -729,11 +729,13 @@ int join_streams(QuantStreams* q, cudaStream_t s) {
   return GPTQ_OK;
 }
 
-int launch_quantize(const WRows& W, int w_dtype, int out, int w_cols, int n, const float* U, const int32_t* perm,
-                    const uint8_t* dead, int bits, int gs, int sym, int block, int32_t* qweight,
-                    uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq,
-                    void* ws, int32_t* st, cudaStream_t s) {
-  (void)block;
+namespace {
+
+// The whole stage enqueued on stream s (and the library's streams, joined back to s).
+int enqueue_quantize(const WRows& W, int w_dtype, int out, int w_cols, int n, const float* U, const int32_t* perm,
+                     const uint8_t* dead, int bits, int gs, int sym, int32_t* qweight, uint16_t* scales,
+                     uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq, void* ws, int32_t* st,
+                     cudaStream_t s) {
   QuantWs w = carve(ws, out, n);
   {
     dim3 blk(32, 8), grd((unsigned)cdiv(n, 128), (unsigned)cdiv(std::max(out, 1), 8));
@@ -807,6 +809,27 @@ int launch_quantize(const WRows& W, int w_dtype, int out, int w_cols, int n, con
     GPTQ_LAUNCH_CHECK();
   }
   return GPTQ_OK;
+}
+
+}  // namespace
+
+// The stage's sweeps and trailing updates are a chain of dependent launches on two
+// streams: replayed as a CUDA graph when the same arguments come again
+// (run_graph_cached).  The key is every argument the launches hold by value.
+int launch_quantize(const WRows& W, int w_dtype, int out, int w_cols, int n, const float* U, const int32_t* perm,
+                    const uint8_t* dead, int bits, int gs, int sym, int block, int32_t* qweight,
+                    uint16_t* scales, uint16_t* zeros, int32_t* g_idx, uint8_t* codes, float* err_sq,
+                    void* ws, int32_t* st, cudaStream_t s) {
+  (void)block;
+  GraphKey key;
+  key.add(2).add(W.count);
+  for (int i = 0; i < W.count; ++i) key.add(W.W[i]).add(W.row0[i]);
+  key.add(W.row0[W.count]).add(w_dtype).add(out).add(w_cols).add(n).add(U).add(perm).add(dead).add(bits).add(gs);
+  key.add(sym).add(qweight).add(scales).add(zeros).add(g_idx).add(codes).add(err_sq).add(ws).add(st);
+  return run_graph_cached(key, s, [&](cudaStream_t strm) {
+    return enqueue_quantize(W, w_dtype, out, w_cols, n, U, perm, dead, bits, gs, sym, qweight, scales, zeros, g_idx,
+                            codes, err_sq, ws, st, strm);
+  });
 }
 
 }  // namespace gptq

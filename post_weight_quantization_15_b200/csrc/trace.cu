@@ -26,6 +26,7 @@ struct Rec {
   double work;
   cudaEvent_t a, b;
   int dev;            // the device the events were created on
+  cudaStream_t s;     // the stream the launch went to
 };
 
 std::atomic<int> g_on{0};
@@ -77,6 +78,8 @@ struct Agg {
 
 }  // namespace
 
+bool trace_enabled() { return g_on.load(std::memory_order_relaxed) != 0; }
+
 TraceScope::TraceScope(const char* kernel, const char* unit, double work, cudaStream_t s)
     : kernel_(kernel), unit_(unit), work_(work), s_(s), a_(nullptr) {
   if (g_on.load(std::memory_order_relaxed) == 0) return;
@@ -100,7 +103,7 @@ TraceScope::~TraceScope() {
   int dev = -1;
   cudaGetDevice(&dev);
   std::lock_guard<std::mutex> lock(g_mu);
-  g_recs.push_back(Rec{kernel_, unit_, work_, static_cast<cudaEvent_t>(a_), b, dev});
+  g_recs.push_back(Rec{kernel_, unit_, work_, static_cast<cudaEvent_t>(a_), b, dev, s_});
 }
 
 }  // namespace gptq
@@ -154,6 +157,41 @@ int gptq_trace_read(gptq_trace_row* rows, int max_rows, int* n_rows) {
     ++k;
   }
   *n_rows = k;
+  return rc;
+}
+
+int gptq_trace_read_timeline(gptq_trace_event* events, int max_events, int* n_events) {
+  if (n_events == nullptr || max_events < 0 || (max_events > 0 && events == nullptr)) return GPTQ_ERR_INVALID_ARG;
+  std::vector<Rec> recs;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    recs.swap(g_recs);
+  }
+  int rc = GPTQ_OK;
+  for (const Rec& r : recs)
+    if (cudaEventSynchronize(r.b) != cudaSuccess) rc = GPTQ_ERR_CUDA;
+  // the origin: the earliest start among the records of the first record's device
+  size_t origin = 0;
+  for (size_t i = 1; i < recs.size(); ++i) {
+    if (recs[i].dev != recs[0].dev) continue;
+    float d = 0.f;
+    if (cudaEventElapsedTime(&d, recs[origin].a, recs[i].a) == cudaSuccess && d < 0.f) origin = i;
+  }
+  int k = 0;
+  for (const Rec& r : recs) {
+    float t0 = 0.f, t1 = 0.f;
+    if (r.dev == recs[origin].dev && k < max_events &&
+        cudaEventElapsedTime(&t0, recs[origin].a, r.a) == cudaSuccess &&
+        cudaEventElapsedTime(&t1, recs[origin].a, r.b) == cudaSuccess) {
+      events[k++] = gptq_trace_event{r.kernel, reinterpret_cast<uint64_t>(r.s), t0, t1};
+    }
+  }
+  for (const Rec& r : recs) {   // the events go back to their device's pool
+    std::lock_guard<std::mutex> lock(g_mu);
+    g_pool[r.dev].push_back(r.a);
+    g_pool[r.dev].push_back(r.b);
+  }
+  *n_events = k;
   return rc;
 }
 

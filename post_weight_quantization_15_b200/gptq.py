@@ -50,6 +50,11 @@ class _TraceRow(ctypes.Structure):
                 ("ms", ctypes.c_double), ("work", ctypes.c_double)]
 
 
+class _TraceEvent(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_char_p), ("stream", ctypes.c_uint64), ("start_ms", ctypes.c_double),
+                ("end_ms", ctypes.c_double)]
+
+
 class GptqError(RuntimeError):
     def __init__(self, code: int, where: str, info: Optional[int] = None):
         self.code = code
@@ -94,6 +99,8 @@ def lib() -> ctypes.CDLL:
     L.gptq_prepare.argtypes = [P, P, I, F, I, P, P, P, P, SZ, P, P]
     L.gptq_prepare_set_deferred_min_n.restype = I
     L.gptq_prepare_set_deferred_min_n.argtypes = [I]
+    L.gptq_set_graph_replay.restype = I
+    L.gptq_set_graph_replay.argtypes = [I]
     L.gptq_quantize_workspace_size.restype = SZ
     L.gptq_quantize_workspace_size.argtypes = [I, I, I]
     L.gptq_quantize_layer.restype = I
@@ -114,6 +121,8 @@ def lib() -> ctypes.CDLL:
     L.gptq_trace_enable.argtypes = [I]
     L.gptq_trace_read.restype = I
     L.gptq_trace_read.argtypes = [ctypes.POINTER(_TraceRow), I, ctypes.POINTER(ctypes.c_int)]
+    L.gptq_trace_read_timeline.restype = I
+    L.gptq_trace_read_timeline.argtypes = [ctypes.POINTER(_TraceEvent), I, ctypes.POINTER(ctypes.c_int)]
     L.gptq_dequantize.restype = I
     L.gptq_dequantize.argtypes = [P, P, P, P, I, I, I, I, I, P, P, P]
     L.gptq_qmatvec_workspace_size.restype = SZ
@@ -158,6 +167,16 @@ def trace_read(max_rows: int = 64) -> dict:
     return {rows[i].kernel.decode(): {"launches": int(rows[i].launches), "ms": float(rows[i].ms),
                                       "work": float(rows[i].work), "unit": rows[i].work_unit.decode()}
             for i in range(n.value)}
+
+
+def trace_read_timeline(max_events: int = 1 << 16) -> list:
+    """Synchronize the recorded events and return [(kernel, stream id, start ms, end ms)] per launch, in
+    enqueue order, times from the earliest recorded start; clears the record."""
+    ev = (_TraceEvent * max_events)()
+    n = ctypes.c_int(0)
+    _check(lib().gptq_trace_read_timeline(ev, max_events, ctypes.byref(n)), "gptq_trace_read_timeline")
+    return [(ev[i].kernel.decode(), int(ev[i].stream), float(ev[i].start_ms), float(ev[i].end_ms))
+            for i in range(n.value)]
 
 
 def probe_fp32_peak(blocks: int, iters: int, out: torch.Tensor, stream=None) -> float:
@@ -328,6 +347,12 @@ def prepare_set_deferred_min_n(min_n: int) -> int:
     """gptq_prepare_set_deferred_min_n: prepare groups its bulk updates by 512-wide outer
     panels for n >= min_n (default 8192).  min_n <= 0 only queries.  Returns the previous value."""
     return int(lib().gptq_prepare_set_deferred_min_n(int(min_n)))
+
+
+def set_graph_replay(on: int) -> int:
+    """gptq_set_graph_replay: prepare and quantize replay a captured CUDA graph for repeated
+    calls with the same arguments (on by default); on < 0 only queries.  Returns the previous value."""
+    return int(lib().gptq_set_graph_replay(int(on)))
 
 
 # --------------------------------------------------------------------------- #

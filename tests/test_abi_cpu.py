@@ -44,6 +44,16 @@ def test_prepare_deferred_threshold_round_trips(L):
     assert G.prepare_set_deferred_min_n(0) == cur
 
 
+def test_graph_replay_switch_round_trips(L):
+    import post_weight_quantization_15_b200 as G
+    cur = G.set_graph_replay(-1)
+    assert cur == 1                          # on by default
+    assert G.set_graph_replay(0) == 1
+    assert G.set_graph_replay(-1) == 0
+    assert G.set_graph_replay(cur) == 0
+    assert G.set_graph_replay(-1) == cur
+
+
 def test_version_and_status_strings(L):
     import post_weight_quantization_15_b200 as G
     assert L.gptq_version() == 1

@@ -144,6 +144,80 @@ def test_prepare_u_and_perm():
     assert np.abs(U - ora.U).max() / np.abs(ora.U).max() < 1e-4
 
 
+@pytest.mark.parametrize("act", [False, True])
+def test_prepare_replayed_as_a_graph(act):
+    """gptq_prepare captures the stage as a CUDA graph the second time it sees the same
+    arguments and replays it afterwards: every replay equals a direct call bit for bit,
+    and a replay reads the buffers' current contents (new H values in the same buffer)."""
+    dev = _dev()
+    n = 1024
+    Hs = []
+    for seed in (11, 12):
+        _, x = S.small_case(8, n, 2 * n, seed=seed)
+        Hs.append(torch.from_numpy(O.hessian(x).astype(np.float32)).to(dev))
+    hd = [torch.diagonal(h).double().contiguous() for h in Hs]
+    def direct(i):        # graph replay off: enqueued launch by launch
+        old = G.set_graph_replay(0)
+        try:
+            p = G.prepare(Hs[i].clone(), 0.01, act, hd[i].clone(), status=G.new_status(dev))
+            torch.cuda.synchronize()
+        finally:
+            G.set_graph_replay(old)
+        return p.U.clone(), p.perm.clone()
+    ref = [direct(0), direct(1)]
+    H = Hs[0].clone()
+    h = hd[0].clone()
+    st = G.new_status(dev)
+    ws = G.workspace(G.lib().gptq_prepare_workspace_size(n), dev)
+    out = None
+    launches = []
+    for call in range(5):
+        src = 0 if call < 3 else 1
+        H.copy_(Hs[src])
+        h.copy_(hd[src])
+        l0 = G.kernel_launches()
+        out = G.prepare(H, 0.01, act, h, status=st, ws=ws, out=out)
+        torch.cuda.synchronize()
+        launches.append(G.kernel_launches() - l0)
+        G.raise_on_status(st, "prepare")
+        assert torch.equal(out.U, ref[src][0]) and torch.equal(out.perm, ref[src][1]), call
+    assert len(set(launches)) == 1   # a replay counts the kernels it runs
+
+
+def test_quantize_replayed_as_a_graph():
+    """The quantize stage is captured as a CUDA graph at the second call with the same
+    arguments: replays equal direct calls bit for bit, with new weights in the same buffer."""
+    dev = _dev()
+    n, out = 1536, 700
+    _, x = S.small_case(8, n, 3000, seed=31)
+    H = torch.from_numpy(O.hessian(x).astype(np.float32)).to(dev)
+    hd = torch.diagonal(H).double().contiguous()
+    p = G.prepare(H, 0.01, True, hd)
+    Ws = [_w_tensor(S.make_w(S.WSpec(out, n, 0.02, "f16", 3, 40 + i)), dev) for i in range(2)]
+    def direct(i):        # graph replay off: enqueued launch by launch
+        old = G.set_graph_replay(0)
+        try:
+            q = G.quantize_layer(Ws[i].clone(), p, 4, 128, True, want_codes=True, want_err=True)
+            torch.cuda.synchronize()
+        finally:
+            G.set_graph_replay(old)
+        return q
+    ref = [direct(0), direct(1)]
+    W = Ws[0].clone()
+    st = G.new_status(dev)
+    ws = G.workspace(G.quantize_workspace_size(out, n, 128), dev)
+    qo = G.alloc_quantized(out, n, 4, 128, True, dev, want_codes=True, want_err=True)
+    for call in range(5):
+        src = 0 if call < 3 else 1
+        W.copy_(Ws[src])
+        p.status = st
+        q = G.quantize_layer(W, p, 4, 128, True, ws=ws, out=qo, want_codes=True, want_err=True)
+        torch.cuda.synchronize()
+        G.raise_on_status(st, "quantize")
+        for name in ("qweight", "scales", "zeros", "g_idx", "codes", "err_sq"):
+            assert torch.equal(getattr(q, name), getattr(ref[src], name)), (call, name)
+
+
 @pytest.mark.parametrize("n,act", [(1600, True), (2048, False), (2600, True)])
 def test_prepare_outer_panels_against_the_oracle(n, act):
     """The deferred form of the preparation (bulk updates grouped by 512-wide outer panels,
@@ -625,6 +699,27 @@ def test_timing_trace_records_every_stage_on_its_stream():
     # with the trace off nothing is recorded
     _run_gpu(W, x, 4, 128, False, True)
     assert G.trace_read() == {}
+
+
+def test_timing_trace_timeline_orders_each_stream():
+    dev = _dev()
+    W, x = S.small_case(256, 1536, 2048, seed=9)
+    G.trace_read()
+    G.trace_enable(True)
+    _run_gpu(W, x, 4, 128, False, True)
+    G.trace_enable(False)
+    tl = G.trace_read_timeline()
+    assert tl and min(e[2] for e in tl) == 0.0
+    assert all(0.0 <= e[2] <= e[3] for e in tl)
+    # the diagonal-block chain: 12 launches on one stream, one after the other
+    chain = [e for e in tl if e[0] == "potrf_inv"]
+    assert len(chain) == 12 and len({e[1] for e in chain}) == 1
+    assert all(a[3] <= b[2] + 1e-3 for a, b in zip(chain, chain[1:]))
+    # the stages run in order: the Hessian before the preparation, the preparation before the sweep
+    hess_end = max(e[3] for e in tl if e[0] == "hessian_tc")
+    assert hess_end <= chain[0][2] + 1e-3
+    assert chain[-1][3] <= min(e[2] for e in tl if e[0] == "sweep") + 1e-3
+    assert G.trace_read_timeline() == []
 
 
 def test_layer_split_over_two_ranks_on_one_device():
