@@ -198,8 +198,11 @@ GPTQ_API int gptq_prepare_set_deferred_min_n(int min_n);
  * The data behind the pointers is read when the graph runs.  Calls enqueue launch by
  * launch the first time, while the timing trace is on, while the caller's stream is
  * being captured, and once 32 graphs exist (the library keeps them until unload).
+ * Replay pays off in loops that call with the same buffers; a caller that allocates
+ * fresh buffers for every call gains nothing from it and pays the captures.
  *   on       1: on; 0: off; < 0: only query.
- * Returns the previous setting.  Process-wide.
+ * Returns the previous setting.  Per host thread: it governs the calls the calling
+ * thread makes (each thread starts with replay on).
  */
 GPTQ_API int gptq_set_graph_replay(int on);
 

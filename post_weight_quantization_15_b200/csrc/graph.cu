@@ -12,7 +12,6 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -33,7 +32,7 @@ struct Entry {
 constexpr size_t kMaxGraphs = 32;
 constexpr size_t kMaxSeen = 64;
 
-std::atomic<int> g_replay{1};
+thread_local int g_replay = 1;   // per host thread: the calls a thread makes
 std::mutex g_mu;
 std::vector<Entry> g_graphs;
 std::vector<std::pair<GraphKey, int>> g_seen;   // keys seen once, oldest first
@@ -65,7 +64,7 @@ int graph_stream(int dev, GraphStream** out) {
 
 int run_graph_cached(const GraphKey& key, cudaStream_t s, const std::function<int(cudaStream_t)>& enqueue) {
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-  if (!key.ok || g_replay.load(std::memory_order_relaxed) == 0 || trace_enabled() ||
+  if (!key.ok || g_replay == 0 || trace_enabled() ||
       cudaStreamIsCapturing(s, &cap) != cudaSuccess ||
       cap != cudaStreamCaptureStatusNone) {
     cudaGetLastError();
@@ -133,5 +132,7 @@ int run_graph_cached(const GraphKey& key, cudaStream_t s, const std::function<in
 }  // namespace gptq
 
 extern "C" int gptq_set_graph_replay(int on) {
-  return on < 0 ? gptq::g_replay.load() : gptq::g_replay.exchange(on ? 1 : 0);
+  const int prev = gptq::g_replay;
+  if (on >= 0) gptq::g_replay = on ? 1 : 0;
+  return prev;
 }

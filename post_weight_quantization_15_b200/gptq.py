@@ -351,7 +351,8 @@ def prepare_set_deferred_min_n(min_n: int) -> int:
 
 def set_graph_replay(on: int) -> int:
     """gptq_set_graph_replay: prepare and quantize replay a captured CUDA graph for repeated
-    calls with the same arguments (on by default); on < 0 only queries.  Returns the previous value."""
+    calls with the same arguments (on by default, per host thread); on < 0 only queries.
+    Returns the previous value."""
     return int(lib().gptq_set_graph_replay(int(on)))
 
 
@@ -667,6 +668,8 @@ def gptq_quantize(W: torch.Tensor, X: torch.Tensor, bits: int = 4, group_size: i
     to the device in token chunks while the Hessian of the previous chunk is formed.
     pad: quantize the layer zero-padded to padded_width(in, group_size) inputs (the
     outputs then describe the padded layer).
+    Every call allocates its buffers, so its calls run without graph replay (see
+    set_graph_replay); loops that reuse buffers call prepare / quantize_layer themselves.
     """
     n = padded_width(X.shape[0], group_size) if pad else X.shape[0]
     host = X.device.type == "cpu"
@@ -679,8 +682,12 @@ def gptq_quantize(W: torch.Tensor, X: torch.Tensor, bits: int = 4, group_size: i
         hessian_accumulate_host(H, X, hdiag, st)
     else:
         hessian_accumulate(H, X, hdiag, st)
-    prep = prepare(H, damp_percent, desc_act, hdiag, st)
-    q = quantize_layer(W, prep, bits, group_size, sym, block, want_codes, want_err)
+    replay = set_graph_replay(0)
+    try:
+        prep = prepare(H, damp_percent, desc_act, hdiag, st)
+        q = quantize_layer(W, prep, bits, group_size, sym, block, want_codes, want_err)
+    finally:
+        set_graph_replay(replay)
     if check:
         raise_on_status(st, "gptq_quantize")
     return q, prep, H
