@@ -277,12 +277,12 @@ def run_reference(args):
     return 0
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one hessian_tc_kernel launch on
-# layer-1024x4096, from one ncu capture of this bench command, valid while the kernel's sources
-# are the ones that were captured (their SHA-256 below); otherwise the traffic is null.
-HESSIAN_TRAFFIC = {"n": 4096, "tokens": 65536, "bytes": 941675008 + 24184064,
-                   "sha256": {"post_weight_quantization_15_b200/csrc/hessian.cu": "4e15e91d4ea22356",
-                              "post_weight_quantization_15_b200/csrc/tc_common.cuh": "7955f242938f18ca"}}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one hessian_pair_kernel launch
+# on layer-1024x4096, from one ncu capture of this bench command, valid while the kernel's
+# sources are the ones that were captured (their SHA-256 below); otherwise the traffic is null.
+HESSIAN_TRAFFIC = {"n": 4096, "tokens": 65536, "bytes": 1008786688 + 26257920,
+                   "sha256": {"post_weight_quantization_15_b200/csrc/hessian.cu": "4ea0a4d9c5f6d896",
+                              "post_weight_quantization_15_b200/csrc/tc_common.cuh": "397409833b5bb824"}}
 
 
 def hessian_traffic(n: int, tokens: int):
