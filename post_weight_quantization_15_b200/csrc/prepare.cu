@@ -518,20 +518,35 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tp
   // the diagonal block's, so that the two latencies overlap.
   constexpr int PF = (PB * 8 + DT - 1) / DT;
   float4 pa[PF], ph[PF], pl[PF];
-  auto fetch = [&](int kc) {
+  auto fetch_a = [&](int kc) {
 #pragma unroll
     for (int u = 0; u < PF; ++u) {
       const int idx = tid + u * DT;
       const int r = idx >> 3, c = kc * 32 + 4 * (idx & 7);
-      pa[u] = ph[u] = pl[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      pa[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (idx < PB * 8 && r < nb) pa[u] = *reinterpret_cast<const float4*>(A + (int64_t)(k0 + r) * lda + kp + c);
+    }
+  };
+  auto fetch_t = [&](int kc) {
+#pragma unroll
+    for (int u = 0; u < PF; ++u) {
+      const int idx = tid + u * DT;
+      const int r = idx >> 3, c = kc * 32 + 4 * (idx & 7);
+      ph[u] = pl[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (idx < PB * 8) {
-        if (r < nb) pa[u] = *reinterpret_cast<const float4*>(A + (int64_t)(k0 + r) * lda + kp + c);
         ph[u] = *reinterpret_cast<const float4*>(Tphi + r * PB + c);
         pl[u] = *reinterpret_cast<const float4*>(Tplo + r * PB + c);
       }
     }
   };
-  if (kp >= 0) fetch(0);
+  // Consecutive launches of the chain are programmatic dependents (launch_potrf_inv): the
+  // next panel's kernel may start once this one has begun and issue what the other streams'
+  // kernels produced (its diagonal block, A(k, k-1)), which are complete when it starts.
+  // T' = L_{k-1,k-1}^-1, the previous launch's output, is read only after
+  // griddepcontrol.wait, which returns once the previous launch has completed and its
+  // writes are visible.  (Launched without the attribute, both instructions do nothing.)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (kp >= 0) fetch_a(0);
   // The diagonal block: for a full panel, 16-byte asynchronous copies that land while the
   // prologue's products run (the block is first read after them).  Its upper triangle is
   // copied as it lies in A (never written there): every reader of the block masks or
@@ -549,6 +564,8 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tp
   } else {
     load_diag_block(A, lda, k0, nb, Ls, tid);
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (kp >= 0) fetch_t(0);
   if (kp >= 0) {
     if (tid == 0) {
       for (int i = 0; i < 6; ++i) tc::mbar_init(&pbar[i], 1);
@@ -587,7 +604,10 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tp
           sw_store4(ob + 49152, r, j, pl[u]);
         }
       }
-      if (kc + 1 < 4) fetch(kc + 1);
+      if (kc + 1 < 4) {
+        fetch_a(kc + 1);
+        fetch_t(kc + 1);
+      }
       fence_proxy_async();
       __syncthreads();
       if (tid == 0 && !*fail) {
@@ -782,6 +802,7 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tp
 
   // output: the TF32 split of T (L_kk itself is not needed later: the trailing
   // steps use L21 and T; the block of Xt comes from this split, off this chain)
+#pragma unroll 4
   for (int idx = tid; idx < PB * PB / 4; idx += DT) {
     const int i = idx / (PB / 4), k = 4 * (idx % (PB / 4));
     const float4 v = *reinterpret_cast<const float4*>(Ts + i * LDL + k);
@@ -851,7 +872,27 @@ __global__ void __launch_bounds__(256) write_u_kernel(const float* Xt, int n, in
   }
 }
 
-// The panel loop runs on four streams.  High priority, so that their small
+// One launch of the diagonal-block chain, as a programmatic dependent of the previous
+// launch on its stream (the kernel orders its reads of the previous launch's output).
+int launch_potrf_inv(const PrepWs& w, int ldn, int k0, int nb, int n, int b1, int kp, int b, int32_t* st,
+                     cudaStream_t c) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(DT);
+  cfg.dynamicSmemBytes = POTRF_SMEM;
+  cfg.stream = c;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  GPTQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, potrf_inv_kernel, (const float*)w.A, ldn, k0, nb, n,
+                                   (const float*)w.LIhi[b1], (const float*)w.LIlo[b1], kp, w.LIhi[b], w.LIlo[b], st));
+  GPTQ_LAUNCH_CHECK();
+  return GPTQ_OK;
+}
+
+// The panel loop runs on four streams.// The panel loop runs on four streams.  High priority, so that their small
 // launches get SMs ahead of the bulk work: the chain of diagonal blocks (one
 // launch per panel), and the rest of each panel's factorization (all rows of
 // L21, and the update of the next block column below its diagonal block).  Low
@@ -937,9 +978,8 @@ int panel_loop(const PrepWs& w, int n, int ldn, AuxStream* aux, int32_t* st) {
     // useful flops: the previous panel's two 128-deep products (when there is one), the
     // block's Cholesky factorization and its triangular inverse
     TraceScope ts_d("potrf_inv", "flop", (panel > 0 ? 4.0 * nb * nb * PB : 0.0) + 2.0 / 3.0 * nb * nb * nb, c);
-    potrf_inv_kernel<<<1, DT, POTRF_SMEM, c>>>(w.A, ldn, k0, nb, n, w.LIhi[b1], w.LIlo[b1],
-                                               panel > 0 ? k0 - PB : -1, w.LIhi[b], w.LIlo[b], st);
-    GPTQ_LAUNCH_CHECK();
+    rc = launch_potrf_inv(w, ldn, k0, nb, n, b1, panel > 0 ? k0 - PB : -1, b, st, c);
+    if (rc != GPTQ_OK) return rc;
     GPTQ_CUDA_TRY(cudaEventRecord(aux->diag[b], c));
     if (rest > 0) {
       // ---- L21 and the next block column ----
@@ -1049,9 +1089,8 @@ int panel_loop_deferred(const PrepWs& w, int n, int ldn, AuxStream* aux, int32_t
       }
       if (panel >= NLI) GPTQ_CUDA_TRY(wait(c, aux->done[b]));   // LI[b] is free again
       TraceScope ts_d("potrf_inv", "flop", (j > 0 ? 4.0 * nb * nb * PB : 0.0) + 2.0 / 3.0 * nb * nb * nb, c);
-      potrf_inv_kernel<<<1, DT, POTRF_SMEM, c>>>(w.A, ldn, k0, nb, n, w.LIhi[b1], w.LIlo[b1], j > 0 ? k0 - PB : -1,
-                                                 w.LIhi[b], w.LIlo[b], st);
-      GPTQ_LAUNCH_CHECK();
+      rc = launch_potrf_inv(w, ldn, k0, nb, n, b1, j > 0 ? k0 - PB : -1, b, st, c);
+      if (rc != GPTQ_OK) return rc;
       GPTQ_CUDA_TRY(cudaEventRecord(aux->diag[b], c));
       if (rest > 0) {
         // ---- L21 and the next block column ----
