@@ -220,6 +220,11 @@ GPTQ_API int gptq_set_graph_replay(int on);
  *
  *   W          [out, n] row-major, dtype w_dtype (F32, F16 or BF16); not modified.
  *   U, perm, dead   from gptq_prepare (perm and dead may be NULL: identity / none).
+ *              With perm NULL the sweep also packs: it writes qweight itself,
+ *              block by block, and the separate packing launch is skipped (the
+ *              same bits; the packing then joins the sweep's dependent chain, which
+ *              measured slower than the separate launch: pass the identity perm
+ *              from gptq_prepare to keep the separate packing).
  *   bits       2, 3, 4 or 8.     group_size 32, 64, 128, or -1 (one group per row).
  *   block      128 (the pages' batch); block % group_size == 0 when group_size > 0.
  *   n % 32 == 0, and n % group_size == 0 when group_size > 0.

@@ -232,15 +232,16 @@ struct SweepShape {
   static constexpr int THREADS = TPR == 32 ? 256 : 128;
   static constexpr int ROWS = THREADS / TPR;     // rows per CTA
   static constexpr int LDE = BLK + 4;            // error row stride (16-byte aligned rows)
-  // two U stages (the block's U, then the near passes alternating), 1/U_jj, errors
-  static constexpr size_t SMEM =
-      2 * (size_t)BLK * LDU * sizeof(float) + BLK * sizeof(float) + (size_t)ROWS * LDE * sizeof(float);
+  // two U stages (the block's U, then the near passes alternating), 1/U_jj, errors, and
+  // the block's codes of the CTA's rows (the fused packing)
+  static constexpr size_t SMEM = 2 * (size_t)BLK * LDU * sizeof(float) + BLK * sizeof(float) +
+                                 (size_t)ROWS * LDE * sizeof(float) + (size_t)ROWS * BLK;
 };
 
 template <int GS, int TPR, bool SYM>
 __global__ void __launch_bounds__(SweepShape<TPR>::THREADS)
 sweep_kernel(float* Wf, int out, int n, int s0, int se, const float* U, float* Ehi, float* Elo,
-             uint8_t* codes_p,
+             uint8_t* codes_p, int32_t* qweight,
              uint16_t* scales, uint16_t* zeros, const float* rows, float* err_sq, int bits, int sym,
              const int32_t* st) {
   using SS = SweepShape<TPR>;
@@ -421,6 +422,37 @@ sweep_kernel(float* Wf, int out, int n, int s0, int se, const float* U, float* E
       *reinterpret_cast<uint2*>(crow) = make_uint2(cw[0], cw[1]);
     } else {
       *reinterpret_cast<uint32_t*>(crow) = cw[0];
+    }
+    if (qweight != nullptr) {   // the codes of the CTA's rows for the fused packing below
+      uint32_t* cs = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(dinv + BLK + SS::ROWS * SS::LDE) +
+                                                 (threadIdx.x / TPR) * BLK + seg * SEG);
+#pragma unroll
+      for (int k = 0; k < SEG / 4; ++k) cs[k] = cw[k];
+    }
+  }
+  // Packing fused into the sweep (identity column order, qweight given): the block's words
+  // of the bit stream (column k at bits k.bits; a 128-column block holds whole words for
+  // every width) straight from the staged codes; word wi of row r goes to
+  // qweight[b0 . bits / 32 + wi][r], consecutive threads on consecutive rows.
+  if (qweight != nullptr) {
+    __syncthreads();
+    const uint8_t* cs = reinterpret_cast<const uint8_t*>(dinv + BLK + SS::ROWS * SS::LDE);
+    const int wpr = bw * bits / 32;
+    const int64_t wbase = (int64_t)b0 * bits / 32;
+    const uint32_t mask = (1u << bits) - 1u;
+    for (int idx = threadIdx.x; idx < SS::ROWS * wpr; idx += blockDim.x) {
+      const int rl = idx % SS::ROWS, wi = idx / SS::ROWS;
+      const int row = blockIdx.x * SS::ROWS + rl;
+      if (row >= out) continue;
+      const int pos0 = wi * 32;
+      const int k_lo = pos0 / bits, k_hi = min((pos0 + 31) / bits, bw - 1);
+      uint64_t acc = 0;
+      for (int k = k_lo; k <= k_hi; ++k) {
+        const uint64_t c = cs[rl * BLK + k] & mask;
+        const int sh = k * bits - pos0;   // negative for a code straddling in from the left
+        acc |= sh >= 0 ? c << sh : c >> -sh;
+      }
+      qweight[(wbase + wi) * out + row] = (int32_t)(uint32_t)acc;
     }
   }
   GPTQ_SWEEP_MARK(3);
@@ -671,8 +703,8 @@ int launch_pack_zeros(const uint16_t* zeros, int groups, int out, int bits, int 
 // The super-blocks of one layer on the two library streams (ordering: see launch_quantize).
 template <typename SweepFn>
 int super_block_loop(QuantStreams* q, const QuantWs& w, int out, int n, const float* U, int bits, int sym,
-                     uint16_t* scales, uint16_t* zeros, float* err_sq, int32_t* st, SweepFn sweep, size_t smem,
-                     int rows_per_cta, int threads) {
+                     int32_t* qweight_fused, uint16_t* scales, uint16_t* zeros, float* err_sq, int32_t* st,
+                     SweepFn sweep, size_t smem, int rows_per_cta, int threads) {
   int rc = GPTQ_OK;
   const int S = (int)cdiv(n, SBK);
   // U[super-block sb rows, the columns after it]^T, split, into B[sb & 1] (on lo)
@@ -693,8 +725,8 @@ int super_block_loop(QuantStreams* q, const QuantWs& w, int out, int n, const fl
     // bytes of the section's work: W in, both error halves and the codes out, U's block
     TraceScope ts_s("sweep", "byte", (double)out * (se - s0) * 13.0 + 4.0 * (se - s0) * (se - s0), q->hi);
     sweep<<<(unsigned)cdiv(out, rows_per_cta), threads, smem, q->hi>>>(w.Wf, out, n, s0, se, U, w.Ehi[b], w.Elo[b],
-                                                                    w.codes_p, scales, zeros, w.rows, err_sq, bits,
-                                                                    sym, st);
+                                                                    w.codes_p, qweight_fused, scales, zeros, w.rows,
+                                                                    err_sq, bits, sym, st);
     GPTQ_LAUNCH_CHECK();
     if (se >= n) break;
     const int kn = std::min(SBK, n - se);   // the next super-block's width
@@ -795,14 +827,20 @@ int enqueue_quantize(const WRows& W, int w_dtype, int out, int w_cols, int n, co
   GPTQ_CUDA_TRY(cudaEventRecord(q->fork, s));
   GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->hi, q->fork, 0));
   GPTQ_CUDA_TRY(cudaStreamWaitEvent(q->lo, q->fork, 0));
-  rc = super_block_loop(q, w, out, n, U, bits, sym, scales, zeros, err_sq, st, sweep, smem, rows_per_cta, threads);
+  // With the identity column order (perm NULL) the sweep writes qweight itself and the
+  // separate packing launch is skipped.
+  int32_t* qweight_fused = perm == nullptr ? qweight : nullptr;
+  rc = super_block_loop(q, w, out, n, U, bits, sym, qweight_fused, scales, zeros, err_sq, st, sweep, smem,
+                        rows_per_cta, threads);
   // both library streams join the caller's stream, after an error too, so that the
   // caller's stream is ordered after everything this call enqueued
   const int jrc = join_streams(q, s);
   if (rc != GPTQ_OK) return rc;
   if (jrc != GPTQ_OK) return jrc;
-  rc = launch_pack(w.codes_p, w.invperm, out, n, n, bits, qweight, st, s);
-  if (rc != GPTQ_OK) return rc;
+  if (qweight_fused == nullptr) {
+    rc = launch_pack(w.codes_p, w.invperm, out, n, n, bits, qweight, st, s);
+    if (rc != GPTQ_OK) return rc;
+  }
   if (codes) {
     dim3 blk(32, 8), grd((unsigned)cdiv(n, 32), (unsigned)cdiv(out, 8));
     codes_out_kernel<<<grd, blk, 0, s>>>(w.codes_p, w.invperm, out, n, codes, st);

@@ -316,7 +316,13 @@ class Prepared:
     perm: torch.Tensor    # int32 [n]
     dead: torch.Tensor    # uint8 [n]
     status: torch.Tensor  # int32 [4]
-    desc_act: bool
+    desc_act: bool        # False: perm is the identity
+
+
+def _perm_arg(prep: "Prepared", fused_pack: bool = False):
+    """The perm argument of the quantize calls: NULL (the identity) selects the packing fused
+    into the sweep; allowed only when the order is the identity (desc_act False)."""
+    return None if (fused_pack and not prep.desc_act) else prep.perm
 
 
 def prepare(H: torch.Tensor, damp_percent: float = 0.01, desc_act: bool = False,
@@ -422,8 +428,11 @@ def _check_quantized(out: QuantizedLayer, o: int, n: int):
 def quantize_layer(W: torch.Tensor, prep: Prepared, bits: int = 4, group_size: int = 128, sym: bool = False,
                    block: int = 128, want_codes: bool = False, want_err: bool = False,
                    ws: Optional[torch.Tensor] = None, out: Optional[QuantizedLayer] = None,
-                   stream=None) -> QuantizedLayer:
+                   stream=None, fused_pack: bool = False) -> QuantizedLayer:
     """Sweep, lazy trailing update and packing of W [out, in] given ``prep`` (n = U's size).
+
+    fused_pack: without act-order, let the sweep write qweight itself instead of a separate
+    packing launch (same bits; measured slower, so off by default).
 
     in == n is the ordinary call.  in < n quantizes W zero-padded to n columns (the
     outputs then describe the padded layer: qweight, g_idx and codes have n columns);
@@ -446,7 +455,7 @@ def quantize_layer(W: torch.Tensor, prep: Prepared, bits: int = 4, group_size: i
         _check_quantized(out, o, n)
     # w_cols < n: W is zero-padded to n columns (gptq_quantize_layer_padded)
     _check(lib().gptq_quantize_layer_padded(_ptr(W), _DTYPE_CODE[W.dtype], o, w_cols, n, _ptr(prep.U),
-                                            _ptr(prep.perm), _ptr(prep.dead), int(bits), int(group_size),
+                                            _ptr(_perm_arg(prep, fused_pack)), _ptr(prep.dead), int(bits), int(group_size),
                                             int(bool(sym)), int(block), _ptr(out.qweight), _ptr(out.scales),
                                             _ptr(out.zeros), _ptr(out.g_idx), _ptr(out.codes), _ptr(out.err_sq),
                                             _ptr(ws), ws.numel(), _ptr(prep.status), _stream(stream)),
@@ -459,8 +468,10 @@ MAX_LAYERS = 8
 
 def quantize_layers(Ws, prep: Prepared, bits: int = 4, group_size: int = 128, sym: bool = False,
                     block: int = 128, want_codes: bool = False, want_err: bool = False,
-                    ws: Optional[torch.Tensor] = None, out: Optional[QuantizedLayer] = None, stream=None):
-    """Several layers that read the same input (share ``prep``), in one call.
+                    ws: Optional[torch.Tensor] = None, out: Optional[QuantizedLayer] = None, stream=None,
+                    fused_pack: bool = False):
+    """Several layers that read the same input (share ``prep``), in one call (fused_pack: as
+    in quantize_layer).
 
     Returns (stacked, views): ``stacked`` is the QuantizedLayer of the layers stacked
     along the outputs, ``views`` one QuantizedLayer per layer whose tensors are views of
@@ -489,7 +500,7 @@ def quantize_layers(Ws, prep: Prepared, bits: int = 4, group_size: int = 128, sy
         _check_quantized(out, o, n)
     ptrs = (ctypes.c_void_p * len(Ws))(*[W.data_ptr() for W in Ws])
     rows = (ctypes.c_int * len(Ws))(*outs)
-    _check(lib().gptq_quantize_layers(ptrs, rows, len(Ws), _DTYPE_CODE[dt], n, _ptr(prep.U), _ptr(prep.perm),
+    _check(lib().gptq_quantize_layers(ptrs, rows, len(Ws), _DTYPE_CODE[dt], n, _ptr(prep.U), _ptr(_perm_arg(prep, fused_pack)),
                                       _ptr(prep.dead), int(bits), int(group_size), int(bool(sym)), int(block),
                                       _ptr(out.qweight), _ptr(out.scales), _ptr(out.zeros), _ptr(out.g_idx),
                                       _ptr(out.codes), _ptr(out.err_sq), _ptr(ws), ws.numel(), _ptr(prep.status),

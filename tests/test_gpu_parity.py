@@ -184,6 +184,36 @@ def test_prepare_replayed_as_a_graph(act):
     assert len(set(launches)) == 1   # a replay counts the kernels it runs
 
 
+@pytest.mark.parametrize("bits,gs,out", [(4, 128, 300), (3, 64, 257), (2, 32, 64), (8, 128, 33), (3, -1, 130),
+                                         (4, 32, 1000)])
+def test_packing_fused_into_the_sweep_matches_the_pack_kernel(bits, gs, out):
+    """Without act-order the sweep can write qweight itself (fused_pack: the perm argument
+    is NULL, the identity); by default the separate pack kernel does.  Same bits."""
+    dev = _dev()
+    n = 1536
+    W, x = S.small_case(out, n, 3000, seed=bits * 100 + out)
+    H = torch.from_numpy(O.hessian(x).astype(np.float32)).to(dev)
+    p = G.prepare(H, 0.01, False)
+    assert torch.equal(p.perm.cpu(), torch.arange(n, dtype=torch.int32))
+    Wt = _w_tensor(W, dev)
+    fused = G.quantize_layer(Wt, p, bits, gs, False, want_codes=True, fused_pack=True)
+    packed = G.quantize_layer(Wt, p, bits, gs, False, want_codes=True)
+    torch.cuda.synchronize()
+    G.raise_on_status(p.status, "fused packing")
+    for name in ("qweight", "scales", "zeros", "g_idx", "codes"):
+        assert torch.equal(getattr(fused, name), getattr(packed, name)), name
+    assert np.array_equal(O.pack(fused.codes.cpu().numpy(), bits).view(np.int32), fused.qweight.cpu().numpy())
+    # the stacked and zero-padded entry points take the same path
+    W2 = _w_tensor(S.make_w(S.WSpec(out, n, 0.02, "f32", 3, 77)), dev)
+    _, (a, b) = G.quantize_layers([Wt, W2], p, bits, gs, False, fused_pack=True)
+    _, (c, d) = G.quantize_layers([Wt, W2], p, bits, gs, False)
+    assert torch.equal(a.qweight, c.qweight) and torch.equal(b.qweight, d.qweight)
+    Wn = Wt[:, : n - 32].contiguous()
+    e = G.quantize_layer(Wn, p, bits, gs, False, fused_pack=True)
+    f = G.quantize_layer(Wn, p, bits, gs, False)
+    assert torch.equal(e.qweight, f.qweight)
+
+
 def test_quantize_replayed_as_a_graph():
     """The quantize stage is captured as a CUDA graph at the second call with the same
     arguments: replays equal direct calls bit for bit, with new weights in the same buffer."""
