@@ -368,8 +368,12 @@ GPTQ_API int gptq_pack_zeros(const uint16_t* zeros, int groups, int out, int bit
  *   reads qweight once, so HBM bandwidth bounds it.  X of dtype x_dtype (F16, BF16 or
  *   F32), row stride ld_x; Y fp32, row stride ld_y (>= out).  xperm: NULL, or int32 [n]
  *   (column k of the packed layer multiplies column xperm[k] of X: the form that
- *   gptq_reorder_groups writes).  Sums in fp32, in an order fixed by the shapes
- *   (deterministic).  ws: >= gptq_qmatvec_workspace_size(M, n, out) bytes, 256-byte
+ *   gptq_reorder_groups writes).  Sums in fp32, in an order fixed by the shapes and
+ *   the data's group layout (deterministic).  With 4-bit codes, M <= 2, F16 / BF16
+ *   activations, integer zero points in [0, 127] and every 32 consecutive columns of a
+ *   block in one group, the products x . (c - z) (exact) are summed on the tensor cores
+ *   (mma.sync, fp32 accumulation, at most 128 columns per accumulation) and scaled in
+ *   fp32; otherwise by fp32 fma.  ws: >= gptq_qmatvec_workspace_size(M, n, out) bytes, 256-byte
  *   aligned (the partial sums of the k splits).  Fastest when the groups of nearby
  *   columns are contiguous (no act-order, or a reordered layer): their scales and zero
  *   points are then staged once per block of columns.

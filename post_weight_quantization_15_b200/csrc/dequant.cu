@@ -18,6 +18,7 @@
 // 32 / bits whole codes).
 #include <algorithm>
 #include <climits>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -99,7 +100,68 @@ constexpr int QMV_UNROLL = 4;         // words in flight per thread
 // staged groups: the range's groups when groups of 64 or more columns are contiguous
 __host__ __device__ constexpr int qmv_maxg(int M) { return qmv_kc(M) / 64 + 1; }
 __host__ __device__ constexpr size_t qmv_smem(int M) {
-  return (size_t)M * qmv_kc(M) * 4 + (size_t)qmv_kc(M) * 4 + 8 * 128 * 4 + (size_t)qmv_maxg(M) * 64 * 16;
+  return (size_t)M * qmv_kc(M) * 4 + (size_t)qmv_kc(M) * 4 + 8 * 128 * 4 + (size_t)qmv_maxg(M) * 64 * 16 +
+         (size_t)M * (qmv_kc(M) + 8) * 2;
+}
+
+// ---------------------------------------------------------------------------
+// The tensor-core form of the product (4-bit codes, fp16 or bf16 activations, a block
+// whose groups are staged and constant over each 32-column tile): per 32 columns and 8
+// outputs, two mma.sync m16n8k16 (fp32 accumulate) of the activations (16 rows, the
+// rows past M zero) with the codes minus the zero points, exact in fp16 / bf16:
+//   lane (g, t) of a warp loads the packed word of columns [8t, 8t + 8) of the tile for
+//   output g of the eight, and its nibble pairs (p, p + 4), p = 0..3, become the pairs
+//   (B + c_p, B + c_{p+4}) by one mask-or with the bits of B (1024 in fp16, 128 in
+//   bf16: c < 16 sits in the mantissa exactly); one packed subtraction of (B + z) leaves
+//   the exact integers c - z.  Pair p feeds the k slots of mma p / 2, b-register p % 2,
+//   so the tile's k slot s holds column perm(s) = 8t + 2h + j + 4i for s = 16h + 8j +
+//   2t + i; the activations are staged in that order, so each product pairs the right
+//   column.  The accumulator is scaled by s (per output) and added into fp32 registers
+//   at every group change and every 128 columns (at most 8 mma per accumulation).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int qmv_tc_slot(int c) {     // the k slot of tile column c
+  const int t = c >> 3, i = (c >> 2) & 1, h = (c >> 1) & 1, j = c & 1;
+  return 16 * h + 8 * j + 2 * t + i;
+}
+
+template <typename TX>
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1);
+template <>
+__device__ __forceinline__ void mma_16816<__half>(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+template <>
+__device__ __forceinline__ void mma_16816<__nv_bfloat16>(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// (B + c_lo, B + c_hi) - (B + z, B + z) as a packed pair, exactly
+template <typename TX>
+__device__ __forceinline__ uint32_t qmv_code_pair(uint32_t bits, uint32_t bz);
+template <>
+__device__ __forceinline__ uint32_t qmv_code_pair<__half>(uint32_t bits, uint32_t bz) {
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&bits), *reinterpret_cast<const __half2*>(&bz));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+template <>
+__device__ __forceinline__ uint32_t qmv_code_pair<__nv_bfloat16>(uint32_t bits, uint32_t bz) {
+  const __nv_bfloat162 r =
+      __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&bits), *reinterpret_cast<const __nv_bfloat162*>(&bz));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+template <typename TX> struct QmvMagic;
+template <> struct QmvMagic<__half> { static constexpr uint32_t bits = 0x64006400u; static constexpr float base = 1024.f; };
+template <> struct QmvMagic<__nv_bfloat16> { static constexpr uint32_t bits = 0x43004300u; static constexpr float base = 128.f; };
+template <typename TX> __device__ __forceinline__ uint16_t qmv_to_bits(float v);
+template <> __device__ __forceinline__ uint16_t qmv_to_bits<__half>(float v) { return __half_as_ushort(__float2half_rn(v)); }
+template <> __device__ __forceinline__ uint16_t qmv_to_bits<__nv_bfloat16>(float v) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
 
 template <typename TX, int BITS, int M>
@@ -119,54 +181,245 @@ __global__ void __launch_bounds__(256) qmatvec_kernel(const int32_t* qweight, co
   // szs[gi][l] = (s0, s1, s2, s3), szs[gi][32 + l] = (z0, z1, z2, z3)
   float4* szs = reinterpret_cast<float4*>(red + 8 * 128);             // [QMV_MAXG][64]
   __shared__ int grange[3];
+  // the activations in the tensor-core order (fp16 / bf16 bits), [M][XHS]: rows 16 bytes
+  // longer than kc columns, so that the eight rows of a fragment load sit in distinct banks
+  constexpr int XHS = kc + 8;
+  uint16_t* xh = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(szs) + (size_t)QMV_MAXG * 64 * 16);
+  // the tensor-core form for one or two rows (measured: from four rows on, the fma form's
+  // shorter prologue and reduction win)
+  constexpr bool kTC = BITS == 4 && M <= 2 && !std::is_same<TX, float>::value;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int o0 = blockIdx.x * 128;
   const int k0 = blockIdx.y * kc;
   const int k1 = min(n, k0 + kc);
+  {
+    // the block's packed words (its kc / PER rows, 128 outputs) requested into L2 before the
+    // staging below: their DRAM latency overlaps the staging's dependent loads
+    const int nl = (min(128, out - o0) + 31) / 32;       // 128-byte lines per row
+    const int rows = k1 / PER - k0 / PER;
+    for (int i = threadIdx.x; i < rows * nl; i += blockDim.x)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(qweight + (int64_t)(k0 / PER + i / nl) * out + o0 + 32 * (i % nl)));
+  }
   if (threadIdx.x == 0) { grange[0] = INT_MAX; grange[1] = -1; grange[2] = 0; }
+  // Every global load of the staging is issued before any is used: the range's group
+  // indices and its activations (column k of the range multiplies X column xperm[k], or
+  // k); thread i holds columns i + 256 r.
+  constexpr int KPT = kc / 256;
+  int gv[KPT], xk[KPT];
+#pragma unroll
+  for (int r = 0; r < KPT; ++r) {
+    const int k = k0 + threadIdx.x + 256 * r;
+    gv[r] = k < k1 ? __ldg(g_idx + k) : -1;
+    xk[r] = k < k1 ? (xperm ? __ldg(xperm + k) : k) : -1;
+  }
+  float xv[M][KPT];
+#pragma unroll
+  for (int m = 0; m < M; ++m)
+#pragma unroll
+    for (int r = 0; r < KPT; ++r)
+      xv[m][r] = (xk[r] >= 0 && m < m_real) ? load_as_float<TX>(X + (int64_t)m * ldx + xk[r]) : 0.f;
   __syncthreads();
-  int gmin = INT_MAX, gmax = -1;
-  for (int i = threadIdx.x; i < kc; i += blockDim.x) {
-    int g = k0 + i < k1 ? g_idx[k0 + i] : -1;
-    if (g >= groups || (g < 0 && k0 + i < k1)) {     // a group index the scales do not have
+  // the range's groups: their span, and whether every packed word (PER columns; k0 is a
+  // multiple of PER) and every 32-column tile holds columns of one group
+  int gmin = INT_MAX, gmax = -1, split_word = 0, split_tile = 0;
+#pragma unroll
+  for (int r = 0; r < KPT; ++r) {
+    const int i = threadIdx.x + 256 * r;
+    const bool in = k0 + i < k1;
+    int g = gv[r];
+    if (g >= groups || (g < 0 && in)) {               // a group index the scales do not have
       set_error(st, GPTQ_ERR_INVALID_ARG, k0 + i, STAGE_DEQUANT);
       g = 0;
     }
-    if (k0 + i < k1) { gmin = min(gmin, g); gmax = max(gmax, g); }
-    gsm[i] = g < 0 ? 0 : g;
+    g = g < 0 ? 0 : g;
+    if (in) { gmin = min(gmin, g); gmax = max(gmax, g); }
+    gsm[i] = g;
+    const int gw = __shfl_sync(0xffffffffu, g, lane - lane % PER), gt = __shfl_sync(0xffffffffu, g, 0);
+    if (in && g != gw) split_word = 1;
+    if (in && g != gt) split_tile = 1;
   }
-  __syncthreads();
-  // does every packed word of the range hold columns of one group?  (k0 is a multiple of
-  // PER, so the words start at multiples of PER within the range)
-  int split_word = 0;
-  for (int i = threadIdx.x; i < k1 - k0; i += blockDim.x)
-    if (gsm[i] != gsm[i - i % PER]) split_word = 1;
-  if (__any_sync(0xffffffffu, split_word) && lane == 0) atomicOr(&grange[2], 1);
   for (int o = 16; o > 0; o >>= 1) {
     gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, o));
     gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
   }
-  if (lane == 0) { atomicMin(&grange[0], gmin); atomicMax(&grange[1], gmax); }
-  for (int i = threadIdx.x; i < M * kc; i += blockDim.x) {
-    const int m = i / kc, k = k0 + i % kc;
-    const int xk = k < k1 ? (xperm ? xperm[k] : k) : 0;
-    xs[i] = (k < k1 && m < m_real) ? load_as_float<TX>(X + (int64_t)m * ldx + xk) : 0.f;
+  split_word = __any_sync(0xffffffffu, split_word);
+  split_tile = __any_sync(0xffffffffu, split_tile);
+  if (lane == 0) {
+    atomicMin(&grange[0], gmin);
+    atomicMax(&grange[1], gmax);
+    if (split_word | split_tile) atomicOr(&grange[2], split_word | (split_tile << 1));
   }
   __syncthreads();
   const int g_lo = grange[0];
   const bool staged = grange[1] - g_lo < QMV_MAXG;
-  const bool uniform = grange[2] == 0;
+  const bool uniform = (grange[2] & 1) == 0;
+  // the tensor-core form (block-uniform): staged groups constant over each 32-column tile
+  bool tc = kTC && staged && (grange[2] & 2) == 0 && ((k1 - k0) & 31) == 0;
+  // the staged groups' scales and zero points, loaded before the activations are stored
+  constexpr int SZPT = (QMV_MAXG * 128 + 255) / 256;
+  const int nsz = staged ? (grange[1] - g_lo + 1) * 128 : 0;
+  uint16_t sv[SZPT], zv[SZPT];
+#pragma unroll
+  for (int r = 0; r < SZPT; ++r) {
+    const int i = threadIdx.x + 256 * r, oo = o0 + i % 128;
+    const bool in = i < nsz && oo < out;
+    sv[r] = in ? __ldg(scales + (int64_t)(g_lo + i / 128) * out + oo) : (uint16_t)0;
+    zv[r] = in ? __ldg(zeros + (int64_t)(g_lo + i / 128) * out + oo) : (uint16_t)0;
+  }
+  auto stage_xs = [&]() {
+#pragma unroll
+    for (int m = 0; m < M; ++m)
+#pragma unroll
+      for (int r = 0; r < KPT; ++r) xs[m * kc + threadIdx.x + 256 * r] = xv[m][r];
+  };
+  if constexpr (kTC) {
+    if (tc) {
+#pragma unroll
+      for (int m = 0; m < M; ++m)
+#pragma unroll
+        for (int r = 0; r < KPT; ++r) {
+          const int c = threadIdx.x + 256 * r;
+          xh[m * XHS + (c & ~31) + qmv_tc_slot(c & 31)] = qmv_to_bits<TX>(xv[m][r]);
+        }
+    } else {
+      stage_xs();
+    }
+  } else {
+    stage_xs();
+  }
   if (staged) {
     float* szf = reinterpret_cast<float*>(szs);
-    for (int i = threadIdx.x; i < (grange[1] - g_lo + 1) * 128; i += blockDim.x) {
-      const int gi = i / 128, oi = i % 128, oo = o0 + oi;
-      const bool in = oo < out;
-      szf[(gi * 64 + oi / 4) * 4 + oi % 4] =
-          in ? __half2float(__ushort_as_half(scales[(int64_t)(g_lo + gi) * out + oo])) : 0.f;
-      szf[(gi * 64 + 32 + oi / 4) * 4 + oi % 4] =
-          in ? __half2float(__ushort_as_half(zeros[(int64_t)(g_lo + gi) * out + oo])) : 0.f;
+    int odd_zero = 0;
+#pragma unroll
+    for (int r = 0; r < SZPT; ++r) {
+      const int i = threadIdx.x + 256 * r, gi = i / 128, oi = i % 128;
+      if (i < nsz) {
+        const float zf = __half2float(__ushort_as_half(zv[r]));
+        szf[(gi * 64 + oi / 4) * 4 + oi % 4] = __half2float(__ushort_as_half(sv[r]));
+        szf[(gi * 64 + 32 + oi / 4) * 4 + oi % 4] = zf;
+        // the tensor-core form subtracts z in fp16 / bf16: exact for integers in [0, 127]
+        if (!(zf >= 0.f && zf <= 127.f && zf == rintf(zf))) odd_zero = 1;
+      }
     }
-    __syncthreads();
+    if (kTC && __any_sync(0xffffffffu, odd_zero) && lane == 0) atomicOr(&grange[2], 4);
+  }
+  __syncthreads();
+  if constexpr (kTC) {
+    // the tensor-core form also wants integer zero points; a block that finds others (a
+    // layer edited by hand) stores the fp32 activations after all and takes the fma form
+    if (tc && (grange[2] & 4) != 0) {
+      tc = false;
+      stage_xs();
+      __syncthreads();
+    }
+    if (tc) {
+      const float* szf = reinterpret_cast<const float*>(szs);
+      const int g = lane >> 2, t = lane & 3;
+      const int qo = warp & 3, kh = warp >> 2;                 // output quarter, k half
+      const int ntile = (k1 - k0) >> 5;
+      const int tb = kh * ((ntile + 1) >> 1), te = min(ntile, tb + ((ntile + 1) >> 1));
+      float yacc[4][4], dacc[4][4];
+      uint32_t bz[4];
+#pragma unroll
+      for (int og = 0; og < 4; ++og)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) { yacc[og][e] = 0.f; dacc[og][e] = 0.f; }
+      int gcur = -1, nacc = 0;
+      auto flush = [&]() {
+#pragma unroll
+        for (int og = 0; og < 4; ++og) {
+          const int oi = 32 * qo + 8 * og + 2 * t;             // this lane's two accumulator columns
+          const float s0 = szf[(gcur * 64 + oi / 4) * 4 + oi % 4];
+          const float s1 = szf[(gcur * 64 + (oi + 1) / 4) * 4 + (oi + 1) % 4];
+          yacc[og][0] = fmaf(s0, dacc[og][0], yacc[og][0]);
+          yacc[og][1] = fmaf(s1, dacc[og][1], yacc[og][1]);
+          yacc[og][2] = fmaf(s0, dacc[og][2], yacc[og][2]);
+          yacc[og][3] = fmaf(s1, dacc[og][3], yacc[og][3]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dacc[og][e] = 0.f;
+        }
+        nacc = 0;
+      };
+      for (int tq = tb; tq < te; tq += 4) {
+      uint32_t q4[4][4];                                       // four tiles' words in flight
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t wrow = (int64_t)((k0 + (tq + u) * 32) / 8 + t) * out;
+#pragma unroll
+        for (int og = 0; og < 4; ++og) {
+          const int oo = o0 + 32 * qo + 8 * og + g;
+          q4[u][og] = (tq + u < te && oo < out) ? (uint32_t)__ldg(qweight + wrow + oo) : 0u;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int tt = tq + u;
+        if (tt >= te) break;
+        const int c0 = tt * 32;
+        const int gi = gsm[c0] - g_lo;
+        if (gi != gcur || nacc == 4) {                         // a group change, or 128 columns
+          if (gcur >= 0) flush();
+          if (gi != gcur) {
+            gcur = gi;
+#pragma unroll
+            for (int og = 0; og < 4; ++og) {                   // B + z for this lane's output
+              const int oi = 32 * qo + 8 * og + g;
+              const float zb = QmvMagic<TX>::base + szf[(gcur * 64 + 32 + oi / 4) * 4 + oi % 4];
+              const uint32_t h = qmv_to_bits<TX>(zb);
+              bz[og] = h | (h << 16);
+            }
+          }
+        }
+        // the activations: rows g and g + 8 of the two k halves of each mma
+        uint32_t a[2][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int sb = c0 + 16 * h + 2 * t;
+          a[h][0] = g < M ? *reinterpret_cast<const uint32_t*>(xh + g * XHS + sb) : 0u;
+          a[h][2] = g < M ? *reinterpret_cast<const uint32_t*>(xh + g * XHS + sb + 8) : 0u;
+          a[h][1] = g + 8 < M ? *reinterpret_cast<const uint32_t*>(xh + (g + 8) * XHS + sb) : 0u;
+          a[h][3] = g + 8 < M ? *reinterpret_cast<const uint32_t*>(xh + (g + 8) * XHS + sb + 8) : 0u;
+        }
+        const uint32_t* q = q4[u];
+#pragma unroll
+        for (int og = 0; og < 4; ++og) {
+          uint32_t b[4];
+#pragma unroll
+          for (int p = 0; p < 4; ++p)
+            b[p] = qmv_code_pair<TX>(((q[og] >> (4 * p)) & 0x000F000Fu) | QmvMagic<TX>::bits, bz[og]);
+          mma_16816<TX>(dacc[og], a[0], b[0], b[1]);
+          mma_16816<TX>(dacc[og], a[1], b[2], b[3]);
+        }
+        ++nacc;
+      }
+      }
+      if (gcur >= 0) flush();
+      // the 8 warps' sums in warp order (each output has two warps' terms, the rest zero)
+#pragma unroll 1
+      for (int m = 0; m < M; ++m) {
+        if (m >= m_real) break;
+        __syncthreads();
+        for (int i = lane; i < 128; i += 32) red[warp * 128 + i] = 0.f;
+        __syncwarp();
+        if (g == m || g + 8 == m) {
+          const int e0 = g == m ? 0 : 2;
+#pragma unroll
+          for (int og = 0; og < 4; ++og) {
+            red[warp * 128 + 32 * qo + 8 * og + 2 * t] = yacc[og][e0];
+            red[warp * 128 + 32 * qo + 8 * og + 2 * t + 1] = yacc[og][e0 + 1];
+          }
+        }
+        __syncthreads();
+        if (threadIdx.x < 128) {
+          const int oo = o0 + threadIdx.x;
+          float tsum = 0.f;
+#pragma unroll
+          for (int wp = 0; wp < 8; ++wp) tsum += red[wp * 128 + threadIdx.x];
+          if (oo < out) part[((int64_t)blockIdx.y * m_real + m) * out + oo] = tsum;
+        }
+      }
+      return;
+    }
   }
   const int o = o0 + 4 * lane;
   float acc[M][4];
@@ -178,6 +431,7 @@ __global__ void __launch_bounds__(256) qmatvec_kernel(const int32_t* qweight, co
   const int w0 = k0 / PER, w1 = k1 / PER;
   int g_prev = -1;
   float s[4] = {0.f, 0.f, 0.f, 0.f}, z[4] = {0.f, 0.f, 0.f, 0.f};
+  constexpr int I1U = M * PER >= 256 ? 4 : PER;     // the per-column loop's unrolling
   for (int wb = w0 + warp; wb < w1; wb += 8 * QMV_UNROLL) {
     uint32_t q[QMV_UNROLL][4];
 #pragma unroll
@@ -214,7 +468,10 @@ __global__ void __launch_bounds__(256) qmatvec_kernel(const int32_t* qweight, co
         const float n4[4] = {-sv.x * ((float)(1 << BITS) + zv.x), -sv.y * ((float)(1 << BITS) + zv.y),
                              -sv.z * ((float)(1 << BITS) + zv.z), -sv.w * ((float)(1 << BITS) + zv.w)};
         constexpr int POS = 23 - BITS;                 // where the code goes in the mantissa
-#pragma unroll
+        // fully unrolled unless the body is large (16 rows of 2-bit codes): then four
+        // columns at a time, the shift a register operand
+        constexpr int I0U = M * PER >= 256 ? 1 : PER / 4;
+#pragma unroll I0U
         for (int i0 = 0; i0 < PER; i0 += 4) {
           float wv[4][4];
 #pragma unroll
@@ -239,7 +496,7 @@ __global__ void __launch_bounds__(256) qmatvec_kernel(const int32_t* qweight, co
         }
         continue;
       }
-#pragma unroll
+#pragma unroll I1U
       for (int i = 0; i < PER; ++i) {
         const int kl = w * PER + i - k0;
         const int g = gsm[kl];

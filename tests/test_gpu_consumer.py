@@ -41,13 +41,22 @@ def _oracle_what(q):
 
 
 def _matvec_bound(X64, What):
-    """|Y_gpu - Y| <= (n + 24) . 2^-24 . sum_k |x_k . what_k|: every term is an exact product
-    of fp32 values (fp16 / bf16 activations and the exact What) added by one fma (one
-    rounding of at most 2^-24 of the running sum, itself at most the sum of |terms|); a
-    thread adds at most n terms, then the 8 warps' sums and the k splits (at most 16 more
-    additions at the tested sizes)."""
+    """|Y_gpu - Y| <= c . 2^-24 . sum_k |x_k . what_k|, c the larger of the two forms' counts.
+
+    CUDA cores: every term is an exact product of fp32 values (the activations and the exact
+    What) added by one fma (one rounding of at most 2^-24 of the running sum, itself at most
+    the sum of |terms|); a thread adds at most n terms, then the 8 warps' sums and the k
+    splits (at most 24 more additions): c = n + 24.
+    Tensor cores (4-bit codes, fp16 / bf16 activations): the products x . (code - z) are
+    exact; an accumulation holds at most 8 mma.sync of 16 columns, each summing 17 aligned
+    terms (16 products and the accumulator), each off by at most one ulp of that sum
+    whether the hardware rounds or truncates: <= 8 . 17 . 2^-23 of the accumulation's sum of
+    |terms|, which times s (> 0) is at most the sum of its |x . what|; each accumulation is
+    scaled and added by one fma (at most one per 32 columns), then the warps and the splits:
+    c = 272 + n / 32 + 9 + n / 256."""
     n = X64.shape[1]
-    return (n + 24) * 2.0 ** -24 * (np.abs(X64) @ np.abs(What).T)
+    c = max(n + 24, 272 + n // 32 + 9 + n // 256)
+    return c * 2.0 ** -24 * (np.abs(X64) @ np.abs(What).T)
 
 
 @pytest.mark.parametrize("bits,gs,sym,act", [(4, 128, False, False), (4, 64, True, True), (2, 32, False, True),
@@ -71,8 +80,8 @@ def test_dequantize_is_bit_exact(bits, gs, sym, act, dtype):
 
 
 @pytest.mark.parametrize("M", [1, 3, 8, 16])
-@pytest.mark.parametrize("bits,gs,act,xdt", [(4, 128, False, "f16"), (4, 128, True, "bf16"), (2, 64, True, "f16"),
-                                             (8, 32, False, "f32")])
+@pytest.mark.parametrize("bits,gs,act,xdt", [(4, 128, False, "f16"), (4, 128, True, "bf16"), (4, 64, False, "bf16"),
+                                             (2, 64, True, "f16"), (8, 32, False, "f32")])
 def test_qmatvec_against_the_oracle(M, bits, gs, act, xdt):
     # n = 1536: three 512-wide k splits; out = 250: a ragged last block of outputs (out % 4 != 0)
     q = _stored_layer(250, 1536, 3072, bits, gs, False, act, seed=M + bits)
@@ -91,9 +100,11 @@ def test_qmatvec_against_the_oracle(M, bits, gs, act, xdt):
     assert np.all(err <= _matvec_bound(X64, What)), float(np.max(err / _matvec_bound(X64, What)))
 
 
-def test_qmatvec_decode_shape_of_the_70b_mlp():
-    """gate of the 70B block, [28672 x 8192] 4-bit g128 act-order, one token: sampled
-    outputs against the oracle (rows are read from the stored bits one by one)."""
+@pytest.mark.parametrize("reordered", [False, True])
+def test_qmatvec_decode_shape_of_the_70b_mlp(reordered):
+    """gate of the 70B block, [28672 x 8192] 4-bit g128 act-order, one token, as stored and
+    reordered by group: sampled outputs against the oracle (rows are read from the stored
+    bits one by one)."""
     dev = _dev()
     out, n = 28672, 8192
     gen = torch.Generator(device=dev)
@@ -107,7 +118,11 @@ def test_qmatvec_decode_shape_of_the_70b_mlp():
                          codes=None, err_sq=None, bits=4, group_size=128, sym=False)
     X = torch.randn((1, n), generator=gen, device=dev).half()
     st = G.new_status(dev)
-    Y = G.qmatvec(q, X, st)
+    if reordered:
+        qg, xperm = G.reorder_groups(q, st)
+        Y = G.qmatvec(qg, X, st, xperm=xperm)
+    else:
+        Y = G.qmatvec(q, X, st)
     G.raise_on_status(st, "decode shape")
     cols = np.sort(np.random.default_rng(0).choice(out, 256, replace=False))
     qw = q.qweight.cpu().numpy()[:, cols]
@@ -154,6 +169,26 @@ def test_reordered_act_order_layer(bits, gs, M):
         q.qweight.device).half()
     Y = G.qmatvec(qg, X, st, xperm=xperm)
     G.raise_on_status(st, "reordered qmatvec")
+    X64 = X.float().cpu().numpy().astype(np.float64)
+    err = np.abs(Y.cpu().numpy().astype(np.float64) - X64 @ What.T)
+    assert np.all(err <= _matvec_bound(X64, What))
+
+
+@pytest.mark.parametrize("xdt", ["f16", "bf16"])
+def test_qmatvec_with_fractional_zero_points(xdt):
+    """Zero points off the integers (a stored layer edited by hand) are still applied in fp32:
+    the product is the oracle's within the summation bound."""
+    q = _stored_layer(256, 1024, 2048, 4, 128, False, False, seed=21)
+    zq = (q.zeros.float() + 0.25).half()
+    q2 = G.QuantizedLayer(q.qweight, q.scales, zq, q.g_idx, None, None, 4, 128, False)
+    dev = q.qweight.device
+    tdt = {"f16": torch.float16, "bf16": torch.bfloat16}[xdt]
+    X = torch.from_numpy(np.random.default_rng(4).standard_normal((3, 1024)).astype(np.float32)).to(dev).to(tdt)
+    st = G.new_status(dev)
+    Y = G.qmatvec(q2, X, st)
+    G.raise_on_status(st, "fractional zeros")
+    What = _oracle_what(q2)
+    assert not np.array_equal(What, _oracle_what(q))
     X64 = X.float().cpu().numpy().astype(np.float64)
     err = np.abs(Y.cpu().numpy().astype(np.float64) - X64 @ What.T)
     assert np.all(err <= _matvec_bound(X64, What))
