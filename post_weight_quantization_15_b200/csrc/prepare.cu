@@ -703,11 +703,76 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tp
   __syncthreads();
   GPTQ_PHASE_MARK(0);
 
+  // The factor-and-invert loop over the four 32-column sub-blocks (q = 32 p):
+  //   A  warp 0 factors the diagonal tile (the one-warp Cholesky).  Meanwhile the other
+  //      warps finish sub-block p - 1: its trailing tiles below the next diagonal tile,
+  //      its rows of T (T[q - 32 + a][c] = -T_pp Y), and they write out the split of
+  //      sub-block p - 2's rows of T, final since.
+  //   B  the rows below by forward substitution (into L and the scratch panel), T_pp,
+  //      and Y = L(p, :q) T(:q, :q).
+  //   C  the next diagonal tile's update (two 16 x 32 tiles), all that A of the next
+  //      sub-block reads.
+  // Lower 16 x 32 tiles of the trailing block of the sub-block at q: row tile rt
+  // (16 rows), column chunk ch <= rt / 2; tasks 0 and 1 are the next diagonal tile.
+  auto trail_task = [&](int q, int task) {
+    int rt = 0, rem = task;
+    while (rem >= rt / 2 + 1) { rem -= rt / 2 + 1; ++rt; }
+    const int ch = rem;
+    float acc[4][4] = {};
+    mma_tile_16x32<false>(Ps + 16 * rt * LDP, LDP, Ps + 32 * ch * LDP, LDP, 32, lane, acc);
+    const int i0 = q + 32 + 16 * rt, c0 = q + 32 + 32 * ch;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      float2* e0 = reinterpret_cast<float2*>(Ls + (i0 + g) * LDL + c0 + 8 * s + 2 * t4);
+      float2* e1 = reinterpret_cast<float2*>(Ls + (i0 + g + 8) * LDL + c0 + 8 * s + 2 * t4);
+      float2 v0 = *e0, v1 = *e1;
+      v0.x -= acc[s][0]; v0.y -= acc[s][1]; v1.x -= acc[s][2]; v1.y -= acc[s][3];
+      *e0 = v0; *e1 = v1;
+    }
+  };
+  auto trail_tasks = [](int q) {
+    const int rt_n = (PB - q - 32) / 16;
+    int ntc = 0;
+    for (int rt = 0; rt < rt_n; ++rt) ntc += rt / 2 + 1;
+    return ntc;
+  };
+  // T[q + a][c] = -sum_b T_pp[a][b] Y[b][c] (T_pp[a][b] = 0 for b > a), rows a0 .. a0 + 16,
+  // columns 32 ch ..
+  auto t_task = [&](int q, int u) {
+    const int a0 = 16 * (u & 1), ch = u >> 1;
+    float acc[4][4] = {};
+    mma_tile_16x32<true>(Ts + (q + a0) * LDL + q, LDL, Ys + 32 * ch, LDY, a0 + 16, lane, acc);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      float* t0 = Ts + (q + a0 + g) * LDL + 32 * ch + 8 * s + 2 * t4;
+      *reinterpret_cast<float2*>(t0) = make_float2(-acc[s][0], -acc[s][1]);
+      *reinterpret_cast<float2*>(t0 + 8 * LDL) = make_float2(-acc[s][2], -acc[s][3]);
+    }
+  };
+  // the TF32 split of T's rows r0 .. r0 + 32 (L_kk itself is not needed later: the
+  // trailing steps use L21 and T; the block of Xt comes from this split, off this chain)
+  auto write_rows = [&](int r0, int first, int stride) {
+#pragma unroll 4
+    for (int idx = first; idx < 32 * PB / 4; idx += stride) {
+      const int i = r0 + idx / (PB / 4), k = 4 * (idx % (PB / 4));
+      const float4 v = *reinterpret_cast<const float4*>(Ts + i * LDL + k);
+      float e[4] = {v.x, v.y, v.z, v.w}, h[4], l[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (i >= nb || k + u >= nb) e[u] = 0.f;
+        h[u] = tf32_hi(e[u]);
+        l[u] = e[u] - h[u];
+      }
+      *reinterpret_cast<float4*>(LIhi + i * PB + k) = make_float4(h[0], h[1], h[2], h[3]);
+      *reinterpret_cast<float4*>(LIlo + i * PB + k) = make_float4(l[0], l[1], l[2], l[3]);
+    }
+  };
+
 #pragma unroll 1
   for (int p = 0; p < 4; ++p) {
     const int q = 32 * p;
     const int R = PB - q - 32;          // rows below the sub-block
-    // ---- A ----
+    // ---- A (and the rest of sub-block p - 1) ----
     if (warp == 0) {
       int bj, bn;
       chol32(Ls, Cs, Rv + q, q, lane, &bj, &bn);
@@ -715,6 +780,15 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tp
         bad = 1;
         set_error(st, bn ? GPTQ_ERR_NONFINITE : GPTQ_ERR_NOT_SPD, n - 1 - (k0 + q + bj), STAGE_POTRF);
       }
+    } else if (p > 0) {
+      const int qp = q - 32;
+      const int nrest = trail_tasks(qp) - 2;
+#pragma unroll 1
+      for (int task = warp - 1; task < nrest + 2 * (p - 1); task += NWARP - 1) {
+        if (task < nrest) trail_task(qp, task + 2);
+        else t_task(qp, task - nrest);
+      }
+      if (p > 1) write_rows(q - 64, tid - 32, DT - 32);
     }
     __syncthreads();
     GPTQ_PHASE_MARK(1 + 3 * p);
@@ -760,62 +834,17 @@ potrf_inv_kernel(const float* A, int lda, int k0, int nb, int n, const float* Tp
     }
     __syncthreads();
     GPTQ_PHASE_MARK(2 + 3 * p);
-    // ---- C ----
-    const int rt_n = R / 16;            // trailing row tiles (16 rows), column chunks <= rt / 2
-    int ntc = 0;
-    for (int rt = 0; rt < rt_n; ++rt) ntc += rt / 2 + 1;
-    const int ntasks = ntc + 2 * p;
-#pragma unroll 1
-    for (int task = warp; task < ntasks; task += NWARP) {
-      float acc[4][4] = {};
-      if (task < ntc) {
-        int rt = 0, rem = task;
-        while (rem >= rt / 2 + 1) { rem -= rt / 2 + 1; ++rt; }
-        const int ch = rem;
-        mma_tile_16x32<false>(Ps + 16 * rt * LDP, LDP, Ps + 32 * ch * LDP, LDP, 32, lane, acc);
-        const int i0 = q + 32 + 16 * rt, c0 = q + 32 + 32 * ch;
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          float2* e0 = reinterpret_cast<float2*>(Ls + (i0 + g) * LDL + c0 + 8 * s + 2 * t4);
-          float2* e1 = reinterpret_cast<float2*>(Ls + (i0 + g + 8) * LDL + c0 + 8 * s + 2 * t4);
-          float2 v0 = *e0, v1 = *e1;
-          v0.x -= acc[s][0]; v0.y -= acc[s][1]; v1.x -= acc[s][2]; v1.y -= acc[s][3];
-          *e0 = v0; *e1 = v1;
-        }
-      } else {
-        // T[q + a][c] = -sum_b T_pp[a][b] Y[b][c]; T_pp[a][b] = 0 for b > a
-        const int u = task - ntc;
-        const int a0 = 16 * (u & 1), ch = u >> 1;
-        mma_tile_16x32<true>(Ts + (q + a0) * LDL + q, LDL, Ys + 32 * ch, LDY, a0 + 16, lane, acc);
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          float* t0 = Ts + (q + a0 + g) * LDL + 32 * ch + 8 * s + 2 * t4;
-          *reinterpret_cast<float2*>(t0) = make_float2(-acc[s][0], -acc[s][1]);
-          *reinterpret_cast<float2*>(t0 + 8 * LDL) = make_float2(-acc[s][2], -acc[s][3]);
-        }
-      }
-    }
+    // ---- C: the next diagonal tile ----
+    if (R > 0 && warp < 2) trail_task(q, warp);
     __syncthreads();
     GPTQ_PHASE_MARK(3 + 3 * p);
   }
+  // the last sub-block's rows of T, sub-block 2's rows written out meanwhile
+  if (warp < 6) t_task(96, warp);
+  else write_rows(64, tid - 192, DT - 192);
+  __syncthreads();
   if (bad) return;
-
-  // output: the TF32 split of T (L_kk itself is not needed later: the trailing
-  // steps use L21 and T; the block of Xt comes from this split, off this chain)
-#pragma unroll 4
-  for (int idx = tid; idx < PB * PB / 4; idx += DT) {
-    const int i = idx / (PB / 4), k = 4 * (idx % (PB / 4));
-    const float4 v = *reinterpret_cast<const float4*>(Ts + i * LDL + k);
-    float e[4] = {v.x, v.y, v.z, v.w}, h[4], l[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (i >= nb || k + u >= nb) e[u] = 0.f;
-      h[u] = tf32_hi(e[u]);
-      l[u] = e[u] - h[u];
-    }
-    *reinterpret_cast<float4*>(LIhi + i * PB + k) = make_float4(h[0], h[1], h[2], h[3]);
-    *reinterpret_cast<float4*>(LIlo + i * PB + k) = make_float4(l[0], l[1], l[2], l[3]);
-  }
+  write_rows(96, tid, DT);
   GPTQ_PHASE_MARK(13);
 }
 
