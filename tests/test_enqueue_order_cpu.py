@@ -378,3 +378,106 @@ def test_deferred_loop_missing_wait_is_reported(label):
 def test_implied_waits(model, label):
     races, err = _check(model, 2600 if model is model_panel_loop_deferred else 1700, skip=(label,))
     assert races == [] and err < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# The quantizer's two streams (`csrc/quantize.cu`, super_block_loop): per super-block
+# of SBK = 512 columns, on the high-priority stream the sweep (its columns, the scaled
+# errors E[b]) and the update of the next super-block's columns (near); on the other
+# stream the operand B[b] = U[super-block, later columns]^T and the update of all
+# columns after that (far).  E and B are double buffers (b = super-block mod 2).
+# The sweep is modelled by GPTQ's column step without the group machinery: round the
+# column, its error over the pivot, the update of the block's later columns; the
+# whole order must then equal the unblocked column loop.
+# ---------------------------------------------------------------------------
+SBK = 512
+
+
+def model_super_block_loop(out, n, skip=(), seed=0):
+    rng = np.random.default_rng(seed)
+    W0 = rng.standard_normal((out, n)) * 4.0
+    U = np.triu(rng.standard_normal((n, n)) * 0.02, 1) + np.diag(1.0 + rng.random(n))
+    Wf = W0.copy()
+    codes = np.full((out, n), np.nan)
+    E = [np.full((out, SBK), np.nan) for _ in range(2)]
+    B = [np.full((n, SBK), np.nan) for _ in range(2)]
+    sim = Sim(skip)
+    hi, lo = "hi", "lo"
+    S = -(-n // SBK)
+
+    def operand(sb):
+        b0, be, bb = sb * SBK, sb * SBK + SBK, sb & 1
+
+        def fn():
+            B[bb][:n - be, :] = U[b0:be, be:n].T
+        sim.op(lo, [], [R(("B", bb), 0, n, 0, SBK)], fn, f"operand{sb}")
+        sim.record(("opnd", bb), lo)
+
+    for sb in range(min(2, S - 1)):
+        operand(sb)
+    for sb in range(S):
+        b, s0 = sb & 1, sb * SBK
+        se = min(n, s0 + SBK)
+
+        def fn(b=b, s0=s0, se=se):
+            for j in range(s0, se):
+                q = np.round(Wf[:, j])
+                codes[:, j] = q
+                e = (Wf[:, j] - q) / U[j, j]
+                E[b][:, j - s0] = e
+                Wf[:, j + 1:se] -= np.outer(e, U[j, j + 1:se])
+        sim.op(hi, [R("W", 0, out, s0, se)], [R("W", 0, out, s0, se), R(("E", b), 0, out, 0, SBK),
+                                              R("codes", 0, out, s0, se)], fn, f"sweep{sb}")
+        if se >= n:
+            break
+        kn = min(SBK, n - se)
+        sim.record("swept", hi)
+        sim.wait(hi, ("opnd", b), "hi_opnd")
+        if sb > 0:
+            sim.wait(hi, "far", "hi_far")
+
+        def fn(b=b, se=se, kn=kn):
+            Wf[:, se:se + kn] -= E[b] @ B[b][:kn].T
+        sim.op(hi, [R(("E", b), 0, out, 0, SBK), R(("B", b), 0, kn, 0, SBK), R("W", 0, out, se, se + kn)],
+               [R("W", 0, out, se, se + kn)], fn, f"near{sb}")
+        sim.record("near", hi)
+        if n - se > kn:
+            sim.wait(lo, "swept", "lo_swept")
+
+            def fn(b=b, se=se, kn=kn):
+                Wf[:, se + kn:] -= E[b] @ B[b][kn:n - se].T
+            sim.op(lo, [R(("E", b), 0, out, 0, SBK), R(("B", b), kn, n - se, 0, SBK), R("W", 0, out, se + kn, n)],
+                   [R("W", 0, out, se + kn, n)], fn, f"far{sb}")
+        sim.record("far", lo)
+        if sb + 2 < S - 1:
+            sim.wait(lo, "near", "lo_near")
+            operand(sb + 2)
+    return sim, W0, U, codes
+
+
+def _check_quantizer(out, n, skip=()):
+    sim, W0, U, codes = model_super_block_loop(out, n, skip)
+    races = sim.races()
+    sim.run()
+    W = W0.copy()
+    ref = np.empty_like(W)
+    for j in range(n):                      # the unblocked column loop
+        q = np.round(W[:, j])
+        ref[:, j] = q
+        e = (W[:, j] - q) / U[j, j]
+        W[:, j + 1:] -= np.outer(e, U[j, j + 1:])
+    return races, np.array_equal(codes, ref)
+
+
+# one super-block, two, and several with a ragged last one (every buffer reused)
+@pytest.mark.parametrize("n", [300, 1024, 1800, 2600])
+def test_quantizer_streams_are_race_free_and_match_the_column_loop(n):
+    races, same = _check_quantizer(8, n)
+    assert races == [], races[:4]
+    assert same
+
+
+@pytest.mark.parametrize("label", ["hi_opnd", "hi_far", "lo_swept", "lo_near"])
+def test_quantizer_missing_wait_is_reported(label):
+    races, _ = _check_quantizer(8, 2600, skip=(label,))
+    assert races, label
