@@ -1,4 +1,4 @@
-"""The preparation's multi-stream enqueue order, replayed on the CPU.
+"""The multi-stream enqueue orders of the preparation and of the quantizer, replayed on the CPU.
 
 `csrc/prepare.cu` factors A = L L^T and builds Xt = (L^-1)^T panel by panel on four
 streams (c: the diagonal blocks, o: L21 and the next block column, t: trailing
@@ -23,6 +23,10 @@ launch's wait for the inverse reach them first), its wait for the previous outer
 bulk update (panel_loop_deferred; the in-panel waits for the trailing stream reach it), and
 the inverse stream's wait for the outer panel's L21 (its per-panel L21 waits reach it).
 They stay in the C++ so that every launch states its own inputs.
+
+The quantizer's two streams (`csrc/quantize.cu`, super_block_loop) are replayed the same
+way at the end of the module; there every wait is load-bearing, and the blocked order
+must give the codes of the unblocked column loop.
 
 The restatement must change with the C++ loops: it is a model of them, not derived
 from them.  The GPU tests check the result of the real enqueue against the oracle.
