@@ -79,7 +79,7 @@ def test_dequantize_is_bit_exact(bits, gs, sym, act, dtype):
         assert np.array_equal(got.view(torch.int16).cpu().numpy().view(np.uint16), bits_ref)
 
 
-@pytest.mark.parametrize("M", [1, 3, 8, 16])
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 16])
 @pytest.mark.parametrize("bits,gs,act,xdt", [(4, 128, False, "f16"), (4, 128, True, "bf16"), (4, 64, False, "bf16"),
                                              (2, 64, True, "f16"), (8, 32, False, "f32")])
 def test_qmatvec_against_the_oracle(M, bits, gs, act, xdt):
@@ -174,16 +174,18 @@ def test_reordered_act_order_layer(bits, gs, M):
     assert np.all(err <= _matvec_bound(X64, What))
 
 
+@pytest.mark.parametrize("rows", [1, 2, 3])
 @pytest.mark.parametrize("xdt", ["f16", "bf16"])
-def test_qmatvec_with_fractional_zero_points(xdt):
-    """Zero points off the integers (a stored layer edited by hand) are still applied in fp32:
+def test_qmatvec_with_fractional_zero_points(xdt, rows):
+    """Zero points off the integers (a stored layer edited by hand) are still applied in fp32
+    (one and two rows: the blocks fall back from the tensor-core form; three: the fma form):
     the product is the oracle's within the summation bound."""
     q = _stored_layer(256, 1024, 2048, 4, 128, False, False, seed=21)
     zq = (q.zeros.float() + 0.25).half()
     q2 = G.QuantizedLayer(q.qweight, q.scales, zq, q.g_idx, None, None, 4, 128, False)
     dev = q.qweight.device
     tdt = {"f16": torch.float16, "bf16": torch.bfloat16}[xdt]
-    X = torch.from_numpy(np.random.default_rng(4).standard_normal((3, 1024)).astype(np.float32)).to(dev).to(tdt)
+    X = torch.from_numpy(np.random.default_rng(4).standard_normal((rows, 1024)).astype(np.float32)).to(dev).to(tdt)
     st = G.new_status(dev)
     Y = G.qmatvec(q2, X, st)
     G.raise_on_status(st, "fractional zeros")
