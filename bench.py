@@ -301,7 +301,7 @@ def hessian_traffic(n: int, tokens: int):
 
 
 def measure_peaks(G, torch, dev):
-    """Denominators the driver does not measure: the dense tf32 tensor-core peak
+    """Denominators MEASURED_PEAKS.json does not hold: the dense tf32 tensor-core peak
     (torch.matmul on fp32 with TF32 allowed, 8192^3, best of 10 — the method of the
     measured bf16 peak) and the FP32 CUDA-core peak (the library's FMA probe, best of 5)."""
     out = {}

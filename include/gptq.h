@@ -60,7 +60,7 @@ extern "C" {
 typedef enum {
   GPTQ_OK = 0,
   GPTQ_ERR_INVALID_ARG = -1,  /* a pointer, size or stride is invalid               */
-  GPTQ_ERR_UNSUPPORTED = -2,  /* a valid combination this build does not implement */
+  GPTQ_ERR_UNSUPPORTED = -2,  /* a valid combination the library does not implement */
   GPTQ_ERR_NOT_SPD = -3,      /* damped Hessian not positive definite; info = pivot  */
   GPTQ_ERR_NONFINITE = -4,    /* NaN/Inf in W or H; info = column or pivot           */
   GPTQ_ERR_CUDA = -5,         /* a CUDA runtime call failed                          */
